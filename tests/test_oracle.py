@@ -1,0 +1,422 @@
+"""Pins of the CPU oracle against what the RouteRelay page and mathematics fix.
+
+Page: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
+Dynamic Sparse Attention" (arXiv 2609.07306), cited as RouteRelay §x.
+Each test names the fact it pins and would fail on a plausible slip in the
+oracle (dropped term, wrong sign/index, transposed operand, wrong tie order,
+wrong counting rule).
+"""
+import math
+import os
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle import Params
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def rownorm(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+# --------------------------------------------------------------- Eq. 1 --
+def test_scores_match_float64_matmul_and_are_not_transposed():
+    rng = np.random.default_rng(1)
+    q = rng.standard_normal((7, 13)).astype(np.float32)
+    k = rng.standard_normal((11, 13)).astype(np.float32)
+    S = oracle.scores(q, k)
+    ref = q.astype(np.float64) @ k.astype(np.float64).T
+    assert S.shape == (7, 11)
+    np.testing.assert_allclose(S, ref, rtol=1e-12, atol=1e-12)
+    # no 1/sqrt(d) scaling (the scaling of Eq. 3 belongs to attention)
+    e = np.eye(13, dtype=np.float32)
+    assert np.array_equal(oracle.scores(e[:3] * 2, e[:3]), np.diag([2.0, 2.0, 2.0]))
+
+
+def test_valid_count_causal():
+    assert [oracle.valid_count(i, 5, True) for i in range(7)] == [1, 2, 3, 4, 5, 5, 5]
+    assert [oracle.valid_count(i, 5, False) for i in range(3)] == [5, 5, 5]
+
+
+# --------------------------------------------------------------- Eq. 2 --
+def _rank_by_counting(s):
+    """Independent definition: rank_j = #{j' : s_j' > s_j or (s_j' == s_j and j' < j)}."""
+    n = len(s)
+    rank = np.empty(n, dtype=np.int64)
+    for j in range(n):
+        rank[j] = sum(1 for jj in range(n) if s[jj] > s[j] or (s[jj] == s[j] and jj < j))
+    order = np.empty(n, dtype=np.int64)
+    order[rank] = np.arange(n)
+    return order
+
+
+@pytest.mark.parametrize("trial", range(40))
+def test_route_row_equals_brute_force_ranks(trial):
+    rng = np.random.default_rng(100 + trial)
+    n = int(rng.integers(1, 17))
+    if trial % 2:
+        s = rng.integers(-3, 4, size=n).astype(np.float64)  # many exact ties
+    else:
+        s = rng.standard_normal(n)
+    order = _rank_by_counting(s)
+    for k in range(1, n + 2):
+        for m in (0, 1, 3, n):
+            route, near, alpha = oracle.route_row(s, n, k, m)
+            nr = min(k, n)
+            nm = min(m, n - nr)
+            assert list(route[:nr]) == list(order[:nr])
+            assert all(x == -1 for x in route[nr:])
+            assert list(near[:nm]) == list(order[nr:nr + nm])
+            assert all(x == -1 for x in near[nm:])
+            assert alpha == min(s[j] for j in order[:nr])
+
+
+def test_route_row_closed_forms():
+    s = np.array([0.5, -1.0, 2.0, 0.25])
+    route, near, alpha = oracle.route_row(s, 4, 4, 2)
+    assert list(route) == [2, 0, 3, 1] and list(near) == [-1, -1]
+    assert alpha == s.min()
+    # causal prefix: only the first n_valid entries are candidates
+    route, near, alpha = oracle.route_row(np.array([1.0, 9.0, 8.0]), 1, 2, 1)
+    assert list(route) == [0, -1] and list(near) == [-1] and alpha == 1.0
+    # equal scores: ascending index wins
+    route, near, _ = oracle.route_row(np.array([1.0, 1.0, 1.0, 0.0]), 4, 2, 1)
+    assert list(route) == [0, 1] and list(near) == [2]
+
+
+# ------------------------------------------------------------ Philox ----
+def test_philox_matches_torch_engine():
+    """Cross-check against torch's own Philox4x32-10 engine (an independent
+    implementation of Salmon et al., SC'11) compiled on the host."""
+    import torch
+    inc = os.path.join(os.path.dirname(torch.__file__), "include")
+    src = os.path.join(HERE, "_philox_torch_check.cpp")
+    exe = os.path.join(HERE, "..", "_build", "philox_torch_check")
+    os.makedirs(os.path.dirname(exe), exist_ok=True)
+    subprocess.check_call(["g++", "-std=c++17", "-O1", "-I" + inc, "-o", exe, src])
+    rng = np.random.default_rng(7)
+    cases = [(0, 0, 0, 0, 0, 0), (0xFFFFFFFF,) * 6]
+    cases += [tuple(int(x) for x in rng.integers(0, 2**32, size=6)) for _ in range(30)]
+    inp = "\n".join(" ".join(str(v) for v in c) for c in cases) + "\n"
+    out = subprocess.run([exe], input=inp, capture_output=True, text=True, check=True).stdout.split("\n")
+    for c, line in zip(cases, out):
+        want = [int(x, 16) for x in line.split()]
+        got = oracle.philox4x32_10(c[:4], c[4:])
+        assert list(got) == want, (c, got, want)
+
+
+# ------------------------------------------------- random sentinels -----
+def test_random_sentinels_distinct_in_pool_and_fill():
+    rng = np.random.default_rng(3)
+    for trial in range(300):
+        n = int(rng.integers(1, 80))
+        n_ex = int(rng.integers(0, min(n, 30) + 1))
+        excl = rng.choice(n, size=n_ex, replace=False).astype(np.int32)
+        excl = np.concatenate([excl, np.full(int(rng.integers(0, 3)), -1, np.int32)])
+        r = int(rng.integers(1, 20))
+        out, draws = oracle.random_sentinels(trial, trial % 5, trial % 97, trial % 31, n, excl, r, 64 * 40)
+        pool = sorted(set(range(n)) - set(int(x) for x in excl if x >= 0))
+        got = [int(x) for x in out if x >= 0]
+        assert len(set(got)) == len(got)
+        assert set(got) <= set(pool)
+        assert len(got) == min(r, len(pool))
+        assert all(x == -1 for x in out[len(got):])
+        if len(pool) <= r:
+            assert got == pool and draws == 0
+
+
+def test_random_sentinels_first_draw_is_multiply_shift_of_philox_word0():
+    seed, bh, row, layer, n = 0x1234_5678_9ABC_DEF0, 3, 17, 5, 1000
+    w = oracle.philox4x32_10([bh, row, layer, 0], [seed & 0xFFFFFFFF, seed >> 32])
+    out, _ = oracle.random_sentinels(seed, bh, row, layer, n, [], 1, 64)
+    assert out[0] == (int(w[0]) * n) >> 32
+
+
+def test_random_sentinels_uniform_chi2():
+    """Uniform over the residual pool (RouteRelay §3.1 item 2, §3.4)."""
+    n, r = 40, 4
+    excl = np.arange(0, 40, 4, dtype=np.int32)  # 10 excluded
+    pool = sorted(set(range(n)) - set(excl.tolist()))
+    counts = {j: 0 for j in pool}
+    trials = 6000
+    for t in range(trials):
+        out, _ = oracle.random_sentinels(11, t % 7, t // 7, 2, n, excl, r, 64 * 24)
+        for j in out:
+            counts[int(j)] += 1
+    obs = np.array([counts[j] for j in pool], dtype=np.float64)
+    exp = trials * r / len(pool)
+    chi2 = float(((obs - exp) ** 2 / exp).sum())
+    # 29 degrees of freedom: the 99.9% quantile is 58.3
+    assert chi2 < 58.3, chi2
+
+
+def test_random_sentinels_miss_probability_eq10():
+    """RouteRelay §3.4 Eq. 10: with u challengers in a residual pool of size
+    N and r draws without replacement, P(miss all) = C(N-u, r)/C(N, r)."""
+    n_valid, u, r = 60, 5, 6
+    excl = np.arange(0, 12, dtype=np.int32)  # pool = 12..59, N = 48
+    Np = n_valid - len(excl)
+    challengers = set(range(30, 30 + u))
+    p = math.comb(Np - u, r) / math.comb(Np, r)
+    assert p <= (1 - u / Np) ** r  # the page's bound
+    trials = 8000
+    miss = 0
+    for t in range(trials):
+        out, _ = oracle.random_sentinels(99, 1, t, 3, n_valid, excl, r, 64 * 30)
+        if not (set(int(x) for x in out) & challengers):
+            miss += 1
+    sd = math.sqrt(p * (1 - p) / trials)
+    assert abs(miss / trials - p) < 3.3 * sd, (miss / trials, p)
+
+
+# ---------------------------------------------------------- layers ------
+def _layer_inputs(seed, bh, n, d, scale=1.0):
+    rng = np.random.default_rng(seed)
+    q = rownorm(rng.standard_normal((bh, n, d))).astype(np.float32)
+    k = rownorm(rng.standard_normal((bh, n, d))).astype(np.float32)
+    return q, k
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_anchor_rows_are_full_routes_with_sentinels(causal):
+    p = Params(nq=40, nk=40, d=16, k=5, m=4, r=3, causal=causal, seed=5)
+    q, k = _layer_inputs(0, 1, 40, 16)
+    led = oracle.HeadLedger.empty(p)
+    flags, beta, ref, pairs, st = oracle.head_layer(p, 0, 0, True, q[0], k[0], led)
+    assert st == 0 and ref == 40 and flags.all()
+    S = q[0].astype(np.float64) @ k[0].astype(np.float64).T
+    nv = [oracle.valid_count(i, 40, causal) for i in range(40)]
+    assert pairs == sum(nv)
+    for i in range(40):
+        order = _rank_by_counting(S[i, : nv[i]])
+        nr = min(5, nv[i]); nm = min(4, nv[i] - nr)
+        assert list(led.ids[i, :nr]) == list(order[:nr])
+        assert list(led.ids[i, 5:5 + nm]) == list(order[nr:nr + nm])
+        assert led.alpha[i] == S[i, order[nr - 1]]
+        rand = [int(x) for x in led.ids[i, 9:] if x >= 0]
+        assert set(rand).isdisjoint(set(order[: nr + nm].tolist()))
+        assert len(rand) == min(3, nv[i] - nr - nm)
+        assert led.anchor_layer[i] == 0
+
+
+def test_zero_drift_relay_keeps_every_route():
+    """Same Q, K at the relay layer, distinct scores: alpha is the rank-k
+    score and beta is at most the rank-(k+1) score, so Eq. 8 holds strictly
+    for every row and no row refreshes."""
+    p = Params(nq=64, nk=96, d=32, k=8, m=6, r=4, seed=1)
+    q, k = _layer_inputs(2, 1, 96, 32)
+    q = q[:, :64]
+    led = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q[0], k[0], led)
+    before = led.copy()
+    flags, beta, ref, pairs, st = oracle.head_layer(p, 0, 1, False, q[0], k[0], led)
+    assert st == 0 and ref == 0 and not flags.any()
+    assert np.array_equal(led.ids, before.ids)
+    assert np.array_equal(led.alpha, before.alpha)
+    assert np.array_equal(led.anchor_layer, before.anchor_layer)
+    assert pairs == 64 * p.c
+
+
+def test_lemma1_bounded_perturbation_keeps_routes_and_raises_no_flag():
+    """RouteRelay §3.3 Lemma 1: max_j |S^l - S^a| <= eps and Delta > 2 eps
+    imply R^l = R^a; the relay test then also passes (alpha^l >= alpha^a -
+    eps > max_{j not in R} S^a + eps >= beta^l)."""
+    p = Params(nq=48, nk=64, d=24, k=6, m=5, r=4, seed=2)
+    rng = np.random.default_rng(4)
+    q, k = _layer_inputs(5, 1, 64, 24)
+    q0 = q[0, :48].astype(np.float32)
+    k0 = k[0]
+    S_a = q0.astype(np.float64) @ k0.astype(np.float64).T
+    srt = -np.sort(-S_a, axis=1)
+    delta = srt[:, p.k - 1] - srt[:, p.k]  # Eq. 9 anchor margin
+    kmax = np.linalg.norm(k0.astype(np.float64), axis=1).max()
+    eps = 0.4 * delta
+    d = rng.standard_normal(q0.shape)
+    d = d / np.linalg.norm(d, axis=1, keepdims=True) * (eps / kmax)[:, None]
+    q1 = (q0.astype(np.float64) + d).astype(np.float32)
+    S_l = q1.astype(np.float64) @ k0.astype(np.float64).T
+    assert (np.abs(S_l - S_a).max(axis=1) <= 0.45 * delta).all()
+    led = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q0, k0, led)
+    anchor_routes = led.ids[:, : p.k].copy()
+    flags, beta, ref, pairs, st = oracle.head_layer(p, 0, 1, False, q1, k0, led)
+    assert not flags.any() and ref == 0
+    exact = oracle.exact_topk(p, q1, k0)
+    for i in range(48):
+        assert set(exact[i].tolist()) == set(anchor_routes[i].tolist())
+
+
+def test_stability_condition_and_refresh_semantics():
+    """Eq. 8 with a guard margin: rows with alpha > beta + gamma keep their
+    ids bit for bit; the others are rebuilt as full routes at this layer."""
+    for gamma in (0.0, 0.05):
+        p = Params(nq=80, nk=80, d=16, k=6, m=6, r=4, causal=True, gamma=gamma, seed=9)
+        rng = np.random.default_rng(6)
+        q0, k0 = _layer_inputs(7, 1, 80, 16)
+        q1 = rownorm(q0[0] + 0.3 * rng.standard_normal(q0[0].shape)).astype(np.float32)
+        k1 = rownorm(k0[0] + 0.3 * rng.standard_normal(k0[0].shape)).astype(np.float32)
+        led = oracle.HeadLedger.empty(p)
+        oracle.head_layer(p, 0, 0, True, q0[0], k0[0], led)
+        before = led.copy()
+        flags, beta, ref, pairs, st = oracle.head_layer(p, 0, 3, False, q1, k1, led)
+        S = q1.astype(np.float64) @ k1.astype(np.float64).T
+        n_cand = 0
+        for i in range(80):
+            nv = oracle.valid_count(i, 80, True)
+            ids = before.ids[i]
+            r_ids = [j for j in ids[: p.k] if j >= 0]
+            c_ids = [j for j in ids[p.k:] if j >= 0]
+            n_cand += len(r_ids) + len(c_ids)
+            a = min(S[i, j] for j in r_ids)
+            b = max((S[i, j] for j in c_ids), default=-np.inf)
+            assert beta[i] == b
+            if a > b + gamma:
+                assert flags[i] == 0
+                assert np.array_equal(led.ids[i], before.ids[i])
+                assert led.alpha[i] == a and led.anchor_layer[i] == 0
+            else:
+                assert flags[i] == 1 and led.anchor_layer[i] == 3
+                route, near, alpha = oracle.route_row(S[i, :nv], nv, p.k, p.m)
+                assert list(led.ids[i, : p.k]) == list(route)
+                assert list(led.ids[i, p.k:p.k + p.m]) == list(near)
+                excl = np.concatenate([route, near])
+                rand, _ = oracle.random_sentinels(p.seed, 0, i, 3, nv, excl, p.r, 64 * p.c)
+                assert list(led.ids[i, p.k + p.m:]) == list(rand)
+                assert led.alpha[i] == alpha
+        assert ref == int(flags.sum())
+        assert pairs == n_cand + sum(oracle.valid_count(i, 80, True) for i in range(80) if flags[i])
+        if gamma > 0:
+            assert flags.sum() > 0
+
+
+def test_rows_with_at_most_k_valid_chunks_never_refresh():
+    p = Params(nq=10, nk=10, d=8, k=4, m=2, r=2, causal=True, seed=0)
+    q0, k0 = _layer_inputs(8, 1, 10, 8)
+    q1, k1 = _layer_inputs(9, 1, 10, 8)
+    led = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q0[0], k0[0], led)
+    flags, beta, *_ = oracle.head_layer(p, 0, 1, False, q1[0], k1[0], led)
+    assert not flags[:4].any()
+    assert np.isneginf(beta[:4]).all()
+
+
+# --------------------------------------------------- counting rules -----
+def _read_golden(name):
+    rows = []
+    with open(os.path.join(HERE, "golden", name)) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def test_counting_rule_reproduces_table3():
+    """RouteRelay §5.2 Table 3: with one anchor at layer 0 of 24, the printed
+    rerouted fraction f and the counting rule (anchor rows count as
+    rerouted and cost n; relay rows cost c plus n when refreshed) must give
+    the printed score-pair fraction, within the tables' rounding."""
+    n, L = 256, 24
+
+    def pairs(f, c, rule):
+        s_rho = L * f - 1.0  # relay-layer sum of refreshed fractions
+        if rule == "page":
+            return oracle.pair_fraction_from_counts(L, n, n, c, [s_rho * n] + [0.0] * (L - 2))
+        if rule == "no_candidates":
+            return (1 + s_rho) / L
+        if rule == "anchor_not_rerouted":
+            return (1 + (L - 1) * c / n + L * f) / L
+        raise ValueError(rule)
+
+    def matches(f_pct, c, p_pct, rule):
+        fs = np.linspace(f_pct - 0.05, f_pct + 0.05, 201) / 100
+        vals = np.array([pairs(f, c, rule) for f in fs]) * 100
+        return bool(((vals >= p_pct - 0.05) & (vals <= p_pct + 0.05)).any())
+
+    rows = _read_golden("table3_sentinel_ablation.txt")
+    assert len(rows) == 4
+    for label, k, m, r, f_pct, p_pct in rows:
+        c = int(k) + int(m) + int(r)
+        assert matches(float(f_pct), c, float(p_pct), "page"), label
+    # the readings that were rejected do not reproduce the table
+    assert not all(matches(float(f), int(k) + int(m) + int(r), float(pp), "no_candidates")
+                   for _, k, m, r, f, pp in rows)
+    assert not all(matches(float(f), int(k) + int(m) + int(r), float(pp), "anchor_not_rerouted")
+                   for _, k, m, r, f, pp in rows)
+
+
+def test_rerouted_rows_count_anchor_layers_table2():
+    """RouteRelay §5.1 Table 2: refreshing every row at every fourth of 32
+    layers is 25.0% rerouted rows; routing every layer is 100.0%."""
+    p = Params(nq=6, nk=6, d=4, k=2, m=1, r=1, seed=0)
+    rng = np.random.default_rng(0)
+    for label, layers, H, pct in _read_golden("table2_fixed_stride.txt"):
+        layers, H = int(layers), int(H)
+        rt = oracle.Router(p, bh=1, anchor_interval=H)
+        for l in range(layers):
+            q = rng.standard_normal((1, 6, 4)).astype(np.float32)
+            k = rng.standard_normal((1, 6, 4)).astype(np.float32)
+            # "fixed stride": every non-anchor layer reuses without testing
+            anchor = oracle.is_anchor(l, H)
+            if anchor:
+                rt.step(l, q, k, recall=False)
+            else:
+                rt.stats.append(oracle.LayerStats(l, False, 0, 0))
+        s = rt.summary()
+        assert abs(100 * s["rerouted_fraction"] - float(pct)) < 0.05, label
+
+
+def test_router_counters_follow_counting_rule():
+    p = Params(nq=32, nk=32, d=8, k=4, m=3, r=2, causal=True, seed=3)
+    rng = np.random.default_rng(1)
+    rt = oracle.Router(p, bh=2, anchor_interval=4)
+    x_q = rownorm(rng.standard_normal((2, 32, 8)))
+    x_k = rownorm(rng.standard_normal((2, 32, 8)))
+    for l in range(6):
+        before = [led.copy() for led in rt.ledgers]
+        res, st = rt.step(l, x_q.astype(np.float32), x_k.astype(np.float32))
+        nv = np.array([oracle.valid_count(i, 32, True) for i in range(32)])
+        if st.anchor:
+            assert st.refreshed == 64 and st.pairs == 2 * nv.sum()
+        else:
+            cand = sum(int((b.ids >= 0).sum()) for b in before)
+            fl = [r[0] for r in res]
+            assert st.refreshed == sum(int(f.sum()) for f in fl)
+            assert st.pairs == cand + sum(int(nv[f.astype(bool)].sum()) for f in fl)
+        x_q = rownorm(x_q + 0.2 * rng.standard_normal(x_q.shape))
+        x_k = rownorm(x_k + 0.2 * rng.standard_normal(x_k.shape))
+
+
+def test_sharded_heads_equal_unsharded():
+    """Heads are independent and the random key carries the global head
+    index, so running heads in two shards reproduces the joint run."""
+    p = Params(nq=24, nk=24, d=8, k=3, m=3, r=3, seed=12)
+    rng = np.random.default_rng(2)
+    qs = [rng.standard_normal((4, 24, 8)).astype(np.float32) for _ in range(3)]
+    ks = [rng.standard_normal((4, 24, 8)).astype(np.float32) for _ in range(3)]
+    full = oracle.Router(p, bh=4, anchor_interval=2)
+    a = oracle.Router(p, bh=2, anchor_interval=2, bh_offset=0)
+    b = oracle.Router(p, bh=2, anchor_interval=2, bh_offset=2)
+    for l in range(3):
+        full.step(l, qs[l], ks[l], recall=False)
+        a.step(l, qs[l][:2], ks[l][:2], recall=False)
+        b.step(l, qs[l][2:], ks[l][2:], recall=False)
+    for h in range(4):
+        part = a.ledgers[h] if h < 2 else b.ledgers[h - 2]
+        assert np.array_equal(full.ledgers[h].ids, part.ids)
+        assert np.array_equal(full.ledgers[h].alpha, part.alpha)
+
+
+def test_recall_is_one_when_every_layer_is_an_anchor():
+    p = Params(nq=16, nk=16, d=8, k=3, m=2, r=2, seed=0)
+    rng = np.random.default_rng(5)
+    rt = oracle.Router(p, bh=1, anchor_interval=1)
+    for l in range(4):
+        rt.step(l, rng.standard_normal((1, 16, 8)).astype(np.float32),
+                rng.standard_normal((1, 16, 8)).astype(np.float32))
+    s = rt.summary()
+    assert s["recall"] == 1.0 and s["rerouted_fraction"] == 1.0 and s["pair_fraction"] == 1.0
