@@ -1,0 +1,471 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 RouteRelay router.
+
+One step = one full routing pass of the workload through every layer: an
+anchor (full routing of every row) at layer 0 and every H layers, relay
+(rescore -> compact -> refresh of the flagged rows) at the others, on
+synthetic drifting chunk representations already resident in HBM.
+
+Default workload: BH = 256 batch x head units, 4096 query and key chunks
+per head (256K tokens at 64-token chunks), d = 128 bf16, causal, 32 layers,
+anchor every 16, top-32 with 32 near-miss and 16 random sentinels, drift
+sigma 0.03.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload NAME]
+
+Prints one JSON line (rank 0).  With N > 1 (launched by torchrun) every
+rank routes its own BH units (heads are independent: no collective on the
+data path) and the step time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import rr_workloads as W  # noqa: E402
+
+METRIC = "routed rows/s per layer & score-pairs/s; % of tensor/HBM roofline; recall"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+# ---------------------------------------------------------------- clocks ----
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        srt = sorted(sm)
+        loaded = [x for x in srt if x >= 0.5 * srt[-1]] or srt
+        return {"sm_mhz": loaded[len(loaded) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def smi_id(device) -> str:
+    """nvidia-smi id of a torch device (its UUID; CUDA_VISIBLE_DEVICES may
+    renumber devices, nvidia-smi does not)."""
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        idx = torch.device(device).index or 0
+        if vis:
+            return vis.split(",")[idx]
+        return str(idx)
+
+
+# ------------------------------------------------------------- workload -----
+def make_inputs(w, device, seed):
+    st = W.LayerStream(w, device, seed=seed)
+    qs, ks = [], []
+    for _ in range(w.layers):
+        _, _, q, k = st.next()
+        qs.append(q.contiguous())
+        ks.append(k.contiguous())
+    del st
+    return qs, ks
+
+
+def full_pairs_per_layer(w) -> int:
+    if not w.causal:
+        return w.bh * w.n * w.n
+    return w.bh * w.n * (w.n + 1) // 2
+
+
+# ---------------------------------------------------------------- ours ------
+def run_ours(args, w, rank, world, device):
+    import cross_layer_route_b200 as rr
+
+    torch.cuda.set_device(device)
+    cfg = rr.Config(bh=w.bh, nq=w.n, nk=w.n, d=w.d, k=w.k, m_near=w.m, r_rand=w.r, dtype=w.dtype,
+                    anchor_interval=w.anchor_interval, causal=w.causal, gamma=w.gamma, seed=w.seed,
+                    bh_offset=rank * w.bh)
+    qs, ks = make_inputs(w, device, seed=w.seed * 1009 + rank)
+    led = rr.RouteLedger(cfg, device)
+    stream = torch.cuda.current_stream(device)
+    L = w.layers
+    anchors = [l for l in range(L) if led.is_anchor(l)]
+    relays = [l for l in range(L) if not led.is_anchor(l)]
+
+    # events: per layer spans of the route kernel (anchor / refresh) and of
+    # the relay rescore and compact kernels, on the launching stream
+    def make_events(n):
+        return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+
+    def step(ev=None):
+        e = 0
+        for l in range(L):
+            if led.is_anchor(l):
+                if ev is not None:
+                    ev["anchor"][e].record(stream)
+                led.full_route(qs[l], ks[l], l)
+                if ev is not None:
+                    ev["anchor_end"][e].record(stream)
+            else:
+                if ev is not None:
+                    ev["rescore"][e].record(stream)
+                led.relay_rescore(qs[l], ks[l], l)
+                if ev is not None:
+                    ev["compact"][e].record(stream)
+                led.relay_compact(l)
+                if ev is not None:
+                    ev["refresh"][e].record(stream)
+                led.relay_refresh(qs[l], ks[l], l)
+                if ev is not None:
+                    ev["refresh_end"][e].record(stream)
+            e += 1
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(device)
+
+    for _ in range(args.warmup):
+        step()
+    barrier()
+    c0 = led.read()["counters"].clone()
+    K = args.steps
+    evs = [{n: make_events(L) for n in ("anchor", "anchor_end", "rescore", "compact", "refresh",
+                                        "refresh_end")} for _ in range(K)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(smi_id(device) if args.smi_index is None else args.smi_index) as clk:
+        barrier()
+        t_start.record(stream)
+        for s in range(K):
+            step(evs[s])
+        t_end.record(stream)
+        barrier()
+    ms_total = t_start.elapsed_time(t_end)
+    c1 = led.read()["counters"].clone()
+
+    route_ms = rescore_ms = compact_ms = 0.0
+    n_route = n_rescore = 0
+    for s in range(K):
+        for l in range(L):
+            if l in anchors:
+                route_ms += evs[s]["anchor"][l].elapsed_time(evs[s]["anchor_end"][l])
+                n_route += 1
+            else:
+                rescore_ms += evs[s]["rescore"][l].elapsed_time(evs[s]["compact"][l])
+                compact_ms += evs[s]["compact"][l].elapsed_time(evs[s]["refresh"][l])
+                route_ms += evs[s]["refresh"][l].elapsed_time(evs[s]["refresh_end"][l])
+                n_route += 1
+                n_rescore += 1
+
+    ms_step = ms_total / K
+    if world > 1:
+        t = torch.tensor([ms_step], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms_step = float(t.item())
+
+    rows_per_step = w.bh * w.n * L
+    d_cnt = (c1 - c0).tolist()
+    pairs_per_step = d_cnt[rr.CNT_PAIRS_TOTAL] / K
+    full_pairs_per_step = d_cnt[rr.CNT_FULL_PAIRS_TOTAL] / K
+    refreshed_per_step = d_cnt[rr.CNT_ROWS_TOTAL] / K
+    relay_rows = w.bh * w.n * len(relays)
+    rho = (refreshed_per_step - w.bh * w.n * len(anchors)) / relay_rows if relay_rows else 0.0
+
+    peaks = load_peaks()
+    esz = 2 if w.dtype == "bf16" else 4
+    # dominant kernel: full routing (anchor + refresh).  Algorithmic work =
+    # one multiply-add per (row, valid key, dim) -> 2*d flops per score pair.
+    route_flops = 2.0 * w.d * full_pairs_per_step * K
+    route_tflops = route_flops / (route_ms * 1e-3) / 1e12
+    alu_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+    roofline = {"kernel": "route_rows (anchor + refresh)", "bound": "alu",
+                "achieved": round(route_tflops, 3), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
+                "frac": round(route_tflops / alu_peak, 4), "traffic": None,
+                "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock (CUDA-core FMA path)",
+                "avg_launch_ms": round(route_ms / max(n_route, 1), 4)}
+    # secondary: relay rescore (HBM-bound): per row q (d*e) + its head's keys
+    # once (N*d*e/N) + ids (4c) + alpha/flag writes (5) bytes
+    rescore_bytes = w.bh * w.n * (2 * w.d * esz + 4 * w.c + 5) * n_rescore
+    rescore_gbs = rescore_bytes / (rescore_ms * 1e-3) / 1e9 if rescore_ms > 0 else None
+    kernels = {
+        "rescore": {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1) if rescore_gbs else None,
+                    "peak_gbs": peaks["hbm_gbs"],
+                    "frac": round(rescore_gbs / peaks["hbm_gbs"], 4) if rescore_gbs else None,
+                    "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)},
+        "compact": {"avg_launch_ms": round(compact_ms / max(n_rescore, 1), 4)},
+    }
+
+    result = {
+        "metric": METRIC, "value": rows_per_step * world / (ms_step * 1e-3), "unit": "rows/s",
+        "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "bh_per_gpu": w.bh, "n_chunks": w.n, "d": w.d,
+                   "layers": L, "anchor_interval": w.anchor_interval, "k": w.k, "near_miss": w.m,
+                   "random": w.r, "causal": w.causal, "drift_sigma": w.sigma,
+                   "l2": f"no flush: inputs {2 * L * w.bh * w.n * w.d * esz / 2**30:.1f} GiB per step exceed L2",
+                   "parallelism": f"bh-sharded x{world}, no collective"},
+        "score_pairs_per_s": pairs_per_step * world / (ms_step * 1e-3),
+        "pair_fraction": pairs_per_step / (full_pairs_per_layer(w) * L),
+        "rho_relay": rho,
+        "roofline": roofline,
+        "kernels": kernels,
+        "gpu_launches": K * (2 * len(anchors) + 4 * len(relays)),
+        "clocks": clk.summary(),
+        "peaks_source": peaks["source"],
+    }
+    return result, (led, qs, ks, cfg)
+
+
+def measure_e2e(args, w, state, device):
+    """Same metric through the public API with the inputs in pinned host
+    memory: each step copies every layer's Qc, Kc host->device (copy stream,
+    double-buffered) and reads the ledger back device->host at its end."""
+    import cross_layer_route_b200 as rr
+    led, qs, ks, cfg = state
+    L = w.layers
+    hq = [q.cpu().pin_memory() for q in qs]
+    hk = [k.cpu().pin_memory() for k in ks]
+    bq = [torch.empty_like(qs[0]) for _ in range(2)]
+    bk = [torch.empty_like(ks[0]) for _ in range(2)]
+    comp = torch.cuda.current_stream(device)
+    copy = torch.cuda.Stream(device)
+    out_ids = torch.empty((cfg.bh, cfg.nq, cfg.c), dtype=torch.int32, pin_memory=True)
+    out_alpha = torch.empty((cfg.bh, cfg.nq), dtype=torch.float32, pin_memory=True)
+    out_cnt = torch.empty((rr.NUM_COUNTERS,), dtype=torch.int64, pin_memory=True)
+    view = rr.rr_ledger_view(out_ids.data_ptr(), out_alpha.data_ptr(), None, None, out_cnt.data_ptr())
+    done = [torch.cuda.Event() for _ in range(2)]
+    ready = [torch.cuda.Event() for _ in range(2)]
+
+    def step():
+        for l in range(L):
+            b = l & 1
+            copy.wait_event(done[b])
+            with torch.cuda.stream(copy):
+                bq[b].copy_(hq[l], non_blocking=True)
+                bk[b].copy_(hk[l], non_blocking=True)
+                ready[b].record(copy)
+            comp.wait_event(ready[b])
+            led.layer(bq[b], bk[b], l, stream=comp)
+            done[b].record(comp)
+        rr.rr_ledger_read(led.handle, view, comp.cuda_stream)
+
+    for b in range(2):
+        done[b].record(comp)
+    step()
+    torch.cuda.synchronize(device)
+    K = max(1, min(args.steps, 3))
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    for _ in range(K):
+        step()
+    t1.record(comp)
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1) / K
+    h2d = sum(q.numel() * q.element_size() + k.numel() * k.element_size() for q, k in zip(qs, ks))
+    d2h = out_ids.numel() * 4 + out_alpha.numel() * 4 + out_cnt.numel() * 8
+    return {"value": w.bh * w.n * L / (ms * 1e-3), "unit": "rows/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms, "steps": K}
+
+
+def measure_recall(w, state, device):
+    """Recall of the relayed routes against exact per-layer top-k (a second
+    ledger that fully routes every layer), pooled over rows, mean over
+    layers."""
+    import cross_layer_route_b200 as rr
+    led, qs, ks, cfg = state
+    exact_cfg = rr.Config(**{**cfg.__dict__, "anchor_interval": 1})
+    ex = rr.RouteLedger(exact_cfg, device)
+    dv, ev = led.device_view(), ex.device_view()
+    rec = []
+    for l in range(w.layers):
+        led.layer(qs[l], ks[l], l)
+        ex.layer(qs[l], ks[l], l)
+        hits = tot = 0
+        for h0 in range(0, w.bh, 16):
+            used = dv["ids"][h0:h0 + 16, :, : w.k]
+            exact = ev["ids"][h0:h0 + 16, :, : w.k]
+            m = (used[..., :, None] == exact[..., None, :]) & (exact[..., None, :] >= 0)
+            hits += int(m.any(-2).sum())
+            tot += int((exact >= 0).sum())
+        rec.append(hits / tot)
+    del ex
+    return sum(rec) / len(rec), min(rec)
+
+
+# ------------------------------------------------------- CPU baseline ------
+def cpu_baseline(w, qs, ks, threads=None, layers=2):
+    """The oracle as it stands, on a bounded sample: `threads` heads (one per
+    thread) through `layers` layers (anchor then relay)."""
+    import numpy as np
+
+    import oracle
+    ncpu = os.cpu_count() or 1
+    T = max(1, min(threads or ncpu, 16, w.bh))
+    p = oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal, gamma=w.gamma,
+                      seed=w.seed)
+    rt = oracle.Router(p, bh=T, anchor_interval=w.anchor_interval, threads=T)
+    xs = [(qs[l][:T].float().cpu().numpy(), ks[l][:T].float().cpu().numpy()) for l in range(layers)]
+    t0 = time.perf_counter()
+    for l in range(layers):
+        rt.step(l, xs[l][0], xs[l][1], recall=False)
+    dt = time.perf_counter() - t0
+    rows = T * w.n * layers
+    return {"value": rows / dt, "unit": "rows/s", "cores": T, "kind": "oracle",
+            "sample": f"{T} heads x {layers} layers (anchor, relay) of {w.name}, one head per thread, "
+                      f"{dt:.1f} s wall on {ncpu} host cores"}
+
+
+def run_reference(args, w):
+    """The oracle timed as a benchmark arm on this workload (rank 0 only)."""
+    import numpy as np
+    st = W.LayerStream(w.with_(bh=min(w.bh, 16)), "cpu")
+    qs, ks = [], []
+    for _ in range(2):
+        _, _, q, k = st.next()
+        qs.append(q)
+        ks.append(k)
+    ncpu = os.cpu_count() or 1
+    T = max(1, min(ncpu, 16, w.bh))
+    for _ in range(args.warmup):
+        cpu_baseline(w, qs, ks, threads=T, layers=1)
+    vals = []
+    t_all = time.perf_counter()
+    for _ in range(args.steps):
+        vals.append(cpu_baseline(w, qs, ks, threads=T, layers=2))
+    ms_step = (time.perf_counter() - t_all) / args.steps * 1e3
+    v = sum(x["value"] for x in vals) / len(vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {"metric": METRIC, "value": v, "unit": "rows/s", "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "sample_heads": T, "sample_layers": 2},
+            "cpu_baseline": cb,
+            "e2e": {"value": v, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.C5.name, choices=sorted(W.BY_NAME))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-recall", action="store_true")
+    ap.add_argument("--smi-index", type=int, default=None)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    w = W.BY_NAME[args.workload]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return 0
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    result, state = run_ours(args, w, rank, world, device)
+    if not args.no_recall:
+        r_mean, r_min = measure_recall(w, state, device)
+        result["recall"] = r_mean
+        result["recall_min_layer"] = r_min
+    if not args.no_e2e:
+        e2e = measure_e2e(args, w, state, device)
+        if world > 1:
+            t = torch.tensor([e2e["ms_per_step"]], device=device, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e["ms_per_step"] = float(t.item())
+            e2e["value"] = w.bh * w.n * w.layers * world / (e2e["ms_per_step"] * 1e-3)
+        result["e2e"] = e2e
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        led, qs, ks, cfg = state
+        result["cpu_baseline"] = cpu_baseline(w, qs, ks)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,274 @@
+"""B200-native RouteRelay router: Python binding of librr.so (include/rr.h).
+
+Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
+Dynamic Sparse Attention" (arXiv 2609.07306).  Anchor layers fully route
+every query chunk (S = Qc Kc^T, top-k, §2.1 Eq. 1-2); intermediate layers
+rescore each row's ledger candidates, test alpha > beta + gamma (§3.2 Eq.
+5-8) and fully re-route only the rows that fail (§4.1-4.2).
+
+This module only marshals arguments: every step of the routing path runs in
+the CUDA kernels of librr.so.  There is no CPU fallback; importing it without
+the built library raises.  PyTorch supplies device memory and streams.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librr.so")
+
+RR_OK, RR_EINVAL, RR_ESTATE, RR_ENOMEM, RR_ECUDA, RR_EDEVICE = range(6)
+RR_F32, RR_BF16 = 0, 1
+CNT_ROWS, CNT_PAIRS, CNT_ERROR, CNT_ROWS_TOTAL, CNT_PAIRS_TOTAL, CNT_LAYERS, CNT_LAST_LAYER, \
+    CNT_DRAW_CAP, CNT_FULL_PAIRS, CNT_FULL_PAIRS_TOTAL = range(10)
+NUM_COUNTERS = 16
+
+
+class rr_config(ctypes.Structure):
+    _fields_ = [("bh", ctypes.c_int32), ("nq", ctypes.c_int32), ("nk", ctypes.c_int32),
+                ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("m_near", ctypes.c_int32), ("r_rand", ctypes.c_int32),
+                ("anchor_interval", ctypes.c_int32), ("causal", ctypes.c_int32),
+                ("gamma", ctypes.c_float), ("bh_offset", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+
+
+class rr_ledger_view(ctypes.Structure):
+    _fields_ = [("ids", ctypes.c_void_p), ("alpha", ctypes.c_void_p),
+                ("anchor_layer", ctypes.c_void_p), ("flags", ctypes.c_void_p),
+                ("counters", ctypes.c_void_p)]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"librr.so is not built ({LIB_PATH}); run python cross_layer_route_b200/build.py")
+    lib = ctypes.CDLL(LIB_PATH)
+    P = ctypes.c_void_p
+    lib.rr_ledger_workspace_bytes.argtypes = [ctypes.POINTER(rr_config)]
+    lib.rr_ledger_workspace_bytes.restype = ctypes.c_size_t
+    lib.rr_ledger_create.argtypes = [ctypes.POINTER(rr_config), P, ctypes.c_size_t, ctypes.POINTER(P)]
+    lib.rr_ledger_create.restype = ctypes.c_int
+    lib.rr_ledger_destroy.argtypes = [P]
+    lib.rr_ledger_destroy.restype = ctypes.c_int
+    for name in ("rr_full_route", "rr_relay_layer", "rr_relay_rescore", "rr_relay_refresh"):
+        f = getattr(lib, name)
+        f.argtypes = [P, P, P, ctypes.c_int32, P]
+        f.restype = ctypes.c_int
+    lib.rr_relay_compact.argtypes = [P, ctypes.c_int32, P]
+    lib.rr_relay_compact.restype = ctypes.c_int
+    lib.rr_ledger_read.argtypes = [P, ctypes.POINTER(rr_ledger_view), P]
+    lib.rr_ledger_read.restype = ctypes.c_int
+    lib.rr_ledger_device_view.argtypes = [P, ctypes.POINTER(rr_ledger_view)]
+    lib.rr_ledger_device_view.restype = ctypes.c_int
+    lib.rr_status_string.argtypes = [ctypes.c_int]
+    lib.rr_status_string.restype = ctypes.c_char_p
+    return lib
+
+
+_lib = _load()
+
+
+class RRError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {rr_status_string(status)}")
+
+
+def _check(status: int, what: str):
+    if status != RR_OK:
+        raise RRError(status, what)
+
+
+# ---- the C ABI, name for name ---------------------------------------------
+def rr_status_string(status: int) -> str:
+    return _lib.rr_status_string(status).decode()
+
+
+def rr_ledger_workspace_bytes(cfg: rr_config) -> int:
+    return int(_lib.rr_ledger_workspace_bytes(ctypes.byref(cfg)))
+
+
+def rr_ledger_create(cfg: rr_config, d_workspace: int, nbytes: int) -> ctypes.c_void_p:
+    out = ctypes.c_void_p()
+    _check(_lib.rr_ledger_create(ctypes.byref(cfg), ctypes.c_void_p(d_workspace), nbytes,
+                                 ctypes.byref(out)), "rr_ledger_create")
+    return out
+
+
+def rr_ledger_destroy(handle) -> None:
+    _check(_lib.rr_ledger_destroy(handle), "rr_ledger_destroy")
+
+
+def rr_full_route(handle, d_qc: int, d_kc: int, layer: int, stream: int) -> None:
+    _check(_lib.rr_full_route(handle, ctypes.c_void_p(d_qc), ctypes.c_void_p(d_kc), layer,
+                              ctypes.c_void_p(stream)), "rr_full_route")
+
+
+def rr_relay_layer(handle, d_qc: int, d_kc: int, layer: int, stream: int) -> None:
+    _check(_lib.rr_relay_layer(handle, ctypes.c_void_p(d_qc), ctypes.c_void_p(d_kc), layer,
+                               ctypes.c_void_p(stream)), "rr_relay_layer")
+
+
+def rr_relay_rescore(handle, d_qc: int, d_kc: int, layer: int, stream: int) -> None:
+    _check(_lib.rr_relay_rescore(handle, ctypes.c_void_p(d_qc), ctypes.c_void_p(d_kc), layer,
+                                 ctypes.c_void_p(stream)), "rr_relay_rescore")
+
+
+def rr_relay_compact(handle, layer: int, stream: int) -> None:
+    _check(_lib.rr_relay_compact(handle, layer, ctypes.c_void_p(stream)), "rr_relay_compact")
+
+
+def rr_relay_refresh(handle, d_qc: int, d_kc: int, layer: int, stream: int) -> None:
+    _check(_lib.rr_relay_refresh(handle, ctypes.c_void_p(d_qc), ctypes.c_void_p(d_kc), layer,
+                                 ctypes.c_void_p(stream)), "rr_relay_refresh")
+
+
+def rr_ledger_read(handle, view: rr_ledger_view, stream: int) -> None:
+    _check(_lib.rr_ledger_read(handle, ctypes.byref(view), ctypes.c_void_p(stream)), "rr_ledger_read")
+
+
+def rr_ledger_device_view(handle) -> rr_ledger_view:
+    v = rr_ledger_view()
+    _check(_lib.rr_ledger_device_view(handle, ctypes.byref(v)), "rr_ledger_device_view")
+    return v
+
+
+# ---- convenience wrapper over torch memory --------------------------------
+@dataclass
+class Config:
+    """Problem statement of one ledger (see rr_config in include/rr.h)."""
+    bh: int
+    nq: int
+    nk: int
+    d: int
+    k: int
+    m_near: int
+    r_rand: int
+    dtype: str = "f32"          # "f32" | "bf16"
+    anchor_interval: int = 0
+    causal: bool = False
+    gamma: float = 0.0
+    seed: int = 0
+    bh_offset: int = 0
+
+    @property
+    def c(self) -> int:
+        return self.k + self.m_near + self.r_rand
+
+    @property
+    def torch_dtype(self) -> torch.dtype:
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    def to_c(self) -> rr_config:
+        return rr_config(self.bh, self.nq, self.nk, self.d, RR_BF16 if self.dtype == "bf16" else RR_F32,
+                         self.k, self.m_near, self.r_rand, self.anchor_interval, int(bool(self.causal)),
+                         float(self.gamma), self.bh_offset, int(self.seed) & 0xFFFFFFFFFFFFFFFF)
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+class RouteLedger:
+    """One ledger (RouteRelay Eq. 4) in a torch-allocated device workspace."""
+
+    def __init__(self, cfg: Config, device=None):
+        self.cfg = cfg
+        self._c = cfg.to_c()
+        dev = torch.device(device if device is not None else "cuda")
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        self.device = dev
+        nbytes = rr_ledger_workspace_bytes(self._c)
+        if nbytes == 0:
+            raise RRError(RR_EINVAL, "rr_ledger_workspace_bytes (invalid config)")
+        self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.handle = rr_ledger_create(self._c, self.workspace.data_ptr(), nbytes)
+
+    def __del__(self):
+        h = getattr(self, "handle", None)
+        if h is not None and _lib is not None:
+            _lib.rr_ledger_destroy(h)
+            self.handle = None
+
+    def _args(self, qc: torch.Tensor, kc: torch.Tensor):
+        c = self.cfg
+        for name, t, n in (("qc", qc, c.nq), ("kc", kc, c.nk)):
+            if t.device != self.device or t.dtype != c.torch_dtype or not t.is_contiguous() \
+                    or tuple(t.shape) != (c.bh, n, c.d):
+                raise ValueError(f"{name}: expected contiguous {c.torch_dtype} [{c.bh}, {n}, {c.d}] on "
+                                 f"{self.device}, got {t.dtype} {tuple(t.shape)} on {t.device}")
+        return qc.data_ptr(), kc.data_ptr()
+
+    def full_route(self, qc, kc, layer: int, stream=None):
+        q, k = self._args(qc, kc)
+        rr_full_route(self.handle, q, k, layer, _stream_handle(stream))
+
+    def relay_layer(self, qc, kc, layer: int, stream=None):
+        q, k = self._args(qc, kc)
+        rr_relay_layer(self.handle, q, k, layer, _stream_handle(stream))
+
+    def relay_rescore(self, qc, kc, layer: int, stream=None):
+        q, k = self._args(qc, kc)
+        rr_relay_rescore(self.handle, q, k, layer, _stream_handle(stream))
+
+    def relay_compact(self, layer: int, stream=None):
+        rr_relay_compact(self.handle, layer, _stream_handle(stream))
+
+    def relay_refresh(self, qc, kc, layer: int, stream=None):
+        q, k = self._args(qc, kc)
+        rr_relay_refresh(self.handle, q, k, layer, _stream_handle(stream))
+
+    def is_anchor(self, layer: int) -> bool:
+        H = self.cfg.anchor_interval
+        return layer == 0 or (H > 0 and layer % H == 0)
+
+    def read(self, device="cpu", stream=None, check: bool = True) -> dict:
+        """Copies the ledger out (ids [bh, nq, c], alpha, anchor_layer, flags,
+        counters), synchronises the stream and raises on a device error."""
+        c = self.cfg
+        pin = torch.device(device).type == "cpu"
+        mk = lambda shape, dt: torch.empty(shape, dtype=dt, device=device, pin_memory=pin)
+        out = {"ids": mk((c.bh, c.nq, c.c), torch.int32), "alpha": mk((c.bh, c.nq), torch.float32),
+               "anchor_layer": mk((c.bh, c.nq), torch.int32), "flags": mk((c.bh, c.nq), torch.uint8),
+               "counters": mk((NUM_COUNTERS,), torch.int64)}
+        v = rr_ledger_view(out["ids"].data_ptr(), out["alpha"].data_ptr(), out["anchor_layer"].data_ptr(),
+                           out["flags"].data_ptr(), out["counters"].data_ptr())
+        rr_ledger_read(self.handle, v, _stream_handle(stream))
+        torch.cuda.synchronize(self.device)
+        if check and int(out["counters"][CNT_ERROR]) != 0:
+            raise RRError(RR_EDEVICE, f"device error word {int(out['counters'][CNT_ERROR]):#x}")
+        return out
+
+    def device_view(self) -> dict:
+        """Zero-copy torch views of the ledger inside the workspace."""
+        v = rr_ledger_device_view(self.handle)
+        c = self.cfg
+        base = self.workspace.data_ptr()
+        ws = self.workspace
+
+        def view(ptr, nbytes, dt, shape):
+            off = ptr - base
+            return ws[off:off + nbytes].view(dt).view(shape)
+
+        rows = c.bh * c.nq
+        return {"ids": view(v.ids, rows * c.c * 4, torch.int32, (c.bh, c.nq, c.c)),
+                "alpha": view(v.alpha, rows * 4, torch.float32, (c.bh, c.nq)),
+                "anchor_layer": view(v.anchor_layer, rows * 4, torch.int32, (c.bh, c.nq)),
+                "flags": view(v.flags, rows, torch.uint8, (c.bh, c.nq)),
+                "counters": view(v.counters, NUM_COUNTERS * 8, torch.int64, (NUM_COUNTERS,))}
+
+    def layer(self, qc, kc, layer: int, stream=None):
+        """Layer l of a sequence: an anchor at l == 0, else rr_relay_layer
+        (which itself turns forced-anchor layers into full routing)."""
+        if layer == 0:
+            self.full_route(qc, kc, layer, stream)
+        else:
+            self.relay_layer(qc, kc, layer, stream)

@@ -1,0 +1,50 @@
+// rr_internal.h -- internal types shared by the host library and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rr {
+
+// Device-side view of one ledger, passed to kernels by value.
+struct LedgerDev {
+    // ledger proper (RouteRelay §3.1 Eq. 4, §4.1)
+    int32_t *ids;           // [bh*nq, c]  route | near-miss | random
+    float *alpha;           // [bh*nq]     weakest selected score at the row's last layer
+    int32_t *anchor_layer;  // [bh*nq]     layer the row was last fully routed at
+    uint8_t *flags;         // [bh*nq]     1 = fully routed at the last layer
+    unsigned long long *counters;  // [16] RR_CNT_* slots (int64 in the C ABI)
+    // per-layer scratch
+    int32_t *list;          // [bh*nq]     per-head segments of flagged row ids, ascending
+    int32_t *head_count;    // [bh]        flagged rows per head
+    int bh, nq, nk, d;
+    int k, m, r, c, ksel;   // ksel = k + m
+    int causal;
+    int bh_offset;
+    int max_draws;          // cap on random draws per row (64 * c)
+    float gamma;
+    uint32_t seed_lo, seed_hi;
+};
+
+enum Dtype { kF32 = 0, kBF16 = 1 };
+
+// Selection buffer capacity of one row: a power of two >= 2 * ksel, >= 64.
+inline int select_capacity(int ksel) {
+    int cap = 64;
+    while (cap < 2 * ksel) cap <<= 1;
+    return cap;
+}
+
+// Launchers (return cudaSuccess or the launch error).
+size_t route_rows_smem_bytes(const LedgerDev &L);
+cudaError_t route_rows_prepare(int dtype, size_t smem_bytes);
+cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
+                              int layer, bool use_list, cudaStream_t s);
+cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
+                                 int layer, cudaStream_t s);
+cudaError_t launch_compact(const LedgerDev &L, cudaStream_t s);
+cudaError_t launch_finalize(const LedgerDev &L, int layer, long long add_rows,
+                            long long add_pairs, long long add_full_pairs, cudaStream_t s);
+
+}  // namespace rr

@@ -1,0 +1,182 @@
+// rr_relay.cu -- relay-layer kernels of the B200 RouteRelay router.
+//
+// Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
+// Dynamic Sparse Attention" (arXiv 2609.07306), cited as RouteRelay §x.
+//
+//  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
+//      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
+//      row"), one warp per query row, one lane per candidate.
+//  compact_flags: the prefix sum that compacts unstable row ids (§4.2), one
+//      CTA per head, writing an ascending per-head list and its length.
+//  finalize_layer: per-layer counters (§4.1: the refreshed-row fraction is
+//      "exposed to the runtime").
+#include <float.h>
+
+#include "rr_device.cuh"
+#include "rr_internal.h"
+
+namespace rr {
+namespace {
+
+constexpr int kRescoreThreads = 256;
+constexpr int kRescoreWarps = kRescoreThreads / 32;
+constexpr int kDMax = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kRescoreThreads)
+relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
+    __shared__ __align__(16) float qs_all[kRescoreWarps][kDMax];
+    __shared__ unsigned long long pair_sum[kRescoreWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const long long rows = (long long)L.bh * L.nq;
+    const long long grow = (long long)blockIdx.x * kRescoreWarps + warp;
+    const int d = L.d;
+    unsigned long long pairs = 0;
+    if (grow < rows) {
+        const int h = (int)(grow / L.nq);
+        const int i = (int)(grow - (long long)h * L.nq);
+        const int n_valid = valid_keys(i, L.nk, L.causal);
+        float *qs = qs_all[warp];
+        for (int t = lane * 4; t < d; t += 128) {
+            float v[4];
+            Elem<T>::load4(Q + grow * d + t, v);
+            *reinterpret_cast<float4 *>(qs + t) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+        __syncwarp();
+        const int32_t *idr = L.ids + grow * L.c;
+        const T *Kh = K + (size_t)h * L.nk * d;
+        float amin = INFINITY, bmax = -INFINITY;
+        bool bad = false;
+        int ncand = 0;
+        for (int e0 = 0; e0 < L.c; e0 += 32) {
+            const int e = e0 + lane;
+            const int j = e < L.c ? idr[e] : -1;
+            const bool valid = j >= 0 && j < n_valid;
+            bad |= j >= n_valid || j < -1;
+            if (valid) {
+                const T *kp = Kh + (size_t)j * d;
+                float s = 0.f;
+                for (int t = 0; t < d; t += 4) {
+                    float kv[4];
+                    Elem<T>::load4(kp + t, kv);
+                    s = fmaf(qs[t], kv[0], s);
+                    s = fmaf(qs[t + 1], kv[1], s);
+                    s = fmaf(qs[t + 2], kv[2], s);
+                    s = fmaf(qs[t + 3], kv[3], s);
+                }
+                if (e < L.k) amin = fminf(amin, s);   // Eq. 6
+                else bmax = fmaxf(bmax, s);           // Eq. 7
+                ++ncand;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
+            bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+            ncand += __shfl_xor_sync(kFull, ncand, o);
+        }
+        const bool any_bad = __any_sync(kFull, bad);
+        if (lane == 0) {
+            const bool refresh = !(amin > bmax + L.gamma);  // Eq. 8
+            L.flags[grow] = refresh ? 1 : 0;
+            if (!refresh) L.alpha[grow] = amin;
+            if (any_bad) atomicOr(&L.counters[2], 1ULL);
+        }
+        pairs = (unsigned long long)ncand;
+    }
+    if (lane == 0) pair_sum[warp] = pairs;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long s = 0;
+        for (int w = 0; w < kRescoreWarps; ++w) s += pair_sum[w];
+        if (s) atomicAdd(&L.counters[1], s);
+    }
+}
+
+constexpr int kCompactThreads = 1024;
+
+__global__ void __launch_bounds__(kCompactThreads) compact_flags_kernel(LedgerDev L) {
+    __shared__ int warp_tot[kCompactThreads / 32];
+    __shared__ unsigned long long warp_pairs[kCompactThreads / 32];
+    const int h = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint8_t *fl = L.flags + (size_t)h * L.nq;
+    int32_t *lst = L.list + (size_t)h * L.nq;
+    int base = 0;
+    unsigned long long pairs = 0;
+    for (int i0 = 0; i0 < L.nq; i0 += kCompactThreads) {
+        const int i = i0 + tid;
+        const bool f = i < L.nq && fl[i] != 0;
+        const unsigned wm = __ballot_sync(kFull, f);
+        if (lane == 0) warp_tot[warp] = __popc(wm);
+        __syncthreads();
+        int before = 0, total = 0;
+        for (int w = 0; w < kCompactThreads / 32; ++w) {
+            const int t = warp_tot[w];
+            before += w < warp ? t : 0;
+            total += t;
+        }
+        if (f) {
+            lst[base + before + __popc(wm & lanemask_lt())] = i;
+            pairs += (unsigned long long)valid_keys(i, L.nk, L.causal);
+        }
+        base += total;
+        __syncthreads();
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) pairs += __shfl_xor_sync(kFull, pairs, o);
+    if (lane == 0) warp_pairs[warp] = pairs;
+    __syncthreads();
+    if (tid == 0) {
+        unsigned long long s = 0;
+        for (int w = 0; w < kCompactThreads / 32; ++w) s += warp_pairs[w];
+        L.head_count[h] = base;
+        if (base) atomicAdd(&L.counters[0], (unsigned long long)base);
+        if (s) {
+            atomicAdd(&L.counters[1], s);
+            atomicAdd(&L.counters[8], s);
+        }
+    }
+}
+
+__global__ void finalize_layer_kernel(LedgerDev L, int layer, long long add_rows,
+                                      long long add_pairs, long long add_full_pairs) {
+    unsigned long long *c = L.counters;
+    c[0] += (unsigned long long)add_rows;
+    c[1] += (unsigned long long)add_pairs;
+    c[8] += (unsigned long long)add_full_pairs;
+    c[3] += c[0];
+    c[4] += c[1];
+    c[9] += c[8];
+    c[5] += 1ULL;
+    c[6] = (unsigned long long)(long long)layer;
+}
+
+}  // namespace
+
+cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
+                                 int layer, cudaStream_t s) {
+    (void)layer;
+    const long long rows = (long long)L.bh * L.nq;
+    const unsigned grid = (unsigned)((rows + kRescoreWarps - 1) / kRescoreWarps);
+    if (dtype == kBF16)
+        relay_rescore_kernel<__nv_bfloat16><<<grid, kRescoreThreads, 0, s>>>(
+            L, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k));
+    else
+        relay_rescore_kernel<float><<<grid, kRescoreThreads, 0, s>>>(
+            L, static_cast<const float *>(q), static_cast<const float *>(k));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_compact(const LedgerDev &L, cudaStream_t s) {
+    compact_flags_kernel<<<L.bh, kCompactThreads, 0, s>>>(L);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize(const LedgerDev &L, int layer, long long add_rows,
+                            long long add_pairs, long long add_full_pairs, cudaStream_t s) {
+    finalize_layer_kernel<<<1, 1, 0, s>>>(L, layer, add_rows, add_pairs, add_full_pairs);
+    return cudaGetLastError();
+}
+
+}  // namespace rr

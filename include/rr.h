@@ -1,0 +1,202 @@
+/*
+ * rr.h -- C ABI of the B200 RouteRelay router (librr.so).
+ *
+ * Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
+ * Dynamic Sparse Attention" (arXiv 2609.07306), cited as RouteRelay §x.
+ *
+ * Per layer l and per head, a chunk-based dynamic sparse router scores
+ * query-chunk representations Qc [nq, d] against key-chunk representations
+ * Kc [nk, d] (S = Qc Kc^T, §2.1 Eq. 1) and routes every query row to its
+ * top-k key chunks (§2.1 Eq. 2).  RouteRelay keeps, per query row, a ledger
+ * (§3.1 Eq. 4, §4.1): the route (k ids), the sentinels (m near-miss ids =
+ * the chunks ranked k+1..k+m, and r random ids drawn from the rest), and the
+ * layer the row was last fully routed at.  Anchor layers fully route every
+ * row.  Intermediate ("relay") layers rescore only the ledger's candidates
+ * (§3.2 Eq. 5), compute alpha = min score over the route (Eq. 6) and
+ * beta = max score over the sentinels (Eq. 7), keep the route when
+ * alpha > beta + gamma (Eq. 8), and fully re-route only the rows that fail
+ * (§4.1-4.2: compaction of the failing rows, then a refresh of only those).
+ *
+ * Conventions shared by every entry point:
+ *  - Device memory is owned by the caller.  The library never allocates or
+ *    frees device memory: the ledger lives in a caller-allocated workspace.
+ *  - Qc and Kc are device pointers to contiguous row-major [bh, nq, d] and
+ *    [bh, nk, d] arrays of the ledger's dtype (fp32 or bf16), 16-byte
+ *    aligned, valid until the stream reaches the call.
+ *  - Every call enqueues work on `stream` (a cudaStream_t; NULL is the
+ *    legacy default stream) and returns without synchronising.  Argument
+ *    and state errors are returned synchronously and enqueue nothing.
+ *    Errors found on the device (an out-of-range ledger id) are recorded
+ *    in the ledger's error word (counters[2]), read back by rr_ledger_read.
+ *  - The device that was current at rr_ledger_create must be current at
+ *    every later call on that ledger.
+ *  - Inputs must be finite.  Ties between equal scores are broken by the
+ *    smaller chunk index; ids are stored best first.
+ *  - Missing ids (a causal row with fewer valid chunks than slots) are -1.
+ *  - No entry point throws; none keeps global state besides the ledger.
+ */
+#ifndef RR_H
+#define RR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    RR_OK = 0,
+    RR_EINVAL = 1,   /* bad argument (null pointer, bad shape or size, misalignment) */
+    RR_ESTATE = 2,   /* call out of order (relay before an anchor, layer not increasing) */
+    RR_ENOMEM = 3,   /* workspace too small, or host memory for the handle */
+    RR_ECUDA = 4,    /* a CUDA runtime call failed (launch, copy, attribute) */
+    RR_EDEVICE = 5   /* the device recorded an error (see the error word) */
+} rr_status;
+
+typedef enum { RR_F32 = 0, RR_BF16 = 1 } rr_dtype;
+
+/* Problem statement of one ledger (RouteRelay §2.1, §3.1, §3.2, Table 1).
+ * Limits: 1 <= k <= nk; k + m_near <= 128; r_rand <= 128; d a multiple of 8
+ * with 8 <= d <= 256; gamma >= 0 and finite; anchor_interval >= 0. */
+typedef struct {
+    int32_t bh;              /* batch x heads held by this ledger */
+    int32_t nq;              /* query chunks per head */
+    int32_t nk;              /* key chunks per head */
+    int32_t d;               /* chunk representation dim */
+    int32_t dtype;           /* rr_dtype of Qc and Kc */
+    int32_t k;               /* route width (top-k, Eq. 2) */
+    int32_t m_near;          /* near-miss sentinels (§3.1 item 1) */
+    int32_t r_rand;          /* random sentinels (§3.1 item 2) */
+    int32_t anchor_interval; /* H: layers with layer % H == 0 are forced anchors (§3.2); 0 = none */
+    int32_t causal;          /* nonzero: query chunk i routes only to key chunks j <= i */
+    float gamma;             /* guard margin of Eq. 8 */
+    int32_t bh_offset;       /* global index of this ledger's head 0 (keys the random draws) */
+    uint64_t seed;           /* seed of the random sentinels */
+} rr_config;
+
+/* Opaque host-side handle.  It holds pointers into the caller's workspace
+ * and the host-side layer state; it owns no device memory. */
+typedef struct rr_ledger rr_ledger;
+
+/* Counter slots of the ledger (int64 each). */
+enum {
+    RR_CNT_ROWS = 0,          /* rows fully routed at the last layer */
+    RR_CNT_PAIRS = 1,         /* score pairs evaluated at the last layer */
+    RR_CNT_ERROR = 2,         /* error word: bit 0 = a ledger id was out of range at relay */
+    RR_CNT_ROWS_TOTAL = 3,    /* rows fully routed since rr_ledger_create */
+    RR_CNT_PAIRS_TOTAL = 4,   /* score pairs since rr_ledger_create */
+    RR_CNT_LAYERS = 5,        /* layers processed since rr_ledger_create */
+    RR_CNT_LAST_LAYER = 6,    /* index of the last layer processed */
+    RR_CNT_DRAW_CAP = 7,      /* rows whose random draws hit the draw cap and were filled in order */
+    RR_CNT_FULL_PAIRS = 8,    /* score pairs of the rows fully routed at the last layer */
+    RR_CNT_FULL_PAIRS_TOTAL = 9, /* the same, since rr_ledger_create */
+    RR_NUM_COUNTERS = 16      /* slots 10..15 are reserved (0) */
+};
+
+/* Bytes of device workspace a ledger with this config needs (0 if the
+ * config is invalid).  The workspace holds the ledger proper -- ids
+ * [bh*nq, c] int32 with c = k + m_near + r_rand (route | near-miss |
+ * random), alpha [bh*nq] f32, anchor layer [bh*nq] int32, refresh flags
+ * [bh*nq] u8, counters [16] int64 -- plus the library's per-layer scratch
+ * (refresh lists and counts).  Pure host arithmetic. */
+size_t rr_ledger_workspace_bytes(const rr_config *cfg);
+
+/* Validates cfg, carves the ledger out of d_workspace (device memory of at
+ * least rr_ledger_workspace_bytes(cfg) bytes, 256-byte aligned, owned by
+ * the caller and kept alive until rr_ledger_destroy) and returns a handle
+ * in *out.  Makes no CUDA call and does not touch device memory; the first
+ * call that enqueues work records the current device, sets the kernels'
+ * shared-memory attributes on it and zeroes the counters (on its stream).  The first layer of a sequence must be
+ * an anchor (rr_full_route).  Errors: RR_EINVAL (bad config or pointer),
+ * RR_ENOMEM (workspace too small / no host memory). */
+rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes,
+                           rr_ledger **out);
+
+/* Frees the host handle (not the workspace).  NULL is allowed. */
+rr_status rr_ledger_destroy(rr_ledger *ledger);
+
+/* Anchor layer: full routing of every row (RouteRelay §2.1 Eq. 1-2; §4.1 "an
+ * anchor layer constructs this state from a complete chunk-score matrix").
+ * For every query row the library scores all valid key chunks, takes the
+ * k + m_near best (score descending, index ascending): the first k become
+ * the route, the next m_near the near-miss sentinels; r_rand random
+ * sentinels are drawn without replacement from the remaining valid chunks
+ * (§3.1 item 2, §3.4) with Philox4x32-10 (Salmon et al., SC'11), key
+ * (seed lo, seed hi), counter (bh_offset + head, row, layer, t/4), word t%4,
+ * chunk = (word * n_valid) >> 32, rejecting repeats; if the pool holds no
+ * more than r_rand chunks it is taken whole in ascending order.  alpha
+ * becomes the route's weakest score, the anchor layer becomes `layer`, every
+ * refresh flag becomes 1.  Starts a new layer sequence at any `layer` >= 0.
+ * The score matrix never reaches device memory.  Errors: RR_EINVAL,
+ * RR_ECUDA. */
+rr_status rr_full_route(rr_ledger *ledger, const void *d_qc, const void *d_kc, int32_t layer,
+                        void *stream);
+
+/* Intermediate layer (RouteRelay §3.2 Eq. 5-8, §4.1-4.2).  When
+ * anchor_interval > 0 and layer % anchor_interval == 0 this is a forced
+ * anchor and behaves as rr_full_route.  Otherwise, for every row: rescore
+ * the ledger's candidates against this layer's Kc, alpha = min over the
+ * route, beta = max over the sentinels (-inf if none), refresh flag =
+ * !(alpha > beta + gamma).  Stable rows keep their ids and store this
+ * layer's alpha.  Flagged rows are compacted into a per-head list and only
+ * they are fully re-routed at this layer (route, near-miss and random
+ * sentinels rebuilt as in rr_full_route; anchor layer <- layer).  No host
+ * synchronisation: the refresh launch reads the device-side list.
+ * Errors: RR_ESTATE if no anchor started the sequence or `layer` is not
+ * greater than the previous layer; RR_EINVAL, RR_ECUDA. */
+rr_status rr_relay_layer(rr_ledger *ledger, const void *d_qc, const void *d_kc, int32_t layer,
+                         void *stream);
+
+/* The three stages of rr_relay_layer, for callers that schedule or time
+ * them one by one (RouteRelay §4.2).  They must be called in this order for
+ * one layer; each does exactly its stage and none applies the forced-anchor
+ * schedule (rr_relay_layer does).
+ *  rr_relay_rescore: candidate rescoring and the challenge test of every row
+ *    (Eq. 5-8): writes the refresh flags and, for stable rows, alpha.  Same
+ *    preconditions as rr_relay_layer (RR_ESTATE otherwise).
+ *  rr_relay_compact: the prefix sum over the flags that writes, per head,
+ *    the ascending list of flagged rows and its length.  RR_ESTATE unless
+ *    rr_relay_rescore of this `layer` came just before.
+ *  rr_relay_refresh: full routing of the listed rows only (their route,
+ *    near-miss and random sentinels rebuilt at `layer`, anchor layer <-
+ *    `layer`) and the layer's counters.  The launch covers every possible
+ *    row tile and tiles past a head's list length exit at once, so nothing
+ *    waits on the host.  RR_ESTATE unless rr_relay_compact of this `layer`
+ *    came just before. */
+rr_status rr_relay_rescore(rr_ledger *ledger, const void *d_qc, const void *d_kc, int32_t layer,
+                           void *stream);
+rr_status rr_relay_compact(rr_ledger *ledger, int32_t layer, void *stream);
+rr_status rr_relay_refresh(rr_ledger *ledger, const void *d_qc, const void *d_kc, int32_t layer,
+                           void *stream);
+
+/* Destination of rr_ledger_read.  Any pointer may be NULL (that part is not
+ * copied).  Sizes: ids bh*nq*c int32 laid out [bh, nq, c] (route, then
+ * near-miss, then random), alpha bh*nq f32, anchor_layer bh*nq int32, flags
+ * bh*nq u8 (1 = the row was fully routed at the last layer), counters 16
+ * int64 (the RR_CNT_* slots).  Host (pinned or pageable) or device memory. */
+typedef struct {
+    int32_t *ids;
+    float *alpha;
+    int32_t *anchor_layer;
+    uint8_t *flags;
+    int64_t *counters;
+} rr_ledger_view;
+
+/* Enqueues copies of the ledger into dst (cudaMemcpyDefault, on `stream`).
+ * The caller synchronises the stream before reading dst.  Errors: RR_EINVAL,
+ * RR_ECUDA. */
+rr_status rr_ledger_read(const rr_ledger *ledger, const rr_ledger_view *dst, void *stream);
+
+/* Fills *view with the device addresses of the ledger's arrays inside the
+ * workspace (no copy), for consumers on the same device. */
+rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view);
+
+/* Human-readable name of a status code (static string). */
+const char *rr_status_string(rr_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RR_H */

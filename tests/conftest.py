@@ -6,5 +6,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_native():
+    """Builds the oracle and librr.so (if stale) before any test imports them."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_rr_build", os.path.join(ROOT, "cross_layer_route_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import oracle
+    oracle.build()
+
+
+_build_native()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")

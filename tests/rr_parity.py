@@ -1,0 +1,179 @@
+"""Parity helpers: compare the CUDA path's ledger with the CPU oracle, layer by
+layer, on the same seeded inputs.
+
+Tie margin: the oracle ranks in fp64, the kernels in fp32.  A row whose
+decision rests on a score gap below TIE_REL x scale (scale = |q_i| x max_j
+|k_j|, about 1 for the row-normalised workloads) may legitimately come out
+either way; such rows are counted and reported, not compared bit for bit.
+The gaps that decide a row are: the rank-k / rank-(k+1) gap (route set), the
+rank-(k+m) / rank-(k+m+1) gap (near-miss set, hence the random pool), and at
+a relay layer alpha - beta - gamma (the refresh decision).  Everything else
+must match: ids bit for bit, order up to equal scores, alpha within the
+margin, flags, anchor layers and counters.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+import oracle
+
+TIE_REL = 1e-5
+
+
+def params_of(w, bh_offset: int = 0) -> oracle.Params:
+    return oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal,
+                         gamma=w.gamma, seed=w.seed)
+
+
+def config_of(w, rr, bh: int | None = None, bh_offset: int = 0):
+    return rr.Config(bh=w.bh if bh is None else bh, nq=w.n, nk=w.n, d=w.d, k=w.k, m_near=w.m,
+                     r_rand=w.r, dtype=w.dtype, anchor_interval=w.anchor_interval, causal=w.causal,
+                     gamma=w.gamma, seed=w.seed, bh_offset=bh_offset)
+
+
+@dataclass
+class Report:
+    rows: int = 0
+    compared: int = 0
+    tie_route: int = 0
+    tie_flag: int = 0
+    refreshed_gpu: int = 0
+    refreshed_oracle: int = 0
+    pairs_oracle: int = 0
+    mismatches: list = field(default_factory=list)
+
+    def add(self, o: "Report"):
+        for f in ("rows", "compared", "tie_route", "tie_flag", "refreshed_gpu", "refreshed_oracle",
+                  "pairs_oracle"):
+            setattr(self, f, getattr(self, f) + getattr(o, f))
+        self.mismatches += o.mismatches
+
+    @property
+    def ties(self) -> int:
+        return self.tie_route + self.tie_flag
+
+
+def _sorted_valid(s_row: np.ndarray, nv: int):
+    idx = np.arange(nv)
+    order = np.lexsort((idx, -s_row[:nv]))
+    return order, s_row[:nv][order]
+
+
+def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndarray, k: np.ndarray,
+                 prev_ids, prev_alpha, prev_anchor, gpu_ids, gpu_alpha, gpu_anchor, gpu_flags,
+                 max_report: int = 10) -> Report:
+    """Runs the oracle on one head from the GPU's previous ledger and checks
+    the GPU's ledger after the same layer."""
+    rep = Report(rows=p.nq)
+    S = oracle.scores(q, k)
+    scale = np.linalg.norm(q.astype(np.float64), axis=1) * np.linalg.norm(k.astype(np.float64), axis=1).max()
+    tol = TIE_REL * np.maximum(scale, 1e-30)
+    if anchor:
+        led = oracle.HeadLedger.empty(p)
+    else:
+        led = oracle.HeadLedger(prev_ids.astype(np.int32).copy(), prev_alpha.astype(np.float64).copy(),
+                                prev_anchor.astype(np.int32).copy())
+    flags_o, beta_o, ref_o, pairs_o, st = oracle.head_layer(p, gh, layer, anchor, q, k, led)
+    assert st == 0
+    rep.refreshed_oracle = ref_o
+    rep.pairs_oracle = pairs_o
+    rep.refreshed_gpu = int(gpu_flags.sum())
+
+    def bad(i, what):
+        if len(rep.mismatches) < max_report:
+            rep.mismatches.append((gh, layer, i, what))
+        else:
+            rep.mismatches.append(None)
+
+    for i in range(p.nq):
+        nv = oracle.valid_count(i, p.nk, p.causal)
+        if not anchor:
+            r_ids = [j for j in prev_ids[i, : p.k] if j >= 0]
+            a = min(S[i, j] for j in r_ids) if r_ids else np.inf
+            if np.isfinite(beta_o[i]) and abs(a - beta_o[i] - p.gamma) < tol[i]:
+                rep.tie_flag += 1
+                continue
+            if int(gpu_flags[i]) != int(flags_o[i]):
+                bad(i, f"flag gpu={int(gpu_flags[i])} oracle={int(flags_o[i])} alpha={a} beta={beta_o[i]}")
+                continue
+            if not flags_o[i]:
+                rep.compared += 1
+                if not np.array_equal(gpu_ids[i], prev_ids[i]):
+                    bad(i, "stable row changed its ids")
+                if abs(float(gpu_alpha[i]) - a) > tol[i]:
+                    bad(i, f"stable alpha gpu={gpu_alpha[i]} oracle={a}")
+                if int(gpu_anchor[i]) != int(prev_anchor[i]):
+                    bad(i, "stable row changed its anchor layer")
+                continue
+        # fully routed row (anchor, or refreshed at relay)
+        order, srt = _sorted_valid(S[i], nv)
+        nr = min(p.k, nv)
+        nm = min(p.m, nv - nr)
+        if nr < nv and srt[nr - 1] - srt[nr] < tol[i]:
+            rep.tie_route += 1
+            continue
+        if nr + nm < nv and nm > 0 and srt[nr + nm - 1] - srt[nr + nm] < tol[i]:
+            rep.tie_route += 1
+            continue
+        rep.compared += 1
+        g = gpu_ids[i]
+        o = led.ids[i]
+        if set(g[:nr].tolist()) != set(o[:nr].tolist()) or any(x != -1 for x in g[nr:p.k]):
+            bad(i, f"route gpu={g[:p.k].tolist()} oracle={o[:p.k].tolist()}")
+            continue
+        if set(g[p.k:p.k + nm].tolist()) != set(o[p.k:p.k + nm].tolist()) \
+                or any(x != -1 for x in g[p.k + nm:p.k + p.m]):
+            bad(i, f"near-miss gpu={g[p.k:p.k + p.m].tolist()} oracle={o[p.k:p.k + p.m].tolist()}")
+            continue
+        pos = list(range(nr)) + [p.k + t for t in range(nm)]
+        for rank, slot in enumerate(pos):
+            if abs(S[i, g[slot]] - srt[rank]) > tol[i]:
+                bad(i, f"order at slot {slot}: gpu id {g[slot]} score {S[i, g[slot]]} vs {srt[rank]}")
+                break
+        if not np.array_equal(g[p.k + p.m:], o[p.k + p.m:]):
+            bad(i, f"random gpu={g[p.k + p.m:].tolist()} oracle={o[p.k + p.m:].tolist()}")
+        if abs(float(gpu_alpha[i]) - srt[nr - 1]) > tol[i]:
+            bad(i, f"alpha gpu={gpu_alpha[i]} oracle={srt[nr - 1]}")
+        if int(gpu_anchor[i]) != layer:
+            bad(i, f"anchor layer gpu={gpu_anchor[i]} expected {layer}")
+        if int(gpu_flags[i]) != 1:
+            bad(i, "fully routed row without flag")
+    return rep
+
+
+def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None):
+    """Runs `layers` layers of workload w through the CUDA ledger `led` and
+    compares every layer of the listed heads with the oracle started from
+    the GPU's own previous ledger.  Returns (total report, per-layer list)."""
+    import rr_workloads
+    import torch
+    st = rr_workloads.LayerStream(w, stream_device)
+    p = params_of(w)
+    total = Report()
+    per_layer = []
+    prev = None
+    for l in range(layers):
+        qf, kf, qs, ks = st.next()
+        qd = qs.to(device).contiguous()
+        kd = ks.to(device).contiguous()
+        anchor = oracle.is_anchor(l, w.anchor_interval)
+        led.layer(qd, kd, l)
+        after = led.read()
+        layer_rep = Report()
+        qn = qf.cpu().numpy()
+        kn = kf.cpu().numpy()
+        for h in heads:
+            pi = prev["ids"][h].numpy() if prev is not None else None
+            pa = prev["alpha"][h].numpy() if prev is not None else None
+            pl = prev["anchor_layer"][h].numpy() if prev is not None else None
+            r = compare_head(p, h, l, anchor, qn[h], kn[h], pi, pa, pl, after["ids"][h].numpy(),
+                             after["alpha"][h].numpy(), after["anchor_layer"][h].numpy(),
+                             after["flags"][h].numpy())
+            layer_rep.add(r)
+        per_layer.append((l, anchor, layer_rep, after["counters"].clone()))
+        total.add(layer_rep)
+        prev = after
+        del qd, kd
+    return total, per_layer

@@ -1,0 +1,115 @@
+"""Host-side checks of the C ABI (include/rr.h): the library loads, exports
+every declared entry point, lays out the workspace as documented and rejects
+bad arguments before touching a device.  No GPU needed: none of these calls
+reaches the CUDA runtime."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import cross_layer_route_b200 as rr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE_WS = 0x7F00_0000_0000      # never dereferenced by these tests
+FAKE_Q = 0x7F10_0000_0000
+
+
+def header_functions():
+    names = set()
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(rr_[a-z_0-9]+)\s*\(", src))
+    return names
+
+
+def test_library_is_built_for_sm100a_and_exports_every_declared_symbol():
+    lib = ctypes.CDLL(rr.LIB_PATH)
+    names = header_functions()
+    assert {"rr_ledger_create", "rr_full_route", "rr_relay_layer", "rr_ledger_read"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+def cfg(**kw):
+    base = dict(bh=2, nq=64, nk=64, d=64, k=8, m_near=8, r_rand=4, dtype="f32", anchor_interval=4)
+    base.update(kw)
+    return rr.Config(**base)
+
+
+def test_workspace_layout_and_ledger_size():
+    # RouteRelay §4.4: a 32-bit index ledger with nq = 1024 and c = 64 holds 256 KB
+    c = cfg(bh=1, nq=1024, nk=1024, k=32, m_near=16, r_rand=16)
+    nbytes = rr.rr_ledger_workspace_bytes(c.to_c())
+    h = rr.rr_ledger_create(c.to_c(), FAKE_WS, nbytes)
+    v = rr.rr_ledger_device_view(h)
+    assert v.ids == FAKE_WS
+    assert v.alpha - v.ids == 1024 * 64 * 4 == 256 * 1024
+    assert v.anchor_layer - v.alpha >= 1024 * 4 and v.flags - v.anchor_layer >= 1024 * 4
+    assert v.counters % 256 == 0 and nbytes >= (v.counters - v.ids) + 64
+    rr.rr_ledger_destroy(h)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(k=0), dict(k=65, nk=64), dict(d=12), dict(d=264), dict(d=0), dict(m_near=-1),
+    dict(k=100, m_near=29), dict(r_rand=129), dict(bh=0), dict(nq=0), dict(nk=0),
+    dict(gamma=-0.1), dict(gamma=float("nan")), dict(gamma=float("inf")), dict(anchor_interval=-1),
+])
+def test_invalid_configs_are_rejected(bad):
+    c = cfg(**bad)
+    assert rr.rr_ledger_workspace_bytes(c.to_c()) == 0
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_ledger_create(c.to_c(), FAKE_WS, 1 << 30)
+    assert e.value.status == rr.RR_EINVAL
+
+
+def test_limits_at_the_edge_are_accepted():
+    for c in (cfg(k=64, nk=64, m_near=64, r_rand=128, d=256), cfg(d=8, k=1, m_near=0, r_rand=0)):
+        nbytes = rr.rr_ledger_workspace_bytes(c.to_c())
+        assert nbytes > 0
+        rr.rr_ledger_destroy(rr.rr_ledger_create(c.to_c(), FAKE_WS, nbytes))
+
+
+def test_create_argument_errors():
+    c = cfg()
+    nbytes = rr.rr_ledger_workspace_bytes(c.to_c())
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_ledger_create(c.to_c(), 0, nbytes)
+    assert e.value.status == rr.RR_EINVAL
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_ledger_create(c.to_c(), FAKE_WS + 16, nbytes)   # not 256-byte aligned
+    assert e.value.status == rr.RR_EINVAL
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_ledger_create(c.to_c(), FAKE_WS, nbytes - 1)
+    assert e.value.status == rr.RR_ENOMEM
+    lib = ctypes.CDLL(rr.LIB_PATH)
+    lib.rr_ledger_create.restype = ctypes.c_int
+    assert lib.rr_ledger_create(None, None, ctypes.c_size_t(0), None) == rr.RR_EINVAL
+
+
+def test_call_order_and_pointer_errors_before_any_device_work():
+    c = cfg()
+    nbytes = rr.rr_ledger_workspace_bytes(c.to_c())
+    h = rr.rr_ledger_create(c.to_c(), FAKE_WS, nbytes)
+    with pytest.raises(rr.RRError) as e:             # relay before any anchor
+        rr.rr_relay_layer(h, FAKE_Q, FAKE_Q, 1, 0)
+    assert e.value.status == rr.RR_ESTATE
+    for q, k, layer in ((0, FAKE_Q, 0), (FAKE_Q, 0, 0), (FAKE_Q + 4, FAKE_Q, 0), (FAKE_Q, FAKE_Q, -1)):
+        with pytest.raises(rr.RRError) as e:
+            rr.rr_full_route(h, q, k, layer, 0)
+        assert e.value.status == rr.RR_EINVAL
+        with pytest.raises(rr.RRError) as e:
+            rr.rr_relay_layer(h, q, k, layer, 0)
+        assert e.value.status == rr.RR_EINVAL
+    with pytest.raises(rr.RRError):
+        rr.rr_ledger_read(None, rr.rr_ledger_view(), 0)
+    rr.rr_ledger_destroy(h)
+    rr.rr_ledger_destroy(None)
+
+
+def test_status_strings():
+    for s in range(6):
+        assert rr.rr_status_string(s).startswith("RR_")
+    assert rr.rr_status_string(99) == "RR_UNKNOWN"
