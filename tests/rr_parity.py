@@ -39,13 +39,14 @@ class Report:
     compared: int = 0
     tie_route: int = 0
     tie_flag: int = 0
+    tie_identical: int = 0
     refreshed_gpu: int = 0
     refreshed_oracle: int = 0
     pairs_oracle: int = 0
     mismatches: list = field(default_factory=list)
 
     def add(self, o: "Report"):
-        for f in ("rows", "compared", "tie_route", "tie_flag", "refreshed_gpu", "refreshed_oracle",
+        for f in ("rows", "compared", "tie_route", "tie_flag", "tie_identical", "refreshed_gpu", "refreshed_oracle",
                   "pairs_oracle"):
             setattr(self, f, getattr(self, f) + getattr(o, f))
         self.mismatches += o.mismatches
@@ -87,6 +88,32 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
         else:
             rep.mismatches.append(None)
 
+    def valid_full_row(i, nv, srt):
+        """A fully routed row whose ranking sits inside the tie margin: check
+        that the GPU's choice is one of the correct ones."""
+        g = gpu_ids[i]
+        nr = min(p.k, nv)
+        nm = min(p.m, nv - nr)
+        route = [int(x) for x in g[: p.k] if x >= 0]
+        near = [int(x) for x in g[p.k:p.k + p.m] if x >= 0]
+        rand = [int(x) for x in g[p.k + p.m:] if x >= 0]
+        allids = route + near + rand
+        if len(route) != nr or len(near) != nm or len(set(allids)) != len(allids):
+            return "wrong counts or repeated ids"
+        if any(x < 0 or x >= nv for x in allids):
+            return "id outside the valid range"
+        if any(S[i, j] < srt[nr - 1] - tol[i] for j in route):
+            return "route member below the k-th score"
+        if nm and any(S[i, j] < srt[nr + nm - 1] - tol[i] or S[i, j] > srt[nr - 1] + tol[i] for j in near):
+            return "near-miss member outside its rank band"
+        if len(rand) != min(p.r, nv - nr - nm):
+            return "wrong random count"
+        if abs(float(gpu_alpha[i]) - srt[nr - 1]) > tol[i]:
+            return "alpha"
+        if int(gpu_anchor[i]) != layer or int(gpu_flags[i]) != 1:
+            return "anchor layer / flag"
+        return None
+
     for i in range(p.nq):
         nv = oracle.valid_count(i, p.nk, p.causal)
         if not anchor:
@@ -94,6 +121,12 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
             a = min(S[i, j] for j in r_ids) if r_ids else np.inf
             if np.isfinite(beta_o[i]) and abs(a - beta_o[i] - p.gamma) < tol[i]:
                 rep.tie_flag += 1
+                if int(gpu_flags[i]):
+                    why = valid_full_row(i, nv, _sorted_valid(S[i], nv)[1])
+                    if why:
+                        bad(i, "tie row refreshed invalidly: " + why)
+                elif not np.array_equal(gpu_ids[i], prev_ids[i]):
+                    bad(i, "tie row kept its route but changed ids")
                 continue
             if int(gpu_flags[i]) != int(flags_o[i]):
                 bad(i, f"flag gpu={int(gpu_flags[i])} oracle={int(flags_o[i])} alpha={a} beta={beta_o[i]}")
@@ -111,11 +144,15 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
         order, srt = _sorted_valid(S[i], nv)
         nr = min(p.k, nv)
         nm = min(p.m, nv - nr)
-        if nr < nv and srt[nr - 1] - srt[nr] < tol[i]:
+        tie = (nr < nv and srt[nr - 1] - srt[nr] < tol[i]) or \
+              (nr + nm < nv and nm > 0 and srt[nr + nm - 1] - srt[nr + nm] < tol[i])
+        if tie:
             rep.tie_route += 1
-            continue
-        if nr + nm < nv and nm > 0 and srt[nr + nm - 1] - srt[nr + nm] < tol[i]:
-            rep.tie_route += 1
+            why = valid_full_row(i, nv, srt)
+            if why:
+                bad(i, "tie row invalid: " + why)
+            elif np.array_equal(gpu_ids[i], led.ids[i]):
+                rep.tie_identical += 1
             continue
         rep.compared += 1
         g = gpu_ids[i]

@@ -21,10 +21,15 @@ def rr():
     return rr
 
 
-def _check(rep: Report, max_tie_frac=0.01):
+def _check(rep: Report, max_tie_frac=0.05):
+    """No mismatch outside the tie margin, every tie row valid, and the tie
+    rows a small share (at 4096 chunks the gap between neighbouring ranks is
+    ~1e-4, so a 1e-5 margin catches a few percent of rows)."""
     assert not rep.mismatches, rep.mismatches[:10]
     assert rep.compared > 0
     assert rep.ties <= max(2, max_tie_frac * rep.rows), (rep.ties, rep.rows)
+    print(f"rows={rep.rows} compared={rep.compared} tie_route={rep.tie_route} "
+          f"tie_flag={rep.tie_flag} tie_identical={rep.tie_identical}")
 
 
 def _workload(name, bh, n, d, dtype, k, m, r, causal, layers=1, H=4, sigma=0.03, seed=0, nk=None):
