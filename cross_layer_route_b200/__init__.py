@@ -21,7 +21,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librr.so")
 
-RR_OK, RR_EINVAL, RR_ESTATE, RR_ENOMEM, RR_ECUDA, RR_EDEVICE = range(6)
+RR_OK, RR_EINVAL, RR_ESTATE, RR_ENOMEM, RR_ECUDA, RR_EDEVICE, RR_ECAPACITY = range(7)
 RR_F32, RR_BF16 = 0, 1
 CNT_ROWS, CNT_PAIRS, CNT_ERROR, CNT_ROWS_TOTAL, CNT_PAIRS_TOTAL, CNT_LAYERS, CNT_LAST_LAYER, \
     CNT_DRAW_CAP, CNT_FULL_PAIRS, CNT_FULL_PAIRS_TOTAL = range(10)
@@ -63,6 +63,8 @@ def _load():
     lib.rr_ledger_read.restype = ctypes.c_int
     lib.rr_ledger_device_view.argtypes = [P, ctypes.POINTER(rr_ledger_view)]
     lib.rr_ledger_device_view.restype = ctypes.c_int
+    lib.rr_route_layer_static.argtypes = [ctypes.POINTER(rr_config), P, P, ctypes.c_int32, P, P, P, P, P, P]
+    lib.rr_route_layer_static.restype = ctypes.c_int
     lib.rr_status_string.argtypes = [ctypes.c_int]
     lib.rr_status_string.restype = ctypes.c_char_p
     return lib
@@ -134,6 +136,19 @@ def rr_ledger_device_view(handle) -> rr_ledger_view:
     v = rr_ledger_view()
     _check(_lib.rr_ledger_device_view(handle, ctypes.byref(v)), "rr_ledger_device_view")
     return v
+
+
+def rr_route_layer_static(cfg: rr_config, d_qc: int, d_kc: int, layer: int, d_ids: int, d_alpha: int,
+                          d_anchor_layer: int, d_flags: int, d_counters: int, stream: int) -> None:
+    """One layer on caller-held ledger arrays with no workspace and no
+    allocation, for callers that cannot allocate device memory (their host
+    framework owns every allocation).  See rr_route_layer_static in
+    include/rr.h for its fixed capacity and its shared static scratch."""
+    _check(_lib.rr_route_layer_static(ctypes.byref(cfg), ctypes.c_void_p(d_qc), ctypes.c_void_p(d_kc), layer,
+                                      ctypes.c_void_p(d_ids), ctypes.c_void_p(d_alpha),
+                                      ctypes.c_void_p(d_anchor_layer), ctypes.c_void_p(d_flags),
+                                      ctypes.c_void_p(d_counters), ctypes.c_void_p(stream)),
+           "rr_route_layer_static")
 
 
 # ---- convenience wrapper over torch memory --------------------------------

@@ -299,6 +299,7 @@ const char *rr_status_string(rr_status status) {
         case RR_ENOMEM: return "RR_ENOMEM: workspace too small or out of host memory";
         case RR_ECUDA: return "RR_ECUDA: CUDA runtime error";
         case RR_EDEVICE: return "RR_EDEVICE: error recorded on the device";
+        case RR_ECAPACITY: return "RR_ECAPACITY: problem exceeds the fixed capacity of the call";
     }
     return "RR_UNKNOWN";
 }

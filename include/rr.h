@@ -51,7 +51,8 @@ typedef enum {
     RR_ESTATE = 2,   /* call out of order (relay before an anchor, layer not increasing) */
     RR_ENOMEM = 3,   /* workspace too small, or host memory for the handle */
     RR_ECUDA = 4,    /* a CUDA runtime call failed (launch, copy, attribute) */
-    RR_EDEVICE = 5   /* the device recorded an error (see the error word) */
+    RR_EDEVICE = 5,  /* the device recorded an error (see the error word) */
+    RR_ECAPACITY = 6 /* the problem exceeds a fixed capacity (rr_route_layer_static) */
 } rr_status;
 
 typedef enum { RR_F32 = 0, RR_BF16 = 1 } rr_dtype;
@@ -191,6 +192,38 @@ rr_status rr_ledger_read(const rr_ledger *ledger, const rr_ledger_view *dst, voi
 /* Fills *view with the device addresses of the ledger's arrays inside the
  * workspace (no copy), for consumers on the same device. */
 rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view);
+
+/* One layer on caller-held ledger arrays, allocating nothing.  The paper
+ * has no counterpart: this is a deployment variant for callers that cannot
+ * call cudaMalloc -- code inside a host framework that owns every device
+ * allocation, or code that must not reach an allocator while it runs.  They
+ * pass the inputs (d_qc, d_kc as for rr_full_route) and the ledger arrays
+ * (in/out, laid out as rr_ledger_read documents: ids [bh, nq, c] int32,
+ * alpha [bh*nq] f32, anchor_layer [bh*nq] int32, flags [bh*nq] u8,
+ * counters [16] int64, zeroed by the caller before the first layer); no
+ * workspace.  Layer 0 and forced-anchor layers (layer % anchor_interval ==
+ * 0) are full routing as in rr_full_route; other layers are one relay layer
+ * as in rr_relay_layer (rescore, compact, refresh).  The only scratch, the
+ * per-head refresh lists and their lengths, lives in a fixed array inside
+ * the library: about 4 MiB of device memory that every GPU loading
+ * librr.so holds until the process exits.  Limits: bh * nq <= 1048576 and
+ * bh <= 4096; larger problems return RR_ECAPACITY and enqueue nothing.
+ * The first call on a device looks up that array's device address (set-up
+ * done once per device, with the device current); make that first call
+ * before any stream capture.  Every call on a device shares the one array
+ * and it keeps the last call's contents; nothing in it has to start at zero
+ * (each call writes every list length it reads).  Calls that can overlap
+ * on the GPU (different streams, or different ledgers run concurrently)
+ * race on it: run them on one stream or serialise them.  The call keeps no
+ * host state, so it cannot check the layer order: the caller must start a
+ * sequence at layer 0 or an anchor layer and pass increasing layers.
+ * Errors: RR_EINVAL (bad config, null or misaligned pointer, layer < 0),
+ * RR_ECAPACITY, RR_ECUDA.  Calls no cudaMalloc, cudaFree or allocating
+ * library routine. */
+rr_status rr_route_layer_static(const rr_config *cfg, const void *d_qc, const void *d_kc,
+                                int32_t layer, int32_t *d_ids, float *d_alpha,
+                                int32_t *d_anchor_layer, uint8_t *d_flags, int64_t *d_counters,
+                                void *stream);
 
 /* Human-readable name of a status code (static string). */
 const char *rr_status_string(rr_status status);

@@ -1,0 +1,86 @@
+"""The allocation-free entry point, rr_route_layer_static, against the regular
+ledger entry points.
+
+rr_route_layer_static serves callers that cannot allocate device memory
+(their host framework owns every allocation): they pass only inputs and the
+ledger arrays, and the call's scratch lives in a fixed array inside librr.so.
+Here it must reproduce, layer after layer, what rr_full_route and
+rr_relay_layer write into a workspace-backed ledger from the same inputs.
+The kernels are the same and deterministic, so ids, flags, anchor layers
+and counters must be identical and alpha equal (the parity tests' margin,
+1e-5, is the bound asserted; exact equality is expected).
+
+The file is named so that pytest collects it last; it also runs alone.
+"""
+import pytest
+import torch
+
+import rr_workloads as W
+from rr_parity import config_of
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def rr():
+    import cross_layer_route_b200 as rr
+    torch.cuda.set_device(0)
+    return rr
+
+
+def _static_arrays(rr, cfg):
+    rows = cfg.bh * cfg.nq
+    return {"ids": torch.full((cfg.bh, cfg.nq, cfg.c), -1, dtype=torch.int32, device=DEV),
+            "alpha": torch.zeros(rows, dtype=torch.float32, device=DEV),
+            "anchor_layer": torch.zeros(rows, dtype=torch.int32, device=DEV),
+            "flags": torch.zeros(rows, dtype=torch.uint8, device=DEV),
+            "counters": torch.zeros(rr.NUM_COUNTERS, dtype=torch.int64, device=DEV)}
+
+
+def _call_static(rr, cfg, q, k, layer, a):
+    rr.rr_route_layer_static(cfg.to_c(), q.data_ptr(), k.data_ptr(), layer, a["ids"].data_ptr(),
+                             a["alpha"].data_ptr(), a["anchor_layer"].data_ptr(), a["flags"].data_ptr(),
+                             a["counters"].data_ptr(), torch.cuda.current_stream().cuda_stream)
+
+
+@pytest.mark.parametrize("w", [W.C3.with_(bh=4, layers=4, anchor_interval=8),
+                               W.C5.with_(bh=2, n=640, layers=4, anchor_interval=16)],
+                         ids=["f32_causal", "bf16_causal"])
+def test_static_entry_point_matches_ledger_entry_points(rr, w):
+    cfg = config_of(w, rr)
+    led = rr.RouteLedger(cfg, DEV)
+    arrs = _static_arrays(rr, cfg)
+    st = W.LayerStream(w, "cpu")
+    for layer in range(w.layers):
+        _, _, qs, ks = st.next()
+        q, k = qs.to(DEV), ks.to(DEV)
+        led.layer(q, k, layer)
+        _call_static(rr, cfg, q, k, layer, arrs)
+        ref = led.read()
+        torch.cuda.synchronize()
+        got = {n: t.cpu() for n, t in arrs.items()}
+        assert torch.equal(got["ids"], ref["ids"]), layer
+        assert torch.equal(got["flags"].view(cfg.bh, cfg.nq), ref["flags"]), layer
+        assert torch.equal(got["anchor_layer"].view(cfg.bh, cfg.nq), ref["anchor_layer"]), layer
+        assert torch.allclose(got["alpha"].view(cfg.bh, cfg.nq), ref["alpha"], rtol=0, atol=1e-5), layer
+        assert torch.equal(got["counters"], ref["counters"]), layer
+        if layer > 0:
+            # relay layers are the ones that use the static scratch
+            assert int(got["counters"][rr.CNT_LAST_LAYER]) == layer
+    # two relay calls in a row ran (layers 1..3); some rows were refreshed
+    assert int(arrs["counters"][rr.CNT_ROWS_TOTAL]) > cfg.bh * cfg.nq
+
+
+def test_static_entry_point_rejects_problems_beyond_its_capacity(rr):
+    cfg = rr.Config(bh=300, nq=4096, nk=4096, d=64, k=8, m_near=8, r_rand=8)   # 1.2M rows > 2^20
+    dummy = torch.zeros(16, dtype=torch.int64, device=DEV)
+    p = dummy.data_ptr()
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_route_layer_static(cfg.to_c(), p, p, 1, p, p, p, p, p, 0)
+    assert e.value.status == rr.RR_ECAPACITY
+    cfg = rr.Config(bh=5000, nq=8, nk=8, d=64, k=4, m_near=2, r_rand=1)         # more heads than 4096
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_route_layer_static(cfg.to_c(), p, p, 1, p, p, p, p, p, 0)
+    assert e.value.status == rr.RR_ECAPACITY
