@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librr.so")
-SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_relay.cu", "rr_noalloc.cu"]
+SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_route_tc.cu", "rr_relay.cu", "rr_noalloc.cu"]
 HEADERS = ["rr_device.cuh", "rr_internal.h"]
 
 

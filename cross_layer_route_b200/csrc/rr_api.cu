@@ -22,7 +22,6 @@ struct rr_ledger {
     size_t ws_bytes;
     int device;         // device current at the first enqueue
     bool prepared;      // kernel attributes set on that device
-    size_t route_smem;
     bool anchored;      // a full route started the current layer sequence
     int32_t last_layer; // last layer completed
     int stage;          // relay stages done at pending_layer (0 = none, 1 = rescore, 2 = compact)
@@ -97,7 +96,7 @@ rr_status prepare(rr_ledger *L, cudaStream_t s) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return RR_ECUDA;
     if (L->prepared) return dev == L->device ? RR_OK : RR_EINVAL;
-    if (rr::route_rows_prepare(L->cfg.dtype, L->route_smem) != cudaSuccess) return RR_ECUDA;
+    if (rr::route_rows_prepare(L->dev, L->cfg.dtype) != cudaSuccess) return RR_ECUDA;
     if (cudaMemsetAsync(L->dev.counters, 0, RR_NUM_COUNTERS * sizeof(int64_t), s) != cudaSuccess)
         return RR_ECUDA;
     L->device = dev;
@@ -211,7 +210,6 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     D.gamma = cfg->gamma;
     D.seed_lo = (uint32_t)(cfg->seed & 0xffffffffu);
     D.seed_hi = (uint32_t)(cfg->seed >> 32);
-    L->route_smem = rr::route_rows_smem_bytes(D);
     *out = L;
     return RR_OK;
 }

@@ -37,8 +37,16 @@ inline int select_capacity(int ksel) {
 }
 
 // Launchers (return cudaSuccess or the launch error).
-size_t route_rows_smem_bytes(const LedgerDev &L);
-cudaError_t route_rows_prepare(int dtype, size_t smem_bytes);
+// Full routing of a set of rows.  bf16 problems with d in {64, 128}, k + m <=
+// 64 and r <= 32 run on the tensor cores (rr_route_tc.cu); the others on the
+// CUDA cores (rr_route_simt.cu).  prepare() sets the chosen kernel's shared
+// memory attribute on the current device.
+cudaError_t route_rows_prepare(const LedgerDev &L, int dtype);
+bool route_rows_tc_supported(const LedgerDev &L, int dtype);
+size_t route_rows_tc_smem_bytes(const LedgerDev &L);
+cudaError_t route_rows_tc_prepare(size_t smem_bytes);
+cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
+                                 bool use_list, cudaStream_t s);
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s);
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,

@@ -97,7 +97,7 @@ extern "C" rr_status rr_route_layer_static(const rr_config *cfg, const void *d_q
     D.seed_hi = (uint32_t)(cfg->seed >> 32);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (rr::route_rows_prepare(cfg->dtype, rr::route_rows_smem_bytes(D)) != cudaSuccess) return RR_ECUDA;
+    if (rr::route_rows_prepare(D, cfg->dtype) != cudaSuccess) return RR_ECUDA;
     const int H = cfg->anchor_interval;
     const bool anchor = layer == 0 || (H > 0 && layer % H == 0);
     cudaError_t e = cudaMemsetAsync(d_counters + RR_CNT_ROWS, 0, 2 * sizeof(int64_t), s);

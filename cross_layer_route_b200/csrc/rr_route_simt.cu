@@ -264,20 +264,19 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
 
 }  // namespace
 
-size_t route_rows_smem_bytes(const LedgerDev &L) {
-    return smem_layout(L.d, select_capacity(L.ksel)).total;
-}
-
-cudaError_t route_rows_prepare(int dtype, size_t smem_bytes) {
+cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
+    if (route_rows_tc_supported(L, dtype)) return route_rows_tc_prepare(route_rows_tc_smem_bytes(L));
+    const int smem = (int)smem_layout(L.d, select_capacity(L.ksel)).total;
     if (dtype == kBF16)
         return cudaFuncSetAttribute(route_rows_kernel<__nv_bfloat16>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
-    return cudaFuncSetAttribute(route_rows_kernel<float>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes);
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    return cudaFuncSetAttribute(route_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                smem);
 }
 
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s) {
+    if (route_rows_tc_supported(L, dtype)) return launch_route_rows_tc(L, q, k, layer, use_list, s);
     const int cap = select_capacity(L.ksel);
     const size_t smem = smem_layout(L.d, cap).total;
     dim3 grid((L.nq + kTileRows - 1) / kTileRows, L.bh);

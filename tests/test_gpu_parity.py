@@ -50,6 +50,12 @@ ANCHOR_SHAPES = [
     ("only_random", 2, 100, 32, "bf16", 10, 0, 30, False),
     ("d256", 1, 96, 256, "f32", 8, 8, 8, True),
     ("seed_big", 2, 150, 64, "f32", 12, 12, 12, True),
+    # shapes of the tensor-core path (bf16, d in {64, 128}, k + m <= 64, r <= 32)
+    ("tc_d64", 3, 1000, 64, "bf16", 12, 12, 8, True),
+    ("tc_d128_noncausal", 2, 300, 128, "bf16", 32, 32, 16, False),
+    ("tc_small_n", 3, 70, 128, "bf16", 32, 32, 16, True),
+    ("tc_exact_tile", 2, 256, 64, "bf16", 40, 24, 32, False),
+    ("tc_k1_r0", 2, 129, 128, "bf16", 1, 0, 0, True),
 ]
 
 
