@@ -137,6 +137,12 @@ def make_inputs(w, device, seed):
     return qs, ks
 
 
+def uses_tensor_cores(w) -> bool:
+    """Which full-routing kernel the library runs for this workload (the
+    rule of route_rows_prepare: bf16, d in {64, 128}, k + m <= 64, r <= 32)."""
+    return w.dtype == "bf16" and w.d in (64, 128) and w.k + w.m <= 64 and w.r <= 32
+
+
 def full_pairs_per_layer(w) -> int:
     if not w.causal:
         return w.bh * w.n * w.n
@@ -244,12 +250,18 @@ def run_ours(args, w, rank, world, device):
     # one multiply-add per (row, valid key, dim) -> 2*d flops per score pair.
     route_flops = 2.0 * w.d * full_pairs_per_step * K
     route_tflops = route_flops / (route_ms * 1e-3) / 1e12
-    alu_peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
-    roofline = {"kernel": "route_rows (anchor + refresh)", "bound": "alu",
-                "achieved": round(route_tflops, 3), "peak": round(alu_peak, 1), "unit": "TFLOP/s",
-                "frac": round(route_tflops / alu_peak, 4), "traffic": None,
-                "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock (CUDA-core FMA path)",
-                "avg_launch_ms": round(route_ms / max(n_route, 1), 4)}
+    if uses_tensor_cores(w):
+        peak = float(peaks["bf16_tflops_sustained"])
+        roofline = {"kernel": "route_rows_tc (tcgen05; anchor + refresh)", "bound": "tensor",
+                    "peak_source": f"{peaks['source']} bf16 dense, sustained (timed inside a long step)"}
+    else:
+        peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
+        roofline = {"kernel": "route_rows (CUDA cores; anchor + refresh)", "bound": "alu",
+                    "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock"}
+    roofline.update({"achieved": round(route_tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
+                     "frac": round(route_tflops / peak, 4), "traffic": None,
+                     "avg_launch_ms": round(route_ms / max(n_route, 1), 4),
+                     "launches": n_route})
     # secondary: relay rescore (HBM-bound): per row q (d*e) + its head's keys
     # once (N*d*e/N) + ids (4c) + alpha/flag writes (5) bytes
     rescore_bytes = w.bh * w.n * (2 * w.d * esz + 4 * w.c + 5) * n_rescore
@@ -275,6 +287,7 @@ def run_ours(args, w, rank, world, device):
         "score_pairs_per_s": pairs_per_step * world / (ms_step * 1e-3),
         "pair_fraction": pairs_per_step / (full_pairs_per_layer(w) * L),
         "rho_relay": rho,
+        "retry_rows_per_step": d_cnt[rr.CNT_RETRY_TOTAL] / K,
         "roofline": roofline,
         "kernels": kernels,
         "gpu_launches": K * (2 * len(anchors) + 4 * len(relays)),
@@ -424,9 +437,15 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-recall", action="store_true")
     ap.add_argument("--smi-index", type=int, default=None)
+    ap.add_argument("--bh", type=int, default=None, help="override BH (profiling a smaller case)")
+    ap.add_argument("--layers", type=int, default=None, help="override the layer count")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
+    if args.bh is not None:
+        w = w.with_(bh=args.bh, name=f"{w.name}@bh{args.bh}")
+    if args.layers is not None:
+        w = w.with_(layers=args.layers, name=f"{w.name}@L{args.layers}")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

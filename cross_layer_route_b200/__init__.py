@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "librr.so")
 RR_OK, RR_EINVAL, RR_ESTATE, RR_ENOMEM, RR_ECUDA, RR_EDEVICE, RR_ECAPACITY = range(7)
 RR_F32, RR_BF16 = 0, 1
 CNT_ROWS, CNT_PAIRS, CNT_ERROR, CNT_ROWS_TOTAL, CNT_PAIRS_TOTAL, CNT_LAYERS, CNT_LAST_LAYER, \
-    CNT_DRAW_CAP, CNT_FULL_PAIRS, CNT_FULL_PAIRS_TOTAL = range(10)
+    CNT_DRAW_CAP, CNT_FULL_PAIRS, CNT_FULL_PAIRS_TOTAL, CNT_RETRY_TOTAL = range(11)
 NUM_COUNTERS = 16
 
 

@@ -35,7 +35,7 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-    size_t ids, alpha, anchor_layer, flags, counters, list, head_count, total;
+    size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count, total;
 };
 
 bool config_ok(const rr_config *c) {
@@ -64,6 +64,8 @@ Layout layout_of(const rr_config *c) {
     L.counters = o;     o = align_up(o + RR_NUM_COUNTERS * sizeof(int64_t));
     L.list = o;         o = align_up(o + rows * sizeof(int32_t));
     L.head_count = o;   o = align_up(o + (size_t)c->bh * sizeof(int32_t));
+    L.retry_list = o;   o = align_up(o + rows * sizeof(int32_t));
+    L.retry_count = o;  o = align_up(o + (size_t)c->bh * sizeof(int32_t));
     L.total = o;
     return L;
 }
@@ -200,6 +202,8 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     D.counters = reinterpret_cast<unsigned long long *>(L->ws + lay.counters);
     D.list = reinterpret_cast<int32_t *>(L->ws + lay.list);
     D.head_count = reinterpret_cast<int32_t *>(L->ws + lay.head_count);
+    D.retry_list = reinterpret_cast<int32_t *>(L->ws + lay.retry_list);
+    D.retry_count = reinterpret_cast<int32_t *>(L->ws + lay.retry_count);
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
     D.c = cfg->k + cfg->m_near + cfg->r_rand;

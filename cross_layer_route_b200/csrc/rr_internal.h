@@ -18,6 +18,8 @@ struct LedgerDev {
     // per-layer scratch
     int32_t *list;          // [bh*nq]     per-head segments of flagged row ids, ascending
     int32_t *head_count;    // [bh]        flagged rows per head
+    int32_t *retry_list;    // [bh*nq]     per-head rows whose tensor-core selection is redone
+    int32_t *retry_count;   // [bh]        rows listed per head
     int bh, nq, nk, d;
     int k, m, r, c, ksel;   // ksel = k + m
     int causal;

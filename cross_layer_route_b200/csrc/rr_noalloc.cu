@@ -7,11 +7,12 @@
 // the outputs (the ledger arrays), but not a scratch workspace.  This file
 // gives it one entry point, rr_route_layer_static, whose only scratch -- the
 // per-head lists of refreshed rows and their lengths, written by the
-// compaction kernel and read by the refresh kernel -- lives in a fixed-size
+// compaction kernel and read by the refresh kernel, and the per-head lists
+// of rows whose tensor-core selection is redone -- lives in a fixed-size
 // array in the library's own device memory.
 //
 // The array below is a file-scope __device__ variable: every GPU that loads
-// this library holds it (about 4 MiB) until the process exits.  In host code
+// this library holds it (about 8 MiB) until the process exits.  In host code
 // its name is only a host-side stand-in, not a device address, so the host
 // looks its address up once per device with cudaGetSymbolAddress and passes
 // that address to the kernels.
@@ -27,9 +28,11 @@ constexpr int kStaticMaxRows = 1 << 20;   // bh * nq of one call, at most
 constexpr int kStaticMaxHeads = 4096;     // bh of one call, at most
 constexpr int kMaxDevices = 64;
 
-// [0, kStaticMaxRows): refresh lists (per-head segments of nq entries);
-// [kStaticMaxRows, + kStaticMaxHeads): rows listed per head.
-static __device__ __align__(256) int32_t g_rr_static_scratch[kStaticMaxRows + kStaticMaxHeads];
+// [0, R): refresh lists (per-head segments of nq entries); [R, R + H): rows
+// listed per head; [R + H, 2R + H): lists of rows whose tensor-core
+// selection is redone; [2R + H, 2R + 2H): their counts per head
+// (R = kStaticMaxRows, H = kStaticMaxHeads).
+static __device__ __align__(256) int32_t g_rr_static_scratch[2 * (kStaticMaxRows + kStaticMaxHeads)];
 
 std::mutex g_setup_mutex;
 int32_t *g_scratch_addr[kMaxDevices] = {nullptr};
@@ -85,6 +88,8 @@ extern "C" rr_status rr_route_layer_static(const rr_config *cfg, const void *d_q
     D.counters = reinterpret_cast<unsigned long long *>(d_counters);
     D.list = scratch;
     D.head_count = scratch + kStaticMaxRows;
+    D.retry_list = scratch + kStaticMaxRows + kStaticMaxHeads;
+    D.retry_count = scratch + 2 * kStaticMaxRows + kStaticMaxHeads;
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
     D.c = cfg->k + cfg->m_near + cfg->r_rand;

@@ -5,7 +5,9 @@
 //
 //  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
 //      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
-//      row"), one warp per query row, one lane per candidate.
+//      row"), one warp per query row, one lane per candidate; each lane
+//      gathers its candidate key row with 16-byte loads (all in flight at
+//      once for d = 64, 128) and sums into 8 independent partials.
 //  compact_flags: the prefix sum that compacts unstable row ids (§4.2), one
 //      CTA per head, writing an ascending per-head list and its length.
 //  finalize_layer: per-layer counters (§4.1: the refreshed-row fraction is
@@ -22,7 +24,61 @@ constexpr int kRescoreThreads = 256;
 constexpr int kRescoreWarps = kRescoreThreads / 32;
 constexpr int kDMax = 256;
 
-template <typename T>
+// Score of one candidate row k_j against the warp's query row (fp32 in
+// shared memory), 16-byte key loads and 8 independent partial sums.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int kElems = 4;
+    static __device__ __forceinline__ void fma16(const float *q, uint4 kv, float *acc, int slot) {
+        const float4 qv = *reinterpret_cast<const float4 *>(q);
+        acc[(slot * 4 + 0) & 7] = fmaf(qv.x, __uint_as_float(kv.x), acc[(slot * 4 + 0) & 7]);
+        acc[(slot * 4 + 1) & 7] = fmaf(qv.y, __uint_as_float(kv.y), acc[(slot * 4 + 1) & 7]);
+        acc[(slot * 4 + 2) & 7] = fmaf(qv.z, __uint_as_float(kv.z), acc[(slot * 4 + 2) & 7]);
+        acc[(slot * 4 + 3) & 7] = fmaf(qv.w, __uint_as_float(kv.w), acc[(slot * 4 + 3) & 7]);
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int kElems = 8;
+    static __device__ __forceinline__ void fma16(const float *q, uint4 kv, float *acc, int) {
+        const float4 qa = *reinterpret_cast<const float4 *>(q);
+        const float4 qb = *reinterpret_cast<const float4 *>(q + 4);
+        // bf16 -> fp32 is exact: the bf16 bits become the high half
+        acc[0] = fmaf(qa.x, __uint_as_float(kv.x << 16), acc[0]);
+        acc[1] = fmaf(qa.y, __uint_as_float(kv.x & 0xffff0000u), acc[1]);
+        acc[2] = fmaf(qa.z, __uint_as_float(kv.y << 16), acc[2]);
+        acc[3] = fmaf(qa.w, __uint_as_float(kv.y & 0xffff0000u), acc[3]);
+        acc[4] = fmaf(qb.x, __uint_as_float(kv.z << 16), acc[4]);
+        acc[5] = fmaf(qb.y, __uint_as_float(kv.z & 0xffff0000u), acc[5]);
+        acc[6] = fmaf(qb.z, __uint_as_float(kv.w << 16), acc[6]);
+        acc[7] = fmaf(qb.w, __uint_as_float(kv.w & 0xffff0000u), acc[7]);
+    }
+};
+
+template <typename T, int D>
+__device__ __forceinline__ float dot_row(const float *qs, const T *kp, int d) {
+    constexpr int E = Vec16<T>::kElems;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4 *k4 = reinterpret_cast<const uint4 *>(kp);
+    if constexpr (D > 0) {
+        uint4 kv[D / E];
+#pragma unroll
+        for (int c = 0; c < D / E; ++c) kv[c] = __ldg(k4 + c);   // all loads in flight together
+#pragma unroll
+        for (int c = 0; c < D / E; ++c) Vec16<T>::fma16(qs + c * E, kv[c], acc, c);
+    } else {
+        const int nc = d / E;
+        int c = 0;
+        for (; c + 1 < nc; c += 2) {
+            Vec16<T>::fma16(qs + c * E, __ldg(k4 + c), acc, 0);
+            Vec16<T>::fma16(qs + (c + 1) * E, __ldg(k4 + c + 1), acc, 1);
+        }
+        if (c < nc) Vec16<T>::fma16(qs + c * E, __ldg(k4 + c), acc, 0);
+    }
+    return ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+}
+
+// One warp per query row, one lane per candidate (RouteRelay §3.2 Eq. 5-8).
+template <typename T, int D>
 __global__ void __launch_bounds__(kRescoreThreads)
 relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
     __shared__ __align__(16) float qs_all[kRescoreWarps][kDMax];
@@ -30,7 +86,7 @@ relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const long long rows = (long long)L.bh * L.nq;
     const long long grow = (long long)blockIdx.x * kRescoreWarps + warp;
-    const int d = L.d;
+    const int d = D > 0 ? D : L.d;
     unsigned long long pairs = 0;
     if (grow < rows) {
         const int h = (int)(grow / L.nq);
@@ -54,18 +110,9 @@ relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__
             const bool valid = j >= 0 && j < n_valid;
             bad |= j >= n_valid || j < -1;
             if (valid) {
-                const T *kp = Kh + (size_t)j * d;
-                float s = 0.f;
-                for (int t = 0; t < d; t += 4) {
-                    float kv[4];
-                    Elem<T>::load4(kp + t, kv);
-                    s = fmaf(qs[t], kv[0], s);
-                    s = fmaf(qs[t + 1], kv[1], s);
-                    s = fmaf(qs[t + 2], kv[2], s);
-                    s = fmaf(qs[t + 3], kv[3], s);
-                }
-                if (e < L.k) amin = fminf(amin, s);   // Eq. 6
-                else bmax = fmaxf(bmax, s);           // Eq. 7
+                const float sc = dot_row<T, D>(qs, Kh + (size_t)j * d, d);
+                if (e < L.k) amin = fminf(amin, sc);   // Eq. 6
+                else bmax = fmaxf(bmax, sc);           // Eq. 7
                 ++ncand;
             }
         }
@@ -154,17 +201,25 @@ __global__ void finalize_layer_kernel(LedgerDev L, int layer, long long add_rows
 
 }  // namespace
 
+template <typename T>
+static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, unsigned grid,
+                             cudaStream_t s) {
+    const T *Q = static_cast<const T *>(q);
+    const T *K = static_cast<const T *>(k);
+    switch (L.d) {
+        case 64: relay_rescore_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 128: relay_rescore_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        default: relay_rescore_kernel<T, 0><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+    }
+}
+
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
                                  int layer, cudaStream_t s) {
     (void)layer;
     const long long rows = (long long)L.bh * L.nq;
     const unsigned grid = (unsigned)((rows + kRescoreWarps - 1) / kRescoreWarps);
-    if (dtype == kBF16)
-        relay_rescore_kernel<__nv_bfloat16><<<grid, kRescoreThreads, 0, s>>>(
-            L, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k));
-    else
-        relay_rescore_kernel<float><<<grid, kRescoreThreads, 0, s>>>(
-            L, static_cast<const float *>(q), static_cast<const float *>(k));
+    if (dtype == kBF16) rescore_dispatch<__nv_bfloat16>(L, q, k, grid, s);
+    else rescore_dispatch<float>(L, q, k, grid, s);
     return cudaGetLastError();
 }
 

@@ -11,20 +11,39 @@
 // refresh of the compacted unstable rows (§4.2, rows taken from the
 // per-head list).
 //
-// CTA layout (one CTA = one head x 128 query rows; 6 warps):
-//   warp 0   TMA producer: 128-key x d tiles of Kc (bf16, 128-byte swizzle)
-//            into a 2-stage shared-memory ring.
-//   warp 1   allocates 256 TMEM columns (two 128x128 fp32 accumulators) and
-//            one lane issues tcgen05.mma (M=128, N=128, K=16 per op) for
-//            every key tile, committing to mbarriers.
-//   warps 2-5  epilogue, one thread per query row (= TMEM lane): reads its
-//            row's 128 scores of a tile with tcgen05.ld, keeps those at or
-//            above the row's running threshold in a small append buffer, and
-//            folds the buffer into a per-row min-heap of the k + m best (the
-//            heap's root is the threshold).  Finally heap-sorts, draws the
-//            random sentinels and writes the ledger row.
-// The query tile is gathered by row index into the same swizzled layout
-// the TMA would produce, so anchor and refresh share one code path.
+// CTA layout (one CTA = one head x 128 query rows):
+//   warp 0     TMA producer: 128-key x d tiles of Kc (bf16, 128-byte
+//              swizzle) into a ring of shared-memory stages.
+//   warp 1     allocates 256 TMEM columns (two 128x128 fp32 accumulators);
+//              one lane issues tcgen05.mma (M=128, N=128, K=16 per op) for
+//              every key tile and commits to mbarriers.
+//   warps 2-   epilogue, reading the score tile with tcgen05.ld; a warp may
+//              only read the 32 TMEM lanes (= query rows) of its sub-partition
+//              (warp index mod 4).  The heap kernel runs 4 such warps, one
+//              thread per row; the three-pass kernel runs 8, the two warps of
+//              a sub-partition splitting each tile's columns.
+// The query tile is gathered by row index into the layout a 128-byte
+// swizzled TMA load would produce, so anchor and refresh share one path.
+//
+// Selection (route_rows_tc_kernel).  The tensor cores are cheap next to the
+// per-score work of an exact top-(k+m), so the key tiles are streamed three
+// times and the MMA recomputed each time:
+//   pass 0  per row: the maximum score M, and Lo = the minimum of the first
+//           k+m valid scores (any k+m scores bound the (k+m)-th best from
+//           below);
+//   pass 1  per row: a histogram of (M - s) over 128 equal bins of [Lo, M]
+//           (scores under Lo fall in the last bin); the first bin b* at
+//           which the running count reaches k+m holds the (k+m)-th best;
+//   pass 2  per row: the histogram's counts of bins 0..b* become start
+//           offsets, and every score of those bins is written to its bin's
+//           next slot (a counting sort; about k+m plus one bin's crowd).
+// An insertion sort then fixes the order inside each bin (exact best-first
+// order), and the first k+m are the route and near-miss ids.  A row whose
+// bins 0..b* hold more than kCap scores (or whose bins did not fill exactly
+// -- a certificate check) is appended to a retry list and routed by
+// route_rows_tc_heap_kernel, which keeps a per-row min-heap of the k+m best
+// over one pass; results are exact either way.
+//
 // Every wait is bounded; a timeout sets bit 1 of the error word and the CTA
 // drains its copies, frees its TMEM and returns.
 #include <cuda.h>
@@ -39,30 +58,53 @@ namespace tc {
 
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
-constexpr int kStages = 2;
-constexpr int kEpiWarps = 4;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kBuf = 32;
+constexpr int kMaxStages = 4;
+constexpr int kHeapThreads = 32 * (2 + 4);     // heap kernel: 4 epilogue warps (one per row)
+constexpr int kPassThreads = 32 * (2 + 8);     // three-pass kernel: 8 epilogue warps (two per row)
 constexpr int kTmemCols = 256;
 constexpr int kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr long long kSpinLimit = 1ll << 31;
-
-struct Layout {
-    uint32_t q, k, heap, bufv, bufi, rows, bars, misc, total;
-};
+// three-pass selection
+constexpr int kNB = 64;                    // histogram bins per row
+constexpr int kCap = 96;                   // kept scores per row (both column halves)
+// heap selection (retry path)
+constexpr int kBuf = 32;
 
 __host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Layout layout_of(int d, int ksel) {
+// Stages of the key ring: the three-pass kernel reuses the query and key
+// buffers (>= 72 KB together) to sort its kept scores at the end.
+__host__ __device__ inline int stages_for(int d, bool three_pass) {
+    return (three_pass && d == 64) ? 4 : 2;
+}
+
+struct Layout {
+    uint32_t q, k, sel, hist, bufv, bufi, rows, red, bars, misc, total;
+    int stages;
+};
+
+// three_pass: q | k | hist [kNB][kRows] u32 | bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16
+//             (bufv + bufi, 72 KB, later hold one membership bitmap per row)
+// heap:       q | k | heap [ksel][kRows] u64 | bufv [kBuf][kRows] f32 | bufi [kBuf][kRows] i32
+__host__ __device__ inline Layout layout_of(int d, int ksel, bool three_pass) {
     Layout s;
+    s.stages = stages_for(d, three_pass);
     uint32_t o = 0;
     s.q = o;    o = up(o + kRows * d * 2, 1024);
-    s.k = o;    o = up(o + kStages * kKeys * d * 2, 1024);
-    s.heap = o; o = up(o + kRows * ksel * 8, 16);
-    s.bufv = o; o = up(o + kRows * kBuf * 4, 16);
-    s.bufi = o; o = up(o + kRows * kBuf * 4, 16);
+    s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
+    s.sel = o;
+    if (three_pass) {
+        s.hist = o; o = up(o + kNB * kRows * 4, 16);
+        s.bufv = o; o = up(o + kCap * kRows * 4, 16);
+        s.bufi = o; o = up(o + kCap * kRows * 2, 16);
+    } else {
+        s.hist = o; o = up(o + kRows * ksel * 8, 16);
+        s.bufv = o; o = up(o + kRows * kBuf * 4, 16);
+        s.bufi = o; o = up(o + kRows * kBuf * 4, 16);
+    }
     s.rows = o; o = up(o + kRows * 4, 16);
-    s.bars = o; o = up(o + 8 * (2 * kStages + 5), 16);
+    s.red = o;  o = up(o + (three_pass ? 6 * kRows * 4 : 0), 16);   // max, min, count per half
+    s.bars = o; o = up(o + 8 * (2 * kMaxStages + 5), 16);
     s.misc = o; o = up(o + 16, 16);
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
@@ -153,6 +195,30 @@ __device__ __forceinline__ void tc_ld32(uint32_t taddr, float *v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// The same load without the wait (pair two loads with one tc_wait_ld).
+__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
+        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
+        "%30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// This thread's 64 scores of a tile half: columns c0..c0+63 of its row.
+__device__ __forceinline__ void tc_ld64(uint32_t taddr, float *v) {
+    uint32_t a[32], b[32];
+    tc_ld32_nowait(taddr, a);
+    tc_ld32_nowait(taddr + 32u, b);
+    tc_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) { v[i] = __uint_as_float(a[i]); v[32 + i] = __uint_as_float(b[i]); }
+}
+
 // Shared-memory matrix descriptor of a K-major operand stored as 128-byte
 // swizzled rows (8-row groups 1024 bytes apart): start address >> 4, leading
 // byte offset 16 B, stride byte offset 1024 B, descriptor version 1,
@@ -166,7 +232,225 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr_bytes) {
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKeys >> 3) << 17) |
                             ((uint32_t)(kRows >> 4) << 24);
 
-// ---- per-row selection (one thread per row) ------------------------------------
+// ---- the CTA machinery shared by both kernels ----------------------------------
+struct Cta {
+    unsigned char *q_s, *k_s;
+    int *rows_s;
+    uint64_t *full, *empty, *acc_full, *acc_empty, *mma_done;
+    uint32_t *tmem_slot;
+    volatile int *abort_flag;
+    int stages, n_rows, ntiles;
+    uint32_t tmem_base;
+};
+
+// Rows, barriers, TMEM and the query tile.  Returns false when the CTA has
+// no rows (all threads return together).
+__device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Layout &lay,
+                                          const LedgerDev &L, const __nv_bfloat16 *Q,
+                                          const int *list, const int *head_count, int use_list) {
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int h = blockIdx.y;
+    const int nq = L.nq, d = L.d;
+    const int count = use_list ? head_count[h] : nq;
+    const int row0 = blockIdx.x * kRows;
+    if (row0 >= count) return false;
+    c.q_s = smem + lay.q;
+    c.k_s = smem + lay.k;
+    c.rows_s = reinterpret_cast<int *>(smem + lay.rows);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
+    c.stages = lay.stages;
+    c.full = bars;
+    c.empty = bars + kMaxStages;
+    c.acc_full = bars + 2 * kMaxStages;
+    c.acc_empty = bars + 2 * kMaxStages + 2;
+    c.mma_done = bars + 2 * kMaxStages + 4;
+    c.tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.misc);
+    c.abort_flag = reinterpret_cast<volatile int *>(smem + lay.misc + 4);
+    c.n_rows = min(kRows, count - row0);
+
+    if (tid < kRows) {
+        int row = -1;
+        if (tid < c.n_rows) row = use_list ? list[(size_t)h * nq + row0 + tid] : row0 + tid;
+        c.rows_s[tid] = row;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < c.stages; ++s) {
+            mbar_init(&c.full[s], 1);
+            mbar_init(&c.empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&c.acc_full[a], 1);
+            mbar_init(&c.acc_empty[a], (blockDim.x >> 5) - 2);
+        }
+        mbar_init(c.mma_done, 1);
+        *c.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         saddr(c.tmem_slot)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+
+    // query tile: gather rows by index into the 128-byte-swizzled K-major
+    // layout (row r, 16-byte chunk c of its 64-element half kb lands at
+    // kb*16KB + r*128 + ((c ^ (r & 7)) * 16)).
+    const int c16 = d >> 3;
+    for (int e = tid; e < kRows * c16; e += blockDim.x) {
+        const int r = e / c16, ch = e - r * c16;
+        const int row = c.rows_s[r];
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (row >= 0) v = *reinterpret_cast<const uint4 *>(Q + ((size_t)h * nq + row) * d + ch * 8);
+        const int kb = ch >> 3, cc = ch & 7;
+        *reinterpret_cast<uint4 *>(c.q_s + kb * kSubTileBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    int max_row = -1;
+    for (int e = 0; e < c.n_rows; ++e) max_row = max(max_row, c.rows_s[e]);
+    const int kend = L.causal ? min(L.nk, max_row + 1) : L.nk;
+    c.ntiles = (kend + kKeys - 1) / kKeys;
+    __syncthreads();
+    tc_fence_after();
+    c.tmem_base = *c.tmem_slot;
+    return true;
+}
+
+// TMA producer (one lane): `total` key tiles; tile g is key tile tile_of(g).
+// With three passes the middle pass runs backwards (its first tiles are the
+// ones still in L2 from the previous pass).
+__device__ __forceinline__ int tile_of(int g, int ntiles, int passes) {
+    const int p = g / ntiles, i = g - p * ntiles;
+    return (passes == 3 && p == 1) ? ntiles - 1 - i : i;
+}
+
+__device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int passes) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap_k)) : "memory");
+    const int total = passes * c.ntiles;
+    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
+    int issued = 0;
+    for (int g = 0; g < total; ++g) {
+        const int s = g % c.stages;
+        if (!mbar_wait(&c.empty[s], ((g / c.stages) & 1) ^ 1, c.abort_flag)) break;
+        mbar_expect_tx(&c.full[s], stage_bytes);
+        const int t = tile_of(g, c.ntiles, passes);
+        for (int kb = 0; kb < (d >> 6); ++kb)
+            tma_load_3d(c.k_s + s * stage_bytes + kb * kSubTileBytes, tmap_k, &c.full[s], kb * 64,
+                        t * kKeys, h);
+        ++issued;
+    }
+    // drain: every issued stage must have landed before the CTA exits
+    for (int g = max(0, issued - c.stages); g < issued; ++g) {
+        const int s = g % c.stages;
+        const long long t0 = clock64();
+        while (!mbar_test(&c.full[s], (g / c.stages) & 1) && clock64() - t0 < kSpinLimit) {
+        }
+    }
+}
+
+// MMA issuer (one lane): score tile g into accumulator g % 2.
+__device__ void mma_issuer(Cta &c, int d, int passes) {
+    const int total = passes * c.ntiles;
+    const uint32_t q_addr = saddr(c.q_s), k_addr = saddr(c.k_s);
+    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
+    for (int g = 0; g < total; ++g) {
+        const int s = g % c.stages, a = g & 1;
+        if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
+        if (!mbar_wait(&c.acc_empty[a], ((g >> 1) & 1) ^ 1, c.abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
+        const uint32_t kst = k_addr + (uint32_t)s * stage_bytes;
+        for (int kk = 0; kk < (d >> 4); ++kk) {
+            const uint32_t off = (uint32_t)((kk >> 2) * kSubTileBytes + (kk & 3) * 32);
+            tc_mma_bf16(d_tmem, sw128_desc(q_addr + off), sw128_desc(kst + off), kIdesc,
+                        kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&c.empty[s]);
+        tc_commit(&c.acc_full[a]);
+    }
+    tc_commit(c.mma_done);
+    const long long t0 = clock64();
+    while (!mbar_test(c.mma_done, 0) && clock64() - t0 < kSpinLimit) {
+    }
+}
+
+__device__ __forceinline__ void cta_teardown(Cta &c, const LedgerDev &L) {
+    tc_fence_before();
+    __syncthreads();
+    if ((threadIdx.x >> 5) == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(c.tmem_base),
+                     "r"(kTmemCols)
+                     : "memory");
+    }
+    if (threadIdx.x == 0 && *c.abort_flag) atomicOr(&L.counters[2], 2ULL);
+}
+
+// Epilogue helpers: wait for accumulator g (warp-uniform outcome) / hand it back.
+__device__ __forceinline__ bool acc_wait(Cta &c, int g) {
+    bool ok = mbar_wait(&c.acc_full[g & 1], (g >> 1) & 1, c.abort_flag);
+    ok = __all_sync(kFull, ok);   // the warp leaves together (tcgen05.ld is .sync.aligned)
+    if (ok) tc_fence_after();
+    return ok;
+}
+__device__ __forceinline__ void acc_release(Cta &c, int g) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&c.acc_empty[g & 1]);
+}
+
+// Random sentinels (RouteRelay §3.1 item 2, §3.4) of one row, one thread:
+// Philox4x32-10 draws keyed (seed; head, row, layer, t/4), chunk = (word *
+// n_valid) >> 32, rejecting repeats and route / near-miss members
+// (`in_excl`); a pool of at most r chunks is taken whole in ascending order,
+// and a row that exhausts max_draws is completed in ascending order.
+// Accepted chunks go to acc_at(0..); with a membership bitmap (`bits`,
+// words at stride kRows, already holding route and near-miss) they are also
+// marked there, which makes in_excl cover them.
+template <typename Excl, typename Acc>
+__device__ __forceinline__ int random_sentinels(const LedgerDev &L, int ghead, int row, int layer,
+                                                int n_valid, int nsel, Excl in_excl, Acc acc_at,
+                                                int32_t *out, uint32_t *bits) {
+    int acc = 0;
+    auto taken = [&](int j) {
+        if (in_excl(j)) return true;
+        if (bits) return false;
+        for (int e = 0; e < acc; ++e)
+            if ((int)acc_at(e) == j) return true;
+        return false;
+    };
+    auto accept = [&](int j) {
+        acc_at(acc) = j;
+        ++acc;
+        if (bits) bits[(j >> 5) * kRows] |= 1u << (j & 31);
+    };
+    if (L.r > 0) {
+        const int np = n_valid - nsel;
+        if (np > L.r) {
+            uint32_t w4[4] = {0u, 0u, 0u, 0u};
+            for (int t = 0; acc < L.r && t < L.max_draws; ++t) {
+                if ((t & 3) == 0) {
+                    const PhiloxOut o = philox4x32_10((uint32_t)ghead, (uint32_t)row, (uint32_t)layer,
+                                                      (uint32_t)(t >> 2), L.seed_lo, L.seed_hi);
+                    w4[0] = o.w[0]; w4[1] = o.w[1]; w4[2] = o.w[2]; w4[3] = o.w[3];
+                }
+                const int sel = t & 3;
+                const uint32_t w = sel == 0 ? w4[0] : sel == 1 ? w4[1] : sel == 2 ? w4[2] : w4[3];
+                const int j = (int)__umulhi(w, (uint32_t)n_valid);
+                if (!taken(j)) accept(j);
+            }
+            if (acc < L.r) atomicAdd(&L.counters[7], 1ULL);
+        }
+        for (int j = 0; acc < L.r && j < n_valid; ++j)
+            if (!taken(j)) accept(j);
+    }
+    for (int e = 0; e < L.r; ++e) out[e] = e < acc ? (int)acc_at(e) : -1;
+    return acc;
+}
+
+// ---- per-row keys for the heap path ---------------------------------------------
 // Keys order (score, chunk) pairs: larger key = higher score, then smaller chunk.
 __device__ __forceinline__ uint32_t ord32(float f) {
     const uint32_t u = __float_as_uint(f);
@@ -199,189 +483,52 @@ __device__ __forceinline__ void heap_sift(uint64_t *H, int n, uint64_t K) {
     H[i * kRows] = K;
 }
 
-__device__ __forceinline__ bool in_keys(const uint64_t *H, int n, int j) {
-    for (int e = 0; e < n; ++e)
-        if (key_chunk(H[e * kRows]) == j) return true;
-    return false;
-}
-__device__ __forceinline__ bool in_ints(const int *B, int n, int j) {
-    for (int e = 0; e < n; ++e)
-        if (B[e * kRows] == j) return true;
-    return false;
-}
-
-__global__ void __launch_bounds__(kThreads, 1)
-route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
-                     const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
+// ---- heap kernel: one pass, per-row min-heap (the retry path) --------------------
+__global__ void __launch_bounds__(kHeapThreads, 1)
+route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+                          const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    const int d = L.d;
-    const int ksel = L.ksel;
-    const Layout lay = layout_of(d, ksel);
-    unsigned char *q_s = smem + lay.q;
-    unsigned char *k_s = smem + lay.k;
-    uint64_t *heap_all = reinterpret_cast<uint64_t *>(smem + lay.heap);
-    float *bufv_all = reinterpret_cast<float *>(smem + lay.bufv);
-    int *bufi_all = reinterpret_cast<int *>(smem + lay.bufi);
-    int *rows_s = reinterpret_cast<int *>(smem + lay.rows);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
-    uint64_t *full = bars;                  // [kStages]
-    uint64_t *empty = bars + kStages;       // [kStages]
-    uint64_t *acc_full = bars + 2 * kStages;       // [2]
-    uint64_t *acc_empty = bars + 2 * kStages + 2;  // [2]
-    uint64_t *mma_done = bars + 2 * kStages + 4;   // [1]
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.misc);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + lay.misc + 4);
-
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int d = L.d, ksel = L.ksel;
+    const Layout lay = layout_of(d, ksel, false);
+    Cta c;
+    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
-    const int nq = L.nq, nk = L.nk;
-    const int count = use_list ? L.head_count[h] : nq;
-    const int row0 = blockIdx.x * kRows;
-    if (row0 >= count) return;
-    const int n_rows = min(kRows, count - row0);
-
-    if (tid < kRows) {
-        int row = -1;
-        if (tid < n_rows) row = use_list ? L.list[(size_t)h * nq + row0 + tid] : row0 + tid;
-        rows_s[tid] = row;
-    }
-    if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        for (int a = 0; a < 2; ++a) {
-            mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], kEpiWarps);
-        }
-        mbar_init(mma_done, 1);
-        *abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         saddr(tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    __syncthreads();
-
-    // query tile: gather rows by index into the 128-byte-swizzled K-major
-    // layout (row r, 16-byte chunk c of its 64-element half kb lands at
-    // kb*16KB + r*128 + ((c ^ (r & 7)) * 16)).
-    const int c16 = d >> 3;  // 16-byte chunks per row
-    for (int e = tid; e < kRows * c16; e += kThreads) {
-        const int r = e / c16, c = e - r * c16;
-        const int row = rows_s[r];
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row >= 0) v = *reinterpret_cast<const uint4 *>(Q + ((size_t)h * nq + row) * d + c * 8);
-        const int kb = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4 *>(q_s + kb * kSubTileBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    int max_row = -1;
-    for (int e = 0; e < n_rows; ++e) max_row = max(max_row, rows_s[e]);
-    const int kend = L.causal ? min(nk, max_row + 1) : nk;
-    const int ntiles = (kend + kKeys - 1) / kKeys;
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_k))
-                         : "memory");
-            int issued = 0;
-            for (int t = 0; t < ntiles; ++t) {
-                const int s = t % kStages;
-                if (!mbar_wait(&empty[s], ((t / kStages) & 1) ^ 1, abort_flag)) break;
-                mbar_expect_tx(&full[s], (uint32_t)(kKeys * d * 2));
-                for (int kb = 0; kb < (d >> 6); ++kb)
-                    tma_load_3d(k_s + s * (kKeys * d * 2) + kb * kSubTileBytes, &tmap_k, &full[s],
-                                kb * 64, t * kKeys, h);
-                ++issued;
-            }
-            // drain: every issued stage must have landed before the CTA exits
-            for (int t = max(0, issued - kStages); t < issued; ++t) {
-                const int s = t % kStages;
-                const long long t0 = clock64();
-                while (!mbar_test(&full[s], (t / kStages) & 1) && clock64() - t0 < kSpinLimit) {
-                }
-            }
-        }
+        if (lane == 0) producer(c, &tmap_k, d, h, 1);
     } else if (warp == 1) {
-        // ---------------- MMA issuer ----------------
-        if (lane == 0) {
-            const uint32_t q_addr = saddr(q_s), k_addr = saddr(k_s);
-            for (int t = 0; t < ntiles; ++t) {
-                const int s = t % kStages, a = t & 1;
-                if (!mbar_wait(&full[s], (t / kStages) & 1, abort_flag)) break;
-                if (!mbar_wait(&acc_empty[a], ((t >> 1) & 1) ^ 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(a * kKeys);
-                const uint32_t kst = k_addr + (uint32_t)(s * kKeys * d * 2);
-                for (int kk = 0; kk < (d >> 4); ++kk) {
-                    const uint32_t off = (uint32_t)((kk >> 2) * kSubTileBytes + (kk & 3) * 32);
-                    tc_mma_bf16(d_tmem, sw128_desc(q_addr + off), sw128_desc(kst + off), kIdesc,
-                                kk > 0 ? 1u : 0u);
-                }
-                tc_commit(&empty[s]);
-                tc_commit(&acc_full[a]);
-            }
-            tc_commit(mma_done);
-            const long long t0 = clock64();
-            while (!mbar_test(mma_done, 0) && clock64() - t0 < kSpinLimit) {
-            }
-        }
+        if (lane == 0) mma_issuer(c, d, 1);
     } else {
-        // ---------------- epilogue: one thread per query row ----------------
-        const int sub = warp & 3;            // TMEM sub-partition this warp may read
-        const int r = sub * 32 + lane;       // row slot = TMEM lane = query tile row
-        const int row = rows_s[r];
-        const int n_valid = row >= 0 ? valid_keys(row, nk, L.causal) : 0;
-        uint64_t *H = heap_all + r;
-        float *bv = bufv_all + r;
-        int *bi = bufi_all + r;
+        const int sub = warp & 3;
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
+        uint64_t *H = reinterpret_cast<uint64_t *>(smem + lay.hist) + r;
+        float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
+        int *bi = reinterpret_cast<int *>(smem + lay.bufi) + r;
         for (int e = 0; e < ksel; ++e) H[e * kRows] = 0ull;
         float thr = -INFINITY;
         bool ok = true;
-        for (int t = 0; t < ntiles && ok; ++t) {
-            const int a = t & 1;
-            ok = mbar_wait(&acc_full[a], (t >> 1) & 1, abort_flag);
-            ok = __all_sync(kFull, ok);   // the warp leaves together (tcgen05.ld is .sync.aligned)
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t tbase = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(a * kKeys);
+        for (int t = 0; t < c.ntiles && ok; ++t) {
+            if (!(ok = acc_wait(c, t))) break;
+            const uint32_t tbase = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)((t & 1) * kKeys);
 #pragma unroll 1
             for (int ch = 0; ch < kKeys / 32; ++ch) {
                 float v[32];
                 tc_ld32(tbase + (uint32_t)(ch * 32), v);
                 const int col0 = t * kKeys + ch * 32;
                 int cnt = 0;
-                if (col0 + 32 <= n_valid) {
 #pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        if (v[jj] >= thr) {
-                            bv[cnt * kRows] = v[jj];
-                            bi[cnt * kRows] = col0 + jj;
-                            ++cnt;
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 32; ++jj) {
-                        if (col0 + jj < n_valid && v[jj] >= thr) {
-                            bv[cnt * kRows] = v[jj];
-                            bi[cnt * kRows] = col0 + jj;
-                            ++cnt;
-                        }
+                for (int jj = 0; jj < 32; ++jj) {
+                    if (col0 + jj < n_valid && v[jj] >= thr) {
+                        bv[cnt * kRows] = v[jj];
+                        bi[cnt * kRows] = col0 + jj;
+                        ++cnt;
                     }
                 }
-                // fold this chunk's survivors into the heap
                 for (int e = 0; e < cnt; ++e) {
                     const uint64_t key = make_key(bv[e * kRows], bi[e * kRows]);
                     if (key > H[0]) heap_sift(H, ksel, key);
@@ -389,13 +536,9 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 const uint64_t root = H[0];
                 thr = root == 0ull ? -INFINITY : key_score(root);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[a]);
+            acc_release(c, t);
         }
-        if (!ok) {
-            if (lane == 0) atomicOr(&L.counters[2], 2ULL);
-        } else if (row >= 0) {
+        if (ok && row >= 0) {
             // best-first order: repeatedly move the heap minimum to the end
             for (int end = ksel - 1; end > 0; --end) {
                 const uint64_t top = H[0];
@@ -406,55 +549,268 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             const int nr = min(L.k, n_valid);
             const int nm = min(L.m, n_valid - nr);
             const int nsel = nr + nm;
-            const size_t grow = (size_t)h * nq + row;
+            const size_t grow = (size_t)h * L.nq + row;
             int32_t *out = L.ids + grow * L.c;
             for (int e = 0; e < L.k; ++e) out[e] = e < nr ? key_chunk(H[e * kRows]) : -1;
             for (int e = 0; e < L.m; ++e) out[L.k + e] = e < nm ? key_chunk(H[(nr + e) * kRows]) : -1;
-            // random sentinels (RouteRelay §3.1 item 2, §3.4); accepted ids in bi[]
-            int acc = 0;
-            if (L.r > 0) {
-                const int np = n_valid - nsel;
-                if (np > L.r) {
-                    uint32_t w4[4] = {0u, 0u, 0u, 0u};
-                    int t = 0;
-                    for (; acc < L.r && t < L.max_draws; ++t) {
-                        if ((t & 3) == 0) {
-                            const PhiloxOut o = philox4x32_10((uint32_t)(L.bh_offset + h), (uint32_t)row,
-                                                              (uint32_t)layer, (uint32_t)(t >> 2),
-                                                              L.seed_lo, L.seed_hi);
-                            w4[0] = o.w[0]; w4[1] = o.w[1]; w4[2] = o.w[2]; w4[3] = o.w[3];
-                        }
-                        const int sel = t & 3;
-                        const uint32_t w = sel == 0 ? w4[0] : sel == 1 ? w4[1] : sel == 2 ? w4[2] : w4[3];
-                        const int j = (int)__umulhi(w, (uint32_t)n_valid);
-                        if (in_keys(H, nsel, j) || in_ints(bi, acc, j)) continue;
-                        bi[acc * kRows] = j;
-                        ++acc;
-                    }
-                    if (acc < L.r) atomicAdd(&L.counters[7], 1ULL);
-                }
-                for (int j = 0; acc < L.r && j < n_valid; ++j) {
-                    if (in_keys(H, nsel, j) || in_ints(bi, acc, j)) continue;
-                    bi[acc * kRows] = j;
-                    ++acc;
-                }
-            }
-            for (int e = 0; e < L.r; ++e) out[L.k + L.m + e] = e < acc ? bi[e * kRows] : -1;
+            random_sentinels(
+                L, L.bh_offset + h, row, layer, n_valid, nsel,
+                [&](int j) {
+                    for (int e = 0; e < nsel; ++e)
+                        if (key_chunk(H[e * kRows]) == j) return true;
+                    return false;
+                },
+                [&](int e) -> int & { return bi[e * kRows]; }, out + L.k + L.m, nullptr);
             L.alpha[grow] = key_score(H[(nr - 1) * kRows]);
             L.anchor_layer[grow] = layer;
             L.flags[grow] = 1;
         }
     }
+    cta_teardown(c, L);
+}
 
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 1) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                     "r"(kTmemCols)
-                     : "memory");
+// ---- three-pass kernel (the main path) ------------------------------------------
+// Bin of a score for one row: bins of width (M - Lo) / kNB counted down from
+// M; scores under Lo land in the last bin.  The same expression is used in
+// every place a bin is computed, so counts and placements agree.
+__device__ __forceinline__ int bin_of(float v, float neg_inv, float hi_inv) {
+    return min((int)fmaf(v, neg_inv, hi_inv), kNB - 1);
+}
+
+__global__ void __launch_bounds__(kPassThreads, 1)
+route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+                     const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const int d = L.d, ksel = L.ksel;
+    const Layout lay = layout_of(d, ksel, true);
+    Cta c;
+    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+
+    if (warp == 0) {
+        if (lane == 0) producer(c, &tmap_k, d, h, 3);
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(c, d, 3);
+    } else {
+        // Two warps per TMEM sub-partition: half 0 reads columns 0..63 of
+        // every tile, half 1 columns 64..127.  Per-row state lives in shared
+        // memory; the 256 epilogue threads meet at named barrier 1 between
+        // phases (every one of them reaches every barrier, also after a
+        // timeout, so none can be left waiting).
+        const int sub = warp & 3;
+        const int half = (warp - 2) >> 2;
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
+        const int first_lim = min(ksel, n_valid);
+        const bool all_mode = n_valid <= ksel;   // every valid key is selected
+        uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist) + r;
+        float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
+        uint16_t *bi = reinterpret_cast<uint16_t *>(smem + lay.bufi) + r;
+        float *red_lo = reinterpret_cast<float *>(smem + lay.red) + 2 * kRows; // [2][kRows]
+        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(half * 64);
+        const int nt = c.ntiles;
+        bool ok = true;
+        int g = 0;
+        auto epi_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+
+        // pass 0: per row, the maximum of each of 64 disjoint column groups
+        // (group = half, column mod 32) and the minimum of the first k+m valid
+        // scores.  M = the largest group maximum; the smallest group maximum
+        // and that minimum are both at most the (k+m)-th best score (each
+        // comes with k+m or more distinct scores at or above it), so the
+        // larger of the two is the histogram's lower end Lo.
+        float gm[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) gm[q] = -INFINITY;
+        float Lo = INFINITY;
+        for (int i = 0; i < nt && ok; ++i, ++g) {
+            if (!(ok = acc_wait(c, g))) break;
+            float v[64];
+            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            const int col0 = i * kKeys + half * 64;
+            if (col0 + 64 <= n_valid) {
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj) gm[jj & 31] = fmaxf(gm[jj & 31], v[jj]);
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj)
+                    if (col0 + jj < n_valid) gm[jj & 31] = fmaxf(gm[jj & 31], v[jj]);
+            }
+            if (col0 < first_lim) {
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj)
+                    if (col0 + jj < first_lim) Lo = fminf(Lo, v[jj]);
+            }
+            acc_release(c, g);
+        }
+        {
+            float *gx = reinterpret_cast<float *>(smem + lay.bufv) + r;   // [64][kRows]
+#pragma unroll
+            for (int q = 0; q < 32; ++q) gx[(half * 32 + q) * kRows] = gm[q];
+        }
+        red_lo[half * kRows + r] = Lo;
+        if (half == 0)
+            for (int b = 0; b < kNB; ++b) hist[b * kRows] = 0u;
+        epi_sync();
+        float M = -INFINITY, gmin = INFINITY;
+        {
+            const float *gx = reinterpret_cast<const float *>(smem + lay.bufv) + r;
+            for (int q = 0; q < 64; ++q) {
+                const float x = gx[q * kRows];
+                M = fmaxf(M, x);
+                gmin = fminf(gmin, x);
+            }
+        }
+        Lo = fmaxf(fminf(red_lo[r], red_lo[kRows + r]), gmin);
+
+        // pass 1: histogram of (M - s) over [Lo, M], tiles in reverse order
+        const float range = M - Lo;
+        const float inv = (!all_mode && range > 0.f) ? (float)kNB / range : 0.f;
+        const float neg_inv = -inv, hi_inv = M * inv;
+        for (int i = 0; i < nt && ok; ++i, ++g) {
+            if (!(ok = acc_wait(c, g))) break;
+            const int t = nt - 1 - i;
+            float v[64];
+            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);   // every lane loads (.sync.aligned)
+            const int col0 = t * kKeys + half * 64;
+            if (!all_mode) {
+                if (col0 + 64 <= n_valid) {
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj)
+                        atomicAdd(&hist[bin_of(v[jj], neg_inv, hi_inv) * kRows], 1u);
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < 64; ++jj)
+                        if (col0 + jj < n_valid)
+                            atomicAdd(&hist[bin_of(v[jj], neg_inv, hi_inv) * kRows], 1u);
+                }
+            }
+            acc_release(c, g);
+        }
+        epi_sync();
+
+        // boundary bin b*: the first bin where the running count reaches k+m;
+        // run = scores in bins 0..b*.  Rows with every valid key selected use
+        // one bin.
+        int bstar = 0;
+        uint32_t run = (uint32_t)n_valid;
+        if (!all_mode) {
+            bstar = kNB - 1;
+            uint32_t cum = 0;
+            for (int b = 0; b < kNB; ++b) {
+                cum += hist[b * kRows];
+                if (cum >= (uint32_t)ksel) { bstar = b; break; }
+            }
+            run = cum;
+        }
+        const bool overflow = run > (uint32_t)kCap;
+        // half 0 turns the counts of bins 0..b* into exclusive start offsets
+        if (half == 0) {
+            if (all_mode) {
+                hist[0] = 0u;
+            } else {
+                uint32_t acc = 0;
+                for (int b = 0; b <= bstar; ++b) {
+                    const uint32_t x = hist[b * kRows];
+                    hist[b * kRows] = acc;
+                    acc += x;
+                }
+            }
+        }
+        epi_sync();
+
+        // pass 2: every score of bins 0..b* goes straight to its bin's next
+        // slot (same bin arithmetic as pass 1, so exactly `run` scores land)
+        for (int i = 0; i < nt && ok; ++i, ++g) {
+            if (!(ok = acc_wait(c, g))) break;
+            float v[64];
+            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            const int col0 = i * kKeys + half * 64;
+            const int lim = overflow ? 0 : n_valid - col0;   // columns jj < lim take part
+#pragma unroll
+            for (int jj = 0; jj < 64; ++jj) {
+                const int b = all_mode ? 0 : bin_of(v[jj], neg_inv, hi_inv);
+                if (jj < lim && b <= bstar) {
+                    const uint32_t pos = atomicAdd(&hist[b * kRows], 1u);
+                    if (pos < (uint32_t)kCap) {
+                        bv[pos * kRows] = v[jj];
+                        bi[pos * kRows] = (uint16_t)(col0 + jj);
+                    }
+                }
+            }
+            acc_release(c, g);
+        }
+        epi_sync();
+
+        // Each row's kept scores now sit in bins order.  The two halves share
+        // the rows: half 0 finishes lanes 0..15, half 1 lanes 16..31.
+        const bool mine = ok && row >= 0 && (lane >> 4) == half;
+        if (mine) {
+            // every bin must have been filled exactly (b*'s next slot == run)
+            const bool fail = overflow || hist[bstar * kRows] != run;
+            if (fail) {
+                const int pos = atomicAdd(&L.retry_count[h], 1);
+                L.retry_list[(size_t)h * L.nq + pos] = row;
+                atomicAdd(&L.counters[10], 1ULL);
+            } else {
+                // insertion sort, best first (score desc, chunk asc): only
+                // within-bin disorder is left
+                const int nsorted = (int)run;
+                for (int e = 1; e < nsorted; ++e) {
+                    const float v = bv[e * kRows];
+                    const uint16_t j = bi[e * kRows];
+                    int p = e - 1;
+                    while (p >= 0) {
+                        const float pv = bv[p * kRows];
+                        const uint16_t pj = bi[p * kRows];
+                        if (!(v > pv || (v == pv && j < pj))) break;
+                        bv[(p + 1) * kRows] = pv;
+                        bi[(p + 1) * kRows] = pj;
+                        --p;
+                    }
+                    bv[(p + 1) * kRows] = v;
+                    bi[(p + 1) * kRows] = j;
+                }
+                const int nr = min(L.k, n_valid);
+                const int nm = min(L.m, n_valid - nr);
+                const int nsel = nr + nm;
+                const size_t grow = (size_t)h * L.nq + row;
+                int32_t *out = L.ids + grow * L.c;
+                for (int e = 0; e < L.k; ++e) out[e] = e < nr ? (int)bi[e * kRows] : -1;
+                for (int e = 0; e < L.m; ++e) out[L.k + e] = e < nm ? (int)bi[(nr + e) * kRows] : -1;
+                // one bit per valid chunk (route, near-miss, accepted sentinels)
+                // in the query/key buffers, free now that every MMA is done
+                uint32_t *bits = reinterpret_cast<uint32_t *>(smem + lay.q) + r;
+                const int words = (n_valid + 31) >> 5;
+                const bool use_bits = words <= (int)(lay.sel / (kRows * 4));
+                if (use_bits) {
+                    for (int w = 0; w < words; ++w) bits[w * kRows] = 0u;
+                    for (int e = 0; e < nsel; ++e) {
+                        const int j = bi[e * kRows];
+                        bits[(j >> 5) * kRows] |= 1u << (j & 31);
+                    }
+                }
+                int32_t *rout = out + L.k + L.m;
+                random_sentinels(
+                    L, L.bh_offset + h, row, layer, n_valid, nsel,
+                    [&](int j) {
+                        if (use_bits) return ((bits[(j >> 5) * kRows] >> (j & 31)) & 1u) != 0u;
+                        for (int e = 0; e < nsel; ++e)
+                            if ((int)bi[e * kRows] == j) return true;
+                        return false;
+                    },
+                    [&](int e) -> int32_t & { return rout[e]; }, rout, use_bits ? bits : nullptr);
+                L.alpha[grow] = bv[(nr - 1) * kRows];
+                L.anchor_layer[grow] = layer;
+                L.flags[grow] = 1;
+            }
+        }
     }
-    if (tid == 0 && *abort_flag) atomicOr(&L.counters[2], 2ULL);
+    cta_teardown(c, L);
 }
 
 // ---- host side -----------------------------------------------------------------
@@ -480,14 +836,27 @@ EncodeTiledFn encode_fn() {
 }  // namespace tc
 
 bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
-    return dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf;
+    return dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf &&
+           L.nk <= 65535;
 }
 
-size_t route_rows_tc_smem_bytes(const LedgerDev &L) { return tc::layout_of(L.d, L.ksel).total; }
+size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
+    const size_t a = tc::layout_of(L.d, L.ksel, true).total;
+    const size_t b = tc::layout_of(L.d, L.ksel, false).total;
+    return a > b ? a : b;
+}
 
 cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
-    return cudaFuncSetAttribute(tc::route_rows_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes);
+    if (smem_bytes > 232448) return cudaErrorInvalidValue;   // 227 KB per block on sm_100
+    // both kernels may be launched with up to their largest layout
+    const int big = (int)tc::layout_of(128, 64, true).total;
+    const int big_heap = (int)tc::layout_of(128, 64, false).total;
+    cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::route_rows_tc_heap_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big_heap);
+    return e;
 }
 
 cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
@@ -503,10 +872,21 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    const size_t smem = tc::layout_of(L.d, L.ksel).total;
+    cudaError_t e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
+    if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
-    tc::route_rows_tc_kernel<<<grid, tc::kThreads, smem, s>>>(
+    const size_t smem3 = tc::layout_of(L.d, L.ksel, true).total;
+    tc::route_rows_tc_kernel<<<grid, tc::kPassThreads, smem3, s>>>(
         L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    // rows whose three-pass certificate failed: exact heap selection
+    LedgerDev R = L;
+    R.list = L.retry_list;
+    R.head_count = L.retry_count;
+    const size_t smemh = tc::layout_of(L.d, L.ksel, false).total;
+    tc::route_rows_tc_heap_kernel<<<grid, tc::kHeapThreads, smemh, s>>>(
+        R, static_cast<const __nv_bfloat16 *>(q), map, layer, 1);
     return cudaGetLastError();
 }
 

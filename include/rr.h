@@ -92,7 +92,9 @@ enum {
     RR_CNT_DRAW_CAP = 7,      /* rows whose random draws hit the draw cap and were filled in order */
     RR_CNT_FULL_PAIRS = 8,    /* score pairs of the rows fully routed at the last layer */
     RR_CNT_FULL_PAIRS_TOTAL = 9, /* the same, since rr_ledger_create */
-    RR_NUM_COUNTERS = 16      /* slots 10..15 are reserved (0) */
+    RR_CNT_RETRY_TOTAL = 10,  /* rows whose tensor-core selection took the one-pass exact
+                                 path (a failed three-pass certificate), since create */
+    RR_NUM_COUNTERS = 16      /* slots 11..15 are reserved (0) */
 };
 
 /* Bytes of device workspace a ledger with this config needs (0 if the
@@ -204,8 +206,9 @@ rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view);
  * workspace.  Layer 0 and forced-anchor layers (layer % anchor_interval ==
  * 0) are full routing as in rr_full_route; other layers are one relay layer
  * as in rr_relay_layer (rescore, compact, refresh).  The only scratch, the
- * per-head refresh lists and their lengths, lives in a fixed array inside
- * the library: about 4 MiB of device memory that every GPU loading
+ * per-head refresh lists and their lengths (and the per-head lists of rows
+ * whose tensor-core selection is redone), lives in a fixed array inside
+ * the library: about 8 MiB of device memory that every GPU loading
  * librr.so holds until the process exits.  Limits: bh * nq <= 1048576 and
  * bh <= 4096; larger problems return RR_ECAPACITY and enqueue nothing.
  * The first call on a device looks up that array's device address (set-up

@@ -226,3 +226,41 @@ def test_layer_order_is_enforced(rr):
     led.full_route(q, k, 0)   # an anchor starts a new sequence at any layer
     led.relay_layer(q, k, 1)
     assert int(led.read()["counters"][rr.CNT_LAST_LAYER]) == 1
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 64)])
+def test_equal_scores_pick_lowest_chunks(rr, dtype, d):
+    """All keys equal -> every score of a row ties: the route is the k lowest
+    valid chunks and the near-miss the next m (ties go to the smaller index).
+    On the tensor-core path this is the case the three-pass certificate
+    rejects, so it also exercises the exact one-pass retry."""
+    bh, n, k, m, r = 2, 300, 8, 6, 4
+    cfg = rr.Config(bh=bh, nq=n, nk=n, d=d, k=k, m_near=m, r_rand=r, dtype=dtype, causal=True)
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn((bh, n, d), generator=g)
+    kk = torch.randn((bh, 1, d), generator=g).expand(bh, n, d).contiguous()
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    led = rr.RouteLedger(cfg, DEV)
+    led.full_route(q.to(td).to(DEV), kk.to(td).to(DEV), 0)
+    out = led.read()
+    ids = out["ids"]
+    for i in (0, 3, 7, 13, 14, 50, 299):
+        nv = i + 1
+        nr = min(k, nv)
+        nm = min(m, nv - nr)
+        assert ids[0, i, :nr].tolist() == list(range(nr))
+        assert ids[0, i, k:k + nm].tolist() == list(range(nr, nr + nm))
+        rand = [x for x in ids[0, i, k + m:].tolist() if x >= 0]
+        assert len(rand) == min(r, nv - nr - nm) and all(nr + nm <= x < nv for x in rand)
+    if dtype == "bf16":
+        assert int(out["counters"][rr.CNT_RETRY_TOTAL]) > 0
+
+
+def test_retry_path_is_rare_on_the_full_size_workload(rr):
+    """On the bf16 workload the three-pass certificate should hold for nearly
+    every row (the retry path is a safety net, not the common case)."""
+    w = W.C5.with_(bh=16, layers=1)
+    led = rr.RouteLedger(config_of(w, rr), DEV)
+    _drive(rr, w, led, 1)
+    c = led.read()["counters"]
+    assert int(c[rr.CNT_RETRY_TOTAL]) <= 0.005 * w.bh * w.n, int(c[rr.CNT_RETRY_TOTAL])
