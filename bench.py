@@ -137,10 +137,45 @@ def make_inputs(w, device, seed):
     return qs, ks
 
 
+def profiled_traffic_per_row(kernel_file: str, summary_glob: str):
+    """DRAM bytes per routed row from a committed ncu summary, or None when
+    the kernel source changed since the counters were taken."""
+    import glob
+    import hashlib
+    src = os.path.join(ROOT, "cross_layer_route_b200", "csrc", kernel_file)
+    if not os.path.exists(src):
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    for path in glob.glob(os.path.join(ROOT, "profiles", summary_glob)):
+        vals = {}
+        for line in open(path):
+            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_row", "source_sha256"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+        if vals.get("source_sha256") == sha and "traffic_bytes_per_row" in vals:
+            return float(vals["traffic_bytes_per_row"])
+    return None
+
+
 def uses_tensor_cores(w) -> bool:
     """Which full-routing kernel the library runs for this workload (the
     rule of route_rows_prepare: bf16, d in {64, 128}, k + m <= 64, r <= 32)."""
     return w.dtype == "bf16" and w.d in (64, 128) and w.k + w.m <= 64 and w.r <= 32
+
+
+def shard_offset(rank: int, w) -> int:
+    """Global index of this rank's first BH unit: every rank routes its own
+    w.bh units (weak scaling) and keys its random draws by the global index."""
+    return rank * w.bh
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The slowest rank's value (step times are compared across ranks)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
 
 
 def full_pairs_per_layer(w) -> int:
@@ -156,7 +191,7 @@ def run_ours(args, w, rank, world, device):
     torch.cuda.set_device(device)
     cfg = rr.Config(bh=w.bh, nq=w.n, nk=w.n, d=w.d, k=w.k, m_near=w.m, r_rand=w.r, dtype=w.dtype,
                     anchor_interval=w.anchor_interval, causal=w.causal, gamma=w.gamma, seed=w.seed,
-                    bh_offset=rank * w.bh)
+                    bh_offset=shard_offset(rank, w))
     qs, ks = make_inputs(w, device, seed=w.seed * 1009 + rank)
     led = rr.RouteLedger(cfg, device)
     stream = torch.cuda.current_stream(device)
@@ -230,11 +265,7 @@ def run_ours(args, w, rank, world, device):
                 n_route += 1
                 n_rescore += 1
 
-    ms_step = ms_total / K
-    if world > 1:
-        t = torch.tensor([ms_step], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms_step = float(t.item())
+    ms_step = max_over_ranks(ms_total / K, world, device)
 
     rows_per_step = w.bh * w.n * L
     d_cnt = (c1 - c0).tolist()
@@ -258,8 +289,13 @@ def run_ours(args, w, rank, world, device):
         peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
         roofline = {"kernel": "route_rows (CUDA cores; anchor + refresh)", "bound": "alu",
                     "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock"}
+    traffic = None
+    if uses_tensor_cores(w):
+        per_row = profiled_traffic_per_row("rr_route_tc.cu", "route_rows_tc_kernel__*.md")
+        if per_row is not None and n_route:
+            traffic = round(per_row * refreshed_per_step * K / n_route)   # bytes per launch
     roofline.update({"achieved": round(route_tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(route_tflops / peak, 4), "traffic": None,
+                     "frac": round(route_tflops / peak, 4), "traffic": traffic,
                      "avg_launch_ms": round(route_ms / max(n_route, 1), 4),
                      "launches": n_route})
     # secondary: relay rescore (HBM-bound): per row q (d*e) + its head's keys
@@ -470,9 +506,7 @@ def main():
     if not args.no_e2e:
         e2e = measure_e2e(args, w, state, device)
         if world > 1:
-            t = torch.tensor([e2e["ms_per_step"]], device=device, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(t.item())
+            e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], world, device)
             e2e["value"] = w.bh * w.n * w.layers * world / (e2e["ms_per_step"] * 1e-3)
         result["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -318,17 +318,28 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Lay
     return true;
 }
 
-// TMA producer (one lane): `total` key tiles; tile g is key tile tile_of(g).
-// With three passes the middle pass runs backwards (its first tiles are the
-// ones still in L2 from the previous pass).
+// Tile schedule.  One pass: key tiles 0..nt-1.  Three passes: pass 0 over
+// the first min(nt, kPass0Tiles) tiles, pass 1 over all tiles backwards
+// (its first tiles are the ones still in L2), pass 2 over all tiles.
+// kPass0Tiles bounds the tiles pass 0 sees; a short pass 0 only estimates
+// the row maximum (larger scores fall in bin 0, which stays exact but
+// widens the bins), which measured no faster, so pass 0 covers every tile.
+constexpr int kPass0Tiles = 1 << 20;
+__device__ __forceinline__ int pass0_tiles(int ntiles) { return min(ntiles, kPass0Tiles); }
+__device__ __forceinline__ int total_tiles(int ntiles, int passes) {
+    return passes == 3 ? pass0_tiles(ntiles) + 2 * ntiles : ntiles;
+}
 __device__ __forceinline__ int tile_of(int g, int ntiles, int passes) {
-    const int p = g / ntiles, i = g - p * ntiles;
-    return (passes == 3 && p == 1) ? ntiles - 1 - i : i;
+    if (passes != 3) return g;
+    const int p0 = pass0_tiles(ntiles);
+    if (g < p0) return g;
+    if (g < p0 + ntiles) return ntiles - 1 - (g - p0);
+    return g - p0 - ntiles;
 }
 
 __device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int passes) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap_k)) : "memory");
-    const int total = passes * c.ntiles;
+    const int total = total_tiles(c.ntiles, passes);
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
     int issued = 0;
     for (int g = 0; g < total; ++g) {
@@ -352,7 +363,7 @@ __device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int pa
 
 // MMA issuer (one lane): score tile g into accumulator g % 2.
 __device__ void mma_issuer(Cta &c, int d, int passes) {
-    const int total = passes * c.ntiles;
+    const int total = total_tiles(c.ntiles, passes);
     const uint32_t q_addr = saddr(c.q_s), k_addr = saddr(c.k_s);
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
     for (int g = 0; g < total; ++g) {
@@ -571,10 +582,10 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 
 // ---- three-pass kernel (the main path) ------------------------------------------
 // Bin of a score for one row: bins of width (M - Lo) / kNB counted down from
-// M; scores under Lo land in the last bin.  The same expression is used in
+// M; scores above M land in bin 0, scores under Lo in the last bin.  The same expression is used in
 // every place a bin is computed, so counts and placements agree.
 __device__ __forceinline__ int bin_of(float v, float neg_inv, float hi_inv) {
-    return min((int)fmaf(v, neg_inv, hi_inv), kNB - 1);
+    return min((int)fmaxf(fmaf(v, neg_inv, hi_inv), 0.f), kNB - 1);
 }
 
 __global__ void __launch_bounds__(kPassThreads, 1)
@@ -619,15 +630,16 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 
         // pass 0: per row, the maximum of each of 64 disjoint column groups
         // (group = half, column mod 32) and the minimum of the first k+m valid
-        // scores.  M = the largest group maximum; the smallest group maximum
-        // and that minimum are both at most the (k+m)-th best score (each
-        // comes with k+m or more distinct scores at or above it), so the
-        // larger of the two is the histogram's lower end Lo.
+        // scores.  M = the largest group maximum (the row maximum); the
+        // smallest group maximum and that minimum are both at most the
+        // (k+m)-th best score (each comes with k+m or more distinct scores at
+        // or above it), so the larger of the two is the histogram's lower end.
         float gm[32];
 #pragma unroll
         for (int q = 0; q < 32; ++q) gm[q] = -INFINITY;
         float Lo = INFINITY;
-        for (int i = 0; i < nt && ok; ++i, ++g) {
+        const int p0 = pass0_tiles(nt);
+        for (int i = 0; i < p0 && ok; ++i, ++g) {
             if (!(ok = acc_wait(c, g))) break;
             float v[64];
             tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
@@ -780,8 +792,20 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 const int nsel = nr + nm;
                 const size_t grow = (size_t)h * L.nq + row;
                 int32_t *out = L.ids + grow * L.c;
-                for (int e = 0; e < L.k; ++e) out[e] = e < nr ? (int)bi[e * kRows] : -1;
-                for (int e = 0; e < L.m; ++e) out[L.k + e] = e < nm ? (int)bi[(nr + e) * kRows] : -1;
+                // route | near-miss: 16-byte stores where the layout allows
+                auto id_at = [&](int e) -> int {   // ledger slot e of route | near-miss
+                    if (e < L.k) return e < nr ? (int)bi[e * kRows] : -1;
+                    const int f = e - L.k;
+                    return f < nm ? (int)bi[(nr + f) * kRows] : -1;
+                };
+                if (((L.c | L.k | L.m) & 3) == 0) {
+                    int4 *o4 = reinterpret_cast<int4 *>(out);
+                    for (int e = 0; e < L.k + L.m; e += 4)
+                        o4[e >> 2] = make_int4(id_at(e), id_at(e + 1), id_at(e + 2), id_at(e + 3));
+                } else {
+                    for (int e = 0; e < L.k + L.m; ++e) out[e] = id_at(e);
+                }
+                const float alpha = bv[(nr - 1) * kRows];
                 // one bit per valid chunk (route, near-miss, accepted sentinels)
                 // in the query/key buffers, free now that every MMA is done
                 uint32_t *bits = reinterpret_cast<uint32_t *>(smem + lay.q) + r;
@@ -794,6 +818,8 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                         bits[(j >> 5) * kRows] |= 1u << (j & 31);
                     }
                 }
+                // accepted sentinels go to the slots after route | near-miss
+                uint16_t *acc_ids = bi + nsel * kRows;
                 int32_t *rout = out + L.k + L.m;
                 random_sentinels(
                     L, L.bh_offset + h, row, layer, n_valid, nsel,
@@ -803,8 +829,9 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                             if ((int)bi[e * kRows] == j) return true;
                         return false;
                     },
-                    [&](int e) -> int32_t & { return rout[e]; }, rout, use_bits ? bits : nullptr);
-                L.alpha[grow] = bv[(nr - 1) * kRows];
+                    [&](int e) -> uint16_t & { return acc_ids[e * kRows]; }, rout,
+                    use_bits ? bits : nullptr);
+                L.alpha[grow] = alpha;
                 L.anchor_layer[grow] = layer;
                 L.flags[grow] = 1;
             }
