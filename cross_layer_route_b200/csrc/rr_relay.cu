@@ -5,9 +5,9 @@
 //
 //  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
 //      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
-//      row"), one warp per query row, one lane per candidate; each lane
-//      gathers its candidate key row with 16-byte loads (all in flight at
-//      once for d = 64, 128) and sums into 8 independent partials.
+//      row"), one warp per query row.  For d in {64, 128, 256} four lanes
+//      share a candidate (each a quarter of the key row, 16-byte loads, its
+//      quarter of q in registers); other d use one lane per candidate.
 //  compact_flags: the prefix sum that compacts unstable row ids (§4.2), one
 //      CTA per head, writing an ascending per-head list and its length.
 //  finalize_layer: per-layer counters (§4.1: the refreshed-row fraction is
@@ -201,14 +201,123 @@ __global__ void finalize_layer_kernel(LedgerDev L, int layer, long long add_rows
 
 }  // namespace
 
+// Four lanes per candidate: lane quad g of the warp scores candidate
+// it*8 + g, each lane one quarter of the key row (R/4 bytes, R = d * elem
+// size, a multiple of 64), with its quarter of the query row in registers.
+// A load instruction of the warp touches 8 whole key rows -- 8 cache lines
+// instead of the 32 of one-lane-per-candidate.
+template <typename T, int D>
+__global__ void __launch_bounds__(kRescoreThreads)
+relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
+    constexpr int E = Vec16<T>::kElems;         // elements per 16-byte load
+    constexpr int kChunks = D / E / 4;          // 16-byte loads per lane
+    __shared__ unsigned long long pair_sum[kRescoreWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quad = lane >> 2, part = lane & 3;
+    const long long rows = (long long)L.bh * L.nq;
+    const long long grow = (long long)blockIdx.x * kRescoreWarps + warp;
+    unsigned long long pairs = 0;
+    if (grow < rows) {
+        const int h = (int)(grow / L.nq);
+        const int i = (int)(grow - (long long)h * L.nq);
+        const int n_valid = valid_keys(i, L.nk, L.causal);
+        // this lane's quarter of q, as fp32
+        float qv[kChunks * E];
+        {
+            const uint4 *q4 = reinterpret_cast<const uint4 *>(Q + grow * D) + part * kChunks;
+#pragma unroll
+            for (int c = 0; c < kChunks; ++c) {
+                const uint4 u = __ldg(q4 + c);
+                if constexpr (E == 8) {
+                    qv[c * 8 + 0] = __uint_as_float(u.x << 16); qv[c * 8 + 1] = __uint_as_float(u.x & 0xffff0000u);
+                    qv[c * 8 + 2] = __uint_as_float(u.y << 16); qv[c * 8 + 3] = __uint_as_float(u.y & 0xffff0000u);
+                    qv[c * 8 + 4] = __uint_as_float(u.z << 16); qv[c * 8 + 5] = __uint_as_float(u.z & 0xffff0000u);
+                    qv[c * 8 + 6] = __uint_as_float(u.w << 16); qv[c * 8 + 7] = __uint_as_float(u.w & 0xffff0000u);
+                } else {
+                    qv[c * 4 + 0] = __uint_as_float(u.x); qv[c * 4 + 1] = __uint_as_float(u.y);
+                    qv[c * 4 + 2] = __uint_as_float(u.z); qv[c * 4 + 3] = __uint_as_float(u.w);
+                }
+            }
+        }
+        const int32_t *idr = L.ids + grow * L.c;
+        const T *Kh = K + (size_t)h * L.nk * D;
+        float amin = INFINITY, bmax = -INFINITY;
+        bool bad = false;
+        int ncand = 0;
+#pragma unroll 2
+        for (int e0 = 0; e0 < L.c; e0 += 8) {
+            const int e = e0 + quad;
+            const int j = e < L.c ? idr[e] : -1;
+            const bool valid = j >= 0 && j < n_valid;
+            bad |= j >= n_valid || j < -1;
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            if (valid) {
+                const uint4 *k4 = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D) + part * kChunks;
+                uint4 kv[kChunks];
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) kv[c] = __ldg(k4 + c);
+#pragma unroll
+                for (int c = 0; c < kChunks; ++c) {
+                    const uint4 u = kv[c];
+                    if constexpr (E == 8) {
+                        acc[0] = fmaf(qv[c * 8 + 0], __uint_as_float(u.x << 16), acc[0]);
+                        acc[1] = fmaf(qv[c * 8 + 1], __uint_as_float(u.x & 0xffff0000u), acc[1]);
+                        acc[2] = fmaf(qv[c * 8 + 2], __uint_as_float(u.y << 16), acc[2]);
+                        acc[3] = fmaf(qv[c * 8 + 3], __uint_as_float(u.y & 0xffff0000u), acc[3]);
+                        acc[0] = fmaf(qv[c * 8 + 4], __uint_as_float(u.z << 16), acc[0]);
+                        acc[1] = fmaf(qv[c * 8 + 5], __uint_as_float(u.z & 0xffff0000u), acc[1]);
+                        acc[2] = fmaf(qv[c * 8 + 6], __uint_as_float(u.w << 16), acc[2]);
+                        acc[3] = fmaf(qv[c * 8 + 7], __uint_as_float(u.w & 0xffff0000u), acc[3]);
+                    } else {
+                        acc[0] = fmaf(qv[c * 4 + 0], __uint_as_float(u.x), acc[0]);
+                        acc[1] = fmaf(qv[c * 4 + 1], __uint_as_float(u.y), acc[1]);
+                        acc[2] = fmaf(qv[c * 4 + 2], __uint_as_float(u.z), acc[2]);
+                        acc[3] = fmaf(qv[c * 4 + 3], __uint_as_float(u.w), acc[3]);
+                    }
+                }
+            }
+            float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            sc += __shfl_xor_sync(kFull, sc, 1);
+            sc += __shfl_xor_sync(kFull, sc, 2);
+            if (valid && part == 0) {
+                if (e < L.k) amin = fminf(amin, sc);   // Eq. 6
+                else bmax = fmaxf(bmax, sc);           // Eq. 7
+                ++ncand;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
+            bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+            ncand += __shfl_xor_sync(kFull, ncand, o);
+        }
+        const bool any_bad = __any_sync(kFull, bad);
+        if (lane == 0) {
+            const bool refresh = !(amin > bmax + L.gamma);  // Eq. 8
+            L.flags[grow] = refresh ? 1 : 0;
+            if (!refresh) L.alpha[grow] = amin;
+            if (any_bad) atomicOr(&L.counters[2], 1ULL);
+        }
+        pairs = (unsigned long long)ncand;
+    }
+    if (lane == 0) pair_sum[warp] = pairs;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long s = 0;
+        for (int w = 0; w < kRescoreWarps; ++w) s += pair_sum[w];
+        if (s) atomicAdd(&L.counters[1], s);
+    }
+}
+
 template <typename T>
 static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, unsigned grid,
                              cudaStream_t s) {
     const T *Q = static_cast<const T *>(q);
     const T *K = static_cast<const T *>(k);
     switch (L.d) {
-        case 64: relay_rescore_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        case 128: relay_rescore_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 64: relay_rescore_quad_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 128: relay_rescore_quad_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 256: relay_rescore_quad_kernel<T, 256><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
         default: relay_rescore_kernel<T, 0><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
     }
 }
