@@ -34,15 +34,15 @@
 //   pass 1  per row: a histogram of (M - s) over 128 equal bins of [Lo, M]
 //           (scores under Lo fall in the last bin); the first bin b* at
 //           which the running count reaches k+m holds the (k+m)-th best;
-//   pass 2  per row: the histogram's counts of bins 0..b* become start
-//           offsets, and every score of those bins is written to its bin's
-//           next slot (a counting sort; about k+m plus one bin's crowd).
-// An insertion sort then fixes the order inside each bin (exact best-first
-// order), and the first k+m are the route and near-miss ids.  A row whose
-// bins 0..b* hold more than kCap scores (or whose bins did not fill exactly
-// -- a certificate check) is appended to a retry list and routed by
-// route_rows_tc_heap_kernel, which keeps a per-row min-heap of the k+m best
-// over one pass; results are exact either way.
+//   pass 2  per row: every score of bins 0..b* is appended to the row's
+//           buffer (about k+m plus one bin's crowd).
+// The kept scores are then placed by bin (a counting sort on the histogram's
+// start offsets), each inserted in order among its bin's earlier arrivals
+// (exact best-first order); the first k+m are the route and near-miss ids.  A row whose bins 0..b* hold more than kCap-2 scores (or
+// whose appended count differs from the histogram's -- a certificate check)
+// is appended to a retry list and routed by route_rows_tc_heap_kernel, which
+// keeps a per-row min-heap of the k+m best over one pass; results are exact
+// either way.
 //
 // Every wait is bounded; a timeout sets bit 1 of the error word and the CTA
 // drains its copies, frees its TMEM and returns.
@@ -643,6 +643,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             if (!(ok = acc_wait(c, g))) break;
             float v[64];
             tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            acc_release(c, g);   // the scores are in registers: the MMA may reuse the accumulator
             const int col0 = i * kKeys + half * 64;
             if (col0 + 64 <= n_valid) {
 #pragma unroll
@@ -657,7 +658,6 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 for (int jj = 0; jj < 64; ++jj)
                     if (col0 + jj < first_lim) Lo = fminf(Lo, v[jj]);
             }
-            acc_release(c, g);
         }
         {
             float *gx = reinterpret_cast<float *>(smem + lay.bufv) + r;   // [64][kRows]
@@ -688,6 +688,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             const int t = nt - 1 - i;
             float v[64];
             tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);   // every lane loads (.sync.aligned)
+            acc_release(c, g);
             const int col0 = t * kKeys + half * 64;
             if (!all_mode) {
                 if (col0 + 64 <= n_valid) {
@@ -701,7 +702,6 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                             atomicAdd(&hist[bin_of(v[jj], neg_inv, hi_inv) * kRows], 1u);
                 }
             }
-            acc_release(c, g);
         }
         epi_sync();
 
@@ -719,122 +719,138 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             }
             run = cum;
         }
-        const bool overflow = run > (uint32_t)kCap;
-        // half 0 turns the counts of bins 0..b* into exclusive start offsets
-        if (half == 0) {
-            if (all_mode) {
-                hist[0] = 0u;
-            } else {
+        const bool overflow = run > (uint32_t)(kCap - 2);
+        // pass 2: append every score of bins 0..b* (same bin arithmetic as
+        // pass 1) to the row's buffer, half 0 upward from slot 0 and half 1
+        // downward from slot kCap-1.  Branch-free: each value is stored at
+        // the half's next free slot and the slot advances only if the value
+        // is kept, so values not kept are overwritten; the two halves never
+        // share a slot while their counts sum to at most kCap-2.
+        int cnt = 0;
+        {
+            const int base = half ? kCap - 1 : 0;
+            const int dir = half ? -1 : 1;
+            for (int i = 0; i < nt && ok; ++i, ++g) {
+                if (!(ok = acc_wait(c, g))) break;
+                float v[64];
+                tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+                acc_release(c, g);
+                const int col0 = i * kKeys + half * 64;
+                const int lim = overflow ? 0 : n_valid - col0;   // columns jj < lim take part
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj) {
+                    const int b = all_mode ? 0 : bin_of(v[jj], neg_inv, hi_inv);
+                    const int slot = base + dir * min(cnt, kCap - 1);
+                    bv[slot * kRows] = v[jj];
+                    bi[slot * kRows] = (uint16_t)(col0 + jj);
+                    cnt += (jj < lim && b <= bstar) ? 1 : 0;
+                }
+            }
+        }
+        int *rcnt = reinterpret_cast<int *>(smem + lay.red) + 4 * kRows;   // [2][kRows]
+        rcnt[half * kRows + r] = cnt;
+        epi_sync();
+
+        // Place the kept scores by bin in the query/key buffers, free now
+        // that every MMA is done, each one inserted in order among the scores
+        // of its bin placed before it (best first: score desc, chunk asc).
+        // Bins hold a handful of scores, so the insertion moves few.  The two
+        // halves share the rows: half 0 finishes lanes 0..15, half 1 lanes
+        // 16..31.
+        float *sv = reinterpret_cast<float *>(smem + lay.q) + r;
+        uint16_t *si = reinterpret_cast<uint16_t *>(smem + lay.q + kCap * kRows * 4) + r;
+        const bool mine = ok && row >= 0 && (lane >> 4) == half;
+        bool fail = false;
+        if (mine) {
+            const int c0 = rcnt[r], c1 = rcnt[kRows + r];
+            fail = overflow || c0 + c1 != (int)run;
+            if (!fail) {
+                // per bin: start offset (low half) and next free slot (high
+                // half); both halves read the counts before pass 2, so this
+                // thread owns the row's histogram now
                 uint32_t acc = 0;
                 for (int b = 0; b <= bstar; ++b) {
                     const uint32_t x = hist[b * kRows];
-                    hist[b * kRows] = acc;
+                    hist[b * kRows] = acc | (acc << 16);
                     acc += x;
                 }
-            }
-        }
-        epi_sync();
-
-        // pass 2: every score of bins 0..b* goes straight to its bin's next
-        // slot (same bin arithmetic as pass 1, so exactly `run` scores land)
-        for (int i = 0; i < nt && ok; ++i, ++g) {
-            if (!(ok = acc_wait(c, g))) break;
-            float v[64];
-            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
-            const int col0 = i * kKeys + half * 64;
-            const int lim = overflow ? 0 : n_valid - col0;   // columns jj < lim take part
-#pragma unroll
-            for (int jj = 0; jj < 64; ++jj) {
-                const int b = all_mode ? 0 : bin_of(v[jj], neg_inv, hi_inv);
-                if (jj < lim && b <= bstar) {
-                    const uint32_t pos = atomicAdd(&hist[b * kRows], 1u);
-                    if (pos < (uint32_t)kCap) {
-                        bv[pos * kRows] = v[jj];
-                        bi[pos * kRows] = (uint16_t)(col0 + jj);
+                for (int e = 0; e < c0 + c1; ++e) {
+                    const int slot = e < c0 ? e : kCap - 1 - (e - c0);
+                    const float v = bv[slot * kRows];
+                    const uint16_t j = bi[slot * kRows];
+                    const int b = all_mode ? 0 : bin_of(v, neg_inv, hi_inv);
+                    const uint32_t x = hist[b * kRows];
+                    hist[b * kRows] = x + (1u << 16);
+                    const int lo = (int)(x & 0xffffu);
+                    int p = (int)(x >> 16);
+                    for (; p > lo; --p) {
+                        const float pv = sv[(p - 1) * kRows];
+                        const uint16_t pj = si[(p - 1) * kRows];
+                        if (!(v > pv || (v == pv && j < pj))) break;
+                        sv[p * kRows] = pv;
+                        si[p * kRows] = pj;
                     }
+                    sv[p * kRows] = v;
+                    si[p * kRows] = j;
                 }
-            }
-            acc_release(c, g);
-        }
-        epi_sync();
-
-        // Each row's kept scores now sit in bins order.  The two halves share
-        // the rows: half 0 finishes lanes 0..15, half 1 lanes 16..31.
-        const bool mine = ok && row >= 0 && (lane >> 4) == half;
-        if (mine) {
-            // every bin must have been filled exactly (b*'s next slot == run)
-            const bool fail = overflow || hist[bstar * kRows] != run;
-            if (fail) {
+            } else {
                 const int pos = atomicAdd(&L.retry_count[h], 1);
                 L.retry_list[(size_t)h * L.nq + pos] = row;
                 atomicAdd(&L.counters[10], 1ULL);
-            } else {
-                // insertion sort, best first (score desc, chunk asc): only
-                // within-bin disorder is left
-                const int nsorted = (int)run;
-                for (int e = 1; e < nsorted; ++e) {
-                    const float v = bv[e * kRows];
-                    const uint16_t j = bi[e * kRows];
-                    int p = e - 1;
-                    while (p >= 0) {
-                        const float pv = bv[p * kRows];
-                        const uint16_t pj = bi[p * kRows];
-                        if (!(v > pv || (v == pv && j < pj))) break;
-                        bv[(p + 1) * kRows] = pv;
-                        bi[(p + 1) * kRows] = pj;
-                        --p;
-                    }
-                    bv[(p + 1) * kRows] = v;
-                    bi[(p + 1) * kRows] = j;
-                }
-                const int nr = min(L.k, n_valid);
-                const int nm = min(L.m, n_valid - nr);
-                const int nsel = nr + nm;
-                const size_t grow = (size_t)h * L.nq + row;
-                int32_t *out = L.ids + grow * L.c;
-                // route | near-miss: 16-byte stores where the layout allows
-                auto id_at = [&](int e) -> int {   // ledger slot e of route | near-miss
-                    if (e < L.k) return e < nr ? (int)bi[e * kRows] : -1;
-                    const int f = e - L.k;
-                    return f < nm ? (int)bi[(nr + f) * kRows] : -1;
-                };
-                if (((L.c | L.k | L.m) & 3) == 0) {
-                    int4 *o4 = reinterpret_cast<int4 *>(out);
-                    for (int e = 0; e < L.k + L.m; e += 4)
-                        o4[e >> 2] = make_int4(id_at(e), id_at(e + 1), id_at(e + 2), id_at(e + 3));
-                } else {
-                    for (int e = 0; e < L.k + L.m; ++e) out[e] = id_at(e);
-                }
-                const float alpha = bv[(nr - 1) * kRows];
-                // one bit per valid chunk (route, near-miss, accepted sentinels)
-                // in the query/key buffers, free now that every MMA is done
-                uint32_t *bits = reinterpret_cast<uint32_t *>(smem + lay.q) + r;
-                const int words = (n_valid + 31) >> 5;
-                const bool use_bits = words <= (int)(lay.sel / (kRows * 4));
-                if (use_bits) {
-                    for (int w = 0; w < words; ++w) bits[w * kRows] = 0u;
-                    for (int e = 0; e < nsel; ++e) {
-                        const int j = bi[e * kRows];
-                        bits[(j >> 5) * kRows] |= 1u << (j & 31);
-                    }
-                }
-                // accepted sentinels go to the slots after route | near-miss
-                uint16_t *acc_ids = bi + nsel * kRows;
-                int32_t *rout = out + L.k + L.m;
-                random_sentinels(
-                    L, L.bh_offset + h, row, layer, n_valid, nsel,
-                    [&](int j) {
-                        if (use_bits) return ((bits[(j >> 5) * kRows] >> (j & 31)) & 1u) != 0u;
-                        for (int e = 0; e < nsel; ++e)
-                            if ((int)bi[e * kRows] == j) return true;
-                        return false;
-                    },
-                    [&](int e) -> uint16_t & { return acc_ids[e * kRows]; }, rout,
-                    use_bits ? bits : nullptr);
-                L.alpha[grow] = alpha;
-                L.anchor_layer[grow] = layer;
-                L.flags[grow] = 1;
             }
+        }
+        // every row is placed: the append buffers become membership bitmaps
+        // (a row's bitmap words past the value buffer overlap other rows'
+        // index slots, so this barrier is needed)
+        epi_sync();
+
+        if (mine && !fail) {
+            const int nr = min(L.k, n_valid);
+            const int nm = min(L.m, n_valid - nr);
+            const int nsel = nr + nm;
+            const size_t grow = (size_t)h * L.nq + row;
+            int32_t *out = L.ids + grow * L.c;
+            // route | near-miss: 16-byte stores where the layout allows
+            auto id_at = [&](int e) -> int {   // ledger slot e of route | near-miss
+                if (e < L.k) return e < nr ? (int)si[e * kRows] : -1;
+                const int f = e - L.k;
+                return f < nm ? (int)si[(nr + f) * kRows] : -1;
+            };
+            if (((L.c | L.k | L.m) & 3) == 0) {
+                int4 *o4 = reinterpret_cast<int4 *>(out);
+                for (int e = 0; e < L.k + L.m; e += 4)
+                    o4[e >> 2] = make_int4(id_at(e), id_at(e + 1), id_at(e + 2), id_at(e + 3));
+            } else {
+                for (int e = 0; e < L.k + L.m; ++e) out[e] = id_at(e);
+            }
+            const float alpha = sv[(nr - 1) * kRows];
+            // one bit per valid chunk (route, near-miss, accepted sentinels)
+            uint32_t *bits = reinterpret_cast<uint32_t *>(smem + lay.bufv) + r;
+            const int words = (n_valid + 31) >> 5;
+            const bool use_bits = words <= (int)(kCap * 6 / 4);   // 144 words fit the buffers
+            if (use_bits) {
+                for (int w = 0; w < words; ++w) bits[w * kRows] = 0u;
+                for (int e = 0; e < nsel; ++e) {
+                    const int j = si[e * kRows];
+                    bits[(j >> 5) * kRows] |= 1u << (j & 31);
+                }
+            }
+            // accepted sentinels are kept in the sorted area past route | near-miss
+            uint16_t *acc_ids = si + nsel * kRows;
+            int32_t *rout = out + L.k + L.m;
+            random_sentinels(
+                L, L.bh_offset + h, row, layer, n_valid, nsel,
+                [&](int jx) {
+                    if (use_bits) return ((bits[(jx >> 5) * kRows] >> (jx & 31)) & 1u) != 0u;
+                    for (int e = 0; e < nsel; ++e)
+                        if ((int)si[e * kRows] == jx) return true;
+                    return false;
+                },
+                [&](int e) -> uint16_t & { return acc_ids[e * kRows]; }, rout,
+                use_bits ? bits : nullptr);
+            L.alpha[grow] = alpha;
+            L.anchor_layer[grow] = layer;
+            L.flags[grow] = 1;
         }
     }
     cta_teardown(c, L);
@@ -863,8 +879,15 @@ EncodeTiledFn encode_fn() {
 }  // namespace tc
 
 bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
-    return dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf &&
-           L.nk <= 65535;
+    if (!(dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf &&
+          L.nk <= 65535))
+        return false;
+    // the selection kernel's sorted scores (f32 + u16 per slot) reuse the
+    // operand buffers, and its per-row bitmaps the append buffers
+    const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
+    return lay.sel - lay.q >= (uint32_t)(tc::kCap * tc::kRows * 6) &&
+           lay.bufi + tc::kCap * tc::kRows * 2 - lay.bufv >= (uint32_t)(144 * tc::kRows * 4) &&
+           L.ksel + L.r <= tc::kCap;
 }
 
 size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
