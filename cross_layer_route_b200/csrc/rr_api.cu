@@ -35,7 +35,10 @@ constexpr size_t kAlign = 256;
 size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
-    size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count, total;
+    size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count;
+    size_t cand_v, cand_i, cand_meta;   // split tensor-core path only (size 0 otherwise)
+    bool cand;
+    size_t total;
 };
 
 bool config_ok(const rr_config *c) {
@@ -66,6 +69,14 @@ Layout layout_of(const rr_config *c) {
     L.head_count = o;   o = align_up(o + (size_t)c->bh * sizeof(int32_t));
     L.retry_list = o;   o = align_up(o + rows * sizeof(int32_t));
     L.retry_count = o;  o = align_up(o + (size_t)c->bh * sizeof(int32_t));
+    rr::LedgerDev t;
+    t.bh = c->bh; t.nq = c->nq; t.nk = c->nk; t.d = c->d;
+    t.k = c->k; t.m = c->m_near; t.r = c->r_rand; t.ksel = c->k + c->m_near;
+    const rr::CandSizes cs = rr::route_rows_tc_candidate_sizes(t, c->dtype);
+    L.cand = cs.v > 0;
+    L.cand_v = o;       o = align_up(o + cs.v);
+    L.cand_i = o;       o = align_up(o + cs.i);
+    L.cand_meta = o;    o = align_up(o + cs.meta);
     L.total = o;
     return L;
 }
@@ -204,6 +215,11 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     D.head_count = reinterpret_cast<int32_t *>(L->ws + lay.head_count);
     D.retry_list = reinterpret_cast<int32_t *>(L->ws + lay.retry_list);
     D.retry_count = reinterpret_cast<int32_t *>(L->ws + lay.retry_count);
+    if (lay.cand) {
+        D.cand_v = reinterpret_cast<float *>(L->ws + lay.cand_v);
+        D.cand_i = reinterpret_cast<uint16_t *>(L->ws + lay.cand_i);
+        D.cand_meta = reinterpret_cast<int32_t *>(L->ws + lay.cand_meta);
+    }
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
     D.c = cfg->k + cfg->m_near + cfg->r_rand;

@@ -20,6 +20,11 @@ struct LedgerDev {
     int32_t *head_count;    // [bh]        flagged rows per head
     int32_t *retry_list;    // [bh*nq]     per-head rows whose tensor-core selection is redone
     int32_t *retry_count;   // [bh]        rows listed per head
+    // candidate buffers of the split tensor-core path (null: the route kernel
+    // finishes its rows itself); per 128-row block of one head:
+    float *cand_v = nullptr;       // [blocks, kCap, 128] kept scores
+    uint16_t *cand_i = nullptr;    // [blocks, kCap, 128] their key chunks
+    int32_t *cand_meta = nullptr;  // [blocks, 128] kept counts of the two halves, or -1
     int bh, nq, nk, d;
     int k, m, r, c, ksel;   // ksel = k + m
     int causal;
@@ -46,6 +51,10 @@ inline int select_capacity(int ksel) {
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype);
 bool route_rows_tc_supported(const LedgerDev &L, int dtype);
 size_t route_rows_tc_smem_bytes(const LedgerDev &L);
+// Bytes of the candidate buffers the split tensor-core path needs (all 0 when
+// the problem does not run on the tensor cores).
+struct CandSizes { size_t v, i, meta; };
+CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype);
 cudaError_t route_rows_tc_prepare(size_t smem_bytes);
 cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                  bool use_list, cudaStream_t s);

@@ -588,6 +588,12 @@ __device__ __forceinline__ int bin_of(float v, float neg_inv, float hi_inv) {
     return min((int)fmaxf(fmaf(v, neg_inv, hi_inv), 0.f), kNB - 1);
 }
 
+// kSplit: the kernel ends after pass 2 by writing each row's kept scores
+// (both column halves' buffers, as they are) and their counts to the
+// candidate buffers; route_rows_finalize_kernel orders them and writes the
+// ledger rows.  Otherwise the CTA finishes its rows itself (no candidate
+// buffers needed).
+template <bool kSplit>
 __global__ void __launch_bounds__(kPassThreads, 1)
 route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                      const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
@@ -751,6 +757,34 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         rcnt[half * kRows + r] = cnt;
         epi_sync();
 
+        if constexpr (kSplit) {
+            // candidate slot (blk, slot, r) at cand[(blk * kCap + slot) * kRows + r];
+            // meta (blk, r) = c0 | c1 << 16, or -1 when the row has nothing to finish
+            const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+            const int c0 = rcnt[r], c1 = rcnt[kRows + r];
+            const bool good = ok && row >= 0 && !overflow && c0 + c1 == (int)run;
+            if (half == 0) {
+                L.cand_meta[blk * kRows + r] = good ? (c0 | (c1 << 16)) : -1;
+                if (ok && row >= 0 && !good) {
+                    const int pos = atomicAdd(&L.retry_count[h], 1);
+                    L.retry_list[(size_t)h * L.nq + pos] = row;
+                    atomicAdd(&L.counters[10], 1ULL);
+                }
+            }
+            if (good) {
+                // half 0 writes slots 0..kCap/2-1, half 1 the rest (only used ones)
+                float *gv = L.cand_v + blk * kCap * kRows + r;
+                uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
+                const int s0 = half * (kCap / 2);
+                for (int sl = s0; sl < s0 + kCap / 2; ++sl) {
+                    if (sl < c0 || sl >= kCap - c1) {
+                        gv[sl * kRows] = bv[sl * kRows];
+                        gi[sl * kRows] = bi[sl * kRows];
+                    }
+                }
+            }
+        } else {
+
         // Place the kept scores by bin in the query/key buffers, free now
         // that every MMA is done, each one inserted in order among the scores
         // of its bin placed before it (best first: score desc, chunk asc).
@@ -852,8 +886,221 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             L.anchor_layer[grow] = layer;
             L.flags[grow] = 1;
         }
+        }   // fused tail
     }
     cta_teardown(c, L);
+}
+
+// ---- finalize kernel (split path): one warp per row ---------------------------
+// Reads a row's kept scores (at most kCap - 2, written by
+// route_rows_tc_kernel<true>) and writes its ledger row: route | near-miss in
+// best-first order (score desc, chunk asc), alpha (the k-th score) and the
+// random sentinels (RouteRelay §3.1 items 1-2).
+//
+// Order: the row's kept scores are binned over their own range (128 bins,
+// larger score = lower bin, ties share a bin), placed by bin, and each one's
+// final position is its bin's start plus the number of better keys in its
+// bin.  Sentinels: 32 draws at a time, one per lane (the same Philox words,
+// rejection rule and ascending completion as random_sentinels above); a draw
+// is accepted if its chunk is not selected, not accepted earlier and not
+// drawn by an earlier lane of the round (warp match), in draw order.
+constexpr int kFinWarps = 8;
+constexpr int kFinBins = 128;
+constexpr int kFinBitsWords = 128;   // membership bitmap: rows with <= 4096 valid keys
+
+struct FinWarp {
+    uint64_t keys[kCap];             // kept scores placed by bin
+    uint32_t hist[kFinBins];         // counts, then start offsets
+    uint32_t bits[kFinBitsWords];    // selected and accepted chunks
+    int32_t acc[32];                 // accepted sentinels, in order
+};
+
+// Larger key = better: score desc, then chunk asc (-0 counts as +0).
+__device__ __forceinline__ uint64_t cand_key(float v, int j) {
+    const float z = v == 0.0f ? 0.0f : v;
+    return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
+}
+
+__global__ void __launch_bounds__(32 * kFinWarps)
+route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
+    __shared__ FinWarp fw_all[kFinWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    FinWarp &w = fw_all[warp];
+    const int h = blockIdx.y;
+    constexpr int kPerBlk = kRows / kFinWarps;   // finalize CTAs per route CTA
+    const int bx = blockIdx.x / kPerBlk;
+    const int r = (blockIdx.x % kPerBlk) * kFinWarps + warp;
+    const int count = use_list ? L.head_count[h] : L.nq;
+    const int row0 = bx * kRows;
+    if (row0 + r >= count) return;
+    const size_t blk = (size_t)h * ((L.nq + kRows - 1) / kRows) + bx;
+    const int meta = L.cand_meta[blk * kRows + r];
+    if (meta < 0) return;   // no row, or a row left to the retry path
+    const int row = use_list ? L.list[(size_t)h * L.nq + row0 + r] : row0 + r;
+    const int c0 = meta & 0xffff, c1 = meta >> 16, run = c0 + c1;
+    const int n_valid = valid_keys(row, L.nk, L.causal);
+    const uint32_t lt_mask = (1u << lane) - 1u;
+
+    // the row's kept scores, three per lane
+    const float *gv = L.cand_v + blk * kCap * kRows + r;
+    const uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
+    float v[3];
+    int jc[3];
+    bool live[3];
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        const int e = lane + 32 * i;
+        live[i] = e < run;
+        v[i] = 0.f;
+        jc[i] = -1;
+        if (live[i]) {
+            const int sl = e < c0 ? e : kCap - 1 - (e - c0);
+            v[i] = gv[sl * kRows];
+            jc[i] = gi[sl * kRows];
+            mx = fmaxf(mx, v[i]);
+            mn = fminf(mn, v[i]);
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+    }
+    const float inv = mx > mn ? (float)kFinBins / (mx - mn) : 0.f;
+    const float neg_inv = -inv, hi_inv = mx * inv;
+
+    // counting sort by bin
+#pragma unroll
+    for (int q = 0; q < kFinBins / 32; ++q) w.hist[lane + 32 * q] = 0u;
+    __syncwarp();
+    int bin[3];
+    uint32_t in_bin[3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        bin[i] = min((int)fmaxf(fmaf(v[i], neg_inv, hi_inv), 0.f), kFinBins - 1);
+        in_bin[i] = live[i] ? atomicAdd(&w.hist[bin[i]], 1u) : 0u;
+    }
+    __syncwarp();
+    {
+        uint32_t hc[kFinBins / 32], tot = 0;
+#pragma unroll
+        for (int q = 0; q < kFinBins / 32; ++q) { hc[q] = w.hist[lane * (kFinBins / 32) + q]; tot += hc[q]; }
+        uint32_t incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += x;
+        }
+        uint32_t run_start = incl - tot;
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < kFinBins / 32; ++q) {
+            w.hist[lane * (kFinBins / 32) + q] = run_start;
+            run_start += hc[q];
+        }
+    }
+    __syncwarp();
+    uint64_t key[3];
+    int start[3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        key[i] = cand_key(v[i], jc[i] < 0 ? 0 : jc[i]);
+        start[i] = (int)w.hist[bin[i]];
+        if (live[i]) w.keys[start[i] + (int)in_bin[i]] = key[i];
+    }
+    __syncwarp();
+    const int nr = min(L.k, n_valid);
+    const int nm = min(L.m, n_valid - nr);
+    const int nsel = nr + nm;
+    const size_t grow = (size_t)h * L.nq + row;
+    int32_t *out = L.ids + grow * L.c;
+    bool sel[3];
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+        sel[i] = false;
+        if (!live[i]) continue;
+        const int end = bin[i] + 1 < kFinBins ? (int)w.hist[bin[i] + 1] : run;
+        int rank = 0;
+        for (int p = start[i]; p < end; ++p) rank += w.keys[p] > key[i] ? 1 : 0;
+        const int pos = start[i] + rank;
+        if (pos < nsel) {
+            sel[i] = true;
+            out[pos < nr ? pos : L.k + (pos - nr)] = jc[i];
+            if (pos == nr - 1) L.alpha[grow] = v[i];
+        }
+    }
+    for (int sl = lane; sl < L.k + L.m; sl += 32) {   // padding of short rows
+        if (sl < L.k ? sl >= nr : sl - L.k >= nm) out[sl] = -1;
+    }
+
+    // random sentinels
+    const bool use_bits = n_valid <= 32 * kFinBitsWords;
+    if (use_bits) {
+        const int words = (n_valid + 31) >> 5;
+        for (int q = lane; q < words; q += 32) w.bits[q] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 3; ++i)
+            if (sel[i]) atomicOr(&w.bits[jc[i] >> 5], 1u << (jc[i] & 31));
+        __syncwarp();
+    }
+    int acc = 0;
+    // chunk j selected or accepted (this lane's j; accepted ones in w.acc[0..acc))
+    auto taken = [&](int j) -> bool {
+        if (use_bits) return ((w.bits[j >> 5] >> (j & 31)) & 1u) != 0u;
+        bool hit = false;
+        for (int src = 0; src < 32; ++src) {
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                const int cj = __shfl_sync(kFull, sel[i] ? jc[i] : -1, src);
+                hit |= cj == j;
+            }
+        }
+        for (int a = 0; a < acc; ++a) hit |= w.acc[a] == j;
+        return hit;
+    };
+    // accept this round's free lanes in lane order, up to r in total
+    auto accept = [&](bool is_free, int j) {
+        const uint32_t fm = __ballot_sync(kFull, is_free);
+        const int idx = acc + __popc(fm & lt_mask);
+        if (is_free && idx < L.r) {
+            w.acc[idx] = j;
+            if (use_bits) atomicOr(&w.bits[j >> 5], 1u << (j & 31));
+        }
+        acc = min(L.r, acc + __popc(fm));
+        __syncwarp();
+    };
+    if (L.r > 0) {
+        if (n_valid - nsel > L.r) {
+            for (int t0 = 0; acc < L.r && t0 < L.max_draws; t0 += 32) {
+                const int t = t0 + lane;
+                const PhiloxOut o = philox4x32_10((uint32_t)(L.bh_offset + h), (uint32_t)row,
+                                                  (uint32_t)layer, (uint32_t)(t >> 2), L.seed_lo,
+                                                  L.seed_hi);
+                const int q = t & 3;
+                const uint32_t word = q == 0 ? o.w[0] : q == 1 ? o.w[1] : q == 2 ? o.w[2] : o.w[3];
+                const int j = (int)__umulhi(word, (uint32_t)n_valid);
+                const bool tk = taken(j);   // every lane calls it (it may shuffle)
+                const bool ok_t = t < L.max_draws && !tk;
+                // first draw of its chunk among this round's free draws
+                const uint32_t same = __match_any_sync(kFull, j) & __ballot_sync(kFull, ok_t);
+                accept(ok_t && (same & lt_mask) == 0u, j);
+            }
+            if (acc < L.r && lane == 0) atomicAdd(&L.counters[7], 1ULL);
+        }
+        for (int j0 = 0; acc < L.r && j0 < n_valid; j0 += 32) {
+            const int j = j0 + lane;
+            const bool tk = taken(min(j, n_valid - 1));
+            accept(j < n_valid && !tk, j);
+        }
+    }
+    __syncwarp();
+    if (lane < L.r) out[L.k + L.m + lane] = lane < acc ? w.acc[lane] : -1;
+    if (lane == 0) {
+        L.anchor_layer[grow] = layer;
+        L.flags[grow] = 1;
+    }
 }
 
 // ---- host side -----------------------------------------------------------------
@@ -896,13 +1143,26 @@ size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
     return a > b ? a : b;
 }
 
+CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype) {
+    CandSizes z{0, 0, 0};
+    if (!route_rows_tc_supported(L, dtype)) return z;
+    const size_t blocks = (size_t)L.bh * ((L.nq + tc::kRows - 1) / tc::kRows);
+    z.v = blocks * tc::kCap * tc::kRows * sizeof(float);
+    z.i = blocks * tc::kCap * tc::kRows * sizeof(uint16_t);
+    z.meta = blocks * tc::kRows * sizeof(int32_t);
+    return z;
+}
+
 cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
     if (smem_bytes > 232448) return cudaErrorInvalidValue;   // 227 KB per block on sm_100
-    // both kernels may be launched with up to their largest layout
+    // the kernels may be launched with up to their largest layout
     const int big = (int)tc::layout_of(128, 64, true).total;
     const int big_heap = (int)tc::layout_of(128, 64, false).total;
-    cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel,
+    cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<true>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc::route_rows_tc_heap_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big_heap);
@@ -926,8 +1186,18 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     const size_t smem3 = tc::layout_of(L.d, L.ksel, true).total;
-    tc::route_rows_tc_kernel<<<grid, tc::kPassThreads, smem3, s>>>(
-        L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
+    if (L.cand_v && L.cand_i && L.cand_meta) {
+        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem3, s>>>(
+            L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        dim3 fgrid(grid.x * (tc::kRows / tc::kFinWarps), L.bh);
+        tc::route_rows_finalize_kernel<<<fgrid, 32 * tc::kFinWarps, 0, s>>>(L, layer,
+                                                                             use_list ? 1 : 0);
+    } else {
+        tc::route_rows_tc_kernel<false><<<grid, tc::kPassThreads, smem3, s>>>(
+            L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     // rows whose three-pass certificate failed: exact heap selection

@@ -56,6 +56,8 @@ ANCHOR_SHAPES = [
     ("tc_small_n", 3, 70, 128, "bf16", 32, 32, 16, True),
     ("tc_exact_tile", 2, 256, 64, "bf16", 40, 24, 32, False),
     ("tc_k1_r0", 2, 129, 128, "bf16", 1, 0, 0, True),
+    # rows longer than the finalize kernel's 4096-chunk membership bitmap
+    ("tc_wide_rows", 1, 4700, 64, "bf16", 12, 12, 8, False),
 ]
 
 
