@@ -6,8 +6,9 @@
 //  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
 //      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
 //      row"), one warp per query row.  For d in {64, 128, 256} four lanes
-//      share a candidate (each a quarter of the key row, 16-byte loads, its
-//      quarter of q in registers); other d use one lane per candidate.
+//      share a candidate (16-byte loads interleaved so that the four read 64
+//      contiguous bytes at a time; each keeps its quarter of q in registers);
+//      other d use one lane per candidate.
 //  compact_flags: the prefix sum that compacts unstable row ids (§4.2), one
 //      CTA per head, writing an ascending per-head list and its length.
 //  finalize_layer: per-layer counters (§4.1: the refreshed-row fraction is
@@ -221,13 +222,14 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
         const int h = (int)(grow / L.nq);
         const int i = (int)(grow - (long long)h * L.nq);
         const int n_valid = valid_keys(i, L.nk, L.causal);
-        // this lane's quarter of q, as fp32
+        // this lane's quarter of q, as fp32: the 16-byte chunks part, part + 4,
+        // part + 8, ... (a quad reads 64 contiguous bytes per load)
         float qv[kChunks * E];
         {
-            const uint4 *q4 = reinterpret_cast<const uint4 *>(Q + grow * D) + part * kChunks;
+            const uint4 *q4 = reinterpret_cast<const uint4 *>(Q + grow * D) + part;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
-                const uint4 u = __ldg(q4 + c);
+                const uint4 u = __ldg(q4 + 4 * c);
                 if constexpr (E == 8) {
                     qv[c * 8 + 0] = __uint_as_float(u.x << 16); qv[c * 8 + 1] = __uint_as_float(u.x & 0xffff0000u);
                     qv[c * 8 + 2] = __uint_as_float(u.y << 16); qv[c * 8 + 3] = __uint_as_float(u.y & 0xffff0000u);
@@ -252,10 +254,10 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
             bad |= j >= n_valid || j < -1;
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
             if (valid) {
-                const uint4 *k4 = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D) + part * kChunks;
+                const uint4 *k4 = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D) + part;
                 uint4 kv[kChunks];
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) kv[c] = __ldg(k4 + c);
+                for (int c = 0; c < kChunks; ++c) kv[c] = __ldg(k4 + 4 * c);
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
                     const uint4 u = kv[c];

@@ -58,7 +58,7 @@ namespace tc {
 
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kHeapThreads = 32 * (2 + 4);     // heap kernel: 4 epilogue warps (one per row)
 constexpr int kPassThreads = 32 * (2 + 8);     // three-pass kernel: 8 epilogue warps (two per row)
 constexpr int kTmemCols = 256;
@@ -72,9 +72,12 @@ constexpr int kBuf = 32;
 
 __host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-// Stages of the key ring: the three-pass kernel reuses the query and key
-// buffers (>= 72 KB together) to sort its kept scores at the end.
-__host__ __device__ inline int stages_for(int d, bool three_pass) {
+// Stages of the key ring.  The fused three-pass kernel reuses the query and
+// key buffers (>= 72 KB together) to sort its kept scores at the end; the
+// split kernel keeps its histogram inside the append buffers and spends the
+// space saved on a deeper ring.
+__host__ __device__ inline int stages_for(int d, bool three_pass, bool split) {
+    if (three_pass && split) return d == 64 ? 6 : 3;
     return (three_pass && d == 64) ? 4 : 2;
 }
 
@@ -84,17 +87,19 @@ struct Layout {
 };
 
 // three_pass: q | k | hist [kNB][kRows] u32 | bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16
-//             (bufv + bufi, 72 KB, later hold one membership bitmap per row)
+//             fused: bufv + bufi (72 KB) later hold one membership bitmap per row
+//             split: no separate hist; passes 0-1 use bufv + bufi (hist at
+//             +0, the group maxima at +32 KB), pass 2 appends into them
 // heap:       q | k | heap [ksel][kRows] u64 | bufv [kBuf][kRows] f32 | bufi [kBuf][kRows] i32
-__host__ __device__ inline Layout layout_of(int d, int ksel, bool three_pass) {
+__host__ __device__ inline Layout layout_of(int d, int ksel, bool three_pass, bool split = false) {
     Layout s;
-    s.stages = stages_for(d, three_pass);
+    s.stages = stages_for(d, three_pass, split);
     uint32_t o = 0;
     s.q = o;    o = up(o + kRows * d * 2, 1024);
     s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
     s.sel = o;
     if (three_pass) {
-        s.hist = o; o = up(o + kNB * kRows * 4, 16);
+        s.hist = o; o = up(o + (split ? 0 : kNB * kRows * 4), 16);
         s.bufv = o; o = up(o + kCap * kRows * 4, 16);
         s.bufi = o; o = up(o + kCap * kRows * 2, 16);
     } else {
@@ -584,8 +589,13 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 // Bin of a score for one row: bins of width (M - Lo) / kNB counted down from
 // M; scores above M land in bin 0, scores under Lo in the last bin.  The same expression is used in
 // every place a bin is computed, so counts and placements agree.
+//   x = fma(v, -inv, M * inv),  bin = floor(min(max(x, 0), kNB - 1))
+// (NaN lands in bin 0).  The floor is taken by adding 2^23 rounding down: for
+// 0 <= y < 2^23 the sum's low mantissa bits are floor(y).  bin <= b holds
+// exactly when !(x >= b + 1) for b < kNB - 1, which pass 2 tests directly.
 __device__ __forceinline__ int bin_of(float v, float neg_inv, float hi_inv) {
-    return min((int)fmaxf(fmaf(v, neg_inv, hi_inv), 0.f), kNB - 1);
+    const float y = fminf(fmaxf(fmaf(v, neg_inv, hi_inv), 0.f), (float)(kNB - 1));
+    return __float_as_int(__fadd_rd(y, 8388608.f)) & 0x7fffff;
 }
 
 // kSplit: the kernel ends after pass 2 by writing each row's kept scores
@@ -601,7 +611,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
     const int d = L.d, ksel = L.ksel;
-    const Layout lay = layout_of(d, ksel, true);
+    const Layout lay = layout_of(d, ksel, true, kSplit);
     Cta c;
     if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -665,8 +675,10 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                     if (col0 + jj < first_lim) Lo = fminf(Lo, v[jj]);
             }
         }
+        // group maxima [64][kRows]: clear of the histogram in both layouts
+        const uint32_t gx_off = kSplit ? lay.bufv + kNB * kRows * 4 : lay.bufv;
         {
-            float *gx = reinterpret_cast<float *>(smem + lay.bufv) + r;   // [64][kRows]
+            float *gx = reinterpret_cast<float *>(smem + gx_off) + r;
 #pragma unroll
             for (int q = 0; q < 32; ++q) gx[(half * 32 + q) * kRows] = gm[q];
         }
@@ -676,7 +688,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         epi_sync();
         float M = -INFINITY, gmin = INFINITY;
         {
-            const float *gx = reinterpret_cast<const float *>(smem + lay.bufv) + r;
+            const float *gx = reinterpret_cast<const float *>(smem + gx_off) + r;
             for (int q = 0; q < 64; ++q) {
                 const float x = gx[q * kRows];
                 M = fmaxf(M, x);
@@ -726,12 +738,17 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             run = cum;
         }
         const bool overflow = run > (uint32_t)(kCap - 2);
-        // pass 2: append every score of bins 0..b* (same bin arithmetic as
-        // pass 1) to the row's buffer, half 0 upward from slot 0 and half 1
-        // downward from slot kCap-1.  Branch-free: each value is stored at
-        // the half's next free slot and the slot advances only if the value
-        // is kept, so values not kept are overwritten; the two halves never
-        // share a slot while their counts sum to at most kCap-2.
+        if constexpr (kSplit) epi_sync();   // the histogram's space becomes the append buffers
+
+        // pass 2: append every score of bins 0..b* to the row's buffer, half 0
+        // upward from slot 0 and half 1 downward from slot kCap-1.  A score is
+        // in bins 0..b* exactly when !(x >= b* + 1), x as in bin_of (with a
+        // NaN threshold every score is).  The halves' counts sum to run <=
+        // kCap-2 when the passes agree; a half stops appending once it holds
+        // more than kCap-9 (checked every 8 columns, so no slot leaves the
+        // buffer), and a row whose counts then differ from run is retried.
+        const float thr = (all_mode || bstar >= kNB - 1) ? __int_as_float(0x7fc00000)
+                                                         : (float)(bstar + 1);
         int cnt = 0;
         {
             const int base = half ? kCap - 1 : 0;
@@ -744,12 +761,18 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 const int col0 = i * kKeys + half * 64;
                 const int lim = overflow ? 0 : n_valid - col0;   // columns jj < lim take part
 #pragma unroll
-                for (int jj = 0; jj < 64; ++jj) {
-                    const int b = all_mode ? 0 : bin_of(v[jj], neg_inv, hi_inv);
-                    const int slot = base + dir * min(cnt, kCap - 1);
-                    bv[slot * kRows] = v[jj];
-                    bi[slot * kRows] = (uint16_t)(col0 + jj);
-                    cnt += (jj < lim && b <= bstar) ? 1 : 0;
+                for (int g8 = 0; g8 < 64; g8 += 8) {
+                    const int lim8 = cnt <= kCap - 9 ? lim : 0;
+#pragma unroll
+                    for (int jj = g8; jj < g8 + 8; ++jj) {
+                        const float x = fmaf(v[jj], neg_inv, hi_inv);
+                        if (jj < lim8 && !(x >= thr)) {
+                            const int slot = base + dir * cnt;
+                            bv[slot * kRows] = v[jj];
+                            bi[slot * kRows] = (uint16_t)(col0 + jj);
+                            ++cnt;
+                        }
+                    }
                 }
             }
         }
@@ -1132,15 +1155,19 @@ bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     // the selection kernel's sorted scores (f32 + u16 per slot) reuse the
     // operand buffers, and its per-row bitmaps the append buffers
     const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
-    return lay.sel - lay.q >= (uint32_t)(tc::kCap * tc::kRows * 6) &&
+    const tc::Layout lays = tc::layout_of(L.d, L.ksel, true, true);
+    return lay.total <= 232448 && lays.total <= 232448 &&
+           lay.sel - lay.q >= (uint32_t)(tc::kCap * tc::kRows * 6) &&
            lay.bufi + tc::kCap * tc::kRows * 2 - lay.bufv >= (uint32_t)(144 * tc::kRows * 4) &&
            L.ksel + L.r <= tc::kCap;
 }
 
 size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
-    const size_t a = tc::layout_of(L.d, L.ksel, true).total;
+    size_t a = tc::layout_of(L.d, L.ksel, true).total;
     const size_t b = tc::layout_of(L.d, L.ksel, false).total;
-    return a > b ? a : b;
+    const size_t c = tc::layout_of(L.d, L.ksel, true, true).total;
+    if (b > a) a = b;
+    return c > a ? c : a;
 }
 
 CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype) {
@@ -1157,9 +1184,10 @@ cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
     if (smem_bytes > 232448) return cudaErrorInvalidValue;   // 227 KB per block on sm_100
     // the kernels may be launched with up to their largest layout
     const int big = (int)tc::layout_of(128, 64, true).total;
+    const int big_split = (int)tc::layout_of(128, 64, true, true).total;
     const int big_heap = (int)tc::layout_of(128, 64, false).total;
     cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, big_split);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big);
@@ -1186,8 +1214,9 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     const size_t smem3 = tc::layout_of(L.d, L.ksel, true).total;
+    const size_t smem3s = tc::layout_of(L.d, L.ksel, true, true).total;
     if (L.cand_v && L.cand_i && L.cand_meta) {
-        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem3, s>>>(
+        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem3s, s>>>(
             L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
