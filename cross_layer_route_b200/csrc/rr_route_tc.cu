@@ -20,29 +20,26 @@
 //   warps 2-   epilogue, reading the score tile with tcgen05.ld; a warp may
 //              only read the 32 TMEM lanes (= query rows) of its sub-partition
 //              (warp index mod 4).  The heap kernel runs 4 such warps, one
-//              thread per row; the three-pass kernel runs 8, the two warps of
+//              thread per row; the two-pass kernel runs 8, the two warps of
 //              a sub-partition splitting each tile's columns.
 // The query tile is gathered by row index into the layout a 128-byte
 // swizzled TMA load would produce, so anchor and refresh share one path.
 //
 // Selection (route_rows_tc_kernel).  The tensor cores are cheap next to the
-// per-score work of an exact top-(k+m), so the key tiles are streamed three
-// times and the MMA recomputed each time:
-//   pass 0  per row: the maximum score M, and Lo = the minimum of the first
-//           k+m valid scores (any k+m scores bound the (k+m)-th best from
-//           below);
-//   pass 1  per row: a histogram of (M - s) over 128 equal bins of [Lo, M]
-//           (scores under Lo fall in the last bin); the first bin b* at
-//           which the running count reaches k+m holds the (k+m)-th best;
-//   pass 2  per row: every score of bins 0..b* is appended to the row's
-//           buffer (about k+m plus one bin's crowd).
-// The kept scores are then placed by bin (a counting sort on the histogram's
-// start offsets), each inserted in order among its bin's earlier arrivals
-// (exact best-first order); the first k+m are the route and near-miss ids.  A row whose bins 0..b* hold more than kCap-2 scores (or
-// whose appended count differs from the histogram's -- a certificate check)
-// is appended to a retry list and routed by route_rows_tc_heap_kernel, which
-// keeps a per-row min-heap of the k+m best over one pass; results are exact
-// either way.
+// per-score work of an exact top-(k+m), so the key tiles are streamed twice
+// and the MMA recomputed:
+//   pass 0  per row: the two largest valid scores of each of 64 column
+//           groups; T = the (k+m)-th largest of these 128 values (a lower
+//           bound of the row's (k+m)-th best score, since that many distinct
+//           scores reach it);
+//   pass 1  per row: every valid score >= T is appended to the row's buffer
+//           (on Gaussian-like rows about 10% more than k+m).
+// The kept scores are then ordered (score desc, chunk asc) and the row's
+// ledger entry written by one warp per row (finish_row): in a separate
+// kernel reading the kept scores from global memory, or by the same CTA.  A
+// row whose kept scores do not fit the buffer (kCap-2) is appended to a retry
+// list and routed by route_rows_tc_heap_kernel, which keeps a per-row
+// min-heap of the k+m best over one pass; results are exact either way.
 //
 // Every wait is bounded; a timeout sets bit 1 of the error word and the CTA
 // drains its copies, frees its TMEM and returns.
@@ -60,55 +57,59 @@ constexpr int kRows = 128;
 constexpr int kKeys = 128;
 constexpr int kMaxStages = 6;
 constexpr int kHeapThreads = 32 * (2 + 4);     // heap kernel: 4 epilogue warps (one per row)
-constexpr int kPassThreads = 32 * (2 + 8);     // three-pass kernel: 8 epilogue warps (two per row)
+constexpr int kPassThreads = 32 * (2 + 8);     // two-pass kernel: 8 epilogue warps (two per row)
 constexpr int kTmemCols = 256;
 constexpr int kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr long long kSpinLimit = 1ll << 31;
-// three-pass selection
-constexpr int kNB = 64;                    // histogram bins per row
-constexpr int kCap = 96;                   // kept scores per row (both column halves)
+// two-pass selection
+constexpr int kGroups = 32;                // column groups per half row (two halves per row)
+constexpr int kTops = 4 * kGroups;         // group top-2 values per row
+constexpr int kTopStride = kTops + 1;      // padded row of the group tops in shared memory
+constexpr int kCap = 128;                  // kept scores per row (both column halves)
+constexpr int kStageCols = 16;             // columns per staging round of the collect pass
+constexpr int kThrLowBit = 16;             // threshold search stops at this key bit
 // heap selection (retry path)
 constexpr int kBuf = 32;
 
 __host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
-// Stages of the key ring.  The fused three-pass kernel reuses the query and
-// key buffers (>= 72 KB together) to sort its kept scores at the end; the
-// split kernel keeps its histogram inside the append buffers and spends the
-// space saved on a deeper ring.
-__host__ __device__ inline int stages_for(int d, bool three_pass, bool split) {
-    if (three_pass && split) return d == 64 ? 6 : 3;
-    return (three_pass && d == 64) ? 4 : 2;
+// Stages of the key ring (what the shared memory left by the selection
+// buffers allows).
+__host__ __device__ inline int stages_for(int d, bool two_pass) {
+    if (two_pass) return d == 64 ? 4 : 2;
+    return 2;
 }
 
 struct Layout {
-    uint32_t q, k, sel, hist, bufv, bufi, rows, red, bars, misc, total;
+    uint32_t q, k, sel, bufv, bufi, stg, rows, red, bars, misc, total;
     int stages;
 };
 
-// three_pass: q | k | hist [kNB][kRows] u32 | bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16
-//             fused: bufv + bufi (72 KB) later hold one membership bitmap per row
-//             split: no separate hist; passes 0-1 use bufv + bufi (hist at
-//             +0, the group maxima at +32 KB), pass 2 appends into them
-// heap:       q | k | heap [ksel][kRows] u64 | bufv [kBuf][kRows] f32 | bufi [kBuf][kRows] i32
-__host__ __device__ inline Layout layout_of(int d, int ksel, bool three_pass, bool split = false) {
+// two_pass: q | k | sel (96 KB: the group tops [kRows][kTopStride] f32 after
+//           pass 0, then bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16) |
+//           stg [256 threads][kStageCols] f32 | rows | red (threshold and
+//           two kept counts per row)
+// heap:     q | k | heap [ksel][kRows] u64 | bufv [kBuf][kRows] f32 | bufi [kBuf][kRows] i32
+__host__ __device__ inline Layout layout_of(int d, int ksel, bool two_pass) {
     Layout s;
-    s.stages = stages_for(d, three_pass, split);
+    s.stages = stages_for(d, two_pass);
     uint32_t o = 0;
     s.q = o;    o = up(o + kRows * d * 2, 1024);
     s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
     s.sel = o;
-    if (three_pass) {
-        s.hist = o; o = up(o + (split ? 0 : kNB * kRows * 4), 16);
+    if (two_pass) {
         s.bufv = o; o = up(o + kCap * kRows * 4, 16);
         s.bufi = o; o = up(o + kCap * kRows * 2, 16);
+        o = up(s.sel + (kRows * kTopStride * 4 > o - s.sel ? kRows * kTopStride * 4 : o - s.sel), 16);
+        s.stg = o;  o = up(o + 256 * kStageCols * 4, 16);
     } else {
-        s.hist = o; o = up(o + kRows * ksel * 8, 16);
+        s.stg = 0;
+        o = up(o + kRows * ksel * 8, 16);   // the heap, at sel
         s.bufv = o; o = up(o + kRows * kBuf * 4, 16);
         s.bufi = o; o = up(o + kRows * kBuf * 4, 16);
     }
     s.rows = o; o = up(o + kRows * 4, 16);
-    s.red = o;  o = up(o + (three_pass ? 6 * kRows * 4 : 0), 16);   // max, min, count per half
+    s.red = o;  o = up(o + (two_pass ? 3 * kRows * 4 : 0), 16);
     s.bars = o; o = up(o + 8 * (2 * kMaxStages + 5), 16);
     s.misc = o; o = up(o + 16, 16);
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
@@ -323,23 +324,12 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Lay
     return true;
 }
 
-// Tile schedule.  One pass: key tiles 0..nt-1.  Three passes: pass 0 over
-// the first min(nt, kPass0Tiles) tiles, pass 1 over all tiles backwards
-// (its first tiles are the ones still in L2), pass 2 over all tiles.
-// kPass0Tiles bounds the tiles pass 0 sees; a short pass 0 only estimates
-// the row maximum (larger scores fall in bin 0, which stays exact but
-// widens the bins), which measured no faster, so pass 0 covers every tile.
-constexpr int kPass0Tiles = 1 << 20;
-__device__ __forceinline__ int pass0_tiles(int ntiles) { return min(ntiles, kPass0Tiles); }
-__device__ __forceinline__ int total_tiles(int ntiles, int passes) {
-    return passes == 3 ? pass0_tiles(ntiles) + 2 * ntiles : ntiles;
-}
+// Tile schedule: pass p covers key tiles 0..nt-1, the second pass backwards
+// (its first tiles are the ones most recently loaded).
+__device__ __forceinline__ int total_tiles(int ntiles, int passes) { return passes * ntiles; }
 __device__ __forceinline__ int tile_of(int g, int ntiles, int passes) {
-    if (passes != 3) return g;
-    const int p0 = pass0_tiles(ntiles);
-    if (g < p0) return g;
-    if (g < p0 + ntiles) return ntiles - 1 - (g - p0);
-    return g - p0 - ntiles;
+    (void)passes;
+    return g < ntiles ? g : 2 * ntiles - 1 - g;
 }
 
 __device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int passes) {
@@ -522,7 +512,7 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const int r = sub * 32 + lane;
         const int row = c.rows_s[r];
         const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
-        uint64_t *H = reinterpret_cast<uint64_t *>(smem + lay.hist) + r;
+        uint64_t *H = reinterpret_cast<uint64_t *>(smem + lay.sel) + r;
         float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
         int *bi = reinterpret_cast<int *>(smem + lay.bufi) + r;
         for (int e = 0; e < ksel; ++e) H[e * kRows] = 0ull;
@@ -585,345 +575,16 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     cta_teardown(c, L);
 }
 
-// ---- three-pass kernel (the main path) ------------------------------------------
-// Bin of a score for one row: bins of width (M - Lo) / kNB counted down from
-// M; scores above M land in bin 0, scores under Lo in the last bin.  The same expression is used in
-// every place a bin is computed, so counts and placements agree.
-//   x = fma(v, -inv, M * inv),  bin = floor(min(max(x, 0), kNB - 1))
-// (NaN lands in bin 0).  The floor is taken by adding 2^23 rounding down: for
-// 0 <= y < 2^23 the sum's low mantissa bits are floor(y).  bin <= b holds
-// exactly when !(x >= b + 1) for b < kNB - 1, which pass 2 tests directly.
-__device__ __forceinline__ int bin_of(float v, float neg_inv, float hi_inv) {
-    const float y = fminf(fmaxf(fmaf(v, neg_inv, hi_inv), 0.f), (float)(kNB - 1));
-    return __float_as_int(__fadd_rd(y, 8388608.f)) & 0x7fffff;
-}
-
-// kSplit: the kernel ends after pass 2 by writing each row's kept scores
-// (both column halves' buffers, as they are) and their counts to the
-// candidate buffers; route_rows_finalize_kernel orders them and writes the
-// ledger rows.  Otherwise the CTA finishes its rows itself (no candidate
-// buffers needed).
-template <bool kSplit>
-__global__ void __launch_bounds__(kPassThreads, 1)
-route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
-                     const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
-    extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-    const int d = L.d, ksel = L.ksel;
-    const Layout lay = layout_of(d, ksel, true, kSplit);
-    Cta c;
-    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y;
-
-    if (warp == 0) {
-        if (lane == 0) producer(c, &tmap_k, d, h, 3);
-    } else if (warp == 1) {
-        if (lane == 0) mma_issuer(c, d, 3);
-    } else {
-        // Two warps per TMEM sub-partition: half 0 reads columns 0..63 of
-        // every tile, half 1 columns 64..127.  Per-row state lives in shared
-        // memory; the 256 epilogue threads meet at named barrier 1 between
-        // phases (every one of them reaches every barrier, also after a
-        // timeout, so none can be left waiting).
-        const int sub = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const int r = sub * 32 + lane;
-        const int row = c.rows_s[r];
-        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
-        const int first_lim = min(ksel, n_valid);
-        const bool all_mode = n_valid <= ksel;   // every valid key is selected
-        uint32_t *hist = reinterpret_cast<uint32_t *>(smem + lay.hist) + r;
-        float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
-        uint16_t *bi = reinterpret_cast<uint16_t *>(smem + lay.bufi) + r;
-        float *red_lo = reinterpret_cast<float *>(smem + lay.red) + 2 * kRows; // [2][kRows]
-        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(half * 64);
-        const int nt = c.ntiles;
-        bool ok = true;
-        int g = 0;
-        auto epi_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
-
-        // pass 0: per row, the maximum of each of 64 disjoint column groups
-        // (group = half, column mod 32) and the minimum of the first k+m valid
-        // scores.  M = the largest group maximum (the row maximum); the
-        // smallest group maximum and that minimum are both at most the
-        // (k+m)-th best score (each comes with k+m or more distinct scores at
-        // or above it), so the larger of the two is the histogram's lower end.
-        float gm[32];
-#pragma unroll
-        for (int q = 0; q < 32; ++q) gm[q] = -INFINITY;
-        float Lo = INFINITY;
-        const int p0 = pass0_tiles(nt);
-        for (int i = 0; i < p0 && ok; ++i, ++g) {
-            if (!(ok = acc_wait(c, g))) break;
-            float v[64];
-            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
-            acc_release(c, g);   // the scores are in registers: the MMA may reuse the accumulator
-            const int col0 = i * kKeys + half * 64;
-            if (col0 + 64 <= n_valid) {
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj) gm[jj & 31] = fmaxf(gm[jj & 31], v[jj]);
-            } else {
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj)
-                    if (col0 + jj < n_valid) gm[jj & 31] = fmaxf(gm[jj & 31], v[jj]);
-            }
-            if (col0 < first_lim) {
-#pragma unroll
-                for (int jj = 0; jj < 64; ++jj)
-                    if (col0 + jj < first_lim) Lo = fminf(Lo, v[jj]);
-            }
-        }
-        // group maxima [64][kRows]: clear of the histogram in both layouts
-        const uint32_t gx_off = kSplit ? lay.bufv + kNB * kRows * 4 : lay.bufv;
-        {
-            float *gx = reinterpret_cast<float *>(smem + gx_off) + r;
-#pragma unroll
-            for (int q = 0; q < 32; ++q) gx[(half * 32 + q) * kRows] = gm[q];
-        }
-        red_lo[half * kRows + r] = Lo;
-        if (half == 0)
-            for (int b = 0; b < kNB; ++b) hist[b * kRows] = 0u;
-        epi_sync();
-        float M = -INFINITY, gmin = INFINITY;
-        {
-            const float *gx = reinterpret_cast<const float *>(smem + gx_off) + r;
-            for (int q = 0; q < 64; ++q) {
-                const float x = gx[q * kRows];
-                M = fmaxf(M, x);
-                gmin = fminf(gmin, x);
-            }
-        }
-        Lo = fmaxf(fminf(red_lo[r], red_lo[kRows + r]), gmin);
-
-        // pass 1: histogram of (M - s) over [Lo, M], tiles in reverse order
-        const float range = M - Lo;
-        const float inv = (!all_mode && range > 0.f) ? (float)kNB / range : 0.f;
-        const float neg_inv = -inv, hi_inv = M * inv;
-        for (int i = 0; i < nt && ok; ++i, ++g) {
-            if (!(ok = acc_wait(c, g))) break;
-            const int t = nt - 1 - i;
-            float v[64];
-            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);   // every lane loads (.sync.aligned)
-            acc_release(c, g);
-            const int col0 = t * kKeys + half * 64;
-            if (!all_mode) {
-                if (col0 + 64 <= n_valid) {
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj)
-                        atomicAdd(&hist[bin_of(v[jj], neg_inv, hi_inv) * kRows], 1u);
-                } else {
-#pragma unroll
-                    for (int jj = 0; jj < 64; ++jj)
-                        if (col0 + jj < n_valid)
-                            atomicAdd(&hist[bin_of(v[jj], neg_inv, hi_inv) * kRows], 1u);
-                }
-            }
-        }
-        epi_sync();
-
-        // boundary bin b*: the first bin where the running count reaches k+m;
-        // run = scores in bins 0..b*.  Rows with every valid key selected use
-        // one bin.
-        int bstar = 0;
-        uint32_t run = (uint32_t)n_valid;
-        if (!all_mode) {
-            bstar = kNB - 1;
-            uint32_t cum = 0;
-            for (int b = 0; b < kNB; ++b) {
-                cum += hist[b * kRows];
-                if (cum >= (uint32_t)ksel) { bstar = b; break; }
-            }
-            run = cum;
-        }
-        const bool overflow = run > (uint32_t)(kCap - 2);
-        if constexpr (kSplit) epi_sync();   // the histogram's space becomes the append buffers
-
-        // pass 2: append every score of bins 0..b* to the row's buffer, half 0
-        // upward from slot 0 and half 1 downward from slot kCap-1.  A score is
-        // in bins 0..b* exactly when !(x >= b* + 1), x as in bin_of (with a
-        // NaN threshold every score is).  The halves' counts sum to run <=
-        // kCap-2 when the passes agree; a half stops appending once it holds
-        // more than kCap-9 (checked every 8 columns, so no slot leaves the
-        // buffer), and a row whose counts then differ from run is retried.
-        const float thr = (all_mode || bstar >= kNB - 1) ? __int_as_float(0x7fc00000)
-                                                         : (float)(bstar + 1);
-        int cnt = 0;
-        {
-            const int base = half ? kCap - 1 : 0;
-            const int dir = half ? -1 : 1;
-            for (int i = 0; i < nt && ok; ++i, ++g) {
-                if (!(ok = acc_wait(c, g))) break;
-                float v[64];
-                tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
-                acc_release(c, g);
-                const int col0 = i * kKeys + half * 64;
-                const int lim = overflow ? 0 : n_valid - col0;   // columns jj < lim take part
-#pragma unroll
-                for (int g8 = 0; g8 < 64; g8 += 8) {
-                    const int lim8 = cnt <= kCap - 9 ? lim : 0;
-#pragma unroll
-                    for (int jj = g8; jj < g8 + 8; ++jj) {
-                        const float x = fmaf(v[jj], neg_inv, hi_inv);
-                        if (jj < lim8 && !(x >= thr)) {
-                            const int slot = base + dir * cnt;
-                            bv[slot * kRows] = v[jj];
-                            bi[slot * kRows] = (uint16_t)(col0 + jj);
-                            ++cnt;
-                        }
-                    }
-                }
-            }
-        }
-        int *rcnt = reinterpret_cast<int *>(smem + lay.red) + 4 * kRows;   // [2][kRows]
-        rcnt[half * kRows + r] = cnt;
-        epi_sync();
-
-        if constexpr (kSplit) {
-            // candidate slot (blk, slot, r) at cand[(blk * kCap + slot) * kRows + r];
-            // meta (blk, r) = c0 | c1 << 16, or -1 when the row has nothing to finish
-            const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-            const int c0 = rcnt[r], c1 = rcnt[kRows + r];
-            const bool good = ok && row >= 0 && !overflow && c0 + c1 == (int)run;
-            if (half == 0) {
-                L.cand_meta[blk * kRows + r] = good ? (c0 | (c1 << 16)) : -1;
-                if (ok && row >= 0 && !good) {
-                    const int pos = atomicAdd(&L.retry_count[h], 1);
-                    L.retry_list[(size_t)h * L.nq + pos] = row;
-                    atomicAdd(&L.counters[10], 1ULL);
-                }
-            }
-            if (good) {
-                // half 0 writes slots 0..kCap/2-1, half 1 the rest (only used ones)
-                float *gv = L.cand_v + blk * kCap * kRows + r;
-                uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
-                const int s0 = half * (kCap / 2);
-                for (int sl = s0; sl < s0 + kCap / 2; ++sl) {
-                    if (sl < c0 || sl >= kCap - c1) {
-                        gv[sl * kRows] = bv[sl * kRows];
-                        gi[sl * kRows] = bi[sl * kRows];
-                    }
-                }
-            }
-        } else {
-
-        // Place the kept scores by bin in the query/key buffers, free now
-        // that every MMA is done, each one inserted in order among the scores
-        // of its bin placed before it (best first: score desc, chunk asc).
-        // Bins hold a handful of scores, so the insertion moves few.  The two
-        // halves share the rows: half 0 finishes lanes 0..15, half 1 lanes
-        // 16..31.
-        float *sv = reinterpret_cast<float *>(smem + lay.q) + r;
-        uint16_t *si = reinterpret_cast<uint16_t *>(smem + lay.q + kCap * kRows * 4) + r;
-        const bool mine = ok && row >= 0 && (lane >> 4) == half;
-        bool fail = false;
-        if (mine) {
-            const int c0 = rcnt[r], c1 = rcnt[kRows + r];
-            fail = overflow || c0 + c1 != (int)run;
-            if (!fail) {
-                // per bin: start offset (low half) and next free slot (high
-                // half); both halves read the counts before pass 2, so this
-                // thread owns the row's histogram now
-                uint32_t acc = 0;
-                for (int b = 0; b <= bstar; ++b) {
-                    const uint32_t x = hist[b * kRows];
-                    hist[b * kRows] = acc | (acc << 16);
-                    acc += x;
-                }
-                for (int e = 0; e < c0 + c1; ++e) {
-                    const int slot = e < c0 ? e : kCap - 1 - (e - c0);
-                    const float v = bv[slot * kRows];
-                    const uint16_t j = bi[slot * kRows];
-                    const int b = all_mode ? 0 : bin_of(v, neg_inv, hi_inv);
-                    const uint32_t x = hist[b * kRows];
-                    hist[b * kRows] = x + (1u << 16);
-                    const int lo = (int)(x & 0xffffu);
-                    int p = (int)(x >> 16);
-                    for (; p > lo; --p) {
-                        const float pv = sv[(p - 1) * kRows];
-                        const uint16_t pj = si[(p - 1) * kRows];
-                        if (!(v > pv || (v == pv && j < pj))) break;
-                        sv[p * kRows] = pv;
-                        si[p * kRows] = pj;
-                    }
-                    sv[p * kRows] = v;
-                    si[p * kRows] = j;
-                }
-            } else {
-                const int pos = atomicAdd(&L.retry_count[h], 1);
-                L.retry_list[(size_t)h * L.nq + pos] = row;
-                atomicAdd(&L.counters[10], 1ULL);
-            }
-        }
-        // every row is placed: the append buffers become membership bitmaps
-        // (a row's bitmap words past the value buffer overlap other rows'
-        // index slots, so this barrier is needed)
-        epi_sync();
-
-        if (mine && !fail) {
-            const int nr = min(L.k, n_valid);
-            const int nm = min(L.m, n_valid - nr);
-            const int nsel = nr + nm;
-            const size_t grow = (size_t)h * L.nq + row;
-            int32_t *out = L.ids + grow * L.c;
-            // route | near-miss: 16-byte stores where the layout allows
-            auto id_at = [&](int e) -> int {   // ledger slot e of route | near-miss
-                if (e < L.k) return e < nr ? (int)si[e * kRows] : -1;
-                const int f = e - L.k;
-                return f < nm ? (int)si[(nr + f) * kRows] : -1;
-            };
-            if (((L.c | L.k | L.m) & 3) == 0) {
-                int4 *o4 = reinterpret_cast<int4 *>(out);
-                for (int e = 0; e < L.k + L.m; e += 4)
-                    o4[e >> 2] = make_int4(id_at(e), id_at(e + 1), id_at(e + 2), id_at(e + 3));
-            } else {
-                for (int e = 0; e < L.k + L.m; ++e) out[e] = id_at(e);
-            }
-            const float alpha = sv[(nr - 1) * kRows];
-            // one bit per valid chunk (route, near-miss, accepted sentinels)
-            uint32_t *bits = reinterpret_cast<uint32_t *>(smem + lay.bufv) + r;
-            const int words = (n_valid + 31) >> 5;
-            const bool use_bits = words <= (int)(kCap * 6 / 4);   // 144 words fit the buffers
-            if (use_bits) {
-                for (int w = 0; w < words; ++w) bits[w * kRows] = 0u;
-                for (int e = 0; e < nsel; ++e) {
-                    const int j = si[e * kRows];
-                    bits[(j >> 5) * kRows] |= 1u << (j & 31);
-                }
-            }
-            // accepted sentinels are kept in the sorted area past route | near-miss
-            uint16_t *acc_ids = si + nsel * kRows;
-            int32_t *rout = out + L.k + L.m;
-            random_sentinels(
-                L, L.bh_offset + h, row, layer, n_valid, nsel,
-                [&](int jx) {
-                    if (use_bits) return ((bits[(jx >> 5) * kRows] >> (jx & 31)) & 1u) != 0u;
-                    for (int e = 0; e < nsel; ++e)
-                        if ((int)si[e * kRows] == jx) return true;
-                    return false;
-                },
-                [&](int e) -> uint16_t & { return acc_ids[e * kRows]; }, rout,
-                use_bits ? bits : nullptr);
-            L.alpha[grow] = alpha;
-            L.anchor_layer[grow] = layer;
-            L.flags[grow] = 1;
-        }
-        }   // fused tail
-    }
-    cta_teardown(c, L);
-}
-
-// ---- finalize kernel (split path): one warp per row ---------------------------
-// Reads a row's kept scores (at most kCap - 2, written by
-// route_rows_tc_kernel<true>) and writes its ledger row: route | near-miss in
-// best-first order (score desc, chunk asc), alpha (the k-th score) and the
-// random sentinels (RouteRelay §3.1 items 1-2).
+// ---- finishing a row from its kept scores (one warp per row) ---------------------
+// The ledger row of one query row from its kept scores (a superset of its
+// k + m best): route | near-miss in best-first order (score desc, chunk asc),
+// alpha (the k-th score) and the random sentinels (RouteRelay §3.1 items
+// 1-2).
 //
-// Order: the row's kept scores are binned over their own range (128 bins,
-// larger score = lower bin, ties share a bin), placed by bin, and each one's
-// final position is its bin's start plus the number of better keys in its
-// bin.  Sentinels: 32 draws at a time, one per lane (the same Philox words,
+// Order: the kept scores are binned over their own range (128 bins, larger
+// score = lower bin, ties share a bin), placed by bin, and each one's final
+// position is its bin's start plus the number of better keys in its bin.
+// Sentinels: 32 draws at a time, one per lane (the same Philox words,
 // rejection rule and ascending completion as random_sentinels above); a draw
 // is accepted if its chunk is not selected, not accepted earlier and not
 // drawn by an earlier lane of the round (warp match), in draw order.
@@ -944,43 +605,31 @@ __device__ __forceinline__ uint64_t cand_key(float v, int j) {
     return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
 }
 
-__global__ void __launch_bounds__(32 * kFinWarps)
-route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
-    __shared__ FinWarp fw_all[kFinWarps];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    FinWarp &w = fw_all[warp];
-    const int h = blockIdx.y;
-    constexpr int kPerBlk = kRows / kFinWarps;   // finalize CTAs per route CTA
-    const int bx = blockIdx.x / kPerBlk;
-    const int r = (blockIdx.x % kPerBlk) * kFinWarps + warp;
-    const int count = use_list ? L.head_count[h] : L.nq;
-    const int row0 = bx * kRows;
-    if (row0 + r >= count) return;
-    const size_t blk = (size_t)h * ((L.nq + kRows - 1) / kRows) + bx;
-    const int meta = L.cand_meta[blk * kRows + r];
-    if (meta < 0) return;   // no row, or a row left to the retry path
-    const int row = use_list ? L.list[(size_t)h * L.nq + row0 + r] : row0 + r;
-    const int c0 = meta & 0xffff, c1 = meta >> 16, run = c0 + c1;
+// One warp, every lane with the same arguments.  The row's kept scores sit in
+// a two-ended buffer: c0 at slots 0.., c1 at slots kCap-1 downwards, read
+// through getv(slot) / geti(slot).  Needs c0 + c1 <= kCap and at least
+// min(k + m, valid keys) of them.
+template <typename GetV, typename GetI>
+__device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h, int row, int c0,
+                                           int c1, GetV getv, GetI geti, FinWarp &w, int lane) {
+    const int run = c0 + c1;
     const int n_valid = valid_keys(row, L.nk, L.causal);
     const uint32_t lt_mask = (1u << lane) - 1u;
 
-    // the row's kept scores, three per lane
-    const float *gv = L.cand_v + blk * kCap * kRows + r;
-    const uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
-    float v[3];
-    int jc[3];
-    bool live[3];
+    float v[4];
+    int jc[4];
+    bool live[4];
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         const int e = lane + 32 * i;
         live[i] = e < run;
         v[i] = 0.f;
         jc[i] = -1;
         if (live[i]) {
             const int sl = e < c0 ? e : kCap - 1 - (e - c0);
-            v[i] = gv[sl * kRows];
-            jc[i] = gi[sl * kRows];
+            v[i] = getv(sl);
+            jc[i] = geti(sl);
             mx = fmaxf(mx, v[i]);
             mn = fminf(mn, v[i]);
         }
@@ -997,10 +646,10 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
 #pragma unroll
     for (int q = 0; q < kFinBins / 32; ++q) w.hist[lane + 32 * q] = 0u;
     __syncwarp();
-    int bin[3];
-    uint32_t in_bin[3];
+    int bin[4];
+    uint32_t in_bin[4];
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         bin[i] = min((int)fmaxf(fmaf(v[i], neg_inv, hi_inv), 0.f), kFinBins - 1);
         in_bin[i] = live[i] ? atomicAdd(&w.hist[bin[i]], 1u) : 0u;
     }
@@ -1024,10 +673,10 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
         }
     }
     __syncwarp();
-    uint64_t key[3];
-    int start[3];
+    uint64_t key[4];
+    int start[4];
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         key[i] = cand_key(v[i], jc[i] < 0 ? 0 : jc[i]);
         start[i] = (int)w.hist[bin[i]];
         if (live[i]) w.keys[start[i] + (int)in_bin[i]] = key[i];
@@ -1038,9 +687,9 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
     const int nsel = nr + nm;
     const size_t grow = (size_t)h * L.nq + row;
     int32_t *out = L.ids + grow * L.c;
-    bool sel[3];
+    bool sel[4];
 #pragma unroll
-    for (int i = 0; i < 3; ++i) {
+    for (int i = 0; i < 4; ++i) {
         sel[i] = false;
         if (!live[i]) continue;
         const int end = bin[i] + 1 < kFinBins ? (int)w.hist[bin[i] + 1] : run;
@@ -1064,7 +713,7 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
         for (int q = lane; q < words; q += 32) w.bits[q] = 0u;
         __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 3; ++i)
+        for (int i = 0; i < 4; ++i)
             if (sel[i]) atomicOr(&w.bits[jc[i] >> 5], 1u << (jc[i] & 31));
         __syncwarp();
     }
@@ -1075,7 +724,7 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
         bool hit = false;
         for (int src = 0; src < 32; ++src) {
 #pragma unroll
-            for (int i = 0; i < 3; ++i) {
+            for (int i = 0; i < 4; ++i) {
                 const int cj = __shfl_sync(kFull, sel[i] ? jc[i] : -1, src);
                 hit |= cj == j;
             }
@@ -1126,6 +775,253 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
     }
 }
 
+// ---- two-pass kernel (the main path) ---------------------------------------------
+// kSplit: the kernel ends by writing each row's kept scores (both halves'
+// buffers, as they are) and their counts to the candidate buffers;
+// route_rows_finalize_kernel finishes the rows.  Otherwise the epilogue warps
+// finish them here (one warp per row, from shared memory).
+template <bool kSplit>
+__global__ void __launch_bounds__(kPassThreads, 1)
+route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+                     const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const int d = L.d, ksel = L.ksel;
+    const Layout lay = layout_of(d, ksel, true);
+    Cta c;
+    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+
+    if (warp == 0) {
+        if (lane == 0) producer(c, &tmap_k, d, h, 2);
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(c, d, 2);
+    } else {
+        // Two warps per TMEM sub-partition: half 0 reads columns 0..63 of
+        // every tile, half 1 columns 64..127.  The 256 epilogue threads meet
+        // at named barrier 1 between phases (every one of them reaches every
+        // barrier, also after a timeout, so none can be left waiting).
+        const int ew = warp - 2;   // epilogue warp 0..7
+        const int sub = warp & 3;
+        const int half = ew >> 2;
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
+        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(half * 64);
+        const int nt = c.ntiles;
+        bool ok = true;
+        int g = 0;
+        auto epi_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+
+        // pass 0: the two largest valid scores of each column group (this
+        // half's columns, group = column mod 32)
+        float m1[kGroups], m2[kGroups];
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) { m1[q] = -INFINITY; m2[q] = -INFINITY; }
+        for (int i = 0; i < nt && ok; ++i, ++g) {
+            if (!(ok = acc_wait(c, g))) break;
+            float v[64];
+            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            acc_release(c, g);   // the scores are in registers: the MMA may reuse the accumulator
+            const int col0 = i * kKeys + half * 64;
+            if (col0 + 64 <= n_valid) {
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj) {
+                    const int q = jj & (kGroups - 1);
+                    m2[q] = fmaxf(m2[q], fminf(m1[q], v[jj]));
+                    m1[q] = fmaxf(m1[q], v[jj]);
+                }
+            } else {
+#pragma unroll
+                for (int jj = 0; jj < 64; ++jj) {
+                    const int q = jj & (kGroups - 1);
+                    const float x = col0 + jj < n_valid ? v[jj] : -INFINITY;
+                    m2[q] = fmaxf(m2[q], fminf(m1[q], x));
+                    m1[q] = fmaxf(m1[q], x);
+                }
+            }
+        }
+        // the row's 128 group tops: [r][kTopStride], this half at half * 64
+        float *tops = reinterpret_cast<float *>(smem + lay.sel);
+#pragma unroll
+        for (int q = 0; q < kGroups; ++q) {
+            tops[r * kTopStride + half * 2 * kGroups + q] = m1[q];
+            tops[r * kTopStride + half * 2 * kGroups + kGroups + q] = m2[q];
+        }
+        epi_sync();
+
+        // threshold T of each row (one warp per row, 16 rows per warp): the
+        // largest key K, a multiple of 2^kThrLowBit, that at least k + m of
+        // the group tops' order-preserving keys reach.  At least k + m
+        // distinct valid scores are >= T, so T is at most the row's
+        // (k + m)-th best score.  Rows with at most k + m valid keys keep
+        // all of them (T = -inf).
+        float *thr_s = reinterpret_cast<float *>(smem + lay.red);   // [kRows]
+        {
+            constexpr int kRowsPerWarp = kRows / 8;
+            uint32_t key[kRowsPerWarp][4], K[kRowsPerWarp];
+#pragma unroll
+            for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                const int rr = ew * kRowsPerWarp + k2;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) key[k2][i] = ord32(tops[rr * kTopStride + i * 32 + lane]);
+                K[k2] = 0u;
+            }
+            // all 16 rows' searches interleaved (independent chains)
+            for (int bit = 31; bit >= kThrLowBit; --bit) {
+#pragma unroll
+                for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                    const uint32_t cand = K[k2] | (1u << bit);
+                    const unsigned mine = (key[k2][0] >= cand ? 1u : 0u) + (key[k2][1] >= cand ? 1u : 0u) +
+                                          (key[k2][2] >= cand ? 1u : 0u) + (key[k2][3] >= cand ? 1u : 0u);
+                    if ((int)__reduce_add_sync(kFull, mine) >= ksel) K[k2] = cand;
+                }
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                const int rr = ew * kRowsPerWarp + k2;
+                const int rowr = c.rows_s[rr];
+                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
+                float t = unord32(K[k2]);
+                if (nv <= ksel || t != t) t = -INFINITY;
+                if (lane == k2) thr_s[rr] = t;
+            }
+        }
+        epi_sync();
+        const float T = thr_s[r];
+
+        // pass 1: keep every valid score >= T.  Each thread builds a bit mask
+        // of its kept columns, stages the 16 scores of a round in shared
+        // memory (16-byte chunks swizzled by lane, so the stores do not
+        // collide) and appends the kept ones: half 0 upward from slot 0, half
+        // 1 downward from slot kCap-1; no slot leaves the buffer.
+        float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
+        uint16_t *bi = reinterpret_cast<uint16_t *>(smem + lay.bufi) + r;
+        float *stg = reinterpret_cast<float *>(smem + lay.stg) + (ew * 32 + lane) * kStageCols;
+        const int sw = (lane >> 1) & 3;   // 16-byte chunk swizzle: 8 lanes, 8 distinct bank groups
+        const int base = half ? kCap - 1 : 0;
+        const int dir = half ? -1 : 1;
+        int cnt = 0;
+        for (int i = 0; i < nt && ok; ++i, ++g) {
+            if (!(ok = acc_wait(c, g))) break;
+            const int t = tile_of(g, nt, 2);
+            float v[64];
+            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            acc_release(c, g);
+            const int col0 = t * kKeys + half * 64;
+            const int lim = n_valid - col0;   // columns jj < lim are valid
+#pragma unroll
+            for (int hq = 0; hq < 64 / kStageCols; ++hq) {
+                const int o = hq * kStageCols;
+                uint32_t mask = 0u;
+                if (lim >= 64) {
+#pragma unroll
+                    for (int jj = 0; jj < kStageCols; ++jj) mask |= v[o + jj] >= T ? (1u << jj) : 0u;
+                } else {
+#pragma unroll
+                    for (int jj = 0; jj < kStageCols; ++jj)
+                        mask |= (o + jj < lim && v[o + jj] >= T) ? (1u << jj) : 0u;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < kStageCols / 4; ++c4)
+                    *reinterpret_cast<float4 *>(stg + ((c4 ^ sw) << 2)) =
+                        make_float4(v[o + 4 * c4], v[o + 4 * c4 + 1], v[o + 4 * c4 + 2], v[o + 4 * c4 + 3]);
+                while (mask != 0u) {
+                    const int jj = __ffs(mask) - 1;
+                    mask &= mask - 1u;
+                    if (cnt < kCap) {
+                        const int sl = base + dir * cnt;
+                        bv[sl * kRows] = stg[(((jj >> 2) ^ sw) << 2) + (jj & 3)];
+                        bi[sl * kRows] = (uint16_t)(col0 + o + jj);
+                    }
+                    ++cnt;
+                }
+            }
+        }
+        int *rcnt = reinterpret_cast<int *>(smem + lay.red) + kRows;   // [2][kRows]
+        rcnt[half * kRows + r] = cnt;
+        epi_sync();
+
+        // A row is finished from its buffer when every wait succeeded, the
+        // two halves' scores fit it without meeting (c0 + c1 <= kCap - 2),
+        // and at least min(k + m, valid keys) were kept; other rows go to
+        // the retry list (exact heap selection).
+        const bool cta_ok = *c.abort_flag == 0;
+        auto row_good = [&](int rw, int nv, int k0, int k1) {
+            const int kept = k0 + k1;
+            return cta_ok && rw >= 0 && kept <= kCap - 2 && (nv <= ksel ? kept == nv : kept >= ksel);
+        };
+        const int c0 = rcnt[r], c1 = rcnt[kRows + r];
+        const bool good = row_good(row, n_valid, c0, c1);
+        if (half == 0 && ok && row >= 0 && !good) {
+            const int pos = atomicAdd(&L.retry_count[h], 1);
+            L.retry_list[(size_t)h * L.nq + pos] = row;
+            atomicAdd(&L.counters[10], 1ULL);
+        }
+
+        if constexpr (kSplit) {
+            // candidate slot (blk, slot, r) at cand[(blk * kCap + slot) * kRows + r];
+            // meta (blk, r) = c0 | c1 << 16, or -1 when the row has nothing to finish
+            const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+            if (half == 0) L.cand_meta[blk * kRows + r] = good ? (c0 | (c1 << 16)) : -1;
+            if (good) {
+                // half 0 writes slots 0..kCap/2-1, half 1 the rest (only used ones)
+                float *gv = L.cand_v + blk * kCap * kRows + r;
+                uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
+                const int s0 = half * (kCap / 2);
+                for (int sl = s0; sl < s0 + kCap / 2; ++sl) {
+                    if (sl < c0 || sl >= kCap - c1) {
+                        gv[sl * kRows] = bv[sl * kRows];
+                        gi[sl * kRows] = bi[sl * kRows];
+                    }
+                }
+            }
+        } else {
+            // finish the rows here: warp ew takes rows ew*16 .. ew*16+15, its
+            // scratch in the query/key buffers (every MMA is done)
+            FinWarp &fw = reinterpret_cast<FinWarp *>(smem + lay.q)[ew];
+            const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
+            const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
+            for (int k2 = 0; k2 < kRows / 8; ++k2) {
+                const int rr = ew * (kRows / 8) + k2;
+                const int rowr = c.rows_s[rr];
+                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
+                const int k0 = rcnt[rr], k1 = rcnt[kRows + rr];
+                if (!row_good(rowr, nv, k0, k1)) continue;   // warp-uniform
+                finish_row(
+                    L, layer, h, rowr, k0, k1, [&](int sl) { return bvb[sl * kRows + rr]; },
+                    [&](int sl) { return (int)bib[sl * kRows + rr]; }, fw, lane);
+            }
+        }
+    }
+    cta_teardown(c, L);
+}
+
+// ---- finalize kernel (split path): one warp per row ---------------------------
+__global__ void __launch_bounds__(32 * kFinWarps)
+route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
+    __shared__ FinWarp fw_all[kFinWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+    constexpr int kPerBlk = kRows / kFinWarps;   // finalize CTAs per route CTA
+    const int bx = blockIdx.x / kPerBlk;
+    const int r = (blockIdx.x % kPerBlk) * kFinWarps + warp;
+    const int count = use_list ? L.head_count[h] : L.nq;
+    const int row0 = bx * kRows;
+    if (row0 + r >= count) return;
+    const size_t blk = (size_t)h * ((L.nq + kRows - 1) / kRows) + bx;
+    const int meta = L.cand_meta[blk * kRows + r];
+    if (meta < 0) return;   // no row, or a row left to the retry path
+    const int row = use_list ? L.list[(size_t)h * L.nq + row0 + r] : row0 + r;
+    const float *gv = L.cand_v + blk * kCap * kRows + r;
+    const uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
+    finish_row(
+        L, layer, h, row, meta & 0xffff, meta >> 16, [&](int sl) { return gv[sl * kRows]; },
+        [&](int sl) { return (int)gi[sl * kRows]; }, fw_all[warp], lane);
+}
+
 // ---- host side -----------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1152,22 +1048,18 @@ bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     if (!(dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf &&
           L.nk <= 65535))
         return false;
-    // the selection kernel's sorted scores (f32 + u16 per slot) reuse the
-    // operand buffers, and its per-row bitmaps the append buffers
+    // the fused kernel finishes its rows with per-warp scratch in the
+    // query/key buffers
     const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
-    const tc::Layout lays = tc::layout_of(L.d, L.ksel, true, true);
-    return lay.total <= 232448 && lays.total <= 232448 &&
-           lay.sel - lay.q >= (uint32_t)(tc::kCap * tc::kRows * 6) &&
-           lay.bufi + tc::kCap * tc::kRows * 2 - lay.bufv >= (uint32_t)(144 * tc::kRows * 4) &&
-           L.ksel + L.r <= tc::kCap;
+    const tc::Layout layh = tc::layout_of(L.d, L.ksel, false);
+    return lay.total <= 232448 && layh.total <= 232448 &&
+           lay.sel - lay.q >= (uint32_t)(tc::kFinWarps * sizeof(tc::FinWarp));
 }
 
 size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
-    size_t a = tc::layout_of(L.d, L.ksel, true).total;
+    const size_t a = tc::layout_of(L.d, L.ksel, true).total;
     const size_t b = tc::layout_of(L.d, L.ksel, false).total;
-    const size_t c = tc::layout_of(L.d, L.ksel, true, true).total;
-    if (b > a) a = b;
-    return c > a ? c : a;
+    return a > b ? a : b;
 }
 
 CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype) {
@@ -1184,10 +1076,9 @@ cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
     if (smem_bytes > 232448) return cudaErrorInvalidValue;   // 227 KB per block on sm_100
     // the kernels may be launched with up to their largest layout
     const int big = (int)tc::layout_of(128, 64, true).total;
-    const int big_split = (int)tc::layout_of(128, 64, true, true).total;
     const int big_heap = (int)tc::layout_of(128, 64, false).total;
     cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, big_split);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big);
@@ -1213,10 +1104,9 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
     cudaError_t e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
-    const size_t smem3 = tc::layout_of(L.d, L.ksel, true).total;
-    const size_t smem3s = tc::layout_of(L.d, L.ksel, true, true).total;
+    const size_t smem2 = tc::layout_of(L.d, L.ksel, true).total;
     if (L.cand_v && L.cand_i && L.cand_meta) {
-        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem3s, s>>>(
+        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem2, s>>>(
             L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
@@ -1224,12 +1114,12 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
         tc::route_rows_finalize_kernel<<<fgrid, 32 * tc::kFinWarps, 0, s>>>(L, layer,
                                                                              use_list ? 1 : 0);
     } else {
-        tc::route_rows_tc_kernel<false><<<grid, tc::kPassThreads, smem3, s>>>(
+        tc::route_rows_tc_kernel<false><<<grid, tc::kPassThreads, smem2, s>>>(
             L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // rows whose three-pass certificate failed: exact heap selection
+    // rows the two-pass kernel could not finish: exact heap selection
     LedgerDev R = L;
     R.list = L.retry_list;
     R.head_count = L.retry_count;
