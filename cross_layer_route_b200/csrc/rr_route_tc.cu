@@ -65,8 +65,8 @@ constexpr long long kSpinLimit = 1ll << 31;
 constexpr int kGroups = 32;                // column groups per half row (two halves per row)
 constexpr int kTops = 4 * kGroups;         // group top-2 values per row
 constexpr int kTopStride = kTops + 1;      // padded row of the group tops in shared memory
-constexpr int kCap = 128;                  // kept scores per row (both column halves)
-constexpr int kStageCols = 16;             // columns per staging round of the collect pass
+constexpr int kCap = 120;                  // kept scores per row (both column halves)
+constexpr int kStageCols = 32;             // columns per staging round of the collect pass
 constexpr int kThrLowBit = 16;             // threshold search stops at this key bit
 // heap selection (retry path)
 constexpr int kBuf = 32;
@@ -85,7 +85,7 @@ struct Layout {
     int stages;
 };
 
-// two_pass: q | k | sel (96 KB: the group tops [kRows][kTopStride] f32 after
+// two_pass: q | k | sel (90 KB: the group tops [kRows][kTopStride] f32 after
 //           pass 0, then bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16) |
 //           stg [256 threads][kStageCols] f32 | rows | red (threshold and
 //           two kept counts per row)
@@ -893,14 +893,14 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const float T = thr_s[r];
 
         // pass 1: keep every valid score >= T.  Each thread builds a bit mask
-        // of its kept columns, stages the 16 scores of a round in shared
+        // of its kept columns, stages the 32 scores of a round in shared
         // memory (16-byte chunks swizzled by lane, so the stores do not
         // collide) and appends the kept ones: half 0 upward from slot 0, half
         // 1 downward from slot kCap-1; no slot leaves the buffer.
         float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
         uint16_t *bi = reinterpret_cast<uint16_t *>(smem + lay.bufi) + r;
         float *stg = reinterpret_cast<float *>(smem + lay.stg) + (ew * 32 + lane) * kStageCols;
-        const int sw = (lane >> 1) & 3;   // 16-byte chunk swizzle: 8 lanes, 8 distinct bank groups
+        const int sw = lane & 7;   // 16-byte chunk swizzle: 8 lanes, 8 distinct bank groups
         const int base = half ? kCap - 1 : 0;
         const int dir = half ? -1 : 1;
         int cnt = 0;
@@ -915,26 +915,30 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 #pragma unroll
             for (int hq = 0; hq < 64 / kStageCols; ++hq) {
                 const int o = hq * kStageCols;
-                uint32_t mask = 0u;
+                // four independent partial masks (short dependency chains)
+                uint32_t mk[4] = {0u, 0u, 0u, 0u};
                 if (lim >= 64) {
 #pragma unroll
-                    for (int jj = 0; jj < kStageCols; ++jj) mask |= v[o + jj] >= T ? (1u << jj) : 0u;
+                    for (int jj = 0; jj < kStageCols; ++jj)
+                        mk[jj & 3] |= v[o + jj] >= T ? (1u << jj) : 0u;
                 } else {
 #pragma unroll
                     for (int jj = 0; jj < kStageCols; ++jj)
-                        mask |= (o + jj < lim && v[o + jj] >= T) ? (1u << jj) : 0u;
+                        mk[jj & 3] |= (o + jj < lim && v[o + jj] >= T) ? (1u << jj) : 0u;
                 }
+                uint32_t mask = (mk[0] | mk[1]) | (mk[2] | mk[3]);
 #pragma unroll
                 for (int c4 = 0; c4 < kStageCols / 4; ++c4)
                     *reinterpret_cast<float4 *>(stg + ((c4 ^ sw) << 2)) =
                         make_float4(v[o + 4 * c4], v[o + 4 * c4 + 1], v[o + 4 * c4 + 2], v[o + 4 * c4 + 3]);
+                const int colo = col0 + o;
                 while (mask != 0u) {
                     const int jj = __ffs(mask) - 1;
                     mask &= mask - 1u;
                     if (cnt < kCap) {
                         const int sl = base + dir * cnt;
                         bv[sl * kRows] = stg[(((jj >> 2) ^ sw) << 2) + (jj & 3)];
-                        bi[sl * kRows] = (uint16_t)(col0 + o + jj);
+                        bi[sl * kRows] = (uint16_t)(colo + jj);
                     }
                     ++cnt;
                 }
