@@ -22,8 +22,8 @@ struct LedgerDev {
     int32_t *retry_count;   // [bh]        rows listed per head
     // candidate buffers of the split tensor-core path (null: the route kernel
     // finishes its rows itself); per 128-row block of one head:
-    float *cand_v = nullptr;       // [blocks, kCap, 128] kept scores
-    uint16_t *cand_i = nullptr;    // [blocks, kCap, 128] their key chunks
+    float *cand_v = nullptr;       // [blocks, 128, kCap] kept scores (row-contiguous)
+    uint16_t *cand_i = nullptr;    // [blocks, 128, kCap] their key chunks
     int32_t *cand_meta = nullptr;  // [blocks, 128] kept counts of the two halves, or -1
     int bh, nq, nk, d;
     int k, m, r, c, ksel;   // ksel = k + m

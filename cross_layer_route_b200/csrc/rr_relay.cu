@@ -5,9 +5,9 @@
 //
 //  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
 //      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
-//      row"), one warp per query row.  For d in {64, 128, 256} four lanes
-//      share a candidate (16-byte loads interleaved so that the four read 64
-//      contiguous bytes at a time; each keeps its quarter of q in registers);
+//      row"), one warp per query row.  For d in {64, 128, 256} eight lanes
+//      share a candidate (16-byte loads interleaved so that the eight read
+//      one 128-byte line at a time; each keeps its eighth of q in registers);
 //      other d use one lane per candidate.
 //  compact_flags: the prefix sum that compacts unstable row ids (§4.2), one
 //      CTA per head, writing an ascending per-head list and its length.
@@ -202,19 +202,21 @@ __global__ void finalize_layer_kernel(LedgerDev L, int layer, long long add_rows
 
 }  // namespace
 
-// Four lanes per candidate: lane quad g of the warp scores candidate
-// it*8 + g, each lane one quarter of the key row (R/4 bytes, R = d * elem
-// size, a multiple of 64), with its quarter of the query row in registers.
-// A load instruction of the warp touches 8 whole key rows -- 8 cache lines
-// instead of the 32 of one-lane-per-candidate.
+// Eight lanes per candidate: lane octet g of the warp scores candidate
+// it*4 + g, each lane an eighth of the key row (R/8 bytes, R = d * elem
+// size, a multiple of 128), with its eighth of the query row in registers.
+// Per load instruction an octet reads one whole 128-byte line, so the warp
+// touches 4 lines, each in full.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRescoreThreads)
-relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
+relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
     constexpr int E = Vec16<T>::kElems;         // elements per 16-byte load
-    constexpr int kChunks = D / E / 4;          // 16-byte loads per lane
+    constexpr int kLanes = 8;                   // lanes per candidate
+    constexpr int kChunks = D / E / kLanes;     // 16-byte loads per lane
+    static_assert(kChunks >= 1, "one 16-byte load per lane at least");
     __shared__ unsigned long long pair_sum[kRescoreWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quad = lane >> 2, part = lane & 3;
+    const int oct = lane >> 3, part = lane & 7;
     const long long rows = (long long)L.bh * L.nq;
     const long long grow = (long long)blockIdx.x * kRescoreWarps + warp;
     unsigned long long pairs = 0;
@@ -222,14 +224,14 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
         const int h = (int)(grow / L.nq);
         const int i = (int)(grow - (long long)h * L.nq);
         const int n_valid = valid_keys(i, L.nk, L.causal);
-        // this lane's quarter of q, as fp32: the 16-byte chunks part, part + 4,
-        // part + 8, ... (a quad reads 64 contiguous bytes per load)
+        // this lane's eighth of q, as fp32: the 16-byte chunks part, part + 8,
+        // ... (eight lanes read one 128-byte line per load)
         float qv[kChunks * E];
         {
             const uint4 *q4 = reinterpret_cast<const uint4 *>(Q + grow * D) + part;
 #pragma unroll
             for (int c = 0; c < kChunks; ++c) {
-                const uint4 u = __ldg(q4 + 4 * c);
+                const uint4 u = __ldg(q4 + kLanes * c);
                 if constexpr (E == 8) {
                     qv[c * 8 + 0] = __uint_as_float(u.x << 16); qv[c * 8 + 1] = __uint_as_float(u.x & 0xffff0000u);
                     qv[c * 8 + 2] = __uint_as_float(u.y << 16); qv[c * 8 + 3] = __uint_as_float(u.y & 0xffff0000u);
@@ -247,8 +249,8 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
         bool bad = false;
         int ncand = 0;
 #pragma unroll 2
-        for (int e0 = 0; e0 < L.c; e0 += 8) {
-            const int e = e0 + quad;
+        for (int e0 = 0; e0 < L.c; e0 += 32 / kLanes) {
+            const int e = e0 + oct;
             const int j = e < L.c ? idr[e] : -1;
             const bool valid = j >= 0 && j < n_valid;
             bad |= j >= n_valid || j < -1;
@@ -257,7 +259,7 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
                 const uint4 *k4 = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D) + part;
                 uint4 kv[kChunks];
 #pragma unroll
-                for (int c = 0; c < kChunks; ++c) kv[c] = __ldg(k4 + 4 * c);
+                for (int c = 0; c < kChunks; ++c) kv[c] = __ldg(k4 + kLanes * c);
 #pragma unroll
                 for (int c = 0; c < kChunks; ++c) {
                     const uint4 u = kv[c];
@@ -281,6 +283,7 @@ relay_rescore_quad_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restr
             float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             sc += __shfl_xor_sync(kFull, sc, 1);
             sc += __shfl_xor_sync(kFull, sc, 2);
+            sc += __shfl_xor_sync(kFull, sc, 4);
             if (valid && part == 0) {
                 if (e < L.k) amin = fminf(amin, sc);   // Eq. 6
                 else bmax = fmaxf(bmax, sc);           // Eq. 7
@@ -317,9 +320,9 @@ static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, u
     const T *Q = static_cast<const T *>(q);
     const T *K = static_cast<const T *>(k);
     switch (L.d) {
-        case 64: relay_rescore_quad_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        case 128: relay_rescore_quad_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        case 256: relay_rescore_quad_kernel<T, 256><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 64: relay_rescore_oct_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 128: relay_rescore_oct_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 256: relay_rescore_oct_kernel<T, 256><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
         default: relay_rescore_kernel<T, 0><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
     }
 }

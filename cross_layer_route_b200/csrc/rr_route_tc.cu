@@ -14,7 +14,7 @@
 // CTA layout (one CTA = one head x 128 query rows):
 //   warp 0     TMA producer: 128-key x d tiles of Kc (bf16, 128-byte
 //              swizzle) into a ring of shared-memory stages.
-//   warp 1     allocates 256 TMEM columns (two 128x128 fp32 accumulators);
+//   warp 1     allocates 512 TMEM columns (four 128x128 fp32 accumulators);
 //              one lane issues tcgen05.mma (M=128, N=128, K=16 per op) for
 //              every key tile and commits to mbarriers.
 //   warps 2-   epilogue, reading the score tile with tcgen05.ld; a warp may
@@ -55,18 +55,22 @@ namespace tc {
 
 constexpr int kRows = 128;
 constexpr int kKeys = 128;
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 4;
 constexpr int kHeapThreads = 32 * (2 + 4);     // heap kernel: 4 epilogue warps (one per row)
-constexpr int kPassThreads = 32 * (2 + 8);     // two-pass kernel: 8 epilogue warps (two per row)
-constexpr int kTmemCols = 256;
+constexpr int kEpiWarps = 16;                  // two-pass kernel: epilogue warps (four per row)
+constexpr int kPassThreads = 32 * (2 + kEpiWarps);
+constexpr int kAcc = 4;                       // TMEM accumulators (128 columns each)
+constexpr int kTmemCols = kAcc * 128;
+static_assert(kAcc >= kMaxStages, "a key stage is freed through the accumulator barriers");
 constexpr int kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr long long kSpinLimit = 1ll << 31;
 // two-pass selection
-constexpr int kGroups = 32;                // column groups per half row (two halves per row)
-constexpr int kTops = 4 * kGroups;         // group top-2 values per row
+constexpr int kGroups = 16;                // column groups per quarter row (four quarters per row)
+constexpr int kTops = 8 * kGroups;         // group top-2 values per row
 constexpr int kTopStride = kTops + 1;      // padded row of the group tops in shared memory
-constexpr int kCap = 120;                  // kept scores per row (both column halves)
-constexpr int kStageCols = 32;             // columns per staging round of the collect pass
+constexpr int kCap = 120;                  // kept scores per row
+constexpr int kBufStride = kRows + 1;      // padded row of the append buffers (slot-major)
+constexpr int kStageCols = 16;             // columns per staging round of the collect pass
 constexpr int kThrLowBit = 16;             // threshold search stops at this key bit
 // heap selection (retry path)
 constexpr int kBuf = 32;
@@ -85,10 +89,11 @@ struct Layout {
     int stages;
 };
 
-// two_pass: q | k | sel (90 KB: the group tops [kRows][kTopStride] f32 after
-//           pass 0, then bufv [kCap][kRows] f32 | bufi [kCap][kRows] u16) |
-//           stg [256 threads][kStageCols] f32 | rows | red (threshold and
-//           two kept counts per row)
+// two_pass: q | k | sel (91 KB: the group tops [kRows][kTopStride] f32 after
+//           pass 0, then bufv [kCap][kBufStride] f32 | bufi [kCap][kBufStride]
+//           u16, padded so that one row's slots fall in distinct banks) |
+//           stg [epilogue threads][kStageCols] f32 | rows | red (threshold
+//           and kept count per row)
 // heap:     q | k | heap [ksel][kRows] u64 | bufv [kBuf][kRows] f32 | bufi [kBuf][kRows] i32
 __host__ __device__ inline Layout layout_of(int d, int ksel, bool two_pass) {
     Layout s;
@@ -98,10 +103,10 @@ __host__ __device__ inline Layout layout_of(int d, int ksel, bool two_pass) {
     s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
     s.sel = o;
     if (two_pass) {
-        s.bufv = o; o = up(o + kCap * kRows * 4, 16);
-        s.bufi = o; o = up(o + kCap * kRows * 2, 16);
+        s.bufv = o; o = up(o + kCap * kBufStride * 4, 16);
+        s.bufi = o; o = up(o + kCap * kBufStride * 2, 16);
         o = up(s.sel + (kRows * kTopStride * 4 > o - s.sel ? kRows * kTopStride * 4 : o - s.sel), 16);
-        s.stg = o;  o = up(o + 256 * kStageCols * 4, 16);
+        s.stg = o;  o = up(o + kEpiWarps * 32 * kStageCols * 4, 16);
     } else {
         s.stg = 0;
         o = up(o + kRows * ksel * 8, 16);   // the heap, at sel
@@ -109,8 +114,8 @@ __host__ __device__ inline Layout layout_of(int d, int ksel, bool two_pass) {
         s.bufi = o; o = up(o + kRows * kBuf * 4, 16);
     }
     s.rows = o; o = up(o + kRows * 4, 16);
-    s.red = o;  o = up(o + (two_pass ? 3 * kRows * 4 : 0), 16);
-    s.bars = o; o = up(o + 8 * (2 * kMaxStages + 5), 16);
+    s.red = o;  o = up(o + (two_pass ? 2 * kRows * 4 : 0), 16);
+    s.bars = o; o = up(o + 8 * (2 * kMaxStages + 2 * kAcc + 1), 16);
     s.misc = o; o = up(o + 16, 16);
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
@@ -141,12 +146,26 @@ __device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// The same test, letting the thread sleep up to ~8 us until the phase
+// completes (a waiting warp then takes no issue slots from the warps that
+// share its scheduler).
+__device__ __forceinline__ bool mbar_test_sleep(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(saddr(b)), "r"(parity), "r"(8192u)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase of the given parity.  Returns false on timeout
 // (and raises the CTA's abort flag) or when another role already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag) {
     if (mbar_test(b, parity)) return true;
     const long long t0 = clock64();
-    while (!mbar_test(b, parity)) {
+    while (!mbar_test_sleep(b, parity)) {
         if (*abort_flag) return false;
         if (clock64() - t0 > kSpinLimit) {
             *abort_flag = 1;
@@ -242,7 +261,7 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKe
 struct Cta {
     unsigned char *q_s, *k_s;
     int *rows_s;
-    uint64_t *full, *empty, *acc_full, *acc_empty, *mma_done;
+    uint64_t *full, *acc_full, *acc_empty, *mma_done;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int stages, n_rows, ntiles;
@@ -266,10 +285,9 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Lay
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
     c.stages = lay.stages;
     c.full = bars;
-    c.empty = bars + kMaxStages;
     c.acc_full = bars + 2 * kMaxStages;
-    c.acc_empty = bars + 2 * kMaxStages + 2;
-    c.mma_done = bars + 2 * kMaxStages + 4;
+    c.acc_empty = bars + 2 * kMaxStages + kAcc;
+    c.mma_done = bars + 2 * kMaxStages + 2 * kAcc;
     c.tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.misc);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + lay.misc + 4);
     c.n_rows = min(kRows, count - row0);
@@ -282,9 +300,8 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Lay
     if (tid == 0) {
         for (int s = 0; s < c.stages; ++s) {
             mbar_init(&c.full[s], 1);
-            mbar_init(&c.empty[s], 1);
         }
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < kAcc; ++a) {
             mbar_init(&c.acc_full[a], 1);
             mbar_init(&c.acc_empty[a], (blockDim.x >> 5) - 2);
         }
@@ -339,7 +356,13 @@ __device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int pa
     int issued = 0;
     for (int g = 0; g < total; ++g) {
         const int s = g % c.stages;
-        if (!mbar_wait(&c.empty[s], ((g / c.stages) & 1) ^ 1, c.abort_flag)) break;
+        // stage s is free once tile g - stages is scored (its accumulator
+        // barrier; the ring never runs more accumulators ahead than exist,
+        // kAcc >= stages, so that barrier cannot have moved on two phases)
+        if (g >= c.stages) {
+            const int gp = g - c.stages;
+            if (!mbar_wait(&c.acc_full[gp % kAcc], (gp / kAcc) & 1, c.abort_flag)) break;
+        }
         mbar_expect_tx(&c.full[s], stage_bytes);
         const int t = tile_of(g, c.ntiles, passes);
         for (int kb = 0; kb < (d >> 6); ++kb)
@@ -356,25 +379,34 @@ __device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int pa
     }
 }
 
-// MMA issuer (one lane): score tile g into accumulator g % 2.
+// MMA issuer (one lane): score tile g into accumulator g % kAcc.
+// The descriptor of a K-major operand at byte offset `off` from another's
+// start is that descriptor plus off / 16 (the start address field, bits
+// 0..13, holds address / 16 and shared memory stays below 256 KB).
+template <int kSteps>
+__device__ __forceinline__ void mma_tile(uint32_t d_tmem, uint64_t qdesc, uint64_t kdesc) {
+#pragma unroll
+    for (int kk = 0; kk < kSteps; ++kk) {
+        const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
+        tc_mma_bf16(d_tmem, qdesc + off16, kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
+    }
+}
+
 __device__ void mma_issuer(Cta &c, int d, int passes) {
     const int total = total_tiles(c.ntiles, passes);
-    const uint32_t q_addr = saddr(c.q_s), k_addr = saddr(c.k_s);
+    const uint64_t qdesc = sw128_desc(saddr(c.q_s));
+    const uint32_t k_addr = saddr(c.k_s);
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
     for (int g = 0; g < total; ++g) {
-        const int s = g % c.stages, a = g & 1;
+        const int s = g % c.stages, a = g % kAcc;
         if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
-        if (!mbar_wait(&c.acc_empty[a], ((g >> 1) & 1) ^ 1, c.abort_flag)) break;
+        if (!mbar_wait(&c.acc_empty[a], ((g / kAcc) & 1) ^ 1, c.abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
-        const uint32_t kst = k_addr + (uint32_t)s * stage_bytes;
-        for (int kk = 0; kk < (d >> 4); ++kk) {
-            const uint32_t off = (uint32_t)((kk >> 2) * kSubTileBytes + (kk & 3) * 32);
-            tc_mma_bf16(d_tmem, sw128_desc(q_addr + off), sw128_desc(kst + off), kIdesc,
-                        kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&c.empty[s]);
-        tc_commit(&c.acc_full[a]);
+        const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
+        if (d == 128) mma_tile<8>(d_tmem, qdesc, kdesc);
+        else mma_tile<4>(d_tmem, qdesc, kdesc);
+        tc_commit(&c.acc_full[a]);   // frees accumulator a's scores and stage s
     }
     tc_commit(c.mma_done);
     const long long t0 = clock64();
@@ -396,7 +428,7 @@ __device__ __forceinline__ void cta_teardown(Cta &c, const LedgerDev &L) {
 
 // Epilogue helpers: wait for accumulator g (warp-uniform outcome) / hand it back.
 __device__ __forceinline__ bool acc_wait(Cta &c, int g) {
-    bool ok = mbar_wait(&c.acc_full[g & 1], (g >> 1) & 1, c.abort_flag);
+    bool ok = mbar_wait(&c.acc_full[g % kAcc], (g / kAcc) & 1, c.abort_flag);
     ok = __all_sync(kFull, ok);   // the warp leaves together (tcgen05.ld is .sync.aligned)
     if (ok) tc_fence_after();
     return ok;
@@ -404,7 +436,7 @@ __device__ __forceinline__ bool acc_wait(Cta &c, int g) {
 __device__ __forceinline__ void acc_release(Cta &c, int g) {
     tc_fence_before();
     __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&c.acc_empty[g & 1]);
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&c.acc_empty[g % kAcc]);
 }
 
 // Random sentinels (RouteRelay §3.1 item 2, §3.4) of one row, one thread:
@@ -520,7 +552,7 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         bool ok = true;
         for (int t = 0; t < c.ntiles && ok; ++t) {
             if (!(ok = acc_wait(c, t))) break;
-            const uint32_t tbase = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)((t & 1) * kKeys);
+            const uint32_t tbase = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)((t % kAcc) * kKeys);
 #pragma unroll 1
             for (int ch = 0; ch < kKeys / 32; ++ch) {
                 float v[32];
@@ -605,14 +637,12 @@ __device__ __forceinline__ uint64_t cand_key(float v, int j) {
     return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
 }
 
-// One warp, every lane with the same arguments.  The row's kept scores sit in
-// a two-ended buffer: c0 at slots 0.., c1 at slots kCap-1 downwards, read
-// through getv(slot) / geti(slot).  Needs c0 + c1 <= kCap and at least
-// min(k + m, valid keys) of them.
+// One warp, every lane with the same arguments.  The row's `run` kept scores
+// are read through getv(e) / geti(e), e < run <= kCap; they include the
+// row's min(k + m, valid keys) best.
 template <typename GetV, typename GetI>
-__device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h, int row, int c0,
-                                           int c1, GetV getv, GetI geti, FinWarp &w, int lane) {
-    const int run = c0 + c1;
+__device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h, int row, int run,
+                                           GetV getv, GetI geti, FinWarp &w, int lane) {
     const int n_valid = valid_keys(row, L.nk, L.causal);
     const uint32_t lt_mask = (1u << lane) - 1u;
 
@@ -627,9 +657,8 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
         v[i] = 0.f;
         jc[i] = -1;
         if (live[i]) {
-            const int sl = e < c0 ? e : kCap - 1 - (e - c0);
-            v[i] = getv(sl);
-            jc[i] = geti(sl);
+            v[i] = getv(e);
+            jc[i] = geti(e);
             mx = fmaxf(mx, v[i]);
             mn = fminf(mn, v[i]);
         }
@@ -776,10 +805,10 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
 }
 
 // ---- two-pass kernel (the main path) ---------------------------------------------
-// kSplit: the kernel ends by writing each row's kept scores (both halves'
-// buffers, as they are) and their counts to the candidate buffers;
-// route_rows_finalize_kernel finishes the rows.  Otherwise the epilogue warps
-// finish them here (one warp per row, from shared memory).
+// kSplit: the kernel ends by writing each row's kept scores and their count
+// to the candidate buffers; route_rows_finalize_kernel finishes the rows.
+// Otherwise the epilogue warps finish them here (one warp per row, from
+// shared memory).
 template <bool kSplit>
 __global__ void __launch_bounds__(kPassThreads, 1)
 route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
@@ -799,43 +828,44 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(c, d, 2);
     } else {
-        // Two warps per TMEM sub-partition: half 0 reads columns 0..63 of
-        // every tile, half 1 columns 64..127.  The 256 epilogue threads meet
-        // at named barrier 1 between phases (every one of them reaches every
-        // barrier, also after a timeout, so none can be left waiting).
-        const int ew = warp - 2;   // epilogue warp 0..7
+        // Four warps per TMEM sub-partition: quarter qt reads columns
+        // 32*qt..32*qt+31 of every tile.  The epilogue threads meet at named
+        // barrier 1 between phases (every one of them reaches every barrier,
+        // also after a timeout, so none can be left waiting).
+        const int ew = warp - 2;   // epilogue warp 0..kEpiWarps-1
         const int sub = warp & 3;
-        const int half = ew >> 2;
+        const int qt = ew >> 2;
         const int r = sub * 32 + lane;
         const int row = c.rows_s[r];
         const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
-        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(half * 64);
+        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(qt * 32);
         const int nt = c.ntiles;
         bool ok = true;
         int g = 0;
-        auto epi_sync = [] { asm volatile("bar.sync 1, 256;" ::: "memory"); };
+        auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
+        int *rowcnt = reinterpret_cast<int *>(smem + lay.red) + kRows;   // [kRows] kept per row
 
         // pass 0: the two largest valid scores of each column group (this
-        // half's columns, group = column mod 32)
+        // quarter's columns, group = column mod 16)
         float m1[kGroups], m2[kGroups];
 #pragma unroll
         for (int q = 0; q < kGroups; ++q) { m1[q] = -INFINITY; m2[q] = -INFINITY; }
         for (int i = 0; i < nt && ok; ++i, ++g) {
             if (!(ok = acc_wait(c, g))) break;
-            float v[64];
-            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            float v[32];
+            tc_ld32(lane_base + (uint32_t)((g % kAcc) * kKeys), v);
             acc_release(c, g);   // the scores are in registers: the MMA may reuse the accumulator
-            const int col0 = i * kKeys + half * 64;
-            if (col0 + 64 <= n_valid) {
+            const int col0 = i * kKeys + qt * 32;
+            if (col0 + 32 <= n_valid) {
 #pragma unroll
-                for (int jj = 0; jj < 64; ++jj) {
+                for (int jj = 0; jj < 32; ++jj) {
                     const int q = jj & (kGroups - 1);
                     m2[q] = fmaxf(m2[q], fminf(m1[q], v[jj]));
                     m1[q] = fmaxf(m1[q], v[jj]);
                 }
             } else {
 #pragma unroll
-                for (int jj = 0; jj < 64; ++jj) {
+                for (int jj = 0; jj < 32; ++jj) {
                     const int q = jj & (kGroups - 1);
                     const float x = col0 + jj < n_valid ? v[jj] : -INFINITY;
                     m2[q] = fmaxf(m2[q], fminf(m1[q], x));
@@ -843,24 +873,25 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 }
             }
         }
-        // the row's 128 group tops: [r][kTopStride], this half at half * 64
+        // the row's 128 group tops: [r][kTopStride], this quarter at qt * 32
         float *tops = reinterpret_cast<float *>(smem + lay.sel);
 #pragma unroll
         for (int q = 0; q < kGroups; ++q) {
-            tops[r * kTopStride + half * 2 * kGroups + q] = m1[q];
-            tops[r * kTopStride + half * 2 * kGroups + kGroups + q] = m2[q];
+            tops[r * kTopStride + qt * 2 * kGroups + q] = m1[q];
+            tops[r * kTopStride + qt * 2 * kGroups + kGroups + q] = m2[q];
         }
+        if (qt == 0) rowcnt[r] = 0;
         epi_sync();
 
-        // threshold T of each row (one warp per row, 16 rows per warp): the
+        // threshold T of each row (kRows / kEpiWarps rows per warp): the
         // largest key K, a multiple of 2^kThrLowBit, that at least k + m of
         // the group tops' order-preserving keys reach.  At least k + m
-        // distinct valid scores are >= T, so T is at most the row's
-        // (k + m)-th best score.  Rows with at most k + m valid keys keep
-        // all of them (T = -inf).
+        // distinct valid scores are >= T, so T is at most the row's (k + m)-th
+        // best score.  Rows with at most k + m valid keys keep all of them
+        // (T = -inf).
         float *thr_s = reinterpret_cast<float *>(smem + lay.red);   // [kRows]
         {
-            constexpr int kRowsPerWarp = kRows / 8;
+            constexpr int kRowsPerWarp = kRows / kEpiWarps;
             uint32_t key[kRowsPerWarp][4], K[kRowsPerWarp];
 #pragma unroll
             for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
@@ -869,7 +900,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 for (int i = 0; i < 4; ++i) key[k2][i] = ord32(tops[rr * kTopStride + i * 32 + lane]);
                 K[k2] = 0u;
             }
-            // all 16 rows' searches interleaved (independent chains)
+            // the rows' searches interleaved (independent chains)
             for (int bit = 31; bit >= kThrLowBit; --bit) {
 #pragma unroll
                 for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
@@ -893,31 +924,28 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const float T = thr_s[r];
 
         // pass 1: keep every valid score >= T.  Each thread builds a bit mask
-        // of its kept columns, stages the 32 scores of a round in shared
-        // memory (16-byte chunks swizzled by lane, so the stores do not
-        // collide) and appends the kept ones: half 0 upward from slot 0, half
-        // 1 downward from slot kCap-1; no slot leaves the buffer.
+        // of its kept columns for a round of 16, stages the round's scores
+        // in shared memory (16-byte chunks swizzled by lane, so the stores do
+        // not collide), claims that many slots of the row's buffer with one
+        // atomic and appends the kept ones; no slot leaves the buffer.
         float *bv = reinterpret_cast<float *>(smem + lay.bufv) + r;
         uint16_t *bi = reinterpret_cast<uint16_t *>(smem + lay.bufi) + r;
         float *stg = reinterpret_cast<float *>(smem + lay.stg) + (ew * 32 + lane) * kStageCols;
-        const int sw = lane & 7;   // 16-byte chunk swizzle: 8 lanes, 8 distinct bank groups
-        const int base = half ? kCap - 1 : 0;
-        const int dir = half ? -1 : 1;
-        int cnt = 0;
+        const int sw = (lane >> 1) & 3;   // 8 lanes of a 64-byte row stride: 8 distinct bank groups
         for (int i = 0; i < nt && ok; ++i, ++g) {
             if (!(ok = acc_wait(c, g))) break;
             const int t = tile_of(g, nt, 2);
-            float v[64];
-            tc_ld64(lane_base + (uint32_t)((g & 1) * kKeys), v);
+            float v[32];
+            tc_ld32(lane_base + (uint32_t)((g % kAcc) * kKeys), v);
             acc_release(c, g);
-            const int col0 = t * kKeys + half * 64;
+            const int col0 = t * kKeys + qt * 32;
             const int lim = n_valid - col0;   // columns jj < lim are valid
 #pragma unroll
-            for (int hq = 0; hq < 64 / kStageCols; ++hq) {
+            for (int hq = 0; hq < 32 / kStageCols; ++hq) {
                 const int o = hq * kStageCols;
                 // four independent partial masks (short dependency chains)
                 uint32_t mk[4] = {0u, 0u, 0u, 0u};
-                if (lim >= 64) {
+                if (lim >= 32) {
 #pragma unroll
                     for (int jj = 0; jj < kStageCols; ++jj)
                         mk[jj & 3] |= v[o + jj] >= T ? (1u << jj) : 0u;
@@ -931,72 +959,74 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 for (int c4 = 0; c4 < kStageCols / 4; ++c4)
                     *reinterpret_cast<float4 *>(stg + ((c4 ^ sw) << 2)) =
                         make_float4(v[o + 4 * c4], v[o + 4 * c4 + 1], v[o + 4 * c4 + 2], v[o + 4 * c4 + 3]);
-                const int colo = col0 + o;
-                while (mask != 0u) {
-                    const int jj = __ffs(mask) - 1;
-                    mask &= mask - 1u;
-                    if (cnt < kCap) {
-                        const int sl = base + dir * cnt;
-                        bv[sl * kRows] = stg[(((jj >> 2) ^ sw) << 2) + (jj & 3)];
-                        bi[sl * kRows] = (uint16_t)(colo + jj);
-                    }
-                    ++cnt;
+                if (mask != 0u) {
+                    int sl = atomicAdd(&rowcnt[r], __popc(mask));
+                    const int colo = col0 + o;
+                    do {
+                        const int jj = __ffs(mask) - 1;
+                        mask &= mask - 1u;
+                        if (sl < kCap) {
+                            bv[sl * kBufStride] = stg[(((jj >> 2) ^ sw) << 2) + (jj & 3)];
+                            bi[sl * kBufStride] = (uint16_t)(colo + jj);
+                        }
+                        ++sl;
+                    } while (mask != 0u);
                 }
             }
         }
-        int *rcnt = reinterpret_cast<int *>(smem + lay.red) + kRows;   // [2][kRows]
-        rcnt[half * kRows + r] = cnt;
         epi_sync();
 
-        // A row is finished from its buffer when every wait succeeded, the
-        // two halves' scores fit it without meeting (c0 + c1 <= kCap - 2),
-        // and at least min(k + m, valid keys) were kept; other rows go to
-        // the retry list (exact heap selection).
+        // A row is finished from its buffer when every wait succeeded, its
+        // kept scores fit the buffer, and at least min(k + m, valid keys) were
+        // kept; other rows go to the retry list (exact heap selection).
         const bool cta_ok = *c.abort_flag == 0;
-        auto row_good = [&](int rw, int nv, int k0, int k1) {
-            const int kept = k0 + k1;
-            return cta_ok && rw >= 0 && kept <= kCap - 2 && (nv <= ksel ? kept == nv : kept >= ksel);
+        auto row_good = [&](int rw, int nv, int kept) {
+            return cta_ok && rw >= 0 && kept <= kCap && (nv <= ksel ? kept == nv : kept >= ksel);
         };
-        const int c0 = rcnt[r], c1 = rcnt[kRows + r];
-        const bool good = row_good(row, n_valid, c0, c1);
-        if (half == 0 && ok && row >= 0 && !good) {
+        const int kept = rowcnt[r];
+        const bool good = row_good(row, n_valid, kept);
+        if (qt == 0 && ok && row >= 0 && !good) {
             const int pos = atomicAdd(&L.retry_count[h], 1);
             L.retry_list[(size_t)h * L.nq + pos] = row;
             atomicAdd(&L.counters[10], 1ULL);
         }
 
         if constexpr (kSplit) {
-            // candidate slot (blk, slot, r) at cand[(blk * kCap + slot) * kRows + r];
-            // meta (blk, r) = c0 | c1 << 16, or -1 when the row has nothing to finish
+            // candidates of row r of block blk at cand[(blk * kRows + r) * kCap + e];
+            // meta (blk, r) = the kept count, or -1 when the row has nothing to finish
             const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-            if (half == 0) L.cand_meta[blk * kRows + r] = good ? (c0 | (c1 << 16)) : -1;
-            if (good) {
-                // half 0 writes slots 0..kCap/2-1, half 1 the rest (only used ones)
-                float *gv = L.cand_v + blk * kCap * kRows + r;
-                uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
-                const int s0 = half * (kCap / 2);
-                for (int sl = s0; sl < s0 + kCap / 2; ++sl) {
-                    if (sl < c0 || sl >= kCap - c1) {
-                        gv[sl * kRows] = bv[sl * kRows];
-                        gi[sl * kRows] = bi[sl * kRows];
-                    }
+            if (qt == 0) L.cand_meta[blk * kRows + r] = good ? kept : -1;
+            // one warp per row: 128-byte stores of the row's slots
+            const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
+            const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
+            for (int k2 = 0; k2 < kRows / kEpiWarps; ++k2) {
+                const int rr = ew * (kRows / kEpiWarps) + k2;
+                const int rowr = c.rows_s[rr];
+                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
+                const int kr = rowcnt[rr];
+                if (!row_good(rowr, nv, kr)) continue;   // warp-uniform
+                float *gv = L.cand_v + (blk * kRows + rr) * kCap;
+                uint16_t *gi = L.cand_i + (blk * kRows + rr) * kCap;
+                for (int e = lane; e < kr; e += 32) {
+                    gv[e] = bvb[e * kBufStride + rr];
+                    gi[e] = bib[e * kBufStride + rr];
                 }
             }
         } else {
-            // finish the rows here: warp ew takes rows ew*16 .. ew*16+15, its
+            // finish the rows here (kRows / kEpiWarps per warp), the warps'
             // scratch in the query/key buffers (every MMA is done)
             FinWarp &fw = reinterpret_cast<FinWarp *>(smem + lay.q)[ew];
             const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
             const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
-            for (int k2 = 0; k2 < kRows / 8; ++k2) {
-                const int rr = ew * (kRows / 8) + k2;
+            for (int k2 = 0; k2 < kRows / kEpiWarps; ++k2) {
+                const int rr = ew * (kRows / kEpiWarps) + k2;
                 const int rowr = c.rows_s[rr];
                 const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
-                const int k0 = rcnt[rr], k1 = rcnt[kRows + rr];
-                if (!row_good(rowr, nv, k0, k1)) continue;   // warp-uniform
+                const int kr = rowcnt[rr];
+                if (!row_good(rowr, nv, kr)) continue;   // warp-uniform
                 finish_row(
-                    L, layer, h, rowr, k0, k1, [&](int sl) { return bvb[sl * kRows + rr]; },
-                    [&](int sl) { return (int)bib[sl * kRows + rr]; }, fw, lane);
+                    L, layer, h, rowr, kr, [&](int e) { return bvb[e * kBufStride + rr]; },
+                    [&](int e) { return (int)bib[e * kBufStride + rr]; }, fw, lane);
             }
         }
     }
@@ -1019,11 +1049,11 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
     const int meta = L.cand_meta[blk * kRows + r];
     if (meta < 0) return;   // no row, or a row left to the retry path
     const int row = use_list ? L.list[(size_t)h * L.nq + row0 + r] : row0 + r;
-    const float *gv = L.cand_v + blk * kCap * kRows + r;
-    const uint16_t *gi = L.cand_i + blk * kCap * kRows + r;
+    const float *gv = L.cand_v + (blk * kRows + r) * kCap;
+    const uint16_t *gi = L.cand_i + (blk * kRows + r) * kCap;
     finish_row(
-        L, layer, h, row, meta & 0xffff, meta >> 16, [&](int sl) { return gv[sl * kRows]; },
-        [&](int sl) { return (int)gi[sl * kRows]; }, fw_all[warp], lane);
+        L, layer, h, row, meta, [&](int e) { return gv[e]; }, [&](int e) { return (int)gi[e]; },
+        fw_all[warp], lane);
 }
 
 // ---- host side -----------------------------------------------------------------
@@ -1057,7 +1087,7 @@ bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
     const tc::Layout layh = tc::layout_of(L.d, L.ksel, false);
     return lay.total <= 232448 && layh.total <= 232448 &&
-           lay.sel - lay.q >= (uint32_t)(tc::kFinWarps * sizeof(tc::FinWarp));
+           lay.sel - lay.q >= (uint32_t)(tc::kEpiWarps * sizeof(tc::FinWarp));
 }
 
 size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
