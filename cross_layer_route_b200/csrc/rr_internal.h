@@ -62,6 +62,10 @@ cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, cons
                               int layer, bool use_list, cudaStream_t s);
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
                                  int layer, cudaStream_t s);
+// Relay rescoring from dense tensor-core score tiles (rr_route_tc.cu); used
+// for the problems route_rows_tc_supported accepts.
+cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k,
+                                    cudaStream_t s);
 cudaError_t launch_compact(const LedgerDev &L, cudaStream_t s);
 cudaError_t launch_finalize(const LedgerDev &L, int layer, long long add_rows,
                             long long add_pairs, long long add_full_pairs, cudaStream_t s);

@@ -330,6 +330,7 @@ static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, u
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
                                  int layer, cudaStream_t s) {
     (void)layer;
+    if (route_rows_tc_supported(L, dtype)) return launch_relay_rescore_tc(L, q, k, s);
     const long long rows = (long long)L.bh * L.nq;
     const unsigned grid = (unsigned)((rows + kRescoreWarps - 1) / kRescoreWarps);
     if (dtype == kBF16) rescore_dispatch<__nv_bfloat16>(L, q, k, grid, s);

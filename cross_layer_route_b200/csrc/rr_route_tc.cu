@@ -1056,6 +1056,150 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
         fw_all[warp], lane);
 }
 
+// ---- relay rescoring on the tensor cores ---------------------------------------
+// The relay test of RouteRelay §3.2 (Eq. 5-8) for every row of a head: alpha =
+// min over the row's route ids of s_ij, beta = max over its sentinel ids
+// (near-miss and random), flag = !(alpha > beta + gamma); a stable row keeps
+// its ids and stores alpha.  The candidates' scores are read from dense
+// 128 x 128 score tiles (one MMA pass over the row block's key tiles): on
+// B200 the tensor cores score a whole tile in about the time it takes to
+// gather the 80 candidate key rows of a few query rows.  Each row's
+// candidates are marked in two bitmaps (route, sentinel) of one 2048-column
+// segment at a time; the epilogue folds every marked score of a tile into the
+// row's running min / max.
+constexpr int kSegCols = 2048;                  // key columns per bitmap segment
+constexpr int kSegWords = kSegCols / 32;
+constexpr int kSegStride = kSegWords + 1;       // padded row: distinct banks across rows
+
+__host__ __device__ inline Layout rescore_layout(int d) {
+    Layout s;
+    s.stages = d == 64 ? 4 : 3;
+    uint32_t o = 0;
+    s.q = o;    o = up(o + kRows * d * 2, 1024);
+    s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
+    s.sel = o;  o = up(o + 2 * kRows * kSegStride * 4, 16);   // route bits | sentinel bits
+    s.bufv = s.bufi = s.stg = 0;
+    s.rows = o; o = up(o + kRows * 4, 16);
+    s.red = o;  o = up(o + 3 * 4 * kRows * 4, 16);   // per quarter: alpha, beta, candidates | bad
+    s.bars = o; o = up(o + 8 * (2 * kMaxStages + 2 * kAcc + 1), 16);
+    s.misc = o; o = up(o + 16, 16);
+    s.total = o + 1024;
+    return s;
+}
+
+__global__ void __launch_bounds__(kPassThreads, 1)
+relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+                        const __grid_constant__ CUtensorMap tmap_k) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const int d = L.d;
+    const Layout lay = rescore_layout(d);
+    Cta c;
+    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, 0)) return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+
+    if (warp == 0) {
+        if (lane == 0) producer(c, &tmap_k, d, h, 1);
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(c, d, 1);
+    } else {
+        const int ew = warp - 2;
+        const int sub = warp & 3;
+        const int qt = ew >> 2;   // quarter of the tile's columns
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
+        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(qt * 32);
+        const int nt = c.ntiles;
+        auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
+        uint32_t *rbits = reinterpret_cast<uint32_t *>(smem + lay.sel);   // [kRows][kSegStride]
+        uint32_t *sbits = rbits + kRows * kSegStride;
+        const int32_t *idr = row >= 0 ? L.ids + ((size_t)h * L.nq + row) * L.c : nullptr;
+
+        // this quarter's share of the row's ids: count the valid candidates
+        // (Eq. 5) and flag out-of-range ids
+        int ncand = 0;
+        bool bad = false;
+        if (row >= 0) {
+            for (int e = qt; e < L.c; e += 4) {
+                const int j = idr[e];
+                ncand += (j >= 0 && j < n_valid) ? 1 : 0;
+                bad |= j >= n_valid || j < -1;
+            }
+        }
+        float amin = INFINITY, bmax = -INFINITY;
+        bool ok = true;
+        int g = 0;
+        const int nseg = (nt * kKeys + kSegCols - 1) / kSegCols;
+        for (int sg = 0; sg < nseg; ++sg) {
+            for (int w = qt; w < kSegWords; w += 4) {
+                rbits[r * kSegStride + w] = 0u;
+                sbits[r * kSegStride + w] = 0u;
+            }
+            epi_sync();
+            if (row >= 0) {
+                for (int e = qt; e < L.c; e += 4) {
+                    const int j = idr[e];
+                    if (j >= 0 && j < n_valid && j / kSegCols == sg) {
+                        const int jj = j - sg * kSegCols;
+                        atomicOr(&(e < L.k ? rbits : sbits)[r * kSegStride + (jj >> 5)], 1u << (jj & 31));
+                    }
+                }
+            }
+            epi_sync();
+            const int t_end = min(nt, (sg + 1) * (kSegCols / kKeys));
+            for (; g < t_end && ok; ++g) {   // one pass: tile index = g
+                if (!(ok = acc_wait(c, g))) break;
+                float v[32];
+                tc_ld32(lane_base + (uint32_t)((g % kAcc) * kKeys), v);
+                acc_release(c, g);
+                const int wi = (g * kKeys + qt * 32 - sg * kSegCols) >> 5;
+                const uint32_t rw = rbits[r * kSegStride + wi];
+                const uint32_t sw = sbits[r * kSegStride + wi];
+#pragma unroll
+                for (int jj = 0; jj < 32; ++jj) {
+                    amin = fminf(amin, ((rw >> jj) & 1u) ? v[jj] : INFINITY);   // Eq. 6
+                    bmax = fmaxf(bmax, ((sw >> jj) & 1u) ? v[jj] : -INFINITY);  // Eq. 7
+                }
+            }
+            epi_sync();   // the segment's bitmaps are no longer read
+        }
+
+        float *red_a = reinterpret_cast<float *>(smem + lay.red);   // [4][kRows]
+        float *red_b = red_a + 4 * kRows;
+        int *red_n = reinterpret_cast<int *>(red_b + 4 * kRows);
+        red_a[qt * kRows + r] = amin;
+        red_b[qt * kRows + r] = bmax;
+        red_n[qt * kRows + r] = ncand | (bad ? (1 << 30) : 0);
+        epi_sync();
+        const bool cta_ok = *c.abort_flag == 0;
+        unsigned pairs = 0;
+        if (qt == 0) {
+            float a = red_a[r], b = red_b[r];
+            int n = red_n[r];
+            for (int q = 1; q < 4; ++q) {
+                a = fminf(a, red_a[q * kRows + r]);
+                b = fmaxf(b, red_b[q * kRows + r]);
+                n |= red_n[q * kRows + r] & (1 << 30);
+                n += red_n[q * kRows + r] & ((1 << 30) - 1);
+            }
+            if (cta_ok && row >= 0) {
+                const size_t grow = (size_t)h * L.nq + row;
+                const bool refresh = !(a > b + L.gamma);   // Eq. 8
+                L.flags[grow] = refresh ? 1 : 0;
+                if (!refresh) L.alpha[grow] = a;
+                if (n & (1 << 30)) atomicOr(&L.counters[2], 1ULL);
+                pairs = (unsigned)(n & ((1 << 30) - 1));
+            }
+            const unsigned wsum = __reduce_add_sync(kFull, pairs);
+            if (lane == 0 && wsum) atomicAdd(&L.counters[1], (unsigned long long)wsum);
+        }
+    }
+    cta_teardown(c, L);
+}
+
 // ---- host side -----------------------------------------------------------------
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
@@ -1086,7 +1230,7 @@ bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     // query/key buffers
     const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
     const tc::Layout layh = tc::layout_of(L.d, L.ksel, false);
-    return lay.total <= 232448 && layh.total <= 232448 &&
+    return lay.total <= 232448 && layh.total <= 232448 && tc::rescore_layout(L.d).total <= 232448 &&
            lay.sel - lay.q >= (uint32_t)(tc::kEpiWarps * sizeof(tc::FinWarp));
 }
 
@@ -1119,23 +1263,44 @@ cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc::route_rows_tc_heap_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big_heap);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::relay_rescore_tc_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc::rescore_layout(128).total);
     return e;
 }
 
-cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
-                                 bool use_list, cudaStream_t s) {
+// Tensor map of Kc [bh, nk, d] bf16: boxes of 128 keys x 64 dims, 128-byte swizzle.
+static cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map) {
     tc::EncodeTiledFn enc = tc::encode_fn();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap map;
     const cuuint64_t dims[3] = {(cuuint64_t)L.d, (cuuint64_t)L.nk, (cuuint64_t)L.bh};
     const cuuint64_t strides[2] = {(cuuint64_t)L.d * 2, (cuuint64_t)L.nk * L.d * 2};
     const cuuint32_t box[3] = {64u, (cuuint32_t)tc::kKeys, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
-    const CUresult cr = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims,
+    const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
-    cudaError_t e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
+    return cr == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k,
+                                    cudaStream_t s) {
+    CUtensorMap map;
+    cudaError_t e = key_tensor_map(L, k, &map);
+    if (e != cudaSuccess) return e;
+    dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
+    tc::relay_rescore_tc_kernel<<<grid, tc::kPassThreads, tc::rescore_layout(L.d).total, s>>>(
+        L, static_cast<const __nv_bfloat16 *>(q), map);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
+                                 bool use_list, cudaStream_t s) {
+    CUtensorMap map;
+    cudaError_t e = key_tensor_map(L, k, &map);
+    if (e != cudaSuccess) return e;
+    e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     const size_t smem2 = tc::layout_of(L.d, L.ksel, true).total;
