@@ -1070,6 +1070,7 @@ route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
 constexpr int kSegCols = 2048;                  // key columns per bitmap segment
 constexpr int kSegWords = kSegCols / 32;
 constexpr int kSegStride = kSegWords + 1;       // padded row: distinct banks across rows
+constexpr int kRescoreIdsPerThread = (64 + kBuf + 3) / 4;   // ledger ids per quarter thread (c <= 96)
 
 __host__ __device__ inline Layout rescore_layout(int d) {
     Layout s;
@@ -1116,18 +1117,22 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kEpiWarps * 32) : "memory"); };
         uint32_t *rbits = reinterpret_cast<uint32_t *>(smem + lay.sel);   // [kRows][kSegStride]
         uint32_t *sbits = rbits + kRows * kSegStride;
-        const int32_t *idr = row >= 0 ? L.ids + ((size_t)h * L.nq + row) * L.c : nullptr;
+        const int32_t *idr = L.ids + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * L.c;
 
-        // this quarter's share of the row's ids: count the valid candidates
-        // (Eq. 5) and flag out-of-range ids
+        // this quarter's share of the row's ids (slots qt, qt+4, ...), loaded
+        // once: count the valid candidates (Eq. 5) and flag out-of-range ids;
+        // invalid slots become -1
+        int jid[kRescoreIdsPerThread];
         int ncand = 0;
         bool bad = false;
-        if (row >= 0) {
-            for (int e = qt; e < L.c; e += 4) {
-                const int j = idr[e];
-                ncand += (j >= 0 && j < n_valid) ? 1 : 0;
-                bad |= j >= n_valid || j < -1;
-            }
+#pragma unroll
+        for (int i = 0; i < kRescoreIdsPerThread; ++i) {
+            const int e = qt + 4 * i;
+            const int j = (row >= 0 && e < L.c) ? idr[e] : -1;
+            const bool valid = j >= 0 && j < n_valid;
+            ncand += valid ? 1 : 0;
+            bad |= j >= n_valid || j < -1;
+            jid[i] = valid ? j : -1;
         }
         float amin = INFINITY, bmax = -INFINITY;
         bool ok = true;
@@ -1139,13 +1144,13 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 sbits[r * kSegStride + w] = 0u;
             }
             epi_sync();
-            if (row >= 0) {
-                for (int e = qt; e < L.c; e += 4) {
-                    const int j = idr[e];
-                    if (j >= 0 && j < n_valid && j / kSegCols == sg) {
-                        const int jj = j - sg * kSegCols;
-                        atomicOr(&(e < L.k ? rbits : sbits)[r * kSegStride + (jj >> 5)], 1u << (jj & 31));
-                    }
+#pragma unroll
+            for (int i = 0; i < kRescoreIdsPerThread; ++i) {
+                const int j = jid[i];
+                if (j >= 0 && j / kSegCols == sg) {
+                    const int jj = j - sg * kSegCols;
+                    atomicOr(&(qt + 4 * i < L.k ? rbits : sbits)[r * kSegStride + (jj >> 5)],
+                             1u << (jj & 31));
                 }
             }
             epi_sync();
