@@ -283,7 +283,9 @@ def run_ours(args, w, rank, world, device):
     route_tflops = route_flops / (route_ms * 1e-3) / 1e12
     if uses_tensor_cores(w):
         peak = float(peaks["bf16_tflops_sustained"])
-        roofline = {"kernel": "route_rows_tc (tcgen05; anchor + refresh)", "bound": "tensor",
+        roofline = {"kernel": "full routing: route_rows_tc_kernel (tcgen05, two-pass selection) "
+                              "+ route_rows_finalize_kernel + retry path; anchor + refresh",
+                    "bound": "tensor",
                     "peak_source": f"{peaks['source']} bf16 dense, sustained (timed inside a long step)"}
     else:
         peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
@@ -298,35 +300,41 @@ def run_ours(args, w, rank, world, device):
                      "frac": round(route_tflops / peak, 4), "traffic": traffic,
                      "avg_launch_ms": round(route_ms / max(n_route, 1), 4),
                      "launches": n_route})
-    # secondary: relay rescore (HBM-bound): per row q (d*e) + its head's keys
-    # once (N*d*e/N) + ids (4c) + alpha/flag writes (5) bytes
+    # secondary: relay rescoring.  Bytes it must move per row: q (d*e) + its
+    # head's keys once (N*d*e/N) + ids (4c) + alpha/flag writes (5).
     rescore_bytes = w.bh * w.n * (2 * w.d * esz + 4 * w.c + 5) * n_rescore
     rescore_gbs = rescore_bytes / (rescore_ms * 1e-3) / 1e9 if rescore_ms > 0 else None
-    kernels = {
-        "rescore": {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1) if rescore_gbs else None,
-                    "peak_gbs": peaks["hbm_gbs"],
-                    "frac": round(rescore_gbs / peaks["hbm_gbs"], 4) if rescore_gbs else None,
-                    "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)},
-        "compact": {"avg_launch_ms": round(compact_ms / max(n_rescore, 1), 4)},
-    }
+    rescore = {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1) if rescore_gbs else None,
+               "peak_gbs": peaks["hbm_gbs"],
+               "frac": round(rescore_gbs / peaks["hbm_gbs"], 4) if rescore_gbs else None,
+               "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)}
+    if uses_tensor_cores(w) and rescore_ms > 0:
+        # the tensor-core rescoring scores every valid pair of the row block
+        # (2*d flops per pair) and reads the candidates' scores from the tiles
+        dense_tflops = 2.0 * w.d * full_pairs_per_layer(w) * n_rescore / (rescore_ms * 1e-3) / 1e12
+        rescore.update({"kernel": "relay_rescore_tc_kernel (tcgen05 dense tiles)", "bound": "tensor",
+                        "dense_tflops": round(dense_tflops, 2),
+                        "dense_frac": round(dense_tflops / float(peaks["bf16_tflops_sustained"]), 4)})
+    kernels = {"rescore": rescore,
+               "compact": {"avg_launch_ms": round(compact_ms / max(n_rescore, 1), 4)}}
 
     result = {
         "metric": METRIC, "value": rows_per_step * world / (ms_step * 1e-3), "unit": "rows/s",
         "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
-        "config": {"workload": w.name, "bh_per_gpu": w.bh, "n_chunks": w.n, "d": w.d,
-                   "layers": L, "anchor_interval": w.anchor_interval, "k": w.k, "near_miss": w.m,
-                   "random": w.r, "causal": w.causal, "drift_sigma": w.sigma,
-                   "l2": f"no flush: inputs {2 * L * w.bh * w.n * w.d * esz / 2**30:.1f} GiB per step exceed L2",
-                   "parallelism": f"bh-sharded x{world}, no collective"},
+        "config": workload_config(w, world),
         "score_pairs_per_s": pairs_per_step * world / (ms_step * 1e-3),
         "pair_fraction": pairs_per_step / (full_pairs_per_layer(w) * L),
         "rho_relay": rho,
         "retry_rows_per_step": d_cnt[rr.CNT_RETRY_TOTAL] / K,
         "roofline": roofline,
         "kernels": kernels,
-        "gpu_launches": K * (2 * len(anchors) + 4 * len(relays)),
+        # our kernels per layer: anchor = route (+ finalize + retry on the
+        # tensor-core path) + counters; relay = rescore + compact + the same
+        # route launches over the refreshed rows + counters
+        "gpu_launches": K * ((4 if uses_tensor_cores(w) else 2) * len(anchors)
+                             + (6 if uses_tensor_cores(w) else 4) * len(relays)),
         "clocks": clk.summary(),
         "peaks_source": peaks["source"],
     }
@@ -433,6 +441,16 @@ def cpu_baseline(w, qs, ks, threads=None, layers=2):
                       f"{dt:.1f} s wall on {ncpu} host cores"}
 
 
+def workload_config(w, world: int) -> dict:
+    """The bench line's config block (both arms)."""
+    esz = 2 if w.dtype == "bf16" else 4
+    return {"workload": w.name, "bh_per_gpu": w.bh, "n_chunks": w.n, "d": w.d,
+            "layers": w.layers, "anchor_interval": w.anchor_interval, "k": w.k, "near_miss": w.m,
+            "random": w.r, "causal": w.causal, "drift_sigma": w.sigma,
+            "l2": f"no flush: inputs {2 * w.layers * w.bh * w.n * w.d * esz / 2**30:.1f} GiB per step exceed L2",
+            "parallelism": f"bh-sharded x{world}, no collective"}
+
+
 def run_reference(args, w):
     """The oracle timed as a benchmark arm on this workload (rank 0 only)."""
     import numpy as np
@@ -454,10 +472,10 @@ def run_reference(args, w):
     v = sum(x["value"] for x in vals) / len(vals)
     cb = dict(vals[-1])
     cb["value"] = v
-    return {"metric": METRIC, "value": v, "unit": "rows/s", "n_gpus": 0, "steps": args.steps,
+    return {"metric": METRIC, "value": v, "unit": "rows/s", "n_gpus": args.gpus, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "sample_heads": T, "sample_layers": 2},
+            "config": workload_config(w, args.gpus),
             "cpu_baseline": cb,
             "e2e": {"value": v, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
