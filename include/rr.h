@@ -93,7 +93,7 @@ enum {
     RR_CNT_FULL_PAIRS = 8,    /* score pairs of the rows fully routed at the last layer */
     RR_CNT_FULL_PAIRS_TOTAL = 9, /* the same, since rr_ledger_create */
     RR_CNT_RETRY_TOTAL = 10,  /* rows whose tensor-core selection took the one-pass exact
-                                 path (a failed three-pass certificate), since create */
+                                 path (kept scores overflowed the two-pass buffer), since create */
     RR_NUM_COUNTERS = 16      /* slots 11..15 are reserved (0) */
 };
 
@@ -102,7 +102,10 @@ enum {
  * [bh*nq, c] int32 with c = k + m_near + r_rand (route | near-miss |
  * random), alpha [bh*nq] f32, anchor layer [bh*nq] int32, refresh flags
  * [bh*nq] u8, counters [16] int64 -- plus the library's per-layer scratch
- * (refresh lists and counts).  Pure host arithmetic. */
+ * (refresh lists and counts; for problems routed on the tensor cores also
+ * the kept scores each row hands from the selection kernel to the kernel
+ * that orders them: 120 x 6 bytes + 4 per row, rows rounded up to 128 per
+ * head).  Pure host arithmetic. */
 size_t rr_ledger_workspace_bytes(const rr_config *cfg);
 
 /* Validates cfg, carves the ledger out of d_workspace (device memory of at
