@@ -45,7 +45,8 @@ class _Params(ctypes.Structure):
     _fields_ = [("nq", ctypes.c_int32), ("nk", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("k", ctypes.c_int32), ("m", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("max_draws", ctypes.c_int32),
-                ("gamma", ctypes.c_double), ("seed", ctypes.c_uint64)]
+                ("gamma", ctypes.c_double), ("seed", ctypes.c_uint64),
+                ("max_age", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 def lib():
@@ -63,7 +64,7 @@ def lib():
             _lib.rro_philox4x32_10.argtypes = [P, P, P]
             _lib.rro_random_sentinels.argtypes = [ctypes.c_uint64, i32, i32, i32, i32, P, i32, i32, i32, P]
             _lib.rro_random_sentinels.restype = i32
-            _lib.rro_head_layer.argtypes = [ctypes.POINTER(_Params), i32, i32, i32, P, P, P, P, P, P, P, P]
+            _lib.rro_head_layer.argtypes = [ctypes.POINTER(_Params), i32, i32, i32, P, P, P, P, P, P, P, P, P]
             _lib.rro_head_layer.restype = i32
             _lib.rro_exact_topk.argtypes = [ctypes.POINTER(_Params), P, P, P]
     return _lib
@@ -87,6 +88,7 @@ class Params:
     gamma: float = 0.0
     seed: int = 0
     max_draws: int | None = None  # default 64 * (k + m + r)
+    max_age: int = 0              # per-row lifetime bound (0: off)
 
     @property
     def c(self) -> int:
@@ -95,7 +97,7 @@ class Params:
     def _c(self) -> _Params:
         md = self.max_draws if self.max_draws is not None else 64 * self.c
         return _Params(self.nq, self.nk, self.d, self.k, self.m, self.r, int(bool(self.causal)), md,
-                       float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF)
+                       float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.max_age), 0)
 
 
 def _f32(a) -> np.ndarray:
@@ -171,10 +173,15 @@ class HeadLedger:
         return HeadLedger(self.ids.copy(), self.alpha.copy(), self.anchor_layer.copy())
 
 
-def head_layer(p: Params, bh: int, layer: int, anchor: bool, q, k, led: HeadLedger):
-    """One layer of one head, in place on ``led``.  Returns (flags, beta,
-    refreshed_rows, score_pairs, status)."""
+def head_layer(p: Params, bh: int, layer: int, anchor: bool, q, k, led: HeadLedger, gamma_rows=None):
+    """One layer of one head, in place on ``led``.  gamma_rows: per-row
+    guard margins [nq] (RouteRelay Eq. 8 gamma_i), or None for p.gamma on
+    every row.  Returns (flags, beta, refreshed_rows, score_pairs, status)."""
     q = _f32(q); k = _f32(k)
+    g = None
+    if gamma_rows is not None:
+        g = np.ascontiguousarray(np.asarray(gamma_rows, dtype=np.float64))
+        assert g.shape == (p.nq,)
     assert q.shape == (p.nq, p.d) and k.shape == (p.nk, p.d)
     flags = np.zeros(p.nq, dtype=np.uint8)
     beta = np.empty(p.nq, dtype=np.float64)
@@ -182,7 +189,7 @@ def head_layer(p: Params, bh: int, layer: int, anchor: bool, q, k, led: HeadLedg
     cp = p._c()
     st = lib().rro_head_layer(ctypes.byref(cp), bh, layer, int(bool(anchor)), _ptr(q), _ptr(k),
                               _ptr(led.ids), _ptr(led.alpha), _ptr(led.anchor_layer),
-                              _ptr(flags), _ptr(beta), _ptr(counts))
+                              _ptr(flags), _ptr(beta), _ptr(counts), _ptr(g) if g is not None else None)
     return flags, beta, int(counts[0]), int(counts[1]), int(st)
 
 
@@ -211,6 +218,7 @@ class Router:
     anchor_interval: int
     bh_offset: int = 0
     threads: int = 1
+    gamma_rows: object = None   # [bh, nq] per-row guard margins, or None
     ledgers: list = field(default_factory=list)
     stats: list = field(default_factory=list)
 
@@ -230,8 +238,9 @@ class Router:
         heads = list(range(self.bh)) if heads is None else list(heads)
 
         def one(h):
+            g = None if self.gamma_rows is None else self.gamma_rows[h]
             flags, beta, ref, pairs, st = head_layer(self.p, self.bh_offset + h, layer, anchor,
-                                                      q[h], k[h], self.ledgers[h])
+                                                      q[h], k[h], self.ledgers[h], gamma_rows=g)
             hits = tot = 0
             if recall:
                 ex = exact_topk(self.p, q[h], k[h])

@@ -180,6 +180,8 @@ typedef struct {
     int32_t nq, nk, d, k, m, r, causal, max_draws;
     double gamma;
     uint64_t seed;
+    int32_t max_age;   /* 0: off; else a row whose ledger is max_age layers old refreshes */
+    int32_t reserved;
 } rro_params;
 
 static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
@@ -199,10 +201,18 @@ static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
  *     anchors, §3.2).
  *  anchor == 0: relay (RouteRelay §3.2 Eq. 5-8 and §4.1-4.2): candidate set
  *     A_i = R_i U C_i, alpha = min over R, beta = max over C, reuse iff
- *     alpha > beta + gamma; otherwise the row computes all its scores,
+ *     alpha > beta + gamma_i; otherwise the row computes all its scores,
  *     replaces its route and rebuilds its sentinels (anchor_layer <- layer).
  *     Stable rows keep ids; their age advances implicitly (age = layer -
  *     anchor_layer); their stored alpha becomes this layer's alpha.
+ *     gamma_i (Eq. 8, "a configurable guard margin" per row) is
+ *     gamma_rows[i], or p->gamma for every row when gamma_rows is NULL.
+ *     Per-row lifetime bound (reading of §3.2 "Forced anchors ... bound the
+ *     lifetime of stale random sentinels", applied per row): with
+ *     p->max_age > 0, a row with layer - anchor_layer >= max_age refreshes
+ *     whatever the test says, so no ledger row is reused max_age or more
+ *     layers after it was built.  A forced row is rescored first, like any
+ *     relay row, and counted like a challenged one.
  * Outputs: ids [nq*c] (in/out), alpha [nq] (in/out), anchor_layer [nq]
  * (in/out), flags [nq] (out: 1 = row was fully routed at this layer),
  * beta_out [nq] (out, may be NULL; relay only), counts[2] (out: rows fully
@@ -215,7 +225,8 @@ static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
 int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
                        int32_t anchor, const float *q, const float *kc,
                        int32_t *ids, double *alpha, int32_t *anchor_layer,
-                       uint8_t *flags, double *beta_out, int64_t *counts)
+                       uint8_t *flags, double *beta_out, int64_t *counts,
+                       const double *gamma_rows)
 {
     const int32_t c = p->k + p->m + p->r;
     double *S = (double *)malloc(sizeof(double) * (size_t)p->nq * (size_t)p->nk);
@@ -248,7 +259,10 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
         }
         pairs += n_cand;
         if (beta_out) beta_out[i] = b;
-        int refresh = !(a > b + p->gamma);                      /* Eq. 8 */
+        const double g = gamma_rows ? gamma_rows[i] : p->gamma;
+        int refresh = !(a > b + g);                             /* Eq. 8 */
+        if (p->max_age > 0 && layer - anchor_layer[i] >= p->max_age)
+            refresh = 1;                                        /* lifetime bound */
         flags[i] = (uint8_t)refresh;
         if (refresh) {
             rro_rebuild_row(p, bh, layer, i, s_row, row, &alpha[i]);

@@ -420,3 +420,101 @@ def test_recall_is_one_when_every_layer_is_an_anchor():
                 rng.standard_normal((1, 16, 8)).astype(np.float32))
     s = rt.summary()
     assert s["recall"] == 1.0 and s["rerouted_fraction"] == 1.0 and s["pair_fraction"] == 1.0
+
+
+# ---- per-row guard margins and lifetime bound (RouteRelay §3.2 Eq. 8 gamma_i;
+# "Forced anchors ... bound the lifetime of stale random sentinels") ----------
+
+def _drifting_layers(bh, n, d, layers, sigma, seed):
+    rng = np.random.default_rng(seed)
+    q = rownorm(rng.standard_normal((bh, n, d)))
+    k = rownorm(rng.standard_normal((bh, n, d)))
+    out = []
+    for _ in range(layers):
+        out.append((q.astype(np.float32), k.astype(np.float32)))
+        q = rownorm(q + sigma * rng.standard_normal(q.shape))
+        k = rownorm(k + sigma * rng.standard_normal(k.shape))
+    return out
+
+
+def _run(p, bh, layers_qk, H, gamma_rows=None):
+    rt = oracle.Router(p, bh=bh, anchor_interval=H, gamma_rows=gamma_rows)
+    hist = []
+    for l, (q, k) in enumerate(layers_qk):
+        res, _ = rt.step(l, q, k, recall=False)
+        hist.append(([led.copy() for led in rt.ledgers], [r[0].copy() for r in res], [r[1].copy() for r in res]))
+    return hist
+
+
+def test_gamma_rows_equal_to_the_scalar_reproduce_the_scalar_run():
+    p = Params(nq=40, nk=40, d=8, k=4, m=3, r=2, causal=True, gamma=0.02, seed=4)
+    lq = _drifting_layers(2, 40, 8, 7, 0.15, 21)
+    a = _run(p, 2, lq, 8)
+    b = _run(p, 2, lq, 8, gamma_rows=np.full((2, 40), 0.02))
+    for (la, fa, _), (lb, fb, _) in zip(a, b):
+        for h in range(2):
+            assert np.array_equal(la[h].ids, lb[h].ids)
+            assert np.array_equal(la[h].alpha, lb[h].alpha)
+            assert np.array_equal(fa[h], fb[h])
+
+
+def test_mixed_gamma_rows_follow_the_uniform_run_of_each_row():
+    """Rows are independent (own ledger, own random key), so a run with a
+    per-row margin equals, row by row, the run whose margin is that row's for
+    every row."""
+    p0 = Params(nq=48, nk=48, d=8, k=4, m=3, r=3, causal=False, gamma=0.0, seed=9)
+    big = 1e9
+    lq = _drifting_layers(2, 48, 8, 8, 0.1, 33)
+    g = np.where(np.random.default_rng(5).random((2, 48)) < 0.5, 0.0, big)
+    mixed = _run(p0, 2, lq, 8, gamma_rows=g)
+    zero = _run(p0, 2, lq, 8)
+    huge = _run(Params(**{**p0.__dict__, "gamma": big}), 2, lq, 8)
+    assert sum(int(f.sum()) for f in zero[3][1]) < 2 * 48   # margin 0 keeps some rows
+    for l in range(8):
+        for h in range(2):
+            for i in range(48):
+                ref = huge if g[h, i] > 0 else zero
+                assert np.array_equal(mixed[l][0][h].ids[i], ref[l][0][h].ids[i]), (l, h, i)
+                assert mixed[l][0][h].alpha[i] == ref[l][0][h].alpha[i]
+                assert mixed[l][1][h][i] == ref[l][1][h][i]
+            # a huge margin refreshes every relay row
+            if l % 8:
+                assert all(mixed[l][1][h][i] == 1 for i in range(48) if g[h, i] > 0)
+
+
+def test_max_age_one_routes_every_layer_exactly():
+    p = Params(nq=32, nk=32, d=8, k=4, m=2, r=2, causal=True, seed=6, max_age=1)
+    lq = _drifting_layers(1, 32, 8, 6, 0.02, 8)
+    rt = oracle.Router(p, bh=1, anchor_interval=100)
+    for l, (q, k) in enumerate(lq):
+        res, st = rt.step(l, q, k)
+        assert st.refreshed == 32
+        assert all(int(f) == 1 for f in res[0][0])
+    s = rt.summary()
+    assert s["recall"] == 1.0 and s["rerouted_fraction"] == 1.0
+
+
+def test_max_age_bounds_every_rows_ledger_age_and_leaves_younger_rows_to_the_test():
+    A = 3
+    p = Params(nq=40, nk=40, d=8, k=4, m=3, r=2, causal=False, seed=2, max_age=A)
+    lq = _drifting_layers(1, 40, 8, 10, 0.03, 44)   # low drift: many stable rows
+    rt = oracle.Router(p, bh=1, anchor_interval=100)
+    forced_seen = 0
+    for l, (q, k) in enumerate(lq):
+        before = rt.ledgers[0].copy()
+        res, _ = rt.step(l, q, k, recall=False)
+        flags, beta = res[0][0], res[0][1]
+        after = rt.ledgers[0]
+        assert np.all(l - after.anchor_layer < A)        # no row reused A or more layers after it was built
+        if l == 0:
+            continue
+        S = oracle.scores(q[0], k[0])
+        for i in range(40):
+            a = min(S[i, j] for j in before.ids[i, : p.k] if j >= 0)
+            test_refresh = not (a > beta[i] + p.gamma)
+            if l - before.anchor_layer[i] >= A:
+                assert flags[i] == 1
+                forced_seen += int(not test_refresh)
+            else:
+                assert flags[i] == int(test_refresh)
+    assert forced_seen > 0   # the bound actually forced some otherwise stable rows
