@@ -63,6 +63,8 @@ def _load():
     lib.rr_ledger_read.restype = ctypes.c_int
     lib.rr_ledger_device_view.argtypes = [P, ctypes.POINTER(rr_ledger_view)]
     lib.rr_ledger_device_view.restype = ctypes.c_int
+    lib.rr_ledger_set_guard.argtypes = [P, P, ctypes.c_int32]
+    lib.rr_ledger_set_guard.restype = ctypes.c_int
     lib.rr_route_layer_static.argtypes = [ctypes.POINTER(rr_config), P, P, ctypes.c_int32, P, P, P, P, P, P]
     lib.rr_route_layer_static.restype = ctypes.c_int
     lib.rr_status_string.argtypes = [ctypes.c_int]
@@ -136,6 +138,10 @@ def rr_ledger_device_view(handle) -> rr_ledger_view:
     v = rr_ledger_view()
     _check(_lib.rr_ledger_device_view(handle, ctypes.byref(v)), "rr_ledger_device_view")
     return v
+
+
+def rr_ledger_set_guard(handle, d_gamma_rows: int, max_age: int) -> None:
+    _check(_lib.rr_ledger_set_guard(handle, ctypes.c_void_p(d_gamma_rows), max_age), "rr_ledger_set_guard")
 
 
 def rr_route_layer_static(cfg: rr_config, d_qc: int, d_kc: int, layer: int, d_ids: int, d_alpha: int,
@@ -261,6 +267,19 @@ class RouteLedger:
         if check and int(out["counters"][CNT_ERROR]) != 0:
             raise RRError(RR_EDEVICE, f"device error word {int(out['counters'][CNT_ERROR]):#x}")
         return out
+
+    def set_guard(self, gamma_rows=None, max_age: int = 0) -> None:
+        """Per-row relay trigger: gamma_rows, a float32 device tensor of bh*nq
+        guard margins (or None for cfg.gamma on every row), and the per-row
+        lifetime bound max_age (0: off).  The tensor is kept referenced."""
+        ptr = 0
+        if gamma_rows is not None:
+            c = self.cfg
+            assert gamma_rows.dtype == torch.float32 and gamma_rows.is_contiguous()
+            assert gamma_rows.numel() == c.bh * c.nq and gamma_rows.device == self.workspace.device
+            ptr = gamma_rows.data_ptr()
+        rr_ledger_set_guard(self.handle, ptr, int(max_age))
+        self._gamma_rows = gamma_rows
 
     def device_view(self) -> dict:
         """Zero-copy torch views of the ledger inside the workspace."""

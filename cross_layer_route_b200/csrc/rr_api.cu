@@ -309,6 +309,13 @@ rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view) {
     return RR_OK;
 }
 
+rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int32_t max_age) {
+    if (!ledger || max_age < 0) return RR_EINVAL;
+    ledger->dev.gamma_rows = d_gamma_rows;
+    ledger->dev.max_age = max_age;
+    return RR_OK;
+}
+
 const char *rr_status_string(rr_status status) {
     switch (status) {
         case RR_OK: return "RR_OK";

@@ -28,6 +28,18 @@ __device__ __forceinline__ int valid_keys(int row, int nk, int causal) {
     return causal ? min(row + 1, nk) : nk;
 }
 
+// The relay decision of one row (RouteRelay §3.2): refresh unless
+// alpha > beta + gamma_i (Eq. 8; gamma_i from the per-row margins when the
+// ledger has them), and in any case once the row's ledger is max_age layers
+// old (the per-row lifetime bound; max_age 0 = off).
+__device__ __forceinline__ bool relay_refresh(const LedgerDev &L, size_t grow, int layer,
+                                              float alpha, float beta) {
+    const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
+    bool refresh = !(alpha > beta + g);
+    if (L.max_age > 0 && layer - L.anchor_layer[grow] >= L.max_age) refresh = true;
+    return refresh;
+}
+
 // ---- Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) --------------------
 // Ten rounds; each multiplies counter words 0 and 2 by the two Philox
 // multipliers, mixes the high halves with words 1 and 3 and the round key,

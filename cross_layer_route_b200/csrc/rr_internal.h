@@ -31,6 +31,11 @@ struct LedgerDev {
     int bh_offset;
     int max_draws;          // cap on random draws per row (64 * c)
     float gamma;
+    // per-row guard margins gamma_i of Eq. 8 ([bh*nq], caller-owned device
+    // memory), or null for `gamma` on every row; per-row lifetime bound: a
+    // row max_age or more layers past its anchor layer refreshes (0: off)
+    const float *gamma_rows = nullptr;
+    int max_age = 0;
     uint32_t seed_lo, seed_hi;
 };
 
@@ -64,7 +69,7 @@ cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, c
                                  int layer, cudaStream_t s);
 // Relay rescoring from dense tensor-core score tiles (rr_route_tc.cu); used
 // for the problems route_rows_tc_supported accepts.
-cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k,
+cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                     cudaStream_t s);
 cudaError_t launch_compact(const LedgerDev &L, cudaStream_t s);
 cudaError_t launch_finalize(const LedgerDev &L, int layer, long long add_rows,

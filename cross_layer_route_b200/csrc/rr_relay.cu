@@ -81,7 +81,7 @@ __device__ __forceinline__ float dot_row(const float *qs, const T *kp, int d) {
 // One warp per query row, one lane per candidate (RouteRelay §3.2 Eq. 5-8).
 template <typename T, int D>
 __global__ void __launch_bounds__(kRescoreThreads)
-relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
+relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K, int layer) {
     __shared__ __align__(16) float qs_all[kRescoreWarps][kDMax];
     __shared__ unsigned long long pair_sum[kRescoreWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -125,7 +125,7 @@ relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__
         }
         const bool any_bad = __any_sync(kFull, bad);
         if (lane == 0) {
-            const bool refresh = !(amin > bmax + L.gamma);  // Eq. 8
+            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
             L.flags[grow] = refresh ? 1 : 0;
             if (!refresh) L.alpha[grow] = amin;
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
@@ -209,7 +209,7 @@ __global__ void finalize_layer_kernel(LedgerDev L, int layer, long long add_rows
 // touches 4 lines, each in full.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRescoreThreads)
-relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K) {
+relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K, int layer) {
     constexpr int E = Vec16<T>::kElems;         // elements per 16-byte load
     constexpr int kLanes = 8;                   // lanes per candidate
     constexpr int kChunks = D / E / kLanes;     // 16-byte loads per lane
@@ -298,7 +298,7 @@ relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restri
         }
         const bool any_bad = __any_sync(kFull, bad);
         if (lane == 0) {
-            const bool refresh = !(amin > bmax + L.gamma);  // Eq. 8
+            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
             L.flags[grow] = refresh ? 1 : 0;
             if (!refresh) L.alpha[grow] = amin;
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
@@ -315,26 +315,25 @@ relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restri
 }
 
 template <typename T>
-static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, unsigned grid,
-                             cudaStream_t s) {
+static void rescore_dispatch(const LedgerDev &L, const void *q, const void *k, int layer,
+                             unsigned grid, cudaStream_t s) {
     const T *Q = static_cast<const T *>(q);
     const T *K = static_cast<const T *>(k);
     switch (L.d) {
-        case 64: relay_rescore_oct_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        case 128: relay_rescore_oct_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        case 256: relay_rescore_oct_kernel<T, 256><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
-        default: relay_rescore_kernel<T, 0><<<grid, kRescoreThreads, 0, s>>>(L, Q, K); break;
+        case 64: relay_rescore_oct_kernel<T, 64><<<grid, kRescoreThreads, 0, s>>>(L, Q, K, layer); break;
+        case 128: relay_rescore_oct_kernel<T, 128><<<grid, kRescoreThreads, 0, s>>>(L, Q, K, layer); break;
+        case 256: relay_rescore_oct_kernel<T, 256><<<grid, kRescoreThreads, 0, s>>>(L, Q, K, layer); break;
+        default: relay_rescore_kernel<T, 0><<<grid, kRescoreThreads, 0, s>>>(L, Q, K, layer); break;
     }
 }
 
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,
                                  int layer, cudaStream_t s) {
-    (void)layer;
-    if (route_rows_tc_supported(L, dtype)) return launch_relay_rescore_tc(L, q, k, s);
+    if (route_rows_tc_supported(L, dtype)) return launch_relay_rescore_tc(L, q, k, layer, s);
     const long long rows = (long long)L.bh * L.nq;
     const unsigned grid = (unsigned)((rows + kRescoreWarps - 1) / kRescoreWarps);
-    if (dtype == kBF16) rescore_dispatch<__nv_bfloat16>(L, q, k, grid, s);
-    else rescore_dispatch<float>(L, q, k, grid, s);
+    if (dtype == kBF16) rescore_dispatch<__nv_bfloat16>(L, q, k, layer, grid, s);
+    else rescore_dispatch<float>(L, q, k, layer, grid, s);
     return cudaGetLastError();
 }
 

@@ -1090,7 +1090,7 @@ __host__ __device__ inline Layout rescore_layout(int d) {
 
 __global__ void __launch_bounds__(kPassThreads, 1)
 relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
-                        const __grid_constant__ CUtensorMap tmap_k) {
+                        const __grid_constant__ CUtensorMap tmap_k, int layer) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char *smem = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
@@ -1192,7 +1192,7 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             }
             if (cta_ok && row >= 0) {
                 const size_t grow = (size_t)h * L.nq + row;
-                const bool refresh = !(a > b + L.gamma);   // Eq. 8
+                const bool refresh = relay_refresh(L, grow, layer, a, b);   // Eq. 8
                 L.flags[grow] = refresh ? 1 : 0;
                 if (!refresh) L.alpha[grow] = a;
                 if (n & (1 << 30)) atomicOr(&L.counters[2], 1ULL);
@@ -1289,14 +1289,14 @@ static cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap
     return cr == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k,
+cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                     cudaStream_t s) {
     CUtensorMap map;
     cudaError_t e = key_tensor_map(L, k, &map);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     tc::relay_rescore_tc_kernel<<<grid, tc::kPassThreads, tc::rescore_layout(L.d).total, s>>>(
-        L, static_cast<const __nv_bfloat16 *>(q), map);
+        L, static_cast<const __nv_bfloat16 *>(q), map, layer);
     return cudaGetLastError();
 }
 

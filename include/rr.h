@@ -198,6 +198,21 @@ rr_status rr_ledger_read(const rr_ledger *ledger, const rr_ledger_view *dst, voi
  * workspace (no copy), for consumers on the same device. */
 rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view);
 
+/* Per-row relay trigger (RouteRelay §3.2).  d_gamma_rows: NULL (every row
+ * uses cfg->gamma) or device memory of bh*nq floats holding each row's guard
+ * margin gamma_i of Eq. 8 (row-major [bh, nq], values >= 0; a NaN margin
+ * makes its row refresh); the caller owns it and keeps it valid and
+ * unchanged until the relay calls that use it have run on the stream.
+ * max_age: 0 (off) or the per-row lifetime bound -- the reading of the
+ * page's forced anchors, which "bound the lifetime of stale random
+ * sentinels", applied row by row: at a relay layer, a row whose ledger was
+ * built max_age or more layers earlier (layer - anchor_layer >= max_age)
+ * refreshes whatever Eq. 8 says; it is rescored first and counted like a
+ * challenged row.  Takes effect from the next rr_relay_layer /
+ * rr_relay_rescore call; no CUDA call.  Returns RR_EINVAL for a NULL ledger
+ * or max_age < 0. */
+rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int32_t max_age);
+
 /* One layer on caller-held ledger arrays, allocating nothing.  The paper
  * has no counterpart: this is a deployment variant for callers that cannot
  * call cudaMalloc -- code inside a host framework that owns every device

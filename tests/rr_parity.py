@@ -22,9 +22,9 @@ import oracle
 TIE_REL = 1e-5
 
 
-def params_of(w, bh_offset: int = 0) -> oracle.Params:
+def params_of(w, bh_offset: int = 0, max_age: int = 0) -> oracle.Params:
     return oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal,
-                         gamma=w.gamma, seed=w.seed)
+                         gamma=w.gamma, seed=w.seed, max_age=max_age)
 
 
 def config_of(w, rr, bh: int | None = None, bh_offset: int = 0):
@@ -64,9 +64,10 @@ def _sorted_valid(s_row: np.ndarray, nv: int):
 
 def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndarray, k: np.ndarray,
                  prev_ids, prev_alpha, prev_anchor, gpu_ids, gpu_alpha, gpu_anchor, gpu_flags,
-                 max_report: int = 10) -> Report:
+                 max_report: int = 10, gamma_rows=None) -> Report:
     """Runs the oracle on one head from the GPU's previous ledger and checks
-    the GPU's ledger after the same layer."""
+    the GPU's ledger after the same layer.  gamma_rows: this head's per-row
+    guard margins (None: p.gamma)."""
     rep = Report(rows=p.nq)
     S = oracle.scores(q, k)
     scale = np.linalg.norm(q.astype(np.float64), axis=1) * np.linalg.norm(k.astype(np.float64), axis=1).max()
@@ -76,7 +77,8 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
     else:
         led = oracle.HeadLedger(prev_ids.astype(np.int32).copy(), prev_alpha.astype(np.float64).copy(),
                                 prev_anchor.astype(np.int32).copy())
-    flags_o, beta_o, ref_o, pairs_o, st = oracle.head_layer(p, gh, layer, anchor, q, k, led)
+    flags_o, beta_o, ref_o, pairs_o, st = oracle.head_layer(p, gh, layer, anchor, q, k, led,
+                                                             gamma_rows=gamma_rows)
     assert st == 0
     rep.refreshed_oracle = ref_o
     rep.pairs_oracle = pairs_o
@@ -119,7 +121,9 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
         if not anchor:
             r_ids = [j for j in prev_ids[i, : p.k] if j >= 0]
             a = min(S[i, j] for j in r_ids) if r_ids else np.inf
-            if np.isfinite(beta_o[i]) and abs(a - beta_o[i] - p.gamma) < tol[i]:
+            g_i = p.gamma if gamma_rows is None else float(gamma_rows[i])
+            forced = p.max_age > 0 and layer - int(prev_anchor[i]) >= p.max_age
+            if not forced and np.isfinite(beta_o[i]) and abs(a - beta_o[i] - g_i) < tol[i]:
                 rep.tie_flag += 1
                 if int(gpu_flags[i]):
                     why = valid_full_row(i, nv, _sorted_valid(S[i], nv)[1])
@@ -180,14 +184,17 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
     return rep
 
 
-def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None):
+def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None,
+                  gamma_rows=None, max_age: int = 0):
     """Runs `layers` layers of workload w through the CUDA ledger `led` and
     compares every layer of the listed heads with the oracle started from
-    the GPU's own previous ledger.  Returns (total report, per-layer list)."""
+    the GPU's own previous ledger.  gamma_rows ([bh, nq] array) and max_age
+    must match what the ledger was given with set_guard.  Returns (total
+    report, per-layer list)."""
     import rr_workloads
     import torch
     st = rr_workloads.LayerStream(w, stream_device)
-    p = params_of(w)
+    p = params_of(w, max_age=max_age)
     total = Report()
     per_layer = []
     prev = None
@@ -207,7 +214,8 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
             pl = prev["anchor_layer"][h].numpy() if prev is not None else None
             r = compare_head(p, h, l, anchor, qn[h], kn[h], pi, pa, pl, after["ids"][h].numpy(),
                              after["alpha"][h].numpy(), after["anchor_layer"][h].numpy(),
-                             after["flags"][h].numpy())
+                             after["flags"][h].numpy(),
+                             gamma_rows=None if gamma_rows is None else np.asarray(gamma_rows[h]))
             layer_rep.add(r)
         per_layer.append((l, anchor, layer_rep, after["counters"].clone()))
         total.add(layer_rep)

@@ -113,3 +113,22 @@ def test_status_strings():
     for s in range(6):
         assert rr.rr_status_string(s).startswith("RR_")
     assert rr.rr_status_string(99) == "RR_UNKNOWN"
+
+
+def test_set_guard_validates_its_arguments_without_a_cuda_call():
+    import ctypes
+    import cross_layer_route_b200 as rr
+    lib = rr._lib
+    assert lib.rr_ledger_set_guard(None, None, 0) == rr.RR_EINVAL
+    cfg = rr.Config(bh=2, nq=8, nk=8, d=16, k=2, m_near=1, r_rand=1).to_c()
+    nbytes = lib.rr_ledger_workspace_bytes(ctypes.byref(cfg))
+    buf = ctypes.create_string_buffer(nbytes + 256)
+    base = (ctypes.addressof(buf) + 255) // 256 * 256   # host memory: create never touches it
+    h = ctypes.c_void_p()
+    assert lib.rr_ledger_create(ctypes.byref(cfg), ctypes.c_void_p(base), nbytes, ctypes.byref(h)) == rr.RR_OK
+    try:
+        assert lib.rr_ledger_set_guard(h, None, -1) == rr.RR_EINVAL
+        assert lib.rr_ledger_set_guard(h, None, 0) == rr.RR_OK
+        assert lib.rr_ledger_set_guard(h, ctypes.c_void_p(base), 4) == rr.RR_OK
+    finally:
+        lib.rr_ledger_destroy(h)

@@ -266,3 +266,29 @@ def test_retry_path_is_rare_on_the_full_size_workload(rr):
     _drive(rr, w, led, 1)
     c = led.read()["counters"]
     assert int(c[rr.CNT_RETRY_TOTAL]) <= 0.005 * w.bh * w.n, int(c[rr.CNT_RETRY_TOTAL])
+
+
+GUARD = [
+    (W.low_drift(W.C5).with_(bh=2, n=384, layers=10), "bf16_tensor_cores"),
+    (W.low_drift(W.C3).with_(bh=2, layers=8), "f32_cuda_cores"),
+]
+
+
+@pytest.mark.parametrize("case", GUARD, ids=[c[1] for c in GUARD])
+def test_per_row_margins_and_lifetime_bound(rr, case):
+    """Relay with per-row guard margins gamma_i (Eq. 8) and a per-row
+    lifetime bound, layer by layer against the oracle given the same margins
+    and bound; afterwards no row's ledger is max_age or more layers old."""
+    w, _ = case
+    max_age = 3
+    led = rr.RouteLedger(config_of(w, rr), DEV)
+    g = torch.where(torch.rand(w.bh, w.n, generator=torch.Generator().manual_seed(7)) < 0.5,
+                    torch.tensor(0.0), torch.tensor(0.05)).float()
+    led.set_guard(g.reshape(-1).contiguous().to(DEV), max_age=max_age)
+    rep, per_layer = layer_stepped(w, rr, led, w.layers, range(w.bh), DEV, gamma_rows=g.numpy(),
+                                   max_age=max_age)
+    _check(rep)
+    last = led.read()
+    assert int((w.layers - 1 - last["anchor_layer"]).max()) < max_age
+    relay = [lr for l, a, lr, _ in per_layer if not a]
+    assert sum(lr.refreshed_gpu for lr in relay) < sum(lr.rows for lr in relay)   # some rows were kept
