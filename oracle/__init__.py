@@ -46,7 +46,7 @@ class _Params(ctypes.Structure):
                 ("k", ctypes.c_int32), ("m", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("max_draws", ctypes.c_int32),
                 ("gamma", ctypes.c_double), ("seed", ctypes.c_uint64),
-                ("max_age", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("max_age", ctypes.c_int32), ("min_reuse", ctypes.c_int32)]
 
 
 def lib():
@@ -89,6 +89,7 @@ class Params:
     seed: int = 0
     max_draws: int | None = None  # default 64 * (k + m + r)
     max_age: int = 0              # per-row lifetime bound (0: off)
+    min_reuse: int = 0            # hysteresis: layers a rebuilt row is reused without the test
 
     @property
     def c(self) -> int:
@@ -97,7 +98,8 @@ class Params:
     def _c(self) -> _Params:
         md = self.max_draws if self.max_draws is not None else 64 * self.c
         return _Params(self.nq, self.nk, self.d, self.k, self.m, self.r, int(bool(self.causal)), md,
-                       float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.max_age), 0)
+                       float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.max_age),
+                       int(self.min_reuse))
 
 
 def _f32(a) -> np.ndarray:

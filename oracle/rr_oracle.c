@@ -181,7 +181,7 @@ typedef struct {
     double gamma;
     uint64_t seed;
     int32_t max_age;   /* 0: off; else a row whose ledger is max_age layers old refreshes */
-    int32_t reserved;
+    int32_t min_reuse; /* 0: off; else a row is reused for min_reuse layers after it was built */
 } rro_params;
 
 static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
@@ -213,6 +213,13 @@ static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
  *     whatever the test says, so no ledger row is reused max_age or more
  *     layers after it was built.  A forced row is rescored first, like any
  *     relay row, and counted like a challenged one.
+ *     Hysteresis (reading of §3.2 "a refreshed row receives a minimum reuse
+ *     horizon of one layer", the horizon made configurable): with
+ *     p->min_reuse = h > 0, a row built at layer a is reused without the
+ *     test at layers a+1 .. a+h (ids kept, alpha stored).  The lifetime bound
+ *     takes precedence where the two meet.  The page's optional larger guard
+ *     margin after a refresh is not applied (its recovery rule is not
+ *     given).
  * Outputs: ids [nq*c] (in/out), alpha [nq] (in/out), anchor_layer [nq]
  * (in/out), flags [nq] (out: 1 = row was fully routed at this layer),
  * beta_out [nq] (out, may be NULL; relay only), counts[2] (out: rows fully
@@ -263,6 +270,8 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
         int refresh = !(a > b + g);                             /* Eq. 8 */
         if (p->max_age > 0 && layer - anchor_layer[i] >= p->max_age)
             refresh = 1;                                        /* lifetime bound */
+        else if (p->min_reuse > 0 && layer - anchor_layer[i] <= p->min_reuse)
+            refresh = 0;                                        /* hysteresis horizon */
         flags[i] = (uint8_t)refresh;
         if (refresh) {
             rro_rebuild_row(p, bh, layer, i, s_row, row, &alpha[i]);

@@ -518,3 +518,48 @@ def test_max_age_bounds_every_rows_ledger_age_and_leaves_younger_rows_to_the_tes
             else:
                 assert flags[i] == int(test_refresh)
     assert forced_seen > 0   # the bound actually forced some otherwise stable rows
+
+
+# ---- hysteresis: minimum reuse horizon (RouteRelay §3.2 "Hysteresis") --------
+
+def test_min_reuse_keeps_rebuilt_rows_for_the_horizon_and_tests_the_rest():
+    h = 2
+    p = Params(nq=32, nk=32, d=8, k=4, m=2, r=2, causal=True, seed=8, min_reuse=h)
+    lq = _drifting_layers(1, 32, 8, 9, 0.6, 61)   # high drift: the test refreshes most rows
+    rt = oracle.Router(p, bh=1, anchor_interval=100)
+    kept_by_horizon = 0
+    for l, (q, k) in enumerate(lq):
+        before = rt.ledgers[0].copy()
+        res, _ = rt.step(l, q, k, recall=False)
+        if l == 0:
+            continue
+        flags, beta = res[0][0], res[0][1]
+        S = oracle.scores(q[0], k[0])
+        for i in range(32):
+            age = l - before.anchor_layer[i]
+            a = min(S[i, j] for j in before.ids[i, : p.k] if j >= 0)
+            test_refresh = not (a > beta[i] + p.gamma)
+            if age <= h:
+                assert flags[i] == 0 and np.array_equal(rt.ledgers[0].ids[i], before.ids[i])
+                kept_by_horizon += int(test_refresh)
+            else:
+                assert flags[i] == int(test_refresh)
+    assert kept_by_horizon > 0
+
+
+def test_min_reuse_beyond_the_run_never_refreshes_and_the_bound_takes_precedence():
+    lq = _drifting_layers(1, 24, 8, 6, 0.6, 62)
+    p = Params(nq=24, nk=24, d=8, k=3, m=2, r=2, seed=1, min_reuse=10)
+    rt = oracle.Router(p, bh=1, anchor_interval=100)
+    rt.step(0, *lq[0], recall=False)
+    anchor_ids = rt.ledgers[0].ids.copy()
+    for l in range(1, 6):
+        res, st = rt.step(l, *lq[l], recall=False)
+        assert st.refreshed == 0
+    assert np.array_equal(rt.ledgers[0].ids, anchor_ids)
+    # a lifetime bound shorter than the horizon still forces the refresh
+    p2 = Params(nq=24, nk=24, d=8, k=3, m=2, r=2, seed=1, min_reuse=10, max_age=2)
+    rt2 = oracle.Router(p2, bh=1, anchor_interval=100)
+    for l in range(6):
+        res, st = rt2.step(l, *lq[l], recall=False)
+        assert np.all(l - rt2.ledgers[0].anchor_layer < 2)
