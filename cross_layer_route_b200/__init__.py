@@ -65,6 +65,8 @@ def _load():
     lib.rr_ledger_device_view.restype = ctypes.c_int
     lib.rr_ledger_set_guard.argtypes = [P, P, ctypes.c_int32]
     lib.rr_ledger_set_guard.restype = ctypes.c_int
+    lib.rr_ledger_set_hysteresis.argtypes = [P, ctypes.c_int32]
+    lib.rr_ledger_set_hysteresis.restype = ctypes.c_int
     lib.rr_route_layer_static.argtypes = [ctypes.POINTER(rr_config), P, P, ctypes.c_int32, P, P, P, P, P, P]
     lib.rr_route_layer_static.restype = ctypes.c_int
     lib.rr_status_string.argtypes = [ctypes.c_int]
@@ -142,6 +144,10 @@ def rr_ledger_device_view(handle) -> rr_ledger_view:
 
 def rr_ledger_set_guard(handle, d_gamma_rows: int, max_age: int) -> None:
     _check(_lib.rr_ledger_set_guard(handle, ctypes.c_void_p(d_gamma_rows), max_age), "rr_ledger_set_guard")
+
+
+def rr_ledger_set_hysteresis(handle, min_reuse: int) -> None:
+    _check(_lib.rr_ledger_set_hysteresis(handle, min_reuse), "rr_ledger_set_hysteresis")
 
 
 def rr_route_layer_static(cfg: rr_config, d_qc: int, d_kc: int, layer: int, d_ids: int, d_alpha: int,
@@ -280,6 +286,10 @@ class RouteLedger:
             ptr = gamma_rows.data_ptr()
         rr_ledger_set_guard(self.handle, ptr, int(max_age))
         self._gamma_rows = gamma_rows
+
+    def set_hysteresis(self, min_reuse: int) -> None:
+        """Minimum reuse horizon after a row is rebuilt (0: off)."""
+        rr_ledger_set_hysteresis(self.handle, int(min_reuse))
 
     def device_view(self) -> dict:
         """Zero-copy torch views of the ledger inside the workspace."""

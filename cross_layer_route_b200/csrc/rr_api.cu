@@ -316,6 +316,12 @@ rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int3
     return RR_OK;
 }
 
+rr_status rr_ledger_set_hysteresis(rr_ledger *ledger, int32_t min_reuse) {
+    if (!ledger || min_reuse < 0) return RR_EINVAL;
+    ledger->dev.min_reuse = min_reuse;
+    return RR_OK;
+}
+
 const char *rr_status_string(rr_status status) {
     switch (status) {
         case RR_OK: return "RR_OK";

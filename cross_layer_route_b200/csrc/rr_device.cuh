@@ -30,14 +30,17 @@ __device__ __forceinline__ int valid_keys(int row, int nk, int causal) {
 
 // The relay decision of one row (RouteRelay §3.2): refresh unless
 // alpha > beta + gamma_i (Eq. 8; gamma_i from the per-row margins when the
-// ledger has them), and in any case once the row's ledger is max_age layers
-// old (the per-row lifetime bound; max_age 0 = off).
+// ledger has them).  A row whose ledger is max_age layers old refreshes in
+// any case (the per-row lifetime bound; max_age 0 = off); otherwise a row
+// built min_reuse or fewer layers ago is reused without the test (the
+// hysteresis horizon; min_reuse 0 = off).
 __device__ __forceinline__ bool relay_refresh(const LedgerDev &L, size_t grow, int layer,
                                               float alpha, float beta) {
+    const int age = layer - L.anchor_layer[grow];
+    if (L.max_age > 0 && age >= L.max_age) return true;
+    if (L.min_reuse > 0 && age <= L.min_reuse) return false;
     const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
-    bool refresh = !(alpha > beta + g);
-    if (L.max_age > 0 && layer - L.anchor_layer[grow] >= L.max_age) refresh = true;
-    return refresh;
+    return !(alpha > beta + g);
 }
 
 // ---- Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) --------------------

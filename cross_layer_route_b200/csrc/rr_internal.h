@@ -36,6 +36,9 @@ struct LedgerDev {
     // row max_age or more layers past its anchor layer refreshes (0: off)
     const float *gamma_rows = nullptr;
     int max_age = 0;
+    // hysteresis: a row built at layer a is reused without the test at
+    // layers a+1 .. a+min_reuse (0: off)
+    int min_reuse = 0;
     uint32_t seed_lo, seed_hi;
 };
 

@@ -213,6 +213,17 @@ rr_status rr_ledger_device_view(const rr_ledger *ledger, rr_ledger_view *view);
  * or max_age < 0. */
 rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int32_t max_age);
 
+/* Hysteresis (RouteRelay §3.2: "a refreshed row receives a minimum reuse
+ * horizon of one layer"), the horizon made configurable.  min_reuse: 0 (off)
+ * or h > 0 -- a row built at layer a (anchor or refresh) is reused without
+ * the challenge test at layers a+1 .. a+h: its ids stay, its alpha is
+ * stored, it counts as a stable row.  The lifetime bound of
+ * rr_ledger_set_guard takes precedence where the two meet.  The page's
+ * optional larger guard margin after a refresh is not applied (the page
+ * gives no rule for its recovery).  Takes effect from the next relay call;
+ * no CUDA call.  Returns RR_EINVAL for a NULL ledger or min_reuse < 0. */
+rr_status rr_ledger_set_hysteresis(rr_ledger *ledger, int32_t min_reuse);
+
 /* One layer on caller-held ledger arrays, allocating nothing.  The paper
  * has no counterpart: this is a deployment variant for callers that cannot
  * call cudaMalloc -- code inside a host framework that owns every device

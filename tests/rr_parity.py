@@ -22,9 +22,9 @@ import oracle
 TIE_REL = 1e-5
 
 
-def params_of(w, bh_offset: int = 0, max_age: int = 0) -> oracle.Params:
+def params_of(w, bh_offset: int = 0, max_age: int = 0, min_reuse: int = 0) -> oracle.Params:
     return oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal,
-                         gamma=w.gamma, seed=w.seed, max_age=max_age)
+                         gamma=w.gamma, seed=w.seed, max_age=max_age, min_reuse=min_reuse)
 
 
 def config_of(w, rr, bh: int | None = None, bh_offset: int = 0):
@@ -122,7 +122,8 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
             r_ids = [j for j in prev_ids[i, : p.k] if j >= 0]
             a = min(S[i, j] for j in r_ids) if r_ids else np.inf
             g_i = p.gamma if gamma_rows is None else float(gamma_rows[i])
-            forced = p.max_age > 0 and layer - int(prev_anchor[i]) >= p.max_age
+            age = layer - int(prev_anchor[i])
+            forced = (p.max_age > 0 and age >= p.max_age) or (p.min_reuse > 0 and age <= p.min_reuse)
             if not forced and np.isfinite(beta_o[i]) and abs(a - beta_o[i] - g_i) < tol[i]:
                 rep.tie_flag += 1
                 if int(gpu_flags[i]):
@@ -185,7 +186,7 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
 
 
 def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None,
-                  gamma_rows=None, max_age: int = 0):
+                  gamma_rows=None, max_age: int = 0, min_reuse: int = 0):
     """Runs `layers` layers of workload w through the CUDA ledger `led` and
     compares every layer of the listed heads with the oracle started from
     the GPU's own previous ledger.  gamma_rows ([bh, nq] array) and max_age
@@ -194,7 +195,7 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
     import rr_workloads
     import torch
     st = rr_workloads.LayerStream(w, stream_device)
-    p = params_of(w, max_age=max_age)
+    p = params_of(w, max_age=max_age, min_reuse=min_reuse)
     total = Report()
     per_layer = []
     prev = None

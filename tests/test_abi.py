@@ -115,7 +115,7 @@ def test_status_strings():
     assert rr.rr_status_string(99) == "RR_UNKNOWN"
 
 
-def test_set_guard_validates_its_arguments_without_a_cuda_call():
+def test_trigger_setters_validate_their_arguments_without_a_cuda_call():
     import ctypes
     import cross_layer_route_b200 as rr
     lib = rr._lib
@@ -130,5 +130,8 @@ def test_set_guard_validates_its_arguments_without_a_cuda_call():
         assert lib.rr_ledger_set_guard(h, None, -1) == rr.RR_EINVAL
         assert lib.rr_ledger_set_guard(h, None, 0) == rr.RR_OK
         assert lib.rr_ledger_set_guard(h, ctypes.c_void_p(base), 4) == rr.RR_OK
+        assert lib.rr_ledger_set_hysteresis(h, -1) == rr.RR_EINVAL
+        assert lib.rr_ledger_set_hysteresis(h, 1) == rr.RR_OK
+        assert lib.rr_ledger_set_hysteresis(None, 1) == rr.RR_EINVAL
     finally:
         lib.rr_ledger_destroy(h)

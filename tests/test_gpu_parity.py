@@ -292,3 +292,26 @@ def test_per_row_margins_and_lifetime_bound(rr, case):
     assert int((w.layers - 1 - last["anchor_layer"]).max()) < max_age
     relay = [lr for l, a, lr, _ in per_layer if not a]
     assert sum(lr.refreshed_gpu for lr in relay) < sum(lr.rows for lr in relay)   # some rows were kept
+
+
+HYST = [
+    (W.C5.with_(bh=2, n=256, layers=8), "bf16_tensor_cores"),
+    (W.C3.with_(bh=2, n=256, layers=8), "f32_cuda_cores"),
+]
+
+
+@pytest.mark.parametrize("case", HYST, ids=[c[1] for c in HYST])
+def test_hysteresis_horizon(rr, case):
+    """Relay with a one-layer minimum reuse horizon (RouteRelay §3.2,
+    Hysteresis) under the workload's high drift, layer by layer against the
+    oracle given the same horizon: rows rebuilt at the previous layer are
+    kept, the others follow the test."""
+    w, _ = case
+    led = rr.RouteLedger(config_of(w, rr), DEV)
+    led.set_hysteresis(1)
+    rep, per_layer = layer_stepped(w, rr, led, w.layers, range(w.bh), DEV, min_reuse=1)
+    _check(rep)
+    relay = [lr for l, a, lr, _ in per_layer if not a]
+    # under this drift the test refreshes nearly every row, so the horizon
+    # keeps about every other layer's rows
+    assert sum(lr.refreshed_gpu for lr in relay) < 0.75 * sum(lr.rows for lr in relay)
