@@ -46,7 +46,8 @@ class _Params(ctypes.Structure):
                 ("k", ctypes.c_int32), ("m", ctypes.c_int32), ("r", ctypes.c_int32),
                 ("causal", ctypes.c_int32), ("max_draws", ctypes.c_int32),
                 ("gamma", ctypes.c_double), ("seed", ctypes.c_uint64),
-                ("max_age", ctypes.c_int32), ("min_reuse", ctypes.c_int32)]
+                ("max_age", ctypes.c_int32), ("min_reuse", ctypes.c_int32),
+                ("g_sink", ctypes.c_int32), ("g_recent", ctypes.c_int32)]
 
 
 def lib():
@@ -90,16 +91,18 @@ class Params:
     max_draws: int | None = None  # default 64 * (k + m + r)
     max_age: int = 0              # per-row lifetime bound (0: off)
     min_reuse: int = 0            # hysteresis: layers a rebuilt row is reused without the test
+    g_sink: int = 0               # mandatory global sentinels: sink chunks 0..g_sink-1
+    g_recent: int = 0             # ... and the row's recent chunks i-g_recent+1..i
 
     @property
     def c(self) -> int:
-        return self.k + self.m + self.r
+        return self.k + self.m + self.r + self.g_sink + self.g_recent
 
     def _c(self) -> _Params:
         md = self.max_draws if self.max_draws is not None else 64 * self.c
         return _Params(self.nq, self.nk, self.d, self.k, self.m, self.r, int(bool(self.causal)), md,
                        float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.max_age),
-                       int(self.min_reuse))
+                       int(self.min_reuse), int(self.g_sink), int(self.g_recent))
 
 
 def _f32(a) -> np.ndarray:

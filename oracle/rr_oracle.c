@@ -182,6 +182,8 @@ typedef struct {
     uint64_t seed;
     int32_t max_age;   /* 0: off; else a row whose ledger is max_age layers old refreshes */
     int32_t min_reuse; /* 0: off; else a row is reused for min_reuse layers after it was built */
+    int32_t g_sink;    /* mandatory global sentinels: sink chunks 0..g_sink-1 */
+    int32_t g_recent;  /* ... and the row's recent chunks i-g_recent+1..i */
 } rro_params;
 
 static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
@@ -189,9 +191,31 @@ static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
                             double *alpha)
 {
     int32_t n_valid = rro_valid_count(i, p->nk, p->causal);
+    const int32_t ksel = p->k + p->m, g = p->g_sink + p->g_recent;
     rro_route_row(s_row, n_valid, p->k, p->m, ids, ids + p->k, alpha);
-    rro_random_sentinels(p->seed, bh, i, layer, n_valid, ids, p->k + p->m,
-                         p->r, p->max_draws, ids + p->k + p->m);
+    /* Mandatory global candidates (RouteRelay §3.1 item 3, "sink and recent
+     * chunks"): the sink chunks 0..g_sink-1, then the row's recent chunks
+     * i-g_recent+1..i, each kept if valid, not in route U near-miss and not
+     * already listed (a recent chunk below g_sink is a sink chunk); stored in
+     * that order after the random block, -1 padded. */
+    int32_t *glob = ids + ksel + p->r;
+    int32_t ng = 0;
+    for (int32_t t = 0; t < g; ++t) {
+        const int32_t j = t < p->g_sink ? t : i - p->g_recent + 1 + (t - p->g_sink);
+        if (j < 0 || j >= n_valid) continue;
+        if (t >= p->g_sink && j < p->g_sink) continue;
+        if (rro_contains(ids, ksel, j)) continue;
+        glob[ng++] = j;
+    }
+    for (int32_t t = ng; t < g; ++t) glob[t] = -1;
+    /* random sentinels from the valid chunks outside route U near-miss U the
+     * global candidates */
+    int32_t *excl = (int32_t *)malloc(sizeof(int32_t) * (size_t)(ksel + g + 1));
+    memcpy(excl, ids, sizeof(int32_t) * (size_t)ksel);
+    memcpy(excl + ksel, glob, sizeof(int32_t) * (size_t)ng);
+    rro_random_sentinels(p->seed, bh, i, layer, n_valid, excl, ksel + ng,
+                         p->r, p->max_draws, ids + ksel);
+    free(excl);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -235,7 +259,7 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
                        uint8_t *flags, double *beta_out, int64_t *counts,
                        const double *gamma_rows)
 {
-    const int32_t c = p->k + p->m + p->r;
+    const int32_t c = p->k + p->m + p->r + p->g_sink + p->g_recent;
     double *S = (double *)malloc(sizeof(double) * (size_t)p->nq * (size_t)p->nk);
     rro_scores(q, kc, p->nq, p->nk, p->d, S);
     int64_t refreshed = 0, pairs = 0;

@@ -563,3 +563,57 @@ def test_min_reuse_beyond_the_run_never_refreshes_and_the_bound_takes_precedence
     for l in range(6):
         res, st = rt2.step(l, *lq[l], recall=False)
         assert np.all(l - rt2.ledgers[0].anchor_layer < 2)
+
+
+# ---- mandatory global sentinels (RouteRelay §3.1 item 3: sink and recent) ----
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_global_sentinels_are_the_sink_and_recent_chunks_outside_the_route(causal):
+    gs, gr = 2, 3
+    p = Params(nq=40, nk=40, d=8, k=4, m=3, r=3, causal=causal, seed=5, g_sink=gs, g_recent=gr)
+    rng = np.random.default_rng(17)
+    q = rownorm(rng.standard_normal((40, 8))).astype(np.float32)
+    k = rownorm(rng.standard_normal((40, 8))).astype(np.float32)
+    led = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q, k, led)
+    base = oracle.HeadLedger.empty(Params(**{**p.__dict__, "g_sink": 0, "g_recent": 0}))
+    oracle.head_layer(Params(**{**p.__dict__, "g_sink": 0, "g_recent": 0}), 0, 0, True, q, k, base)
+    for i in range(40):
+        nv = oracle.valid_count(i, 40, causal)
+        row = led.ids[i]
+        sel = [int(x) for x in row[: p.k + p.m] if x >= 0]
+        assert np.array_equal(row[: p.k + p.m], base.ids[i, : p.k + p.m])   # route / near-miss unchanged
+        want = []
+        for j in list(range(gs)) + list(range(i - gr + 1, i + 1)):
+            if 0 <= j < nv and j not in sel and j not in want:
+                want.append(j)
+        glob = [int(x) for x in row[p.k + p.m + p.r:]]
+        assert glob == want + [-1] * (gs + gr - len(want)), i
+        rand = [int(x) for x in row[p.k + p.m: p.k + p.m + p.r] if x >= 0]
+        pool = [j for j in range(nv) if j not in sel and j not in want]
+        assert len(set(rand)) == len(rand) and all(j in pool for j in rand)
+        assert len(rand) == min(p.r, len(pool))
+        if len(pool) <= p.r:
+            assert rand == pool                                            # the whole pool, ascending
+
+
+def test_global_sentinels_take_part_in_beta():
+    """At a relay layer beta is the maximum over every sentinel, globals
+    included (Eq. 7 over C_i, which holds near-miss, random and global
+    candidates)."""
+    p = Params(nq=32, nk=32, d=8, k=3, m=2, r=2, causal=True, seed=3, g_sink=2, g_recent=2)
+    lq = _drifting_layers(1, 32, 8, 3, 0.3, 71)
+    led = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, lq[0][0][0], lq[0][1][0], led)
+    before = led.copy()
+    flags, beta, _, _, _ = oracle.head_layer(p, 0, 1, False, lq[1][0][0], lq[1][1][0], led)
+    S = oracle.scores(lq[1][0][0], lq[1][1][0])
+    n_glob_max = 0
+    for i in range(32):
+        sent = [int(j) for j in before.ids[i, p.k:] if j >= 0]
+        if sent:
+            assert beta[i] == max(S[i, j] for j in sent)
+        glob = [int(j) for j in before.ids[i, p.k + p.m + p.r:] if j >= 0]
+        if glob and sent and max(S[i, j] for j in glob) == beta[i]:
+            n_glob_max += 1
+    assert n_glob_max > 0   # some rows' beta comes from a global candidate
