@@ -33,7 +33,8 @@ class rr_config(ctypes.Structure):
                 ("d", ctypes.c_int32), ("dtype", ctypes.c_int32), ("k", ctypes.c_int32),
                 ("m_near", ctypes.c_int32), ("r_rand", ctypes.c_int32),
                 ("anchor_interval", ctypes.c_int32), ("causal", ctypes.c_int32),
-                ("gamma", ctypes.c_float), ("bh_offset", ctypes.c_int32), ("seed", ctypes.c_uint64)]
+                ("gamma", ctypes.c_float), ("bh_offset", ctypes.c_int32), ("seed", ctypes.c_uint64),
+                ("g_sink", ctypes.c_int32), ("g_recent", ctypes.c_int32)]
 
 
 class rr_ledger_view(ctypes.Structure):
@@ -180,10 +181,12 @@ class Config:
     gamma: float = 0.0
     seed: int = 0
     bh_offset: int = 0
+    g_sink: int = 0             # mandatory global sentinels: sink chunks
+    g_recent: int = 0           # ... and recent chunks per row
 
     @property
     def c(self) -> int:
-        return self.k + self.m_near + self.r_rand
+        return self.k + self.m_near + self.r_rand + self.g_sink + self.g_recent
 
     @property
     def torch_dtype(self) -> torch.dtype:
@@ -192,7 +195,8 @@ class Config:
     def to_c(self) -> rr_config:
         return rr_config(self.bh, self.nq, self.nk, self.d, RR_BF16 if self.dtype == "bf16" else RR_F32,
                          self.k, self.m_near, self.r_rand, self.anchor_interval, int(bool(self.causal)),
-                         float(self.gamma), self.bh_offset, int(self.seed) & 0xFFFFFFFFFFFFFFFF)
+                         float(self.gamma), self.bh_offset, int(self.seed) & 0xFFFFFFFFFFFFFFFF,
+                         self.g_sink, self.g_recent)
 
 
 def _stream_handle(stream) -> int:

@@ -49,6 +49,7 @@ bool config_ok(const rr_config *c) {
     if (c->k < 1 || c->k > c->nk) return false;
     if (c->m_near < 0 || c->r_rand < 0) return false;
     if (c->k + c->m_near > 128 || c->r_rand > 128) return false;
+    if (c->g_sink < 0 || c->g_recent < 0 || c->g_sink + c->g_recent > 32) return false;
     if (c->anchor_interval < 0 || c->bh_offset < 0) return false;
     if (!(c->gamma >= 0.0f) || !isfinite(c->gamma)) return false;
     if ((long long)c->bh * (long long)c->nq > (long long)INT32_MAX) return false;
@@ -57,7 +58,7 @@ bool config_ok(const rr_config *c) {
 
 Layout layout_of(const rr_config *c) {
     const size_t rows = (size_t)c->bh * (size_t)c->nq;
-    const size_t cc = (size_t)(c->k + c->m_near + c->r_rand);
+    const size_t cc = (size_t)(c->k + c->m_near + c->r_rand + c->g_sink + c->g_recent);
     Layout L;
     size_t o = 0;
     L.ids = o;          o = align_up(o + rows * cc * sizeof(int32_t));
@@ -72,6 +73,7 @@ Layout layout_of(const rr_config *c) {
     rr::LedgerDev t;
     t.bh = c->bh; t.nq = c->nq; t.nk = c->nk; t.d = c->d;
     t.k = c->k; t.m = c->m_near; t.r = c->r_rand; t.ksel = c->k + c->m_near;
+    t.g_sink = c->g_sink; t.g_recent = c->g_recent; t.c = (int)cc;
     const rr::CandSizes cs = rr::route_rows_tc_candidate_sizes(t, c->dtype);
     L.cand = cs.v > 0;
     L.cand_v = o;       o = align_up(o + cs.v);
@@ -222,7 +224,8 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     }
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
-    D.c = cfg->k + cfg->m_near + cfg->r_rand;
+    D.g_sink = cfg->g_sink; D.g_recent = cfg->g_recent;
+    D.c = cfg->k + cfg->m_near + cfg->r_rand + cfg->g_sink + cfg->g_recent;
     D.ksel = cfg->k + cfg->m_near;
     D.causal = cfg->causal ? 1 : 0;
     D.bh_offset = cfg->bh_offset;

@@ -28,6 +28,23 @@ __device__ __forceinline__ int valid_keys(int row, int nk, int causal) {
     return causal ? min(row + 1, nk) : nk;
 }
 
+// Mandatory global sentinels (RouteRelay §3.1 item 3, "sink and recent
+// chunks"): candidate t < g_sink + g_recent of query row `row` is sink chunk
+// t, then recent chunk row-g_recent+1+(t-g_sink).  A candidate is kept when
+// it is valid, outside route U near-miss, and not a recent chunk that is
+// also a sink chunk (listed once, as a sink).
+__device__ __forceinline__ int global_cand(const LedgerDev &L, int row, int t) {
+    return t < L.g_sink ? t : row - L.g_recent + 1 + (t - L.g_sink);
+}
+__device__ __forceinline__ bool global_cand_listable(const LedgerDev &L, int t, int j, int n_valid) {
+    return j >= 0 && j < n_valid && !(t >= L.g_sink && j < L.g_sink);
+}
+// Whether valid chunk j is one of row's global candidates (such chunks are
+// outside the random sentinels' pool).
+__device__ __forceinline__ bool is_global_cand(const LedgerDev &L, int row, int n_valid, int j) {
+    return j >= 0 && j < n_valid && (j < L.g_sink || (j <= row && j > row - L.g_recent));
+}
+
 // The relay decision of one row (RouteRelay §3.2): refresh unless
 // alpha > beta + gamma_i (Eq. 8; gamma_i from the per-row margins when the
 // ledger has them).  A row whose ledger is max_age layers old refreshes in

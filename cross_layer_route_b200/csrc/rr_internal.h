@@ -26,7 +26,8 @@ struct LedgerDev {
     uint16_t *cand_i = nullptr;    // [blocks, 128, kCap] their key chunks
     int32_t *cand_meta = nullptr;  // [blocks, 128] kept counts of the two halves, or -1
     int bh, nq, nk, d;
-    int k, m, r, c, ksel;   // ksel = k + m
+    int k, m, r, c, ksel;   // ksel = k + m; c = k + m + r + g_sink + g_recent
+    int g_sink = 0, g_recent = 0;   // mandatory global sentinels (sink, recent chunks)
     int causal;
     int bh_offset;
     int max_draws;          // cap on random draws per row (64 * c)

@@ -92,7 +92,8 @@ extern "C" rr_status rr_route_layer_static(const rr_config *cfg, const void *d_q
     D.retry_count = scratch + 2 * kStaticMaxRows + kStaticMaxHeads;
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
-    D.c = cfg->k + cfg->m_near + cfg->r_rand;
+    D.g_sink = cfg->g_sink; D.g_recent = cfg->g_recent;
+    D.c = cfg->k + cfg->m_near + cfg->r_rand + cfg->g_sink + cfg->g_recent;
     D.ksel = cfg->k + cfg->m_near;
     D.causal = cfg->causal ? 1 : 0;
     D.bh_offset = cfg->bh_offset;

@@ -84,12 +84,12 @@ __device__ __forceinline__ bool in_list(const int *lst, int n, int j) {
 // step, accepted in draw order.  A pool of at most r chunks is taken whole in
 // ascending order; a row that exhausts max_draws is filled in ascending order.
 __device__ void draw_random_sentinels(const LedgerDev &L, int ghead, int row, int layer,
-                                      int n_valid, const int *excl, int n_excl, int *acc_buf,
-                                      int32_t *out) {
+                                      int n_valid, const int *excl, int n_excl, int n_glob,
+                                      int *acc_buf, int32_t *out) {
     const int lane = lane_id();
     const int r = L.r;
     if (r == 0) return;
-    const int np = n_valid - n_excl;
+    const int np = n_valid - n_excl - n_glob;   // the global candidates are outside the pool
     int acc = 0;
     if (np > r) {
         for (int t0 = 0; acc < r && t0 < L.max_draws; t0 += 32) {
@@ -99,7 +99,8 @@ __device__ void draw_random_sentinels(const LedgerDev &L, int ghead, int row, in
             const int sel = t & 3;
             const uint32_t w = sel == 0 ? o.w[0] : sel == 1 ? o.w[1] : sel == 2 ? o.w[2] : o.w[3];
             const int j = (int)__umulhi(w, (uint32_t)n_valid);
-            const bool cand = t < L.max_draws && !in_list(excl, n_excl, j) && !in_list(acc_buf, acc, j);
+            const bool cand = t < L.max_draws && !in_list(excl, n_excl, j) &&
+                              !is_global_cand(L, row, n_valid, j) && !in_list(acc_buf, acc, j);
             const unsigned cm = __ballot_sync(kFull, cand);
             const unsigned same = __match_any_sync(kFull, j) & cm;
             const bool first = cand && ((same & lanemask_lt()) == 0);
@@ -113,7 +114,8 @@ __device__ void draw_random_sentinels(const LedgerDev &L, int ghead, int row, in
     }
     for (int j0 = 0; acc < r && j0 < n_valid; j0 += 32) {
         const int j = j0 + lane;
-        const bool cand = j < n_valid && !in_list(excl, n_excl, j) && !in_list(acc_buf, acc, j);
+        const bool cand = j < n_valid && !in_list(excl, n_excl, j) &&
+                          !is_global_cand(L, row, n_valid, j) && !in_list(acc_buf, acc, j);
         const unsigned cm = __ballot_sync(kFull, cand);
         const int pos = acc + __popc(cm & lanemask_lt());
         if (cand && pos < r) acc_buf[pos] = j;
@@ -252,7 +254,20 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
             else id = (e - L.k) < nm ? bi[nr + e - L.k] : -1;
             out[e] = id;
         }
-        draw_random_sentinels(L, L.bh_offset + h, row, layer, n_valid, bi, nr + nm,
+        // mandatory global sentinels (g <= 32), after the random block
+        const int g = L.g_sink + L.g_recent;
+        int n_glob = 0;
+        if (g > 0) {
+            const int jg = lane < g ? global_cand(L, row, lane) : -1;
+            const bool keep = lane < g && global_cand_listable(L, lane, jg, n_valid) &&
+                              !in_list(bi, nr + nm, jg);
+            const unsigned km = __ballot_sync(kFull, keep);
+            n_glob = __popc(km);
+            int32_t *gout = out + L.k + L.m + L.r;
+            if (keep) gout[__popc(km & lanemask_lt())] = jg;
+            if (lane >= n_glob && lane < g) gout[lane] = -1;
+        }
+        draw_random_sentinels(L, L.bh_offset + h, row, layer, n_valid, bi, nr + nm, n_glob,
                               rnd_all + warp * kRandMax, out + L.k + L.m);
         if (lane == 0) {
             L.alpha[grow] = bs[nr - 1];

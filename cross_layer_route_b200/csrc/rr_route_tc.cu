@@ -591,13 +591,23 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             int32_t *out = L.ids + grow * L.c;
             for (int e = 0; e < L.k; ++e) out[e] = e < nr ? key_chunk(H[e * kRows]) : -1;
             for (int e = 0; e < L.m; ++e) out[L.k + e] = e < nm ? key_chunk(H[(nr + e) * kRows]) : -1;
+            auto in_rn = [&](int j) {
+                for (int e = 0; e < nsel; ++e)
+                    if (key_chunk(H[e * kRows]) == j) return true;
+                return false;
+            };
+            // mandatory global sentinels, after the random block
+            const int g = L.g_sink + L.g_recent;
+            int n_glob = 0;
+            int32_t *gout = out + L.k + L.m + L.r;
+            for (int t = 0; t < g; ++t) {
+                const int j = global_cand(L, row, t);
+                if (global_cand_listable(L, t, j, n_valid) && !in_rn(j)) gout[n_glob++] = j;
+            }
+            for (int t = n_glob; t < g; ++t) gout[t] = -1;
             random_sentinels(
-                L, L.bh_offset + h, row, layer, n_valid, nsel,
-                [&](int j) {
-                    for (int e = 0; e < nsel; ++e)
-                        if (key_chunk(H[e * kRows]) == j) return true;
-                    return false;
-                },
+                L, L.bh_offset + h, row, layer, n_valid, nsel + n_glob,
+                [&](int j) { return in_rn(j) || is_global_cand(L, row, n_valid, j); },
                 [&](int e) -> int & { return bi[e * kRows]; }, out + L.k + L.m, nullptr);
             L.alpha[grow] = key_score(H[(nr - 1) * kRows]);
             L.anchor_layer[grow] = layer;
@@ -747,8 +757,9 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
         __syncwarp();
     }
     int acc = 0;
-    // chunk j selected or accepted (this lane's j; accepted ones in w.acc[0..acc))
-    auto taken = [&](int j) -> bool {
+    // chunk j in route U near-miss, or accepted as a random sentinel (this
+    // lane's j; accepted ones are in the bitmap, or in w.acc[0..acc))
+    auto in_sel_or_acc = [&](int j) -> bool {
         if (use_bits) return ((w.bits[j >> 5] >> (j & 31)) & 1u) != 0u;
         bool hit = false;
         for (int src = 0; src < 32; ++src) {
@@ -760,6 +771,25 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
         }
         for (int a = 0; a < acc; ++a) hit |= w.acc[a] == j;
         return hit;
+    };
+    // mandatory global sentinels (g <= 32): lane t examines candidate t; they
+    // are written after the random block and leave the random pool
+    const int g = L.g_sink + L.g_recent;
+    int n_glob = 0;
+    if (g > 0) {
+        const int jg = lane < g ? global_cand(L, row, lane) : -1;
+        const bool listable = lane < g && global_cand_listable(L, lane, jg, n_valid);
+        const bool in_rn = in_sel_or_acc(listable ? jg : 0);   // nothing accepted yet
+        const bool keep = listable && !in_rn;
+        const uint32_t km = __ballot_sync(kFull, keep);
+        n_glob = __popc(km);
+        int32_t *gout = out + L.k + L.m + L.r;
+        if (keep) gout[__popc(km & lt_mask)] = jg;
+        if (lane >= n_glob && lane < g) gout[lane] = -1;
+    }
+    auto taken = [&](int j) -> bool {
+        const bool hit = in_sel_or_acc(j);   // every lane calls it (it may shuffle)
+        return hit || is_global_cand(L, row, n_valid, j);
     };
     // accept this round's free lanes in lane order, up to r in total
     auto accept = [&](bool is_free, int j) {
@@ -773,7 +803,7 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
         __syncwarp();
     };
     if (L.r > 0) {
-        if (n_valid - nsel > L.r) {
+        if (n_valid - nsel - n_glob > L.r) {
             for (int t0 = 0; acc < L.r && t0 < L.max_draws; t0 += 32) {
                 const int t = t0 + lane;
                 const PhiloxOut o = philox4x32_10((uint32_t)(L.bh_offset + h), (uint32_t)row,
@@ -1229,7 +1259,7 @@ EncodeTiledFn encode_fn() {
 
 bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     if (!(dtype == kBF16 && (L.d == 64 || L.d == 128) && L.ksel <= 64 && L.r <= tc::kBuf &&
-          L.nk <= 65535))
+          L.nk <= 65535 && L.c <= 4 * tc::kRescoreIdsPerThread))
         return false;
     // the fused kernel finishes its rows with per-warp scratch in the
     // query/key buffers

@@ -59,7 +59,8 @@ typedef enum { RR_F32 = 0, RR_BF16 = 1 } rr_dtype;
 
 /* Problem statement of one ledger (RouteRelay §2.1, §3.1, §3.2, Table 1).
  * Limits: 1 <= k <= nk; k + m_near <= 128; r_rand <= 128; d a multiple of 8
- * with 8 <= d <= 256; gamma >= 0 and finite; anchor_interval >= 0. */
+ * with 8 <= d <= 256; gamma >= 0 and finite; anchor_interval >= 0;
+ * g_sink, g_recent >= 0 with g_sink + g_recent <= 32. */
 typedef struct {
     int32_t bh;              /* batch x heads held by this ledger */
     int32_t nq;              /* query chunks per head */
@@ -74,6 +75,8 @@ typedef struct {
     float gamma;             /* guard margin of Eq. 8 */
     int32_t bh_offset;       /* global index of this ledger's head 0 (keys the random draws) */
     uint64_t seed;           /* seed of the random sentinels */
+    int32_t g_sink;          /* mandatory global sentinels (§3.1 item 3): sink chunks 0..g_sink-1 */
+    int32_t g_recent;        /* ... and the row's recent chunks i-g_recent+1..i (0: none) */
 } rr_config;
 
 /* Opaque host-side handle.  It holds pointers into the caller's workspace
@@ -99,8 +102,8 @@ enum {
 
 /* Bytes of device workspace a ledger with this config needs (0 if the
  * config is invalid).  The workspace holds the ledger proper -- ids
- * [bh*nq, c] int32 with c = k + m_near + r_rand (route | near-miss |
- * random), alpha [bh*nq] f32, anchor layer [bh*nq] int32, refresh flags
+ * [bh*nq, c] int32 with c = k + m_near + r_rand + g_sink + g_recent
+ * (route | near-miss | random | global), alpha [bh*nq] f32, anchor layer [bh*nq] int32, refresh flags
  * [bh*nq] u8, counters [16] int64 -- plus the library's per-layer scratch
  * (refresh lists and counts; for problems routed on the tensor cores also
  * the kept scores each row hands from the selection kernel to the kernel
@@ -126,12 +129,16 @@ rr_status rr_ledger_destroy(rr_ledger *ledger);
  * anchor layer constructs this state from a complete chunk-score matrix").
  * For every query row the library scores all valid key chunks, takes the
  * k + m_near best (score descending, index ascending): the first k become
- * the route, the next m_near the near-miss sentinels; r_rand random
- * sentinels are drawn without replacement from the remaining valid chunks
- * (§3.1 item 2, §3.4) with Philox4x32-10 (Salmon et al., SC'11), key
- * (seed lo, seed hi), counter (bh_offset + head, row, layer, t/4), word t%4,
- * chunk = (word * n_valid) >> 32, rejecting repeats; if the pool holds no
- * more than r_rand chunks it is taken whole in ascending order.  alpha
+ * the route, the next m_near the near-miss sentinels.  The mandatory
+ * global sentinels (§3.1 item 3) are the sink chunks 0..g_sink-1 and then
+ * the row's recent chunks i-g_recent+1..i, each kept if valid, outside the
+ * route and near-miss and not already listed, in that order, -1 padded to
+ * g_sink + g_recent slots at the end of the row.  r_rand random sentinels
+ * are drawn without replacement from the remaining valid chunks (§3.1 item
+ * 2, §3.4) with Philox4x32-10 (Salmon et al., SC'11), key (seed lo, seed
+ * hi), counter (bh_offset + head, row, layer, t/4), word t%4, chunk = (word
+ * * n_valid) >> 32, rejecting repeats; if the pool holds no more than
+ * r_rand chunks it is taken whole in ascending order.  alpha
  * becomes the route's weakest score, the anchor layer becomes `layer`, every
  * refresh flag becomes 1.  Starts a new layer sequence at any `layer` >= 0.
  * The score matrix never reaches device memory.  Errors: RR_EINVAL,

@@ -22,15 +22,17 @@ import oracle
 TIE_REL = 1e-5
 
 
-def params_of(w, bh_offset: int = 0, max_age: int = 0, min_reuse: int = 0) -> oracle.Params:
+def params_of(w, bh_offset: int = 0, max_age: int = 0, min_reuse: int = 0, g_sink: int = 0,
+              g_recent: int = 0) -> oracle.Params:
     return oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal,
-                         gamma=w.gamma, seed=w.seed, max_age=max_age, min_reuse=min_reuse)
+                         gamma=w.gamma, seed=w.seed, max_age=max_age, min_reuse=min_reuse,
+                         g_sink=g_sink, g_recent=g_recent)
 
 
-def config_of(w, rr, bh: int | None = None, bh_offset: int = 0):
+def config_of(w, rr, bh: int | None = None, bh_offset: int = 0, g_sink: int = 0, g_recent: int = 0):
     return rr.Config(bh=w.bh if bh is None else bh, nq=w.n, nk=w.n, d=w.d, k=w.k, m_near=w.m,
                      r_rand=w.r, dtype=w.dtype, anchor_interval=w.anchor_interval, causal=w.causal,
-                     gamma=w.gamma, seed=w.seed, bh_offset=bh_offset)
+                     gamma=w.gamma, seed=w.seed, bh_offset=bh_offset, g_sink=g_sink, g_recent=g_recent)
 
 
 @dataclass
@@ -98,8 +100,15 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
         nm = min(p.m, nv - nr)
         route = [int(x) for x in g[: p.k] if x >= 0]
         near = [int(x) for x in g[p.k:p.k + p.m] if x >= 0]
-        rand = [int(x) for x in g[p.k + p.m:] if x >= 0]
-        allids = route + near + rand
+        rand = [int(x) for x in g[p.k + p.m:p.k + p.m + p.r] if x >= 0]
+        glob = [int(x) for x in g[p.k + p.m + p.r:]]
+        want = []
+        for t, j in enumerate(list(range(p.g_sink)) + list(range(i - p.g_recent + 1, i + 1))):
+            if 0 <= j < nv and not (t >= p.g_sink and j < p.g_sink) and j not in route + near:
+                want.append(j)
+        if glob != want + [-1] * (p.g_sink + p.g_recent - len(want)):
+            return "global sentinels"
+        allids = route + near + rand + want
         if len(route) != nr or len(near) != nm or len(set(allids)) != len(allids):
             return "wrong counts or repeated ids"
         if any(x < 0 or x >= nv for x in allids):
@@ -108,7 +117,7 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
             return "route member below the k-th score"
         if nm and any(S[i, j] < srt[nr + nm - 1] - tol[i] or S[i, j] > srt[nr - 1] + tol[i] for j in near):
             return "near-miss member outside its rank band"
-        if len(rand) != min(p.r, nv - nr - nm):
+        if len(rand) != min(p.r, nv - nr - nm - len(want)):
             return "wrong random count"
         if abs(float(gpu_alpha[i]) - srt[nr - 1]) > tol[i]:
             return "alpha"
@@ -186,7 +195,8 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
 
 
 def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None,
-                  gamma_rows=None, max_age: int = 0, min_reuse: int = 0):
+                  gamma_rows=None, max_age: int = 0, min_reuse: int = 0, g_sink: int = 0,
+                  g_recent: int = 0):
     """Runs `layers` layers of workload w through the CUDA ledger `led` and
     compares every layer of the listed heads with the oracle started from
     the GPU's own previous ledger.  gamma_rows ([bh, nq] array) and max_age
@@ -195,7 +205,7 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
     import rr_workloads
     import torch
     st = rr_workloads.LayerStream(w, stream_device)
-    p = params_of(w, max_age=max_age, min_reuse=min_reuse)
+    p = params_of(w, max_age=max_age, min_reuse=min_reuse, g_sink=g_sink, g_recent=g_recent)
     total = Report()
     per_layer = []
     prev = None

@@ -315,3 +315,41 @@ def test_hysteresis_horizon(rr, case):
     # under this drift the test refreshes nearly every row, so the horizon
     # keeps about every other layer's rows
     assert sum(lr.refreshed_gpu for lr in relay) < 0.75 * sum(lr.rows for lr in relay)
+
+
+GLOBALS = [
+    (W.C5.with_(bh=2, n=384, layers=5), "bf16_tensor_cores"),
+    (W.C3.with_(bh=2, n=256, layers=5), "f32_cuda_cores"),
+]
+
+
+@pytest.mark.parametrize("case", GLOBALS, ids=[c[1] for c in GLOBALS])
+def test_global_sentinels_layer_by_layer(rr, case):
+    """Mandatory global sentinels (RouteRelay §3.1 item 3: 2 sink and 3
+    recent chunks per row) on anchor and relay layers, against the oracle."""
+    w, _ = case
+    led = rr.RouteLedger(config_of(w, rr, g_sink=2, g_recent=3), DEV)
+    rep, per_layer = layer_stepped(w, rr, led, w.layers, range(w.bh), DEV, g_sink=2, g_recent=3)
+    _check(rep)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_global_sentinels_on_equal_scores_match_the_oracle(rr, dtype, d):
+    """All scores of a row tie, so route, near-miss and globals are fixed by
+    the index order and the random draws by the exclusion set: every id must
+    equal the oracle's.  On the tensor-core path these rows take the retry
+    kernel."""
+    bh, n, k, m, r, gs, gr = 1, 200, 8, 6, 4, 2, 3
+    cfg = rr.Config(bh=bh, nq=n, nk=n, d=d, k=k, m_near=m, r_rand=r, dtype=dtype, causal=True,
+                    g_sink=gs, g_recent=gr, seed=11)
+    g = torch.Generator().manual_seed(6)
+    q = torch.randn((bh, n, d), generator=g)
+    kk = torch.randn((bh, 1, d), generator=g).expand(bh, n, d).contiguous()
+    td = torch.bfloat16 if dtype == "bf16" else torch.float32
+    led = rr.RouteLedger(cfg, DEV)
+    led.full_route(q.to(td).to(DEV), kk.to(td).to(DEV), 0)
+    out = led.read()
+    p = oracle.Params(nq=n, nk=n, d=d, k=k, m=m, r=r, causal=True, seed=11, g_sink=gs, g_recent=gr)
+    ol = oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q.to(td).float()[0].numpy(), kk.to(td).float()[0].numpy(), ol)
+    assert np.array_equal(out["ids"][0].numpy(), ol.ids)
