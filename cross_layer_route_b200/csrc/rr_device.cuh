@@ -53,9 +53,11 @@ __device__ __forceinline__ bool is_global_cand(const LedgerDev &L, int row, int 
 // hysteresis horizon; min_reuse 0 = off).
 __device__ __forceinline__ bool relay_refresh(const LedgerDev &L, size_t grow, int layer,
                                               float alpha, float beta) {
-    const int age = layer - L.anchor_layer[grow];
-    if (L.max_age > 0 && age >= L.max_age) return true;
-    if (L.min_reuse > 0 && age <= L.min_reuse) return false;
+    if (L.max_age > 0 || L.min_reuse > 0) {   // the row's age is read only when needed
+        const int age = layer - L.anchor_layer[grow];
+        if (L.max_age > 0 && age >= L.max_age) return true;
+        if (L.min_reuse > 0 && age <= L.min_reuse) return false;
+    }
     const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
     return !(alpha > beta + g);
 }
