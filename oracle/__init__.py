@@ -12,6 +12,10 @@ Dynamic Sparse Attention" (arXiv 2609.07306), abbreviated RouteRelay:
 §3.2 Eq. 5-8 (relay test and refresh), §3.2 "Forced anchors" (anchor every
 H layers), §4.1 (ledger dataflow), §5.1-5.2 (recall, rerouted rows, score
 pairs).
+
+The submodule ``oracle.attention`` (plain NumPy, fp64) is the oracle of the
+downstream consumer of a route: token expansion and the sparse attention of
+§2.2 Eq. 3.
 """
 from __future__ import annotations
 
@@ -290,3 +294,6 @@ def pair_fraction_from_counts(n_layers: int, rows: int, n_valid_per_row: int, c:
     for ref in refreshed_per_relay_layer:
         total += rows * c + ref * n_valid_per_row
     return total / (n_layers * rows * n_valid_per_row)
+
+
+from .attention import expand_route, sparse_attention, sparse_attention_head, sparse_attention_rows  # noqa: E402,F401
