@@ -4,7 +4,9 @@ Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
 Dynamic Sparse Attention" (arXiv 2609.07306).  Anchor layers fully route
 every query chunk (S = Qc Kc^T, top-k, §2.1 Eq. 1-2); intermediate layers
 rescore each row's ledger candidates, test alpha > beta + gamma (§3.2 Eq.
-5-8) and fully re-route only the rows that fail (§4.1-4.2).
+5-8) and fully re-route only the rows that fail (§4.1-4.2).  The routes feed
+a sparse attention over their chunks' tokens (§2.1, Eq. 3; sparse_attention,
+RouteLedger.sparse_attention).
 
 This module only marshals arguments: every step of the routing path runs in
 the CUDA kernels of librr.so.  There is no CPU fallback; importing it without
@@ -43,6 +45,12 @@ class rr_ledger_view(ctypes.Structure):
                 ("counters", ctypes.c_void_p)]
 
 
+class rr_attn_config(ctypes.Structure):
+    _fields_ = [("bh", ctypes.c_int32), ("nq_tokens", ctypes.c_int32), ("nk_tokens", ctypes.c_int32),
+                ("dh", ctypes.c_int32), ("chunk", ctypes.c_int32), ("width", ctypes.c_int32),
+                ("route_stride", ctypes.c_int32), ("causal", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"librr.so is not built ({LIB_PATH}); run python cross_layer_route_b200/build.py")
@@ -70,6 +78,8 @@ def _load():
     lib.rr_ledger_set_hysteresis.restype = ctypes.c_int
     lib.rr_route_layer_static.argtypes = [ctypes.POINTER(rr_config), P, P, ctypes.c_int32, P, P, P, P, P, P]
     lib.rr_route_layer_static.restype = ctypes.c_int
+    lib.rr_sparse_attention.argtypes = [ctypes.POINTER(rr_attn_config), P, P, P, P, P, P]
+    lib.rr_sparse_attention.restype = ctypes.c_int
     lib.rr_status_string.argtypes = [ctypes.c_int]
     lib.rr_status_string.restype = ctypes.c_char_p
     return lib
@@ -164,6 +174,14 @@ def rr_route_layer_static(cfg: rr_config, d_qc: int, d_kc: int, layer: int, d_id
            "rr_route_layer_static")
 
 
+def rr_sparse_attention(cfg: rr_attn_config, d_q: int, d_k: int, d_v: int, d_route: int, d_out: int,
+                        stream: int) -> None:
+    """Sparse attention over a route (include/rr_attention.h)."""
+    _check(_lib.rr_sparse_attention(ctypes.byref(cfg), ctypes.c_void_p(d_q), ctypes.c_void_p(d_k),
+                                    ctypes.c_void_p(d_v), ctypes.c_void_p(d_route), ctypes.c_void_p(d_out),
+                                    ctypes.c_void_p(stream)), "rr_sparse_attention")
+
+
 # ---- convenience wrapper over torch memory --------------------------------
 @dataclass
 class Config:
@@ -205,6 +223,41 @@ def _stream_handle(stream) -> int:
     if isinstance(stream, int):
         return stream
     return stream.cuda_stream
+
+
+def sparse_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, route: torch.Tensor, chunk: int,
+                     causal: bool = False, width: int | None = None, scale: float | None = None,
+                     out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Attention of every query token over the tokens of its chunk's route
+    (RouteRelay §2.1, Eq. 3).  q [bh, nq_tokens, dh], k and v [bh, nk_tokens,
+    dh]: contiguous bf16 on one CUDA device; route: contiguous int32 [bh,
+    nq_tokens // chunk, stride] of key-chunk ids, of which the first `width`
+    (default: all) are read.  Returns (or fills) fp32 [bh, nq_tokens, dh]."""
+    bh, nq_tok, dh = q.shape
+    nk_tok = k.shape[1]
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous() or t.dim() != 3 \
+                or t.shape[0] != bh or t.shape[2] != dh or t.device != q.device:
+            raise ValueError(f"{name}: expected contiguous bf16 [bh, tokens, {dh}] on {q.device}, "
+                             f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+    if tuple(v.shape) != tuple(k.shape):
+        raise ValueError(f"v {tuple(v.shape)} must match k {tuple(k.shape)}")
+    if route.dtype != torch.int32 or not route.is_contiguous() or route.device != q.device or route.dim() != 3 \
+            or route.shape[0] != bh or route.shape[1] * chunk != nq_tok:
+        raise ValueError(f"route: expected contiguous int32 [{bh}, {nq_tok // max(chunk, 1)}, stride] on "
+                         f"{q.device}, got {route.dtype} {tuple(route.shape)} on {route.device}")
+    stride = route.shape[2]
+    width = stride if width is None else int(width)
+    if out is None:
+        out = torch.empty((bh, nq_tok, dh), dtype=torch.float32, device=q.device)
+    elif out.dtype != torch.float32 or not out.is_contiguous() or tuple(out.shape) != (bh, nq_tok, dh) \
+            or out.device != q.device:
+        raise ValueError("out: expected contiguous float32 [bh, nq_tokens, dh] on the inputs' device")
+    cfg = rr_attn_config(bh, nq_tok, nk_tok, dh, chunk, width, max(stride, 1), int(bool(causal)),
+                         0.0 if scale is None else float(scale))
+    rr_sparse_attention(cfg, q.data_ptr(), k.data_ptr(), v.data_ptr(), route.data_ptr(), out.data_ptr(),
+                        _stream_handle(stream))
+    return out
 
 
 class RouteLedger:
@@ -312,6 +365,18 @@ class RouteLedger:
                 "anchor_layer": view(v.anchor_layer, rows * 4, torch.int32, (c.bh, c.nq)),
                 "flags": view(v.flags, rows, torch.uint8, (c.bh, c.nq)),
                 "counters": view(v.counters, NUM_COUNTERS * 8, torch.int64, (NUM_COUNTERS,))}
+
+    def sparse_attention(self, q, k, v, chunk: int, out=None, stream=None) -> torch.Tensor:
+        """Attention over the ledger's current routes (the first k ids of each
+        row, read in place): q [bh, nq * chunk, dh], k and v [bh, nk * chunk,
+        dh] bf16 token tensors of the same layer, with the ledger's causal rule
+        applied at token level."""
+        c = self.cfg
+        if q.shape[0] != c.bh or q.shape[1] != c.nq * chunk or k.shape[1] != c.nk * chunk:
+            raise ValueError(f"q/k: expected [{c.bh}, {c.nq * chunk}, dh] / [{c.bh}, {c.nk * chunk}, dh], "
+                             f"got {tuple(q.shape)} / {tuple(k.shape)}")
+        ids = self.device_view()["ids"]
+        return sparse_attention(q, k, v, ids, chunk, causal=c.causal, width=c.k, out=out, stream=stream)
 
     def layer(self, qc, kc, layer: int, stream=None):
         """Layer l of a sequence: an anchor at l == 0, else rr_relay_layer

@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librr.so")
-SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_route_tc.cu", "rr_relay.cu", "rr_noalloc.cu"]
+SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_route_tc.cu", "rr_relay.cu", "rr_noalloc.cu", "rr_attention.cu"]
 HEADERS = ["rr_device.cuh", "rr_internal.h"]
 
 
@@ -33,7 +33,8 @@ def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(ROOT, "include", "rr.h")]
+    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + \
+        [os.path.join(ROOT, "include", h) for h in ("rr.h", "rr_attention.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 

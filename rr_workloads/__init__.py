@@ -117,3 +117,58 @@ class LayerStream:
 
 def storage_dtype(w: Workload) -> torch.dtype:
     return torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+
+# ---- token-level inputs of the sparse attention that consumes a route ------
+@dataclass(frozen=True)
+class AttentionWorkload:
+    """One layer's token tensors for the attention over a route: bh heads of
+    n_chunks chunks of `chunk` tokens, head dim dh, route width k."""
+    name: str
+    bh: int
+    n_chunks: int
+    chunk: int
+    dh: int
+    k: int
+    causal: bool
+    seed: int = 0
+
+    @property
+    def tokens(self) -> int:
+        return self.n_chunks * self.chunk
+
+
+# Four heads of the largest routing workload at token level: 4096 chunks of
+# 64 tokens (256K tokens per head), head dim 128, the route width 32.
+ATTN_C5 = AttentionWorkload("attn_bh4_n4096_c64_dh128_bf16_causal", 4, 4096, 64, 128, 32, True)
+
+
+def attention_tokens(bh: int, n_tokens: int, dh: int, seed: int, device="cpu"):
+    """q, k, v with N(0, 1) entries, rounded to bf16: [bh, n_tokens, dh] each
+    (a head's logits q.k / sqrt(dh) are then about N(0, 1))."""
+    g = torch.Generator(device=torch.device(device)).manual_seed(1000 + seed)
+    return tuple(torch.randn((bh, n_tokens, dh), generator=g, device=device, dtype=torch.float32)
+                 .to(torch.bfloat16) for _ in range(3))
+
+
+def random_routes(bh: int, nq_chunks: int, nk_chunks: int, width: int, causal: bool, seed: int,
+                  stride: int | None = None, pad: float = 0.0, junk: int = 0) -> torch.Tensor:
+    """Routes for the attention: per query chunk i, min(width, valid) distinct
+    key-chunk ids drawn uniformly from the valid ones (0..i when causal,
+    else 0..nk_chunks-1), in random order, then a fraction `pad` of the
+    entries replaced by -1; int32 [bh, nq_chunks, stride] on the CPU.
+    Columns width..stride-1 hold `junk` (a reader must not use them)."""
+    import numpy as np
+    stride = width if stride is None else stride
+    rng = np.random.default_rng(5000 + seed)
+    out = np.full((bh, nq_chunks, stride), junk, dtype=np.int32)
+    out[:, :, :width] = -1
+    for h in range(bh):
+        for i in range(nq_chunks):
+            n_valid = min(i + 1, nk_chunks) if causal else nk_chunks
+            ids = rng.choice(n_valid, size=min(width, n_valid), replace=False)
+            out[h, i, :ids.size] = ids
+            if pad > 0:
+                drop = rng.random(width) < pad
+                out[h, i, :width][drop] = -1
+    return torch.from_numpy(out)

@@ -135,3 +135,39 @@ def test_trigger_setters_validate_their_arguments_without_a_cuda_call():
         assert lib.rr_ledger_set_hysteresis(None, 1) == rr.RR_EINVAL
     finally:
         lib.rr_ledger_destroy(h)
+
+
+# ---- rr_sparse_attention (include/rr_attention.h) --------------------------
+def attn_cfg(**kw):
+    base = dict(bh=2, nq_tokens=256, nk_tokens=256, dh=128, chunk=64, width=4, route_stride=8, causal=1,
+                scale=0.0)
+    base.update(kw)
+    return rr.rr_attn_config(*(base[f] for f, _ in rr.rr_attn_config._fields_))
+
+
+@pytest.mark.parametrize("bad", [
+    dict(dh=96), dict(dh=0), dict(chunk=48), dict(chunk=256), dict(nq_tokens=100), dict(nk_tokens=65),
+    dict(width=-1), dict(width=1025, route_stride=2048), dict(route_stride=3), dict(route_stride=0, width=0),
+    dict(bh=-1), dict(nq_tokens=-64), dict(scale=-1.0), dict(scale=float("nan")), dict(scale=float("inf")),
+])
+def test_attention_rejects_bad_shapes_without_a_cuda_call(bad):
+    with pytest.raises(rr.RRError) as e:
+        rr.rr_sparse_attention(attn_cfg(**bad), FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, 0)
+    assert e.value.status == rr.RR_EINVAL
+
+
+def test_attention_rejects_null_and_misaligned_pointers():
+    c = attn_cfg()
+    for args in ((0, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q), (FAKE_Q + 8, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q),
+                 (FAKE_Q, 0, FAKE_Q, FAKE_Q, FAKE_Q), (FAKE_Q, FAKE_Q, FAKE_Q + 2, FAKE_Q, FAKE_Q),
+                 (FAKE_Q, FAKE_Q, FAKE_Q, 0, FAKE_Q), (FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q + 2, FAKE_Q),
+                 (FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q + 4)):
+        with pytest.raises(rr.RRError) as e:
+            rr.rr_sparse_attention(c, *args, 0)
+        assert e.value.status == rr.RR_EINVAL
+
+
+def test_attention_with_nothing_to_do_returns_at_once():
+    # no query token: nothing is launched, so even fake pointers are fine
+    rr.rr_sparse_attention(attn_cfg(bh=0), FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, 0)
+    rr.rr_sparse_attention(attn_cfg(nq_tokens=0), FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, 0)
