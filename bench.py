@@ -12,7 +12,7 @@ anchor every 16, top-32 with 32 near-miss and 16 random sentinels, drift
 sigma 0.03.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload NAME]
+                    [--workload NAME] [--attention]
 
 Prints one JSON line (rank 0).  With N > 1 (launched by torchrun) every
 rank routes its own BH units (heads are independent: no collective on the
@@ -418,6 +418,55 @@ def measure_recall(w, state, device):
     return sum(rec) / len(rec), min(rec)
 
 
+def measure_attention(args, w, state, device):
+    """The consumer of the routes (opt-in, outside the timed step): sparse
+    attention over the ledger's current routes for the first heads of the
+    ledger, at token level (chunks of W.ATTN_C5.chunk tokens, head dim
+    W.ATTN_C5.dh, seeded N(0, 1) bf16 q, k, v).  Useful work = 4 * dh flops
+    per visible (query token, key token) pair: q.k and p.v."""
+    import cross_layer_route_b200 as rr
+    led, qs, ks, cfg = state
+    a = W.ATTN_C5
+    heads = min(a.bh, w.bh)
+    q, k, v = (x.to(device) for x in W.attention_tokens(heads, w.n * a.chunk, a.dh, seed=a.seed))
+    route = led.device_view()["ids"][:heads]               # [heads, n, c], first k ids read
+    out = torch.empty((heads, w.n * a.chunk, a.dh), dtype=torch.float32, device=device)
+    # visible pairs of these routes (host arithmetic on a copy of the ids)
+    ids = route[:, :, :w.k].cpu().long()
+    i_idx = torch.arange(w.n)[None, :, None]
+    valid = (ids >= 0) & (ids < w.n) & ((ids <= i_idx) if w.causal else True)
+    full = valid & ((ids < i_idx) if w.causal else True)
+    diag = valid & (ids == i_idx) if w.causal else torch.zeros_like(valid)
+    pairs = int(full.sum()) * a.chunk * a.chunk + int(diag.sum()) * a.chunk * (a.chunk + 1) // 2
+    stream = torch.cuda.current_stream(device)
+
+    def call():
+        rr.sparse_attention(q, k, v, route, a.chunk, causal=w.causal, width=w.k, out=out, stream=stream)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize(device)
+    n = 10
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(n):
+        call()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = t0.elapsed_time(t1) / n
+    peaks = load_peaks()
+    tflops = 4.0 * a.dh * pairs / (ms * 1e-3) / 1e12
+    return {"kernel": "sparse_attention_kernel (bf16 mma.sync, online softmax)",
+            "workload": f"attn_bh{heads}_n{w.n}_c{a.chunk}_dh{a.dh}_bf16" + ("_causal" if w.causal else ""),
+            "routes": "the ledger's routes after the last layer", "bound": "tensor",
+            "avg_launch_ms": round(ms, 4), "tokens_per_s": heads * w.n * a.chunk / (ms * 1e-3),
+            "achieved": round(tflops, 2), "unit": "TFLOP/s", "peak": float(peaks["bf16_tflops"]),
+            "frac": round(tflops / float(peaks["bf16_tflops"]), 4),
+            "peak_source": f"{peaks['source']} bf16 dense, burst (timed alone)",
+            "visible_pairs": pairs, "launches": n}
+
+
 # ------------------------------------------------------- CPU baseline ------
 def cpu_baseline(w, qs, ks, threads=None, layers=2):
     """The oracle as it stands, on a bounded sample: `threads` heads (one per
@@ -490,6 +539,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-recall", action="store_true")
+    ap.add_argument("--attention", action="store_true",
+                    help="also time the sparse attention over the ledger's routes (not part of the step)")
     ap.add_argument("--smi-index", type=int, default=None)
     ap.add_argument("--bh", type=int, default=None, help="override BH (profiling a smaller case)")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
@@ -521,6 +572,8 @@ def main():
         r_mean, r_min = measure_recall(w, state, device)
         result["recall"] = r_mean
         result["recall_min_layer"] = r_min
+    if args.attention and rank == 0:
+        result["kernels"]["attention"] = measure_attention(args, w, state, device)
     if not args.no_e2e:
         e2e = measure_e2e(args, w, state, device)
         if world > 1:
