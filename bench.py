@@ -418,6 +418,23 @@ def measure_recall(w, state, device):
     return sum(rec) / len(rec), min(rec)
 
 
+def visible_pairs(route: torch.Tensor, nk_chunks: int, chunk: int, causal: bool) -> int:
+    """(query token, key token) pairs the attention over `route` ([bh,
+    nq_chunks, width] key-chunk ids) evaluates: a usable off-diagonal chunk
+    gives chunk^2 pairs, the causal diagonal chunk chunk (chunk + 1) / 2;
+    -1, out-of-range ids and (causal) ids past the query chunk give none."""
+    ids = route.long()
+    i_idx = torch.arange(ids.shape[1])[None, :, None]
+    usable = (ids >= 0) & (ids < nk_chunks)
+    if causal:
+        full = usable & (ids < i_idx)
+        diag = usable & (ids == i_idx)
+    else:
+        full = usable
+        diag = torch.zeros_like(usable)
+    return int(full.sum()) * chunk * chunk + int(diag.sum()) * chunk * (chunk + 1) // 2
+
+
 def measure_attention(args, w, state, device):
     """The consumer of the routes (opt-in, outside the timed step): sparse
     attention over the ledger's current routes for the first heads of the
@@ -431,13 +448,7 @@ def measure_attention(args, w, state, device):
     q, k, v = (x.to(device) for x in W.attention_tokens(heads, w.n * a.chunk, a.dh, seed=a.seed))
     route = led.device_view()["ids"][:heads]               # [heads, n, c], first k ids read
     out = torch.empty((heads, w.n * a.chunk, a.dh), dtype=torch.float32, device=device)
-    # visible pairs of these routes (host arithmetic on a copy of the ids)
-    ids = route[:, :, :w.k].cpu().long()
-    i_idx = torch.arange(w.n)[None, :, None]
-    valid = (ids >= 0) & (ids < w.n) & ((ids <= i_idx) if w.causal else True)
-    full = valid & ((ids < i_idx) if w.causal else True)
-    diag = valid & (ids == i_idx) if w.causal else torch.zeros_like(valid)
-    pairs = int(full.sum()) * a.chunk * a.chunk + int(diag.sum()) * a.chunk * (a.chunk + 1) // 2
+    pairs = visible_pairs(route[:, :, :w.k].cpu(), w.n, a.chunk, w.causal)
     stream = torch.cuda.current_stream(device)
 
     def call():

@@ -1,0 +1,63 @@
+"""Host-side arithmetic of bench.py, checked without a GPU: the visible-pair
+count behind the attention roofline, the clock-record summary that decides
+whether a run is kept, the lookup of a profiled traffic figure by source
+hash, and the config block both arms print."""
+import hashlib
+
+import pytest
+
+import bench
+import oracle
+import rr_workloads as W
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_visible_pairs_match_brute_force(causal):
+    n, chunk, width = 10, 4, 5
+    route = W.random_routes(2, n, n, width, causal, seed=9, pad=0.3)
+    route[0, 3, 0] = n + 2            # out of range: no pairs
+    route[1, 2, 1] = 7                # past the query chunk: none under causal
+    brute = 0
+    for h in range(2):
+        for i in range(n):
+            toks = oracle.expand_route(route[h, i].numpy(), chunk, n)
+            for t in range(i * chunk, (i + 1) * chunk):
+                brute += int((toks <= t).sum()) if causal else toks.size
+    assert bench.visible_pairs(route, n, chunk, causal) == brute
+
+
+def test_clock_summary_reads_reasons_and_the_loaded_median():
+    c = bench.ClockSampler(0)
+    row = "0, {sm}, 1965, 700.0, 0x0, {hw}, Not Active, Not Active, {pc}"
+    c.lines = [row.format(sm=345, hw="Not Active", pc="Not Active")] + \
+              [row.format(sm=s, hw="Not Active", pc="Active" if s == 1900 else "Not Active")
+               for s in (1965, 1965, 1900, 1965)] + ["garbage", "0, N/A, 1965"]
+    s = c.summary()
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965 and s["samples"] == 5
+    assert s["reasons"] == ["sw_power_cap"]
+    c.lines = [row.format(sm=1965, hw="Active", pc="Not Active")]
+    assert c.summary()["reasons"] == ["hw_slowdown"]
+    c.lines = []
+    assert c.summary()["reasons"] == ["unsampled"]
+
+
+def test_profiled_traffic_needs_the_profiled_source(tmp_path, monkeypatch):
+    (tmp_path / "cross_layer_route_b200" / "csrc").mkdir(parents=True)
+    (tmp_path / "profiles").mkdir()
+    src = tmp_path / "cross_layer_route_b200" / "csrc" / "k.cu"
+    src.write_text("kernel v1\n")
+    sha = hashlib.sha256(b"kernel v1\n").hexdigest()
+    (tmp_path / "profiles" / "k__case.md").write_text(f"x\ntraffic_bytes_per_row: 1234\nsource_sha256: {sha}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic_per_row("k.cu", "k__*.md") == 1234.0
+    src.write_text("kernel v2\n")                       # the kernel changed: the counters are stale
+    assert bench.profiled_traffic_per_row("k.cu", "k__*.md") is None
+
+
+def test_config_block_and_shards():
+    cfg = bench.workload_config(W.C5, 4)
+    assert cfg["workload"] == W.C5.name and cfg["bh_per_gpu"] == 256 and cfg["parallelism"].endswith("no collective")
+    assert "16.0 GiB" in cfg["l2"]
+    assert [bench.shard_offset(r, W.C5) for r in range(3)] == [0, 256, 512]
+    assert bench.full_pairs_per_layer(W.C5) == 256 * 4096 * 4097 // 2
+    assert bench.full_pairs_per_layer(W.C2) == 128 * 256 * 256
