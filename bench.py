@@ -178,6 +178,17 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def layer_kinds(rows_per_layer: int, anchor_ms: float, n_anchor: int, relay_ms: float, n_relay: int) -> dict:
+    """Anchor and relay layers apart (this rank): layers timed, mean time per
+    layer, and rows per second through that kind of layer."""
+    out = {}
+    for name, ms, n in (("anchor", anchor_ms, n_anchor), ("relay", relay_ms, n_relay)):
+        if n > 0 and ms > 0:
+            out[name] = {"layers": n, "ms_per_layer": round(ms / n, 4),
+                         "rows_per_s": rows_per_layer * n / (ms * 1e-3)}
+    return out
+
+
 def full_pairs_per_layer(w) -> int:
     if not w.causal:
         return w.bh * w.n * w.n
@@ -252,16 +263,20 @@ def run_ours(args, w, rank, world, device):
     c1 = led.read()["counters"].clone()
 
     route_ms = rescore_ms = compact_ms = 0.0
+    anchor_layer_ms = relay_layer_ms = 0.0
     n_route = n_rescore = 0
     for s in range(K):
         for l in range(L):
             if l in anchors:
-                route_ms += evs[s]["anchor"][l].elapsed_time(evs[s]["anchor_end"][l])
+                span = evs[s]["anchor"][l].elapsed_time(evs[s]["anchor_end"][l])
+                route_ms += span
+                anchor_layer_ms += span
                 n_route += 1
             else:
                 rescore_ms += evs[s]["rescore"][l].elapsed_time(evs[s]["compact"][l])
                 compact_ms += evs[s]["compact"][l].elapsed_time(evs[s]["refresh"][l])
                 route_ms += evs[s]["refresh"][l].elapsed_time(evs[s]["refresh_end"][l])
+                relay_layer_ms += evs[s]["rescore"][l].elapsed_time(evs[s]["refresh_end"][l])
                 n_route += 1
                 n_rescore += 1
 
@@ -327,6 +342,8 @@ def run_ours(args, w, rank, world, device):
         "score_pairs_per_s": pairs_per_step * world / (ms_step * 1e-3),
         "pair_fraction": pairs_per_step / (full_pairs_per_layer(w) * L),
         "rho_relay": rho,
+        "layer_kinds": layer_kinds(w.bh * w.n, anchor_layer_ms, K * len(anchors), relay_layer_ms,
+                                   K * len(relays)),
         "retry_rows_per_step": d_cnt[rr.CNT_RETRY_TOTAL] / K,
         "roofline": roofline,
         "kernels": kernels,

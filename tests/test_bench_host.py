@@ -61,3 +61,11 @@ def test_config_block_and_shards():
     assert [bench.shard_offset(r, W.C5) for r in range(3)] == [0, 256, 512]
     assert bench.full_pairs_per_layer(W.C5) == 256 * 4096 * 4097 // 2
     assert bench.full_pairs_per_layer(W.C2) == 128 * 256 * 256
+
+
+def test_layer_kinds_split():
+    k = bench.layer_kinds(1000, anchor_ms=8.0, n_anchor=4, relay_ms=30.0, n_relay=10)
+    assert k["anchor"] == {"layers": 4, "ms_per_layer": 2.0, "rows_per_s": 1000 * 4 / 8e-3}
+    assert k["relay"]["ms_per_layer"] == 3.0 and k["relay"]["rows_per_s"] == pytest.approx(1000 / 3e-3)
+    assert bench.layer_kinds(1000, 5.0, 2, 0.0, 0) == {"anchor": {"layers": 2, "ms_per_layer": 2.5,
+                                                                  "rows_per_s": 1000 * 2 / 5e-3}}
