@@ -9,7 +9,8 @@
 // memory; then draws the random sentinels (§3.1 item 2) and writes the
 // ledger row (§3.1 Eq. 4).  Serves the anchor layer (all rows) and the
 // refresh of the compacted unstable rows (§4.2, rows taken from the
-// per-head list).
+// per-head list).  The relay rescoring on the same tiles
+// (relay_rescore_tc_kernel, §3.2 Eq. 5-8) sits at the end of the file.
 //
 // CTA layout (one CTA = one head x 128 query rows):
 //   warp 0     TMA producer: 128-key x d tiles of Kc (bf16, 128-byte
@@ -20,8 +21,9 @@
 //   warps 2-   epilogue, reading the score tile with tcgen05.ld; a warp may
 //              only read the 32 TMEM lanes (= query rows) of its sub-partition
 //              (warp index mod 4).  The heap kernel runs 4 such warps, one
-//              thread per row; the two-pass kernel runs 8, the two warps of
-//              a sub-partition splitting each tile's columns.
+//              thread per row; the two-pass kernel and the rescoring kernel
+//              run 16, the four warps of a sub-partition each taking a
+//              quarter of every tile's columns.
 // The query tile is gathered by row index into the layout a 128-byte
 // swizzled TMA load would produce, so anchor and refresh share one path.
 //
@@ -37,7 +39,7 @@
 // The kept scores are then ordered (score desc, chunk asc) and the row's
 // ledger entry written by one warp per row (finish_row): in a separate
 // kernel reading the kept scores from global memory, or by the same CTA.  A
-// row whose kept scores do not fit the buffer (kCap-2) is appended to a retry
+// row whose kept scores do not fit the buffer (kCap) is appended to a retry
 // list and routed by route_rows_tc_heap_kernel, which keeps a per-row
 // min-heap of the k+m best over one pass; results are exact either way.
 //
@@ -234,15 +236,6 @@ __device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
         : "r"(taddr));
 }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-// This thread's 64 scores of a tile half: columns c0..c0+63 of its row.
-__device__ __forceinline__ void tc_ld64(uint32_t taddr, float *v) {
-    uint32_t a[32], b[32];
-    tc_ld32_nowait(taddr, a);
-    tc_ld32_nowait(taddr + 32u, b);
-    tc_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) { v[i] = __uint_as_float(a[i]); v[32 + i] = __uint_as_float(b[i]); }
-}
 
 // Shared-memory matrix descriptor of a K-major operand stored as 128-byte
 // swizzled rows (8-row groups 1024 bytes apart): start address >> 4, leading
