@@ -5,7 +5,10 @@
 //
 //  relay_rescore: candidate rescoring and the challenge test (§3.2 Eq. 5-8,
 //      §4.2 "a GPU kernel computes alpha, beta, and one refresh flag per query
-//      row"), one warp per query row.  For d in {64, 128, 256} eight lanes
+//      row").  Shapes the tensor-core full routing serves are rescored from
+//      dense tensor-core tiles instead (relay_rescore_tc_kernel, in
+//      rr_route_tc.cu); the kernels here take the others, one warp per
+//      query row.  For d in {64, 128, 256} eight lanes
 //      share a candidate (16-byte loads interleaved so that the eight read
 //      one 128-byte line at a time; each keeps its eighth of q in registers);
 //      other d use one lane per candidate.
