@@ -171,3 +171,15 @@ def test_attention_with_nothing_to_do_returns_at_once():
     # no query token: nothing is launched, so even fake pointers are fine
     rr.rr_sparse_attention(attn_cfg(bh=0), FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, 0)
     rr.rr_sparse_attention(attn_cfg(nq_tokens=0), FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, FAKE_Q, 0)
+
+
+def test_attention_binding_checks_tensors_before_the_library():
+    import torch
+    q = torch.zeros((1, 64, 64), dtype=torch.bfloat16)          # host tensors: rejected, nothing launched
+    route = torch.zeros((1, 1, 4), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        rr.sparse_attention(q, q, q, route, 64)
+    with pytest.raises(ValueError):
+        rr.sparse_attention(q.float(), q, q, route, 64)
+    with pytest.raises(ValueError):
+        rr.sparse_attention(q, q, q, route.long(), 64)
