@@ -515,7 +515,20 @@ def cpu_baseline(w, qs, ks, threads=None, layers=2):
     rows = T * w.n * layers
     return {"value": rows / dt, "unit": "rows/s", "cores": T, "kind": "oracle",
             "sample": f"{T} heads x {layers} layers (anchor, relay) of {w.name}, one head per thread, "
-                      f"{dt:.1f} s wall on {ncpu} host cores"}
+                      f"{dt:.1f} s wall on {ncpu} host cores",
+            "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "unknown"."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.lower().startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def workload_config(w, world: int) -> dict:

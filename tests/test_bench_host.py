@@ -69,3 +69,15 @@ def test_layer_kinds_split():
     assert k["relay"]["ms_per_layer"] == 3.0 and k["relay"]["rows_per_s"] == pytest.approx(1000 / 3e-3)
     assert bench.layer_kinds(1000, 5.0, 2, 0.0, 0) == {"anchor": {"layers": 2, "ms_per_layer": 2.5,
                                                                   "rows_per_s": 1000 * 2 / 5e-3}}
+
+
+def test_cpu_baseline_runs_the_oracle_on_a_bounded_sample():
+    st = W.LayerStream(W.PR1, "cpu")
+    qs, ks = [], []
+    for _ in range(2):
+        _, _, q, k = st.next()
+        qs.append(q)
+        ks.append(k)
+    cb = bench.cpu_baseline(W.PR1, qs, ks, threads=1, layers=2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "rows/s" and cb["cores"] == 1 and cb["value"] > 0
+    assert "1 heads x 2 layers" in cb["sample"] and isinstance(cb["cpu_model"], str)
