@@ -189,6 +189,16 @@ def layer_kinds(rows_per_layer: int, anchor_ms: float, n_anchor: int, relay_ms: 
     return out
 
 
+def sum_over_ranks(xs, world: int, device=None) -> list:
+    """Element-wise sum of per-rank counts (refreshed rows, score pairs): the
+    one collective of the sharded path, on the host side of the step."""
+    if world <= 1:
+        return [float(x) for x in xs]
+    t = torch.tensor([float(x) for x in xs], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return [float(x) for x in t.tolist()]
+
+
 def full_pairs_per_layer(w) -> int:
     if not w.causal:
         return w.bh * w.n * w.n
@@ -287,8 +297,11 @@ def run_ours(args, w, rank, world, device):
     pairs_per_step = d_cnt[rr.CNT_PAIRS_TOTAL] / K
     full_pairs_per_step = d_cnt[rr.CNT_FULL_PAIRS_TOTAL] / K
     refreshed_per_step = d_cnt[rr.CNT_ROWS_TOTAL] / K
-    relay_rows = w.bh * w.n * len(relays)
-    rho = (refreshed_per_step - w.bh * w.n * len(anchors)) / relay_rows if relay_rows else 0.0
+    # all ranks' counts (every rank takes this step, in the same place)
+    pairs_all, refreshed_all, retry_all = sum_over_ranks(
+        [pairs_per_step, refreshed_per_step, d_cnt[rr.CNT_RETRY_TOTAL] / K], world, device)
+    relay_rows = w.bh * w.n * len(relays) * world
+    rho = (refreshed_all - w.bh * w.n * len(anchors) * world) / relay_rows if relay_rows else 0.0
 
     peaks = load_peaks()
     esz = 2 if w.dtype == "bf16" else 4
@@ -339,12 +352,12 @@ def run_ours(args, w, rank, world, device):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
         "config": workload_config(w, world),
-        "score_pairs_per_s": pairs_per_step * world / (ms_step * 1e-3),
-        "pair_fraction": pairs_per_step / (full_pairs_per_layer(w) * L),
+        "score_pairs_per_s": pairs_all / (ms_step * 1e-3),
+        "pair_fraction": pairs_all / (full_pairs_per_layer(w) * L * world),
         "rho_relay": rho,
         "layer_kinds": layer_kinds(w.bh * w.n, anchor_layer_ms, K * len(anchors), relay_layer_ms,
                                    K * len(relays)),
-        "retry_rows_per_step": d_cnt[rr.CNT_RETRY_TOTAL] / K,
+        "retry_rows_per_step": retry_all,
         "roofline": roofline,
         "kernels": kernels,
         # our kernels per layer: anchor = route (+ finalize + retry on the

@@ -1,7 +1,8 @@
 """Multi-rank host logic on CPU (gloo, world size 2): each rank routes its own
 BH units with the random draws keyed by the global unit index, so the ranks
 together reproduce one joint run exactly; the step time reported is the
-slowest rank's.  Uses the oracle as the router (no GPU)."""
+slowest rank's and the counts are summed over the ranks.  Uses the oracle as
+the router (no GPU)."""
 import os
 import socket
 
@@ -43,8 +44,9 @@ def _worker(rank, world, port, out):
         parts = [None] * world
         dist.all_gather_object(parts, mine)
         slowest = bench.max_over_ranks(10.0 + rank, world)
+        totals = bench.sum_over_ranks([1.0 + rank, 100.0 * rank], world)
         if rank == 0:
-            out.put((np.concatenate(parts), slowest))
+            out.put((np.concatenate(parts), slowest, totals))
     finally:
         dist.destroy_process_group()
 
@@ -57,7 +59,7 @@ def test_two_ranks_reproduce_the_joint_run_and_report_the_slowest():
     procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
     for pr in procs:
         pr.start()
-    joint_ids, slowest = out.get(timeout=120)
+    joint_ids, slowest, totals = out.get(timeout=120)
     for pr in procs:
         pr.join(timeout=60)
         assert pr.exitcode == 0
@@ -70,3 +72,4 @@ def test_two_ranks_reproduce_the_joint_run_and_report_the_slowest():
         rt.step(l, q, k, recall=False)
     assert np.array_equal(joint_ids, np.stack([led.ids for led in rt.ledgers]))
     assert slowest == 11.0
+    assert totals == [3.0, 100.0]
