@@ -637,6 +637,9 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         led, qs, ks, cfg = state
         result["cpu_baseline"] = cpu_baseline(w, qs, ks)
+        one = cpu_baseline(w, qs, ks, threads=1)
+        result["cpu_baseline"]["single_thread"] = {"value": one["value"], "unit": one["unit"],
+                                                   "sample": one["sample"]}
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:
