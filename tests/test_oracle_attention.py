@@ -183,3 +183,56 @@ def test_planted_mistakes_are_caught(monkeypatch):
         m.setattr(A, "expand_route", lambda row, chunk, nk: np.concatenate(
             [np.arange(j, j + chunk) for j in (int(x) for x in row) if 0 <= j < nk] or [np.zeros(0, np.int64)]))
         assert not _dense_pin_holds(causal=False) or not _dense_pin_holds(causal=True)
+
+
+# ---- properties Eq. 3 must have, on random small problems --------------------
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@st.composite
+def _problem(draw):
+    chunk = draw(st.sampled_from([1, 2, 4]))
+    n_chunks = draw(st.integers(1, 5))
+    dh = draw(st.integers(1, 6))
+    width = draw(st.integers(0, 6))
+    causal = draw(st.booleans())
+    seed = draw(st.integers(0, 2**31 - 1))
+    rng = np.random.default_rng(seed)
+    n_tok = chunk * n_chunks
+    q, k, v = (rng.standard_normal((1, n_tok, dh)) for _ in range(3))
+    route = rng.integers(-2, n_chunks + 2, size=(1, n_chunks, width)).astype(np.int32)
+    return q, k, v, route, chunk, causal, rng
+
+
+@settings(max_examples=60, deadline=None)
+@given(_problem())
+def test_a_common_key_shift_leaves_every_softmax_unchanged(p):
+    # k_s -> k_s + c adds q_t . c / sqrt(d) to every logit of query t
+    q, k, v, route, chunk, causal, rng = p
+    c = rng.standard_normal(k.shape[2])
+    a = oracle.sparse_attention(q, k, v, route, chunk, causal)
+    b = oracle.sparse_attention(q, k + c, v, route, chunk, causal)
+    np.testing.assert_allclose(b, a, rtol=1e-9, atol=1e-9)
+
+
+@settings(max_examples=60, deadline=None)
+@given(_problem())
+def test_outputs_are_affine_in_the_values(p):
+    # o(a v + b) = a o(v) + b on rows that see at least one key (weights sum to 1)
+    q, k, v, route, chunk, causal, rng = p
+    alpha, beta = rng.standard_normal(), rng.standard_normal(v.shape[2])
+    o = oracle.sparse_attention(q, k, v, route, chunk, causal)
+    seen = oracle.sparse_attention(q, k, np.ones_like(v), route, chunk, causal)[0, :, 0] != 0
+    o2 = oracle.sparse_attention(q, k, alpha * v + beta, route, chunk, causal)
+    np.testing.assert_allclose(o2[0, seen], alpha * o[0, seen] + beta, rtol=1e-9, atol=1e-9)
+    assert np.all(o2[0, ~seen] == 0) and np.all(o[0, ~seen] == 0)
+
+
+@settings(max_examples=60, deadline=None)
+@given(_problem())
+def test_route_order_and_padding_are_irrelevant(p):
+    q, k, v, route, chunk, causal, rng = p
+    a = oracle.sparse_attention(q, k, v, route, chunk, causal)
+    perm = route[:, :, rng.permutation(route.shape[2])]
+    padded = np.concatenate([perm, np.full((1, route.shape[1], 2), -1, np.int32)], axis=2)
+    np.testing.assert_allclose(oracle.sparse_attention(q, k, v, padded, chunk, causal), a, rtol=1e-9, atol=1e-12)
