@@ -617,3 +617,52 @@ def test_global_sentinels_take_part_in_beta():
         if glob and sent and max(S[i, j] for j in glob) == beta[i]:
             n_glob_max += 1
     assert n_glob_max > 0   # some rows' beta comes from a global candidate
+
+
+# ---- properties of the routing on random small problems (hypothesis) ---------
+from hypothesis import assume, given, settings, strategies as st  # noqa: E402
+
+
+def _min_gap(S, nv):
+    """Smallest gap between distinct-rank scores of each row's valid prefix."""
+    g = np.inf
+    for i in range(S.shape[0]):
+        s = np.sort(S[i, : nv[i]])
+        if s.size > 1:
+            g = min(g, float(np.min(np.diff(s))))
+    return g
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 2**31 - 1), causal=st.booleans(), scale_exp=st.integers(-2, 3),
+       nq=st.integers(2, 20), nk=st.integers(2, 20), k=st.integers(1, 4), m=st.integers(0, 4),
+       r=st.integers(0, 4))
+def test_a_positive_key_scale_and_a_common_key_shift_keep_every_decision(seed, causal, scale_exp, nq, nk,
+                                                                         k, m, r):
+    """k_j -> 2^e k_j + c scales every score of row i by 2^e and adds q_i . c:
+    each row's order, its alpha - beta sign (gamma = 0) and therefore the
+    whole ledger (random draws depend only on the excluded set) and every
+    refresh flag stay the same, over an anchor and a relay layer."""
+    assume(k <= nk)
+    rng = np.random.default_rng(seed)
+    d = 6
+    p = Params(nq=nq, nk=nk, d=d, k=k, m=m, r=r, causal=causal, seed=seed)
+    layers = [(rng.standard_normal((nq, d)).astype(np.float32), rng.standard_normal((nk, d)).astype(np.float32))
+              for _ in range(2)]
+    a = np.float32(2.0 ** scale_exp)
+    c = rng.standard_normal(d).astype(np.float32)
+    nv = [oracle.valid_count(i, nk, causal) for i in range(nq)]
+    for q, kk in layers:   # no near-ties that fp32 rounding of the shift could flip
+        for kx in (kk, a * kk + c):
+            assume(_min_gap(oracle.scores(q, kx), nv) > 1e-4)
+    A, B = oracle.HeadLedger.empty(p), oracle.HeadLedger.empty(p)
+    for layer, (q, kk) in enumerate(layers):
+        fa, ba, ra, _, _ = oracle.head_layer(p, 0, layer, layer == 0, q, kk, A)
+        fb, bb, rb, _, _ = oracle.head_layer(p, 0, layer, layer == 0, q, a * kk + c, B)
+        if layer > 0:   # the relay margins must not sit at the decision boundary either
+            r_ids = [[j for j in A.ids[i, :k] if j >= 0] for i in range(nq)]
+            S = oracle.scores(q, kk)
+            margin = [min(S[i, j] for j in r_ids[i]) - ba[i] for i in range(nq) if r_ids[i]]
+            assume(all(abs(x) > 1e-4 or not np.isfinite(x) for x in margin))
+        assert np.array_equal(fa, fb) and ra == rb
+        assert np.array_equal(A.ids, B.ids) and np.array_equal(A.anchor_layer, B.anchor_layer)
