@@ -666,3 +666,30 @@ def test_a_positive_key_scale_and_a_common_key_shift_keep_every_decision(seed, c
             assume(all(abs(x) > 1e-4 or not np.isfinite(x) for x in margin))
         assert np.array_equal(fa, fb) and ra == rb
         assert np.array_equal(A.ids, B.ids) and np.array_equal(A.anchor_layer, B.anchor_layer)
+
+
+@settings(max_examples=40, deadline=None)
+@given(seed=st.integers(0, 2**31 - 1), nq=st.integers(1, 16), nk=st.integers(2, 24), k=st.integers(1, 5),
+       m=st.integers(0, 5))
+def test_permuting_queries_and_keys_permutes_routes_and_near_misses(seed, nq, nk, k, m):
+    """Non-causal anchor: relabelling the key chunks by a permutation P and
+    reordering the query rows maps each row's route and near-miss ids
+    through P (distinct scores: no tie to break) and keeps alpha."""
+    assume(k <= nk)
+    rng = np.random.default_rng(seed)
+    d = 5
+    q = rng.standard_normal((nq, d)).astype(np.float32)
+    kk = rng.standard_normal((nk, d)).astype(np.float32)
+    assume(_min_gap(oracle.scores(q, kk), [nk] * nq) > 1e-6)
+    P = rng.permutation(nk)             # new key index of old key j is P[j]
+    R = rng.permutation(nq)             # new row r holds old row R[r]
+    kp = np.empty_like(kk)
+    kp[P] = kk
+    p = Params(nq=nq, nk=nk, d=d, k=k, m=m, r=0, seed=seed)
+    A, B = oracle.HeadLedger.empty(p), oracle.HeadLedger.empty(p)
+    oracle.head_layer(p, 0, 0, True, q, kk, A)
+    oracle.head_layer(p, 0, 0, True, q[R], kp, B)
+    w = k + m
+    mapped = np.where(A.ids[:, :w] >= 0, P[np.maximum(A.ids[:, :w], 0)], -1)
+    assert np.array_equal(B.ids[:, :w], mapped[R])
+    assert np.array_equal(B.alpha, A.alpha[R])
