@@ -199,6 +199,17 @@ def sum_over_ranks(xs, world: int, device=None) -> list:
     return [float(x) for x in t.tolist()]
 
 
+def launches_per_step(w, n_anchor: int, n_relay: int, oneshot: bool) -> int:
+    """Our kernels launched by one step.  Tensor-core path: anchor = select,
+    finish, heap retry, counters (4); one-shot relay = select, finish, exact
+    rescoring, heap retry, counters (5); staged relay = rescore, compact,
+    select, finish, heap retry, counters (6).  CUDA-core path: anchor = route,
+    counters (2); relay = rescore, compact, route, counters (4)."""
+    if uses_tensor_cores(w):
+        return 4 * n_anchor + (5 if oneshot else 6) * n_relay
+    return 2 * n_anchor + 4 * n_relay
+
+
 def full_pairs_per_layer(w) -> int:
     if not w.causal:
         return w.bh * w.n * w.n
@@ -220,33 +231,35 @@ def run_ours(args, w, rank, world, device):
     anchors = [l for l in range(L) if led.is_anchor(l)]
     relays = [l for l in range(L) if not led.is_anchor(l)]
 
-    # events: per layer spans of the route kernel (anchor / refresh) and of
-    # the relay rescore and compact kernels, on the launching stream
+    # On the tensor-core path a relay layer is one C-ABI call (rr_relay_layer:
+    # every row routed, the relay test taken from the kept scores); the
+    # three-stage form (rescore -> compact -> refresh) is timed with --relay
+    # staged, and is what the CUDA-core path runs.
+    oneshot = uses_tensor_cores(w) and args.relay == "oneshot"
+
+    # events on the launching stream: each layer's span, and in the staged
+    # form the boundaries between its three stages
     def make_events(n):
         return [torch.cuda.Event(enable_timing=True) for _ in range(n)]
 
     def step(ev=None):
-        e = 0
         for l in range(L):
+            if ev is not None:
+                ev["start"][l].record(stream)
             if led.is_anchor(l):
-                if ev is not None:
-                    ev["anchor"][e].record(stream)
                 led.full_route(qs[l], ks[l], l)
-                if ev is not None:
-                    ev["anchor_end"][e].record(stream)
+            elif oneshot:
+                led.relay_layer(qs[l], ks[l], l)
             else:
-                if ev is not None:
-                    ev["rescore"][e].record(stream)
                 led.relay_rescore(qs[l], ks[l], l)
                 if ev is not None:
-                    ev["compact"][e].record(stream)
+                    ev["compact"][l].record(stream)
                 led.relay_compact(l)
                 if ev is not None:
-                    ev["refresh"][e].record(stream)
+                    ev["refresh"][l].record(stream)
                 led.relay_refresh(qs[l], ks[l], l)
-                if ev is not None:
-                    ev["refresh_end"][e].record(stream)
-            e += 1
+            if ev is not None:
+                ev["end"][l].record(stream)
 
     def barrier():
         if world > 1:
@@ -258,8 +271,7 @@ def run_ours(args, w, rank, world, device):
     barrier()
     c0 = led.read()["counters"].clone()
     K = args.steps
-    evs = [{n: make_events(L) for n in ("anchor", "anchor_end", "rescore", "compact", "refresh",
-                                        "refresh_end")} for _ in range(K)]
+    evs = [{n: make_events(L) for n in ("start", "compact", "refresh", "end")} for _ in range(K)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(smi_id(device) if args.smi_index is None else args.smi_index) as clk:
@@ -272,23 +284,23 @@ def run_ours(args, w, rank, world, device):
     ms_total = t_start.elapsed_time(t_end)
     c1 = led.read()["counters"].clone()
 
-    route_ms = rescore_ms = compact_ms = 0.0
-    anchor_layer_ms = relay_layer_ms = 0.0
-    n_route = n_rescore = 0
+    anchor_layer_ms = relay_layer_ms = rescore_ms = compact_ms = refresh_ms = 0.0
     for s in range(K):
         for l in range(L):
+            span = evs[s]["start"][l].elapsed_time(evs[s]["end"][l])
             if l in anchors:
-                span = evs[s]["anchor"][l].elapsed_time(evs[s]["anchor_end"][l])
-                route_ms += span
                 anchor_layer_ms += span
-                n_route += 1
             else:
-                rescore_ms += evs[s]["rescore"][l].elapsed_time(evs[s]["compact"][l])
-                compact_ms += evs[s]["compact"][l].elapsed_time(evs[s]["refresh"][l])
-                route_ms += evs[s]["refresh"][l].elapsed_time(evs[s]["refresh_end"][l])
-                relay_layer_ms += evs[s]["rescore"][l].elapsed_time(evs[s]["refresh_end"][l])
-                n_route += 1
-                n_rescore += 1
+                relay_layer_ms += span
+                if not oneshot:
+                    rescore_ms += evs[s]["start"][l].elapsed_time(evs[s]["compact"][l])
+                    compact_ms += evs[s]["compact"][l].elapsed_time(evs[s]["refresh"][l])
+                    refresh_ms += evs[s]["refresh"][l].elapsed_time(evs[s]["end"][l])
+    n_rescore = 0 if oneshot else K * len(relays)
+    # the full-routing stage: anchor layers, and the relay layers' routing
+    # (one-shot: the whole relay call; staged: the refresh launches)
+    route_ms = anchor_layer_ms + (relay_layer_ms if oneshot else refresh_ms)
+    n_route = K * L
 
     ms_step = max_over_ranks(ms_total / K, world, device)
 
@@ -311,9 +323,11 @@ def run_ours(args, w, rank, world, device):
     route_tflops = route_flops / (route_ms * 1e-3) / 1e12
     if uses_tensor_cores(w):
         peak = float(peaks["bf16_tflops_sustained"])
-        roofline = {"kernel": "full routing: route_rows_tc_kernel (tcgen05, two-pass selection) "
-                              "+ route_rows_finalize_kernel + retry path; anchor + refresh",
-                    "bound": "tensor",
+        what = ("route_select_kernel (tcgen05, query tile in TMEM, two-pass selection) + route_finish_kernel"
+                " + exact/heap fallbacks; anchor and relay layers (relay test taken from the kept scores)"
+                if oneshot else
+                "route_select_kernel + route_finish_kernel + heap fallback; anchor layers and refresh launches")
+        roofline = {"kernel": "full routing: " + what, "bound": "tensor",
                     "peak_source": f"{peaks['source']} bf16 dense, sustained (timed inside a long step)"}
     else:
         peak = 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
@@ -321,30 +335,35 @@ def run_ours(args, w, rank, world, device):
                     "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock"}
     traffic = None
     if uses_tensor_cores(w):
-        per_row = profiled_traffic_per_row("rr_route_tc.cu", "route_rows_tc_kernel__*.md")
+        per_row = profiled_traffic_per_row("rr_select_tc.cu", "route_select_kernel__*.md")
         if per_row is not None and n_route:
-            traffic = round(per_row * refreshed_per_step * K / n_route)   # bytes per launch
+            rows_routed = (w.bh * w.n * L) if oneshot else refreshed_per_step
+            traffic = round(per_row * rows_routed * K / n_route)   # bytes per launch
     roofline.update({"achieved": round(route_tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(route_tflops / peak, 4), "traffic": traffic,
                      "avg_launch_ms": round(route_ms / max(n_route, 1), 4),
                      "launches": n_route})
-    # secondary: relay rescoring.  Bytes it must move per row: q (d*e) + its
-    # head's keys once (N*d*e/N) + ids (4c) + alpha/flag writes (5).
-    rescore_bytes = w.bh * w.n * (2 * w.d * esz + 4 * w.c + 5) * n_rescore
-    rescore_gbs = rescore_bytes / (rescore_ms * 1e-3) / 1e9 if rescore_ms > 0 else None
-    rescore = {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1) if rescore_gbs else None,
-               "peak_gbs": peaks["hbm_gbs"],
-               "frac": round(rescore_gbs / peaks["hbm_gbs"], 4) if rescore_gbs else None,
-               "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)}
-    if uses_tensor_cores(w) and rescore_ms > 0:
-        # the tensor-core rescoring scores every valid pair of the row block
-        # (2*d flops per pair) and reads the candidates' scores from the tiles
-        dense_tflops = 2.0 * w.d * full_pairs_per_layer(w) * n_rescore / (rescore_ms * 1e-3) / 1e12
-        rescore.update({"kernel": "relay_rescore_tc_kernel (tcgen05 dense tiles)", "bound": "tensor",
-                        "dense_tflops": round(dense_tflops, 2),
-                        "dense_frac": round(dense_tflops / float(peaks["bf16_tflops_sustained"]), 4)})
-    kernels = {"rescore": rescore,
-               "compact": {"avg_launch_ms": round(compact_ms / max(n_rescore, 1), 4)}}
+    kernels = {}
+    if not oneshot and rescore_ms > 0:
+        # staged relay: rescoring (bytes it must move per row: q (d*e) + its
+        # head's keys once (N*d*e/N) + ids (4c) + alpha/flag writes (5))
+        rescore_bytes = w.bh * w.n * (2 * w.d * esz + 4 * w.c + 5) * n_rescore
+        rescore_gbs = rescore_bytes / (rescore_ms * 1e-3) / 1e9
+        rescore = {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1), "peak_gbs": peaks["hbm_gbs"],
+                   "frac": round(rescore_gbs / peaks["hbm_gbs"], 4),
+                   "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)}
+        if uses_tensor_cores(w):
+            # dense tiles: every valid pair of the row block is scored (2*d flops per pair)
+            dense_tflops = 2.0 * w.d * full_pairs_per_layer(w) * n_rescore / (rescore_ms * 1e-3) / 1e12
+            rescore = {"kernel": "relay_rescore_tc_kernel (tcgen05 dense tiles)", "bound": "tensor",
+                       "achieved": round(dense_tflops, 2), "unit": "TFLOP/s (dense tile work)",
+                       "peak": float(peaks["bf16_tflops_sustained"]),
+                       "frac": round(dense_tflops / float(peaks["bf16_tflops_sustained"]), 4),
+                       "hbm_gbs": round(rescore_gbs, 1),
+                       "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)}
+        kernels["rescore"] = rescore
+        kernels["compact"] = {"avg_launch_ms": round(compact_ms / max(n_rescore, 1), 4)}
+        kernels["refresh"] = {"avg_launch_ms": round(refresh_ms / max(n_rescore, 1), 4)}
 
     result = {
         "metric": METRIC, "value": rows_per_step * world / (ms_step * 1e-3), "unit": "rows/s",
@@ -358,13 +377,10 @@ def run_ours(args, w, rank, world, device):
         "layer_kinds": layer_kinds(w.bh * w.n, anchor_layer_ms, K * len(anchors), relay_layer_ms,
                                    K * len(relays)),
         "retry_rows_per_step": retry_all,
+        "relay": "one-shot (rr_relay_layer)" if oneshot else "staged (rescore, compact, refresh)",
         "roofline": roofline,
         "kernels": kernels,
-        # our kernels per layer: anchor = route (+ finalize + retry on the
-        # tensor-core path) + counters; relay = rescore + compact + the same
-        # route launches over the refreshed rows + counters
-        "gpu_launches": K * ((4 if uses_tensor_cores(w) else 2) * len(anchors)
-                             + (6 if uses_tensor_cores(w) else 4) * len(relays)),
+        "gpu_launches": K * launches_per_step(w, len(anchors), len(relays), oneshot),
         "clocks": clk.summary(),
         "peaks_source": peaks["source"],
     }
@@ -595,6 +611,8 @@ def main():
     ap.add_argument("--no-recall", action="store_true")
     ap.add_argument("--attention", action="store_true",
                     help="also time the sparse attention over the ledger's routes (not part of the step)")
+    ap.add_argument("--relay", default="oneshot", choices=["oneshot", "staged"],
+                    help="tensor-core path: time relay layers as one rr_relay_layer call or as its three stages")
     ap.add_argument("--smi-index", type=int, default=None)
     ap.add_argument("--bh", type=int, default=None, help="override BH (profiling a smaller case)")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")

@@ -13,8 +13,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "librr.so")
-SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_route_tc.cu", "rr_relay.cu", "rr_noalloc.cu", "rr_attention.cu"]
-HEADERS = ["rr_device.cuh", "rr_internal.h"]
+SOURCES = ["rr_api.cu", "rr_route_simt.cu", "rr_route_tc.cu", "rr_select_tc.cu", "rr_relay.cu", "rr_noalloc.cu",
+           "rr_attention.cu"]
+HEADERS = ["rr_device.cuh", "rr_internal.h", "rr_tc.cuh"]
 
 
 def nvcc() -> str:

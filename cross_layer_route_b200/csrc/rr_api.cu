@@ -36,7 +36,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 
 struct Layout {
     size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count;
-    size_t cand_v, cand_i, cand_meta;   // split tensor-core path only (size 0 otherwise)
+    // tensor-core selection path only (size 0 otherwise)
+    size_t cand_vals, cand_masks, cand_meta, und_list, und_count;
     bool cand;
     size_t total;
 };
@@ -74,11 +75,14 @@ Layout layout_of(const rr_config *c) {
     t.bh = c->bh; t.nq = c->nq; t.nk = c->nk; t.d = c->d;
     t.k = c->k; t.m = c->m_near; t.r = c->r_rand; t.ksel = c->k + c->m_near;
     t.g_sink = c->g_sink; t.g_recent = c->g_recent; t.c = (int)cc;
-    const rr::CandSizes cs = rr::route_rows_tc_candidate_sizes(t, c->dtype);
-    L.cand = cs.v > 0;
-    L.cand_v = o;       o = align_up(o + cs.v);
-    L.cand_i = o;       o = align_up(o + cs.i);
+    t.mt = (c->nk + 127) / 128;
+    const rr::CandSizes cs = rr::route_select_candidate_sizes(t, c->dtype);
+    L.cand = cs.vals > 0;
+    L.cand_vals = o;    o = align_up(o + cs.vals);
+    L.cand_masks = o;   o = align_up(o + cs.masks);
     L.cand_meta = o;    o = align_up(o + cs.meta);
+    L.und_list = o;     o = align_up(o + cs.und);
+    L.und_count = o;    o = align_up(o + (L.cand ? sizeof(int32_t) : 0));
     L.total = o;
     return L;
 }
@@ -179,6 +183,21 @@ rr_status do_full_route(rr_ledger *L, const void *q, const void *k, int32_t laye
     return RR_OK;
 }
 
+// A relay layer on the tensor-core selection path (rr_select_tc.cu): every
+// row is routed, the relay test is taken from the kept scores, and the
+// ledger, flags and counters come out as the three stages would leave them.
+rr_status do_relay_oneshot(rr_ledger *L, const void *q, const void *k, int32_t layer, cudaStream_t s) {
+    const rr_status st = prepare(L, s);
+    if (st != RR_OK) return st;
+    cudaError_t e = reset_layer_counters(L, s);
+    if (e == cudaSuccess) e = rr::launch_relay_oneshot(L->dev, q, k, layer, s);
+    if (e == cudaSuccess) e = rr::launch_finalize(L->dev, layer, 0, 0, 0, s);
+    if (e != cudaSuccess) return RR_ECUDA;
+    L->stage = 0;
+    L->last_layer = layer;
+    return RR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -218,10 +237,13 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     D.retry_list = reinterpret_cast<int32_t *>(L->ws + lay.retry_list);
     D.retry_count = reinterpret_cast<int32_t *>(L->ws + lay.retry_count);
     if (lay.cand) {
-        D.cand_v = reinterpret_cast<float *>(L->ws + lay.cand_v);
-        D.cand_i = reinterpret_cast<uint16_t *>(L->ws + lay.cand_i);
-        D.cand_meta = reinterpret_cast<int32_t *>(L->ws + lay.cand_meta);
+        D.cand_vals = reinterpret_cast<float *>(L->ws + lay.cand_vals);
+        D.cand_masks = reinterpret_cast<uint32_t *>(L->ws + lay.cand_masks);
+        D.cand_meta = reinterpret_cast<uint2 *>(L->ws + lay.cand_meta);
+        D.und_list = reinterpret_cast<int32_t *>(L->ws + lay.und_list);
+        D.und_count = reinterpret_cast<int32_t *>(L->ws + lay.und_count);
     }
+    D.mt = (cfg->nk + 127) / 128;
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;
     D.k = cfg->k; D.m = cfg->m_near; D.r = cfg->r_rand;
     D.g_sink = cfg->g_sink; D.g_recent = cfg->g_recent;
@@ -256,6 +278,7 @@ rr_status rr_relay_layer(rr_ledger *ledger, const void *d_qc, const void *d_kc, 
     if (!ledger->anchored || layer <= ledger->last_layer) return RR_ESTATE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (is_forced_anchor(ledger, layer)) return do_full_route(ledger, d_qc, d_kc, layer, s);
+    if (ledger->dev.cand_vals) return do_relay_oneshot(ledger, d_qc, d_kc, layer, s);
     st = stage_rescore(ledger, d_qc, d_kc, layer, s);
     if (st == RR_OK) st = stage_compact(ledger, layer, s);
     if (st == RR_OK) st = stage_refresh(ledger, d_qc, d_kc, layer, s);

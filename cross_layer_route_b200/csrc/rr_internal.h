@@ -1,6 +1,7 @@
 // rr_internal.h -- internal types shared by the host library and the kernels.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -20,11 +21,15 @@ struct LedgerDev {
     int32_t *head_count;    // [bh]        flagged rows per head
     int32_t *retry_list;    // [bh*nq]     per-head rows whose tensor-core selection is redone
     int32_t *retry_count;   // [bh]        rows listed per head
-    // candidate buffers of the split tensor-core path (null: the route kernel
-    // finishes its rows itself); per 128-row block of one head:
-    float *cand_v = nullptr;       // [blocks, 128, kCap] kept scores (row-contiguous)
-    uint16_t *cand_i = nullptr;    // [blocks, 128, kCap] their key chunks
-    int32_t *cand_meta = nullptr;  // [blocks, 128] kept counts of the two halves, or -1
+    // buffers of the tensor-core selection path (null: the allocation-free
+    // entry point, whose route kernel finishes its rows itself).  Row slot
+    // s = (head * blocks_per_head + block) * 128 + position in the block.
+    float *cand_vals = nullptr;      // [slots, 4, kQCap] kept scores per row quarter
+    uint32_t *cand_masks = nullptr;  // [blocks, mt, 4, 128] kept columns per (tile, quarter, row)
+    uint2 *cand_meta = nullptr;      // [slots] {kept per quarter (bytes, 0xFF = redo), threshold}
+    int32_t *und_list = nullptr;     // [bh*nq] relay rows whose test needs exact rescoring
+    int32_t *und_count = nullptr;    // [1]
+    int mt = 0;                      // key tiles per head: ceil(nk / 128)
     int bh, nq, nk, d;
     int k, m, r, c, ksel;   // ksel = k + m; c = k + m + r + g_sink + g_recent
     int g_sink = 0, g_recent = 0;   // mandatory global sentinels (sink, recent chunks)
@@ -59,14 +64,37 @@ inline int select_capacity(int ksel) {
 // memory attribute on the current device.
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype);
 bool route_rows_tc_supported(const LedgerDev &L, int dtype);
-size_t route_rows_tc_smem_bytes(const LedgerDev &L);
-// Bytes of the candidate buffers the split tensor-core path needs (all 0 when
-// the problem does not run on the tensor cores).
-struct CandSizes { size_t v, i, meta; };
-CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype);
-cudaError_t route_rows_tc_prepare(size_t smem_bytes);
+cudaError_t route_rows_tc_prepare();
 cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                  bool use_list, cudaStream_t s);
+
+// Tensor-core selection path (rr_select_tc.cu): the selection kernel writes
+// every row's kept scores to the candidate buffers, the finishing kernel
+// orders them and writes the ledger row.
+struct CandSizes { size_t vals, masks, meta, und; };
+// Bytes of the buffers (all 0 when the problem does not run on the tensor cores).
+CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype);
+size_t route_select_smem_bytes(const LedgerDev &L);
+cudaError_t route_select_prepare();
+// kAnchor: every row (or every listed row) is rebuilt.  kRelay: every row
+// is routed and the relay test (Eq. 8) decides, row by row, whether the new
+// route or the old one is kept.
+enum class SelectMode { kAnchor = 0, kRelay = 1 };
+cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
+                                bool use_list, SelectMode mode, cudaStream_t s);
+// Exact heap selection of the rows in the per-head retry lists (rr_route_tc.cu).
+cudaError_t launch_route_retry(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
+                               cudaStream_t s);
+// One relay layer on the tensor-core selection path: route every row, take
+// the relay decision from the kept scores, rescore exactly the rows that
+// decision leaves open, rebuild the refreshed rows among them, roll up the
+// counters.
+cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *k, int layer,
+                                 cudaStream_t s);
+namespace tc {
+// Tensor map of Kc [bh, nk, d] bf16: boxes of 128 keys x 64 dims, 128-byte swizzle.
+cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map);
+}
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s);
 cudaError_t launch_relay_rescore(const LedgerDev &L, int dtype, const void *q, const void *k,

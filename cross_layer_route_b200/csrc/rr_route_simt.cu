@@ -280,7 +280,7 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
 }  // namespace
 
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
-    if (route_rows_tc_supported(L, dtype)) return route_rows_tc_prepare(route_rows_tc_smem_bytes(L));
+    if (route_rows_tc_supported(L, dtype)) return route_rows_tc_prepare();
     const int smem = (int)smem_layout(L.d, select_capacity(L.ksel)).total;
     if (dtype == kBF16)
         return cudaFuncSetAttribute(route_rows_kernel<__nv_bfloat16>,

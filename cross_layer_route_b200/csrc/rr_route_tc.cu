@@ -45,27 +45,14 @@
 //
 // Every wait is bounded; a timeout sets bit 1 of the error word and the CTA
 // drains its copies, frees its TMEM and returns.
-#include <cuda.h>
-#include <float.h>
-#include <limits.h>
-
-#include "rr_device.cuh"
-#include "rr_internal.h"
+#include "rr_tc.cuh"
 
 namespace rr {
 namespace tc {
 
-constexpr int kRows = 128;
-constexpr int kKeys = 128;
-constexpr int kMaxStages = 4;
 constexpr int kHeapThreads = 32 * (2 + 4);     // heap kernel: 4 epilogue warps (one per row)
 constexpr int kEpiWarps = 16;                  // two-pass kernel: epilogue warps (four per row)
 constexpr int kPassThreads = 32 * (2 + kEpiWarps);
-constexpr int kAcc = 4;                       // TMEM accumulators (128 columns each)
-constexpr int kTmemCols = kAcc * 128;
-static_assert(kAcc >= kMaxStages, "a key stage is freed through the accumulator barriers");
-constexpr int kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
-constexpr long long kSpinLimit = 1ll << 31;
 // two-pass selection
 constexpr int kGroups = 16;                // column groups per quarter row (four quarters per row)
 constexpr int kTops = 8 * kGroups;         // group top-2 values per row
@@ -77,8 +64,6 @@ constexpr int kThrLowBit = 16;             // threshold search stops at this key
 // heap selection (retry path)
 constexpr int kBuf = 32;
 
-__host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
-
 // Stages of the key ring (what the shared memory left by the selection
 // buffers allows).
 __host__ __device__ inline int stages_for(int d, bool two_pass) {
@@ -89,6 +74,7 @@ __host__ __device__ inline int stages_for(int d, bool two_pass) {
 struct Layout {
     uint32_t q, k, sel, bufv, bufi, stg, rows, red, bars, misc, total;
     int stages;
+    __host__ __device__ CtaLayout cta() const { return CtaLayout{q, k, rows, bars, misc, stages}; }
 };
 
 // two_pass: q | k | sel (91 KB: the group tops [kRows][kTopStride] f32 after
@@ -117,319 +103,10 @@ __host__ __device__ inline Layout layout_of(int d, int ksel, bool two_pass) {
     }
     s.rows = o; o = up(o + kRows * 4, 16);
     s.red = o;  o = up(o + (two_pass ? 2 * kRows * 4 : 0), 16);
-    s.bars = o; o = up(o + 8 * (2 * kMaxStages + 2 * kAcc + 1), 16);
+    s.bars = o; o = up(o + 8 * kNumBars, 16);
     s.misc = o; o = up(o + 16, 16);
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
-}
-
-// ---- PTX wrappers (forms from the PTX ISA for sm_100a) -----------------------
-__device__ __forceinline__ uint32_t saddr(const void *p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t *b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(b)), "r"(bytes)
-                 : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t *b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(b)) : "memory");
-}
-__device__ __forceinline__ bool mbar_test(uint64_t *b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(saddr(b)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-// The same test, letting the thread sleep up to ~8 us until the phase
-// completes (a waiting warp then takes no issue slots from the warps that
-// share its scheduler).
-__device__ __forceinline__ bool mbar_test_sleep(uint64_t *b, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(saddr(b)), "r"(parity), "r"(8192u)
-        : "memory");
-    return ok != 0;
-}
-// Bounded wait for the phase of the given parity.  Returns false on timeout
-// (and raises the CTA's abort flag) or when another role already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag) {
-    if (mbar_test(b, parity)) return true;
-    const long long t0 = clock64();
-    while (!mbar_test_sleep(b, parity)) {
-        if (*abort_flag) return false;
-        if (clock64() - t0 > kSpinLimit) {
-            *abort_flag = 1;
-            return false;
-        }
-    }
-    return true;
-}
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
-                                            int c1, int c2) {
-    asm volatile(
-        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(saddr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(saddr(bar)), "r"(c0), "r"(c1), "r"(c2)
-        : "memory");
-}
-__device__ __forceinline__ void tc_fence_before() {
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_commit(uint64_t *bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     saddr(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-// 32 lanes x 32 consecutive fp32 columns; thread t gets its lane's 32 values.
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, float *v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-        "%30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// The same load without the wait (pair two loads with one tc_wait_ld).
-__device__ __forceinline__ void tc_ld32_nowait(uint32_t taddr, uint32_t *r) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, "
-        "%12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, "
-        "%30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-}
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-
-// Shared-memory matrix descriptor of a K-major operand stored as 128-byte
-// swizzled rows (8-row groups 1024 bytes apart): start address >> 4, leading
-// byte offset 16 B, stride byte offset 1024 B, descriptor version 1,
-// layout "128-byte swizzle".
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr_bytes) {
-    return (uint64_t)((saddr_bytes >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) |
-           ((uint64_t)(1024u >> 4) << 32) | ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
-}
-// Instruction descriptor: fp32 accumulator, bf16 A and B, both K-major,
-// N = 128 (bits 17..22 hold N/8), M = 128 (bits 24..28 hold M/16).
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKeys >> 3) << 17) |
-                            ((uint32_t)(kRows >> 4) << 24);
-
-// ---- the CTA machinery shared by both kernels ----------------------------------
-struct Cta {
-    unsigned char *q_s, *k_s;
-    int *rows_s;
-    uint64_t *full, *acc_full, *acc_empty, *mma_done;
-    uint32_t *tmem_slot;
-    volatile int *abort_flag;
-    int stages, n_rows, ntiles;
-    uint32_t tmem_base;
-};
-
-// Rows, barriers, TMEM and the query tile.  Returns false when the CTA has
-// no rows (all threads return together).
-__device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Layout &lay,
-                                          const LedgerDev &L, const __nv_bfloat16 *Q,
-                                          const int *list, const int *head_count, int use_list) {
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const int h = blockIdx.y;
-    const int nq = L.nq, d = L.d;
-    const int count = use_list ? head_count[h] : nq;
-    const int row0 = blockIdx.x * kRows;
-    if (row0 >= count) return false;
-    c.q_s = smem + lay.q;
-    c.k_s = smem + lay.k;
-    c.rows_s = reinterpret_cast<int *>(smem + lay.rows);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
-    c.stages = lay.stages;
-    c.full = bars;
-    c.acc_full = bars + 2 * kMaxStages;
-    c.acc_empty = bars + 2 * kMaxStages + kAcc;
-    c.mma_done = bars + 2 * kMaxStages + 2 * kAcc;
-    c.tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.misc);
-    c.abort_flag = reinterpret_cast<volatile int *>(smem + lay.misc + 4);
-    c.n_rows = min(kRows, count - row0);
-
-    if (tid < kRows) {
-        int row = -1;
-        if (tid < c.n_rows) row = use_list ? list[(size_t)h * nq + row0 + tid] : row0 + tid;
-        c.rows_s[tid] = row;
-    }
-    if (tid == 0) {
-        for (int s = 0; s < c.stages; ++s) {
-            mbar_init(&c.full[s], 1);
-        }
-        for (int a = 0; a < kAcc; ++a) {
-            mbar_init(&c.acc_full[a], 1);
-            mbar_init(&c.acc_empty[a], (blockDim.x >> 5) - 2);
-        }
-        mbar_init(c.mma_done, 1);
-        *c.abort_flag = 0;
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         saddr(c.tmem_slot)),
-                     "r"(kTmemCols)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-    }
-    __syncthreads();
-
-    // query tile: gather rows by index into the 128-byte-swizzled K-major
-    // layout (row r, 16-byte chunk c of its 64-element half kb lands at
-    // kb*16KB + r*128 + ((c ^ (r & 7)) * 16)).
-    const int c16 = d >> 3;
-    for (int e = tid; e < kRows * c16; e += blockDim.x) {
-        const int r = e / c16, ch = e - r * c16;
-        const int row = c.rows_s[r];
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (row >= 0) v = *reinterpret_cast<const uint4 *>(Q + ((size_t)h * nq + row) * d + ch * 8);
-        const int kb = ch >> 3, cc = ch & 7;
-        *reinterpret_cast<uint4 *>(c.q_s + kb * kSubTileBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
-    }
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    int max_row = -1;
-    for (int e = 0; e < c.n_rows; ++e) max_row = max(max_row, c.rows_s[e]);
-    const int kend = L.causal ? min(L.nk, max_row + 1) : L.nk;
-    c.ntiles = (kend + kKeys - 1) / kKeys;
-    __syncthreads();
-    tc_fence_after();
-    c.tmem_base = *c.tmem_slot;
-    return true;
-}
-
-// Tile schedule: pass p covers key tiles 0..nt-1, the second pass backwards
-// (its first tiles are the ones most recently loaded).
-__device__ __forceinline__ int total_tiles(int ntiles, int passes) { return passes * ntiles; }
-__device__ __forceinline__ int tile_of(int g, int ntiles, int passes) {
-    (void)passes;
-    return g < ntiles ? g : 2 * ntiles - 1 - g;
-}
-
-__device__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int passes) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap_k)) : "memory");
-    const int total = total_tiles(c.ntiles, passes);
-    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
-    int issued = 0;
-    for (int g = 0; g < total; ++g) {
-        const int s = g % c.stages;
-        // stage s is free once tile g - stages is scored (its accumulator
-        // barrier; the ring never runs more accumulators ahead than exist,
-        // kAcc >= stages, so that barrier cannot have moved on two phases)
-        if (g >= c.stages) {
-            const int gp = g - c.stages;
-            if (!mbar_wait(&c.acc_full[gp % kAcc], (gp / kAcc) & 1, c.abort_flag)) break;
-        }
-        mbar_expect_tx(&c.full[s], stage_bytes);
-        const int t = tile_of(g, c.ntiles, passes);
-        for (int kb = 0; kb < (d >> 6); ++kb)
-            tma_load_3d(c.k_s + s * stage_bytes + kb * kSubTileBytes, tmap_k, &c.full[s], kb * 64,
-                        t * kKeys, h);
-        ++issued;
-    }
-    // drain: every issued stage must have landed before the CTA exits
-    for (int g = max(0, issued - c.stages); g < issued; ++g) {
-        const int s = g % c.stages;
-        const long long t0 = clock64();
-        while (!mbar_test(&c.full[s], (g / c.stages) & 1) && clock64() - t0 < kSpinLimit) {
-        }
-    }
-}
-
-// MMA issuer (one lane): score tile g into accumulator g % kAcc.
-// The descriptor of a K-major operand at byte offset `off` from another's
-// start is that descriptor plus off / 16 (the start address field, bits
-// 0..13, holds address / 16 and shared memory stays below 256 KB).
-template <int kSteps>
-__device__ __forceinline__ void mma_tile(uint32_t d_tmem, uint64_t qdesc, uint64_t kdesc) {
-#pragma unroll
-    for (int kk = 0; kk < kSteps; ++kk) {
-        const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
-        tc_mma_bf16(d_tmem, qdesc + off16, kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
-    }
-}
-
-__device__ void mma_issuer(Cta &c, int d, int passes) {
-    const int total = total_tiles(c.ntiles, passes);
-    const uint64_t qdesc = sw128_desc(saddr(c.q_s));
-    const uint32_t k_addr = saddr(c.k_s);
-    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
-    for (int g = 0; g < total; ++g) {
-        const int s = g % c.stages, a = g % kAcc;
-        if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
-        if (!mbar_wait(&c.acc_empty[a], ((g / kAcc) & 1) ^ 1, c.abort_flag)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
-        const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
-        if (d == 128) mma_tile<8>(d_tmem, qdesc, kdesc);
-        else mma_tile<4>(d_tmem, qdesc, kdesc);
-        tc_commit(&c.acc_full[a]);   // frees accumulator a's scores and stage s
-    }
-    tc_commit(c.mma_done);
-    const long long t0 = clock64();
-    while (!mbar_test(c.mma_done, 0) && clock64() - t0 < kSpinLimit) {
-    }
-}
-
-__device__ __forceinline__ void cta_teardown(Cta &c, const LedgerDev &L) {
-    tc_fence_before();
-    __syncthreads();
-    if ((threadIdx.x >> 5) == 1) {
-        tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(c.tmem_base),
-                     "r"(kTmemCols)
-                     : "memory");
-    }
-    if (threadIdx.x == 0 && *c.abort_flag) atomicOr(&L.counters[2], 2ULL);
-}
-
-// Epilogue helpers: wait for accumulator g (warp-uniform outcome) / hand it back.
-__device__ __forceinline__ bool acc_wait(Cta &c, int g) {
-    bool ok = mbar_wait(&c.acc_full[g % kAcc], (g / kAcc) & 1, c.abort_flag);
-    ok = __all_sync(kFull, ok);   // the warp leaves together (tcgen05.ld is .sync.aligned)
-    if (ok) tc_fence_after();
-    return ok;
-}
-__device__ __forceinline__ void acc_release(Cta &c, int g) {
-    tc_fence_before();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&c.acc_empty[g % kAcc]);
 }
 
 // Random sentinels (RouteRelay §3.1 item 2, §3.4) of one row, one thread:
@@ -483,13 +160,6 @@ __device__ __forceinline__ int random_sentinels(const LedgerDev &L, int ghead, i
 
 // ---- per-row keys for the heap path ---------------------------------------------
 // Keys order (score, chunk) pairs: larger key = higher score, then smaller chunk.
-__device__ __forceinline__ uint32_t ord32(float f) {
-    const uint32_t u = __float_as_uint(f);
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float unord32(uint32_t o) {
-    return __uint_as_float((o & 0x80000000u) ? (o & 0x7FFFFFFFu) : ~o);
-}
 __device__ __forceinline__ uint64_t make_key(float s, int j) {
     return ((uint64_t)ord32(s) << 32) | (uint32_t)(~(uint32_t)j);
 }
@@ -524,7 +194,7 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int d = L.d, ksel = L.ksel;
     const Layout lay = layout_of(d, ksel, false);
     Cta c;
-    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
+    if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, use_list)) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
 
@@ -623,7 +293,6 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 // rejection rule and ascending completion as random_sentinels above); a draw
 // is accepted if its chunk is not selected, not accepted earlier and not
 // drawn by an earlier lane of the round (warp match), in draw order.
-constexpr int kFinWarps = 8;
 constexpr int kFinBins = 128;
 constexpr int kFinBitsWords = 128;   // membership bitmap: rows with <= 4096 valid keys
 
@@ -827,12 +496,10 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
     }
 }
 
-// ---- two-pass kernel (the main path) ---------------------------------------------
-// kSplit: the kernel ends by writing each row's kept scores and their count
-// to the candidate buffers; route_rows_finalize_kernel finishes the rows.
-// Otherwise the epilogue warps finish them here (one warp per row, from
-// shared memory).
-template <bool kSplit>
+// ---- two-pass kernel with in-CTA row finishing ---------------------------------
+// The allocation-free entry point's full routing: the epilogue warps finish
+// their rows themselves (one warp per row, from the kept scores in shared
+// memory), so the kernel needs no candidate buffers in device memory.
 __global__ void __launch_bounds__(kPassThreads, 1)
 route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                      const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
@@ -842,7 +509,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int d = L.d, ksel = L.ksel;
     const Layout lay = layout_of(d, ksel, true);
     Cta c;
-    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, use_list)) return;
+    if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, use_list)) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
 
@@ -957,7 +624,7 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const int sw = (lane >> 1) & 3;   // 8 lanes of a 64-byte row stride: 8 distinct bank groups
         for (int i = 0; i < nt && ok; ++i, ++g) {
             if (!(ok = acc_wait(c, g))) break;
-            const int t = tile_of(g, nt, 2);
+            const int t = tile_of(g, nt);
             float v[32];
             tc_ld32(lane_base + (uint32_t)((g % kAcc) * kKeys), v);
             acc_release(c, g);
@@ -1014,69 +681,23 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             atomicAdd(&L.counters[10], 1ULL);
         }
 
-        if constexpr (kSplit) {
-            // candidates of row r of block blk at cand[(blk * kRows + r) * kCap + e];
-            // meta (blk, r) = the kept count, or -1 when the row has nothing to finish
-            const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
-            if (qt == 0) L.cand_meta[blk * kRows + r] = good ? kept : -1;
-            // one warp per row: 128-byte stores of the row's slots
-            const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
-            const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
-            for (int k2 = 0; k2 < kRows / kEpiWarps; ++k2) {
-                const int rr = ew * (kRows / kEpiWarps) + k2;
-                const int rowr = c.rows_s[rr];
-                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
-                const int kr = rowcnt[rr];
-                if (!row_good(rowr, nv, kr)) continue;   // warp-uniform
-                float *gv = L.cand_v + (blk * kRows + rr) * kCap;
-                uint16_t *gi = L.cand_i + (blk * kRows + rr) * kCap;
-                for (int e = lane; e < kr; e += 32) {
-                    gv[e] = bvb[e * kBufStride + rr];
-                    gi[e] = bib[e * kBufStride + rr];
-                }
-            }
-        } else {
-            // finish the rows here (kRows / kEpiWarps per warp), the warps'
-            // scratch in the query/key buffers (every MMA is done)
-            FinWarp &fw = reinterpret_cast<FinWarp *>(smem + lay.q)[ew];
-            const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
-            const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
-            for (int k2 = 0; k2 < kRows / kEpiWarps; ++k2) {
-                const int rr = ew * (kRows / kEpiWarps) + k2;
-                const int rowr = c.rows_s[rr];
-                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
-                const int kr = rowcnt[rr];
-                if (!row_good(rowr, nv, kr)) continue;   // warp-uniform
-                finish_row(
-                    L, layer, h, rowr, kr, [&](int e) { return bvb[e * kBufStride + rr]; },
-                    [&](int e) { return (int)bib[e * kBufStride + rr]; }, fw, lane);
-            }
+        // finish the rows here (kRows / kEpiWarps per warp), the warps'
+        // scratch in the query/key buffers (every MMA is done)
+        FinWarp &fw = reinterpret_cast<FinWarp *>(smem + lay.q)[ew];
+        const float *bvb = reinterpret_cast<const float *>(smem + lay.bufv);
+        const uint16_t *bib = reinterpret_cast<const uint16_t *>(smem + lay.bufi);
+        for (int k2 = 0; k2 < kRows / kEpiWarps; ++k2) {
+            const int rr = ew * (kRows / kEpiWarps) + k2;
+            const int rowr = c.rows_s[rr];
+            const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
+            const int kr = rowcnt[rr];
+            if (!row_good(rowr, nv, kr)) continue;   // warp-uniform
+            finish_row(
+                L, layer, h, rowr, kr, [&](int e) { return bvb[e * kBufStride + rr]; },
+                [&](int e) { return (int)bib[e * kBufStride + rr]; }, fw, lane);
         }
     }
     cta_teardown(c, L);
-}
-
-// ---- finalize kernel (split path): one warp per row ---------------------------
-__global__ void __launch_bounds__(32 * kFinWarps)
-route_rows_finalize_kernel(LedgerDev L, int layer, int use_list) {
-    __shared__ FinWarp fw_all[kFinWarps];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y;
-    constexpr int kPerBlk = kRows / kFinWarps;   // finalize CTAs per route CTA
-    const int bx = blockIdx.x / kPerBlk;
-    const int r = (blockIdx.x % kPerBlk) * kFinWarps + warp;
-    const int count = use_list ? L.head_count[h] : L.nq;
-    const int row0 = bx * kRows;
-    if (row0 + r >= count) return;
-    const size_t blk = (size_t)h * ((L.nq + kRows - 1) / kRows) + bx;
-    const int meta = L.cand_meta[blk * kRows + r];
-    if (meta < 0) return;   // no row, or a row left to the retry path
-    const int row = use_list ? L.list[(size_t)h * L.nq + row0 + r] : row0 + r;
-    const float *gv = L.cand_v + (blk * kRows + r) * kCap;
-    const uint16_t *gi = L.cand_i + (blk * kRows + r) * kCap;
-    finish_row(
-        L, layer, h, row, meta, [&](int e) { return gv[e]; }, [&](int e) { return (int)gi[e]; },
-        fw_all[warp], lane);
 }
 
 // ---- relay rescoring on the tensor cores ---------------------------------------
@@ -1120,7 +741,7 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int d = L.d;
     const Layout lay = rescore_layout(d);
     Cta c;
-    if (!cta_setup(c, smem, lay, L, Q, L.list, L.head_count, 0)) return;
+    if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, 0)) return;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
 
@@ -1220,6 +841,11 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 if (!refresh) L.alpha[grow] = a;
                 if (n & (1 << 30)) atomicOr(&L.counters[2], 1ULL);
                 pairs = (unsigned)(n & ((1 << 30) - 1));
+            } else if (row >= 0) {
+                // a wait timed out (bit 1 of the error word): the row's scores
+                // are unknown, so it is flagged and the refresh rebuilds it
+                // rather than keeping a route no test confirmed
+                L.flags[(size_t)h * L.nq + row] = 1;
             }
             const unsigned wsum = __reduce_add_sync(kFull, pairs);
             if (lane == 0 && wsum) atomicAdd(&L.counters[1], (unsigned long long)wsum);
@@ -1234,7 +860,7 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t
                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn encode_fn() {
+static EncodeTiledFn encode_fn() {
     static EncodeTiledFn fn = nullptr;
     static bool tried = false;
     if (!tried) {
@@ -1248,6 +874,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)L.d, (cuuint64_t)L.nk, (cuuint64_t)L.bh};
+    const cuuint64_t strides[2] = {(cuuint64_t)L.d * 2, (cuuint64_t)L.nk * L.d * 2};
+    const cuuint32_t box[3] = {64u, (cuuint32_t)kKeys, 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return cr == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace tc
 
 bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
@@ -1259,35 +898,16 @@ bool route_rows_tc_supported(const LedgerDev &L, int dtype) {
     const tc::Layout lay = tc::layout_of(L.d, L.ksel, true);
     const tc::Layout layh = tc::layout_of(L.d, L.ksel, false);
     return lay.total <= 232448 && layh.total <= 232448 && tc::rescore_layout(L.d).total <= 232448 &&
-           lay.sel - lay.q >= (uint32_t)(tc::kEpiWarps * sizeof(tc::FinWarp));
+           lay.sel - lay.q >= (uint32_t)(tc::kEpiWarps * sizeof(tc::FinWarp)) &&
+           route_select_smem_bytes(L) <= 232448;
 }
 
-size_t route_rows_tc_smem_bytes(const LedgerDev &L) {
-    const size_t a = tc::layout_of(L.d, L.ksel, true).total;
-    const size_t b = tc::layout_of(L.d, L.ksel, false).total;
-    return a > b ? a : b;
-}
-
-CandSizes route_rows_tc_candidate_sizes(const LedgerDev &L, int dtype) {
-    CandSizes z{0, 0, 0};
-    if (!route_rows_tc_supported(L, dtype)) return z;
-    const size_t blocks = (size_t)L.bh * ((L.nq + tc::kRows - 1) / tc::kRows);
-    z.v = blocks * tc::kCap * tc::kRows * sizeof(float);
-    z.i = blocks * tc::kCap * tc::kRows * sizeof(uint16_t);
-    z.meta = blocks * tc::kRows * sizeof(int32_t);
-    return z;
-}
-
-cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
-    if (smem_bytes > 232448) return cudaErrorInvalidValue;   // 227 KB per block on sm_100
+cudaError_t route_rows_tc_prepare() {
     // the kernels may be launched with up to their largest layout
     const int big = (int)tc::layout_of(128, 64, true).total;
     const int big_heap = (int)tc::layout_of(128, 64, false).total;
-    cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<true>,
+    cudaError_t e = cudaFuncSetAttribute(tc::route_rows_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, big);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::route_rows_tc_kernel<false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, big);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(tc::route_rows_tc_heap_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, big_heap);
@@ -1295,27 +915,14 @@ cudaError_t route_rows_tc_prepare(size_t smem_bytes) {
         e = cudaFuncSetAttribute(tc::relay_rescore_tc_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)tc::rescore_layout(128).total);
+    if (e == cudaSuccess) e = route_select_prepare();
     return e;
-}
-
-// Tensor map of Kc [bh, nk, d] bf16: boxes of 128 keys x 64 dims, 128-byte swizzle.
-static cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map) {
-    tc::EncodeTiledFn enc = tc::encode_fn();
-    if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[3] = {(cuuint64_t)L.d, (cuuint64_t)L.nk, (cuuint64_t)L.bh};
-    const cuuint64_t strides[2] = {(cuuint64_t)L.d * 2, (cuuint64_t)L.nk * L.d * 2};
-    const cuuint32_t box[3] = {64u, (cuuint32_t)tc::kKeys, 1u};
-    const cuuint32_t estr[3] = {1u, 1u, 1u};
-    const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims,
-                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return cr == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                     cudaStream_t s) {
     CUtensorMap map;
-    cudaError_t e = key_tensor_map(L, k, &map);
+    cudaError_t e = tc::key_tensor_map(L, k, &map);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     tc::relay_rescore_tc_kernel<<<grid, tc::kPassThreads, tc::rescore_layout(L.d).total, s>>>(
@@ -1326,30 +933,31 @@ cudaError_t launch_relay_rescore_tc(const LedgerDev &L, const void *q, const voi
 cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
                                  bool use_list, cudaStream_t s) {
     CUtensorMap map;
-    cudaError_t e = key_tensor_map(L, k, &map);
+    cudaError_t e = tc::key_tensor_map(L, k, &map);
     if (e != cudaSuccess) return e;
     e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
-    const size_t smem2 = tc::layout_of(L.d, L.ksel, true).total;
-    if (L.cand_v && L.cand_i && L.cand_meta) {
-        tc::route_rows_tc_kernel<true><<<grid, tc::kPassThreads, smem2, s>>>(
+    if (L.cand_vals) {
+        // selection kernel + row finishing (rr_select_tc.cu)
+        e = launch_route_select(L, q, map, layer, use_list, SelectMode::kAnchor, s);
+    } else {
+        const size_t smem2 = tc::layout_of(L.d, L.ksel, true).total;
+        tc::route_rows_tc_kernel<<<grid, tc::kPassThreads, smem2, s>>>(
             L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
         e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        dim3 fgrid(grid.x * (tc::kRows / tc::kFinWarps), L.bh);
-        tc::route_rows_finalize_kernel<<<fgrid, 32 * tc::kFinWarps, 0, s>>>(L, layer,
-                                                                             use_list ? 1 : 0);
-    } else {
-        tc::route_rows_tc_kernel<false><<<grid, tc::kPassThreads, smem2, s>>>(
-            L, static_cast<const __nv_bfloat16 *>(q), map, layer, use_list ? 1 : 0);
     }
-    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    // rows the two-pass kernel could not finish: exact heap selection
+    return launch_route_retry(L, q, map, layer, s);
+}
+
+cudaError_t launch_route_retry(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
+                               cudaStream_t s) {
+    // rows the two-pass kernels could not finish: exact heap selection
     LedgerDev R = L;
     R.list = L.retry_list;
     R.head_count = L.retry_count;
+    dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     const size_t smemh = tc::layout_of(L.d, L.ksel, false).total;
     tc::route_rows_tc_heap_kernel<<<grid, tc::kHeapThreads, smemh, s>>>(
         R, static_cast<const __nv_bfloat16 *>(q), map, layer, 1);

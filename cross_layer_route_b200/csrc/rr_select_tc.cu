@@ -1,0 +1,925 @@
+// rr_select_tc.cu -- full routing and the relay layer on the tensor cores.
+//
+// Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
+// Dynamic Sparse Attention" (arXiv 2609.07306), cited as RouteRelay §x.
+//
+// Full routing of a row (§2.1 Eq. 1-2, §3.1 items 1-2) takes three steps:
+//
+//   route_select_kernel  (one CTA = one head x 128 query rows, the machinery
+//       of rr_tc.cuh with the query tile in TMEM as the MMA's A operand and
+//       three accumulators) scores the row block against the head's key
+//       tiles twice:
+//         pass 0  per row, the largest score of each of 128 column groups
+//                 (group = column mod 128); T = the (k+m)-th largest of these
+//                 maxima, found by a bit search on their 16-bit order keys
+//                 (floor), is at most the row's (k+m)-th best score since
+//                 that many distinct valid scores reach it;
+//         pass 1  every valid score >= T is kept: the thread owning (row,
+//                 quarter of the columns) appends it to its own slots in
+//                 shared memory and records the kept columns of each tile in
+//                 a 32-bit mask (device memory, one coalesced store per tile).
+//       The kept scores are then copied to the row's record in device memory.
+//   route_finish_kernel  (one CTA per row block, one warp per row) rebuilds
+//       the (score, chunk) pairs from the masks, orders them (score desc,
+//       chunk asc) by a counting sort over 64 bins with exact ranking inside
+//       a bin, writes route | near-miss and alpha (the k-th score), draws the
+//       random sentinels and adds the global ones.  Rows whose kept scores
+//       overflow the slots go to the exact one-pass heap kernel
+//       (rr_route_tc.cu).
+//
+// The relay layer (§3.2 Eq. 5-8, §4.1-4.2) runs the same two kernels over
+// every row and takes the relay decision in route_finish_kernel from the
+// kept scores: a candidate chunk of the old ledger row whose score is kept
+// has that exact score; one that is not kept scores below T.  So alpha (min
+// over the route, Eq. 6) is exact when every route chunk is kept, beta (max
+// over the sentinels, Eq. 7) is exact when at least one sentinel is kept,
+// and Eq. 8 can often be settled with one side bounded by T.  A stable row
+// keeps its ids and stores alpha; a challenged row is rebuilt from the same
+// kept scores at this layer.  Rows the bound cannot settle are rescored
+// exactly (relay_exact_kernel, candidate key rows gathered) and, if
+// challenged, rebuilt by the heap kernel.  On B200 the dense score tiles cost
+// less than the per-score work of the test, so one pass that both tests and
+// re-routes is cheaper than a rescoring pass followed by a re-route pass;
+// the ledger that comes out is the one the pages' two-stage procedure
+// defines, and the counters follow the pages' counting rule (c candidates per
+// relay row plus the valid keys of every refreshed row).
+#include "rr_tc.cuh"
+
+namespace rr {
+namespace tc {
+
+constexpr int kSelEpiWarps = 16;
+constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
+constexpr int kSelAcc = 3;                       // accumulators (TMEM columns 0..383)
+constexpr uint32_t kQCol = kSelAcc * 128;        // TMEM column of the query tile (A operand)
+constexpr int kQCap = 46;                        // kept-score slots per (row, quarter)
+constexpr int kValStride = kRows + 1;            // padded (slot, row) grid of the kept scores
+constexpr int kRowCap = 128;                     // kept scores per row the finishing handles
+constexpr int kTopWords = 65;                    // u32 words per row of 16-bit group maxima
+constexpr int kHalf = 16;                        // columns per capacity check in pass 1
+
+struct SelLayout {
+    uint32_t k, vals, rows, thr, cnt, bars, misc, total;
+    int stages;
+    __host__ __device__ CtaLayout cta() const { return CtaLayout{0u, k, rows, bars, misc, stages}; }
+};
+
+// k (key ring, 128 KB) | vals [4][kQCap][kValStride] f32 (the group maxima
+// [kRows][kTopWords] u32 after pass 0) | rows | thr | cnt | barriers | misc
+__host__ __device__ inline SelLayout sel_layout(int d) {
+    SelLayout s;
+    s.stages = d == 64 ? 8 : 4;
+    uint32_t o = 0;
+    s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
+    s.vals = o; o = up(o + 4 * kQCap * kValStride * 4, 16);
+    s.rows = o; o = up(o + kRows * 4, 16);
+    s.thr = o;  o = up(o + kRows * 4, 16);
+    s.cnt = o;  o = up(o + kRows * 4, 16);
+    s.bars = o; o = up(o + 8 * kNumBars, 16);
+    s.misc = o; o = up(o + 16, 16);
+    s.total = o + 1024;   // slack for aligning the dynamic base to 1024
+    return s;
+}
+
+__device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t *r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// MMA issuer of the selection kernel: A (the query tile) from TMEM.
+__device__ __forceinline__ void sel_mma_issuer(Cta &c, int d) {
+    const int total = 2 * c.ntiles;
+    const uint32_t k_addr = saddr(c.k_s);
+    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
+    const uint32_t a_tmem = c.tmem_base + kQCol;
+    const int steps = d >> 4;
+    for (int g = 0; g < total; ++g) {
+        const int s = g % c.stages, a = g % kSelAcc;
+        if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
+        if (!mbar_wait(&c.acc_empty[a], ((g / kSelAcc) & 1) ^ 1, c.abort_flag)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
+        const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
+        for (int kk = 0; kk < steps; ++kk) {
+            const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
+            tc_mma_bf16_ts(d_tmem, a_tmem + (uint32_t)(kk * 8), kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&c.empty[s]);
+        tc_commit(&c.acc_full[a]);
+    }
+    tc_commit(c.mma_done);
+    const long long t0 = clock64();
+    while (!mbar_test(c.mma_done, 0) && clock64() - t0 < kSpinLimit) {
+    }
+}
+
+// ---- selection kernel ------------------------------------------------------------
+__global__ void __launch_bounds__(kSelThreads, 1)
+route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+                    const __grid_constant__ CUtensorMap tmap_k, int use_list) {
+    extern __shared__ __align__(1024) unsigned char smem_dyn[];
+    unsigned char *smem = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    const int d = L.d, ksel = L.ksel;
+    const SelLayout lay = sel_layout(d);
+    Cta c;
+    if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, use_list, /*q_to_smem=*/false))
+        return;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+
+    // the query tile into TMEM columns kQCol.. (row r in lane r, two bf16 per
+    // column): epilogue warp (sub-partition sub, quarter qt) writes a quarter
+    // of the row's elements for its 32 rows
+    if (warp >= 2) {
+        const int ew = warp - 2, sub = warp & 3, qt = ew >> 2;
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const uint32_t taddr = c.tmem_base + ((uint32_t)(sub * 32) << 16) + kQCol + (uint32_t)(qt * (d >> 3));
+        uint32_t w[16];
+        const uint4 *src = reinterpret_cast<const uint4 *>(Q + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d +
+                                                           qt * (d >> 2));
+        if (d == 128) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+            }
+            tc_st16(taddr, w);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+            }
+            tc_st8(taddr, w);
+        }
+        tc_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    if (warp == 0) {
+        if (lane == 0) producer(c, &tmap_k, d, h, 2);
+    } else if (warp == 1) {
+        if (lane == 0) sel_mma_issuer(c, d);
+    } else {
+        // Four warps per TMEM sub-partition: quarter qt reads columns
+        // 32*qt..32*qt+31 of every tile.  The epilogue threads meet at named
+        // barrier 1 between phases (every one of them reaches every barrier,
+        // also after a timeout, so none can be left waiting).
+        const int ew = warp - 2;
+        const int sub = warp & 3;
+        const int qt = ew >> 2;
+        const int r = sub * 32 + lane;
+        const int row = c.rows_s[r];
+        const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
+        const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(qt * 32);
+        const int nt = c.ntiles;
+        bool ok = true;
+        auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kSelEpiWarps * 32) : "memory"); };
+
+        // pass 0: the largest valid score of each column group (this
+        // quarter's 32 columns of every tile; group = column mod 128)
+        float m[32];
+#pragma unroll
+        for (int q = 0; q < 32; ++q) m[q] = -INFINITY;
+        for (int i = 0; i < nt && ok; ++i) {
+            if (!(ok = acc_wait<kSelAcc>(c, i))) break;
+            float v[32];
+            tc_ld32(lane_base + (uint32_t)((i % kSelAcc) * kKeys), v);
+            acc_release<kSelAcc>(c, i);   // the scores are in registers: the MMA may reuse the accumulator
+            const int col0 = i * kKeys + qt * 32;
+            if (col0 + 32 <= n_valid) {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) m[q] = fmaxf(m[q], v[q]);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 32; ++q) m[q] = fmaxf(m[q], col0 + q < n_valid ? v[q] : -INFINITY);
+            }
+        }
+        // the row's 128 maxima as 16-bit order keys (the top half of the
+        // order-preserving key: a floor), [r][kTopWords] words
+        uint32_t *tops = reinterpret_cast<uint32_t *>(smem + lay.vals);
+#pragma unroll
+        for (int p = 0; p < 16; ++p)
+            tops[r * kTopWords + qt * 16 + p] = (ord32(m[2 * p]) >> 16) | (ord32(m[2 * p + 1]) & 0xFFFF0000u);
+        epi_sync();
+
+        // threshold of each row (kRows / kSelEpiWarps rows per warp): the
+        // largest 16-bit key K that at least k + m of the row's 128 maxima
+        // reach; T = the float of key K << 16.  The search starts below the
+        // bits the largest and smallest maxima share.  Rows with at most
+        // k + m valid keys keep all of them (T = -inf).
+        float *thr_s = reinterpret_cast<float *>(smem + lay.thr);
+        {
+            constexpr int kRowsPerWarp = kRows / kSelEpiWarps;
+            const uint16_t *tops16 = reinterpret_cast<const uint16_t *>(tops);
+            uint32_t key[kRowsPerWarp][4], K[kRowsPerWarp];
+            int hb[kRowsPerWarp];
+            int hbmax = -1;
+#pragma unroll
+            for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                const int rr = ew * kRowsPerWarp + k2;
+                uint32_t kmx = 0u, kmn = 0xFFFFu;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    key[k2][i] = tops16[rr * (2 * kTopWords) + i * 32 + lane];
+                    kmx = max(kmx, key[k2][i]);
+                    kmn = min(kmn, key[k2][i]);
+                }
+                kmx = __reduce_max_sync(kFull, kmx);
+                kmn = __reduce_min_sync(kFull, kmn);
+                const uint32_t x = kmx ^ kmn;
+                hb[k2] = x ? 31 - __clz(x) : -1;
+                K[k2] = hb[k2] >= 0 ? (kmx & ~((2u << hb[k2]) - 1u)) : kmx;
+                hbmax = max(hbmax, hb[k2]);
+            }
+            for (int bit = hbmax; bit >= 0; --bit) {
+#pragma unroll
+                for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                    const uint32_t cand = K[k2] | (1u << bit);
+                    const unsigned mine = (key[k2][0] >= cand ? 1u : 0u) + (key[k2][1] >= cand ? 1u : 0u) +
+                                          (key[k2][2] >= cand ? 1u : 0u) + (key[k2][3] >= cand ? 1u : 0u);
+                    const unsigned tot = __reduce_add_sync(kFull, mine);
+                    if (bit <= hb[k2] && (int)tot >= ksel) K[k2] = cand;
+                }
+            }
+#pragma unroll
+            for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
+                const int rr = ew * kRowsPerWarp + k2;
+                const int rowr = c.rows_s[rr];
+                const int nv = rowr >= 0 ? valid_keys(rowr, L.nk, L.causal) : 0;
+                float t = unord32(K[k2] << 16);
+                if (nv <= ksel || t != t) t = -INFINITY;
+                if (lane == k2) thr_s[rr] = t;
+            }
+        }
+        epi_sync();
+        const float T = thr_s[r];
+
+        // pass 1: keep every valid score >= T (tiles backwards: the first
+        // ones were loaded last).  This thread's slots are column r of rows
+        // qt*kQCap.. of the vals grid; a 16-column half takes the unchecked
+        // path while 16 more slots are free.
+        float *vals = reinterpret_cast<float *>(smem + lay.vals);
+        float *pv = vals + qt * kQCap * kValStride + r;
+        int cur = 0;
+        const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+        uint32_t *gmask = L.cand_masks + (blk * (size_t)L.mt * 4 + qt) * kRows + r;
+        for (int i = 0; i < nt && ok; ++i) {
+            const int g = nt + i;
+            const int t = nt - 1 - i;
+            if (!(ok = acc_wait<kSelAcc>(c, g))) break;
+            float v[32];
+            tc_ld32(lane_base + (uint32_t)((g % kSelAcc) * kKeys), v);
+            acc_release<kSelAcc>(c, g);
+            const int lim = n_valid - (t * kKeys + qt * 32);   // columns jj < lim are valid
+            uint32_t mask = 0u;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                if (lim >= 32 && cur <= kQCap - kHalf) {
+                    uint32_t mh = 0u;
+#pragma unroll
+                    for (int jj = hf * kHalf; jj < (hf + 1) * kHalf; ++jj) {
+                        if (v[jj] >= T) {
+                            *pv = v[jj];
+                            pv += kValStride;
+                            mh |= 1u << jj;
+                        }
+                    }
+                    cur += __popc(mh);
+                    mask |= mh;
+                } else {
+#pragma unroll
+                    for (int jj = hf * kHalf; jj < (hf + 1) * kHalf; ++jj) {
+                        if (jj < lim && v[jj] >= T) {
+                            if (cur < kQCap) {
+                                *pv = v[jj];
+                                pv += kValStride;
+                                mask |= 1u << jj;
+                            }
+                            ++cur;
+                        }
+                    }
+                }
+            }
+            gmask[(size_t)t * 4 * kRows] = mask;
+        }
+        // kept count per quarter, one byte each (0xFF: the row is redone)
+        reinterpret_cast<uint8_t *>(smem + lay.cnt)[r * 4 + qt] = (uint8_t)(cur <= kQCap ? cur : 0xFF);
+        epi_sync();
+
+        // hand-off: each row's kept scores to its record, quarter after
+        // quarter (one warp per row), with the counts and the threshold
+        const bool cta_ok = *c.abort_flag == 0;
+        const uint32_t *cnt_s = reinterpret_cast<const uint32_t *>(smem + lay.cnt);
+        for (int k2 = 0; k2 < kRows / kSelEpiWarps; ++k2) {
+            const int rr = ew * (kRows / kSelEpiWarps) + k2;
+            if (c.rows_s[rr] < 0) continue;   // warp-uniform
+            const uint32_t cw = cta_ok ? cnt_s[rr] : 0xFFFFFFFFu;
+            const size_t slot = blk * kRows + rr;
+            float *rec = L.cand_vals + slot * 4 * kQCap;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int n = (int)((cw >> (8 * q)) & 0xFFu);
+                if (n > kQCap) continue;
+                for (int e = lane; e < n; e += 32) rec[q * kQCap + e] = vals[(q * kQCap + e) * kValStride + rr];
+            }
+            if (lane == 0) L.cand_meta[slot] = make_uint2(cw, __float_as_uint(thr_s[rr]));
+        }
+    }
+    cta_teardown(c, L);
+}
+
+// ---- row finishing ---------------------------------------------------------------
+constexpr int kFinWarps = 16;
+constexpr int kFinThreads = 32 * kFinWarps;
+constexpr int kMaskTilesSmem = 32;     // blocks with at most this many key tiles stage their masks
+constexpr int kMaskStride = kRows + 1;
+constexpr int kBins = 64;
+constexpr int kBitsWords = 128;        // membership bitmaps: rows with <= 4096 valid keys
+
+struct FinScratch {
+    uint64_t keys[kRowCap];            // kept (score, chunk) keys, then in bin order
+    uint32_t hist[kBins];              // bin counts, then bin starts
+    uint32_t bits[kBitsWords];         // selected and accepted chunks
+    uint32_t rbits[kBitsWords];        // relay: chunks of the old route
+    uint32_t sbits[kBitsWords];        // relay: chunks of the old sentinels
+    int32_t acc[32];                   // accepted random sentinels, in order
+};
+
+__host__ __device__ inline size_t fin_smem_bytes() {
+    return (size_t)kMaskTilesSmem * 4 * kMaskStride * 4 + (size_t)kFinWarps * sizeof(FinScratch);
+}
+
+// Larger key = better: score desc, then chunk asc (-0 counts as +0).
+__device__ __forceinline__ uint64_t sel_key(float v, int j) {
+    const float z = v == 0.0f ? 0.0f : v;
+    return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
+}
+__device__ __forceinline__ int sel_key_chunk(uint64_t key) { return (int)(0xffffu - (uint32_t)(key & 0xffffu)); }
+__device__ __forceinline__ float sel_key_score(uint64_t key) { return unord32((uint32_t)(key >> 32)); }
+
+struct FinCounts {
+    unsigned long long rows = 0, pairs = 0, full = 0;
+};
+
+// One warp finishes one row.  Returns with nothing written when the row is
+// handed on: kept scores overflowed (anchor: retry list; relay: exact
+// rescoring), or (relay) the test keeps the old route or needs exact scores.
+template <bool kRelay, typename MaskAt>
+__device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h, int row, size_t slot,
+                                           MaskAt mask_at, FinScratch &w, int lane, FinCounts &cnt) {
+    const int n_valid = valid_keys(row, L.nk, L.causal);
+    const size_t grow = (size_t)h * L.nq + row;
+    const uint32_t lt_mask = (1u << lane) - 1u;
+    const uint2 meta = L.cand_meta[slot];
+    const float T = __uint_as_float(meta.y);
+    int c4[4];
+    bool redo = false;
+    int total = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        c4[q] = (int)((meta.x >> (8 * q)) & 0xFFu);
+        redo |= c4[q] > kQCap;
+        total += c4[q];
+    }
+    redo |= total > kRowCap || total < min(L.ksel, n_valid);
+
+    // the kept (score, chunk) pairs: mask (quarter q, tile t) holds the kept
+    // columns of that tile; a quarter's scores are stored tile by tile from
+    // the last tile down, columns ascending inside a tile
+    const int ntr = (n_valid + kKeys - 1) / kKeys;
+    const int nidx = 4 * ntr;
+    const float *rec = L.cand_vals + slot * 4 * kQCap;
+    int carry = 0;
+    if (!redo) {
+        for (int base = 0; base < nidx; base += 32) {
+            const int idx = base + lane;
+            uint32_t mk = 0u;
+            int q = 0, t = 0;
+            if (idx < nidx) {
+                q = idx / ntr;
+                t = ntr - 1 - (idx - q * ntr);
+                mk = mask_at(t, q);
+            }
+            const int pc = __popc(mk);
+            int incl = pc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int x = __shfl_up_sync(kFull, incl, o);
+                if (lane >= o) incl += x;
+            }
+            int e = carry + incl - pc;
+            const int qs = (q > 0 ? c4[0] : 0) + (q > 1 ? c4[1] : 0) + (q > 2 ? c4[2] : 0);
+            int off = e - qs;
+            while (mk != 0u) {
+                const int b = __ffs(mk) - 1;
+                mk &= mk - 1u;
+                if (e < kRowCap && off < kQCap) w.keys[e] = sel_key(rec[q * kQCap + off], t * kKeys + q * 32 + b);
+                ++e;
+                ++off;
+            }
+            carry += __shfl_sync(kFull, incl, 31);
+        }
+        redo = carry != total;   // masks and counts disagree: redo the row
+    }
+    if (redo) {
+        if (lane == 0) {
+            if (kRelay) {
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
+                L.flags[grow] = 0;
+            } else {
+                const int pos = atomicAdd(&L.retry_count[h], 1);
+                L.retry_list[(size_t)h * L.nq + pos] = row;
+                atomicAdd(&L.counters[10], 1ULL);
+            }
+        }
+        return;
+    }
+    __syncwarp();
+    uint64_t key[4];
+    bool live[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int e = lane + 32 * i;
+        live[i] = e < total;
+        key[i] = live[i] ? w.keys[e] : 0ull;
+    }
+
+    if constexpr (kRelay) {
+        // relay test of the old ledger row (§3.2 Eq. 5-8) from the kept scores
+        const int words = (n_valid + 31) >> 5;
+        if (n_valid > 32 * kBitsWords) {   // no bitmap for such rows: rescore exactly
+            if (lane == 0) {
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
+                L.flags[grow] = 0;
+            }
+            return;
+        }
+        for (int q = lane; q < words; q += 32) {
+            w.rbits[q] = 0u;
+            w.sbits[q] = 0u;
+        }
+        __syncwarp();
+        const int32_t *idr = L.ids + grow * L.c;
+        int rt = 0, st = 0;
+        bool bad = false;
+        for (int e0 = 0; e0 < L.c; e0 += 32) {
+            const int e = e0 + lane;
+            const int j = e < L.c ? idr[e] : -1;
+            const bool valid = j >= 0 && j < n_valid;
+            bad |= j >= n_valid || j < -1;
+            if (valid) atomicOr(&(e < L.k ? w.rbits : w.sbits)[j >> 5], 1u << (j & 31));
+            rt += __popc(__ballot_sync(kFull, valid && e < L.k));
+            st += __popc(__ballot_sync(kFull, valid && e >= L.k));
+        }
+        if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.counters[2], 1ULL);
+        __syncwarp();
+        float amin = INFINITY, bmax = -INFINITY;
+        int rf = 0, sf = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            if (!live[i]) continue;
+            const int j = sel_key_chunk(key[i]);
+            const float v = sel_key_score(key[i]);
+            if ((w.rbits[j >> 5] >> (j & 31)) & 1u) { amin = fminf(amin, v); ++rf; }   // Eq. 6
+            if ((w.sbits[j >> 5] >> (j & 31)) & 1u) { bmax = fmaxf(bmax, v); ++sf; }   // Eq. 7
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
+            bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+        }
+        rf = (int)__reduce_add_sync(kFull, (unsigned)rf);
+        sf = (int)__reduce_add_sync(kFull, (unsigned)sf);
+        // alpha is exact when every route chunk was kept; beta when a
+        // sentinel was kept (the others score below T) or there is none
+        const bool aexact = rf == rt;
+        const bool bexact = sf > 0 || st == 0;
+        int dec = -1;   // 0 keep, 1 refresh, 2 rescore exactly
+        if (L.max_age > 0 || L.min_reuse > 0) {   // the ledger's age rules, as relay_refresh
+            const int age = layer - L.anchor_layer[grow];
+            if (L.max_age > 0 && age >= L.max_age) dec = 1;
+            else if (L.min_reuse > 0 && age <= L.min_reuse) dec = aexact ? 0 : 2;
+        }
+        if (dec < 0) {
+            const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
+            if (aexact && bexact) dec = (amin > bmax + g) ? 0 : 1;   // Eq. 8
+            else if (aexact) dec = (amin > T + g) ? 0 : 2;        // beta < T
+            else if (sf > 0) dec = 1;                             // alpha < T <= beta
+            else dec = 2;
+        }
+        if (dec == 0) {
+            if (lane == 0) {
+                L.alpha[grow] = amin;
+                L.flags[grow] = 0;
+            }
+            cnt.pairs += (unsigned long long)(rt + st);
+            return;
+        }
+        if (dec == 2) {
+            if (lane == 0) {
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
+                L.flags[grow] = 0;
+            }
+            return;
+        }
+        cnt.pairs += (unsigned long long)(rt + st + n_valid);
+        cnt.rows += 1;
+        cnt.full += (unsigned long long)n_valid;
+    }
+
+    // order: counting sort of the kept keys over 64 bins of their score key
+    // (larger key = lower bin), then each key's rank among the keys of its bin
+    uint32_t hmx = 0u, hmn = 0xFFFFFFFFu;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        if (!live[i]) continue;
+        const uint32_t hi = (uint32_t)(key[i] >> 32);
+        hmx = max(hmx, hi);
+        hmn = min(hmn, hi);
+    }
+    hmx = __reduce_max_sync(kFull, hmx);
+    hmn = __reduce_min_sync(kFull, hmn);
+    const float scale = (float)kBins / ((float)(hmx - hmn) + 1.0f);
+    w.hist[lane] = 0u;
+    w.hist[lane + 32] = 0u;
+    __syncwarp();
+    int bin[4];
+    uint32_t in_bin[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        bin[i] = min(kBins - 1, (int)((float)(hmx - (uint32_t)(key[i] >> 32)) * scale));
+        in_bin[i] = live[i] ? atomicAdd(&w.hist[bin[i]], 1u) : 0u;
+    }
+    __syncwarp();
+    {
+        const uint32_t h0 = w.hist[2 * lane], h1 = w.hist[2 * lane + 1];
+        uint32_t incl = h0 + h1;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t x = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += x;
+        }
+        const uint32_t excl = incl - h0 - h1;
+        __syncwarp();
+        w.hist[2 * lane] = excl;
+        w.hist[2 * lane + 1] = excl + h0;
+    }
+    __syncwarp();
+    int start[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        start[i] = (int)w.hist[bin[i]];
+        if (live[i]) w.keys[start[i] + (int)in_bin[i]] = key[i];
+    }
+    __syncwarp();
+    const int nr = min(L.k, n_valid);
+    const int nm = min(L.m, n_valid - nr);
+    const int nsel = nr + nm;
+    int32_t *out = L.ids + grow * L.c;
+    bool sel[4];
+    int jc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        sel[i] = false;
+        jc[i] = live[i] ? sel_key_chunk(key[i]) : -1;
+        if (!live[i]) continue;
+        const int end = bin[i] + 1 < kBins ? (int)w.hist[bin[i] + 1] : total;
+        int rank = 0;
+        for (int p = start[i]; p < end; ++p) rank += w.keys[p] > key[i] ? 1 : 0;
+        const int pos = start[i] + rank;
+        if (pos < nsel) {
+            sel[i] = true;
+            out[pos < nr ? pos : L.k + (pos - nr)] = jc[i];
+            if (pos == nr - 1) L.alpha[grow] = sel_key_score(key[i]);
+        }
+    }
+    for (int sl = lane; sl < L.k + L.m; sl += 32) {   // padding of short rows
+        if (sl < L.k ? sl >= nr : sl - L.k >= nm) out[sl] = -1;
+    }
+
+    // random sentinels (§3.1 item 2, §3.4): Philox4x32-10 words keyed
+    // (seed; global head, row, layer, t/4), chunk = (word * n_valid) >> 32,
+    // repeats and route / near-miss / global members rejected, accepted in
+    // draw order; a pool of at most r chunks is taken whole in ascending
+    // order, and a row that exhausts max_draws is completed in ascending order
+    const bool use_bits = n_valid <= 32 * kBitsWords;
+    if (use_bits) {
+        const int words = (n_valid + 31) >> 5;
+        for (int q = lane; q < words; q += 32) w.bits[q] = 0u;
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (sel[i]) atomicOr(&w.bits[jc[i] >> 5], 1u << (jc[i] & 31));
+        __syncwarp();
+    }
+    int acc = 0;
+    auto in_sel_or_acc = [&](int j) -> bool {
+        if (use_bits) return ((w.bits[j >> 5] >> (j & 31)) & 1u) != 0u;
+        bool hit = false;
+        for (int src = 0; src < 32; ++src) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int cj = __shfl_sync(kFull, sel[i] ? jc[i] : -1, src);
+                hit |= cj == j;
+            }
+        }
+        for (int a = 0; a < acc; ++a) hit |= w.acc[a] == j;
+        return hit;
+    };
+    // mandatory global sentinels (§3.1 item 3; g <= 32): lane t examines
+    // candidate t; they follow the random block and leave the random pool
+    const int g = L.g_sink + L.g_recent;
+    int n_glob = 0;
+    if (g > 0) {
+        const int jg = lane < g ? global_cand(L, row, lane) : -1;
+        const bool listable = lane < g && global_cand_listable(L, lane, jg, n_valid);
+        const bool in_rn = in_sel_or_acc(listable ? jg : 0);   // nothing accepted yet
+        const bool keep = listable && !in_rn;
+        const uint32_t km = __ballot_sync(kFull, keep);
+        n_glob = __popc(km);
+        int32_t *gout = out + L.k + L.m + L.r;
+        if (keep) gout[__popc(km & lt_mask)] = jg;
+        if (lane >= n_glob && lane < g) gout[lane] = -1;
+    }
+    auto taken = [&](int j) -> bool {
+        const bool hit = in_sel_or_acc(j);   // every lane calls it (it may shuffle)
+        return hit || is_global_cand(L, row, n_valid, j);
+    };
+    auto accept = [&](bool is_free, int j) {
+        const uint32_t fm = __ballot_sync(kFull, is_free);
+        const int idx = acc + __popc(fm & lt_mask);
+        if (is_free && idx < L.r) {
+            w.acc[idx] = j;
+            if (use_bits) atomicOr(&w.bits[j >> 5], 1u << (j & 31));
+        }
+        acc = min(L.r, acc + __popc(fm));
+        __syncwarp();
+    };
+    if (L.r > 0) {
+        if (n_valid - nsel - n_glob > L.r) {
+            for (int t0 = 0; acc < L.r && t0 < L.max_draws; t0 += 32) {
+                const int t = t0 + lane;
+                const PhiloxOut o = philox4x32_10((uint32_t)(L.bh_offset + h), (uint32_t)row,
+                                                  (uint32_t)layer, (uint32_t)(t >> 2), L.seed_lo, L.seed_hi);
+                const int q = t & 3;
+                const uint32_t word = q == 0 ? o.w[0] : q == 1 ? o.w[1] : q == 2 ? o.w[2] : o.w[3];
+                const int j = (int)__umulhi(word, (uint32_t)n_valid);
+                const bool tk = taken(j);
+                const bool ok_t = t < L.max_draws && !tk;
+                const uint32_t same = __match_any_sync(kFull, j) & __ballot_sync(kFull, ok_t);
+                accept(ok_t && (same & lt_mask) == 0u, j);
+            }
+            if (acc < L.r && lane == 0) atomicAdd(&L.counters[7], 1ULL);
+        }
+        for (int j0 = 0; acc < L.r && j0 < n_valid; j0 += 32) {
+            const int j = j0 + lane;
+            const bool tk = taken(min(j, n_valid - 1));
+            accept(j < n_valid && !tk, j);
+        }
+    }
+    __syncwarp();
+    if (lane < L.r) out[L.k + L.m + lane] = lane < acc ? w.acc[lane] : -1;
+    if (lane == 0) {
+        L.anchor_layer[grow] = layer;
+        L.flags[grow] = 1;
+    }
+}
+
+template <bool kRelay>
+__global__ void __launch_bounds__(kFinThreads)
+route_finish_kernel(LedgerDev L, int layer, int use_list) {
+    extern __shared__ __align__(16) unsigned char fsm[];
+    __shared__ int red_row[kFinWarps];
+    __shared__ unsigned long long red_cnt[kFinWarps][3];
+    uint32_t *masks_s = reinterpret_cast<uint32_t *>(fsm);
+    FinScratch *scr = reinterpret_cast<FinScratch *>(fsm + (size_t)kMaskTilesSmem * 4 * kMaskStride * 4);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h = blockIdx.y;
+    const int count = use_list ? L.head_count[h] : L.nq;
+    const int row0 = blockIdx.x * kRows;
+    if (row0 >= count) return;
+    const int n_rows = min(kRows, count - row0);
+    // the block's key tiles, as the selection kernel counted them
+    int myrow = -1;
+    if (tid < n_rows) myrow = use_list ? L.list[(size_t)h * L.nq + row0 + tid] : row0 + tid;
+    const int wmax = __reduce_max_sync(kFull, myrow);
+    if (lane == 0) red_row[warp] = wmax;
+    __syncthreads();
+    int max_row = -1;
+    for (int i = 0; i < kFinWarps; ++i) max_row = max(max_row, red_row[i]);
+    const int kend = L.causal ? min(L.nk, max_row + 1) : L.nk;
+    const int nt = (kend + kKeys - 1) / kKeys;
+    const size_t blk = (size_t)h * gridDim.x + blockIdx.x;
+    const uint32_t *gmask = L.cand_masks + blk * (size_t)L.mt * 4 * kRows;
+    const bool staged = nt <= kMaskTilesSmem;
+    if (staged) {
+        for (int e = tid; e < nt * 4 * kRows; e += blockDim.x) {
+            const int tq = e / kRows, r = e - tq * kRows;
+            masks_s[tq * kMaskStride + r] = gmask[e];
+        }
+    }
+    __syncthreads();
+
+    FinCounts cnt;
+    for (int k2 = 0; k2 < kRows / kFinWarps; ++k2) {
+        const int rr = warp * (kRows / kFinWarps) + k2;
+        if (rr >= n_rows) break;   // warp-uniform
+        const int row = use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr;
+        const size_t slot = blk * kRows + rr;
+        if (staged) {
+            finish_one<kRelay>(
+                L, layer, h, row, slot, [&](int t, int q) { return masks_s[(t * 4 + q) * kMaskStride + rr]; },
+                scr[warp], lane, cnt);
+        } else {
+            finish_one<kRelay>(
+                L, layer, h, row, slot, [&](int t, int q) { return gmask[((size_t)t * 4 + q) * kRows + rr]; },
+                scr[warp], lane, cnt);
+        }
+        __syncwarp();
+    }
+    if (kRelay) {
+        if (lane == 0) {
+            red_cnt[warp][0] = cnt.rows;
+            red_cnt[warp][1] = cnt.pairs;
+            red_cnt[warp][2] = cnt.full;
+        }
+        __syncthreads();
+        if (tid < 3) {
+            unsigned long long s = 0;
+            for (int i = 0; i < kFinWarps; ++i) s += red_cnt[i][tid];
+            const int slot_of[3] = {0, 1, 8};   // rows, pairs, full-routing pairs of the layer
+            if (s) atomicAdd(&L.counters[slot_of[tid]], s);
+        }
+    }
+}
+
+// ---- exact rescoring of the relay rows the kept scores leave open ------------------
+// One warp per listed row: alpha and beta from the row's candidate key rows
+// (Eq. 5-7, fp32 products of the bf16 inputs), the decision of Eq. 8 with
+// the ledger's age rules; a challenged row goes to the retry list and is
+// rebuilt by the heap kernel.
+constexpr int kExactWarps = 8;
+
+template <int D>
+__global__ void __launch_bounds__(32 * kExactWarps)
+relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
+                   int layer) {
+    __shared__ __align__(16) float qs[kExactWarps][D];
+    __shared__ unsigned long long red_cnt[kExactWarps][3];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n = *L.und_count;
+    unsigned long long crow = 0, cpair = 0, cfull = 0;
+    for (int u = blockIdx.x * kExactWarps + warp; u < n; u += gridDim.x * kExactWarps) {
+        const int grow = L.und_list[u];
+        const int h = grow / L.nq, i = grow - h * L.nq;
+        const int n_valid = valid_keys(i, L.nk, L.causal);
+        for (int t = lane; t < D; t += 32) qs[warp][t] = __bfloat162float(Q[(size_t)grow * D + t]);
+        __syncwarp();
+        const int32_t *idr = L.ids + (size_t)grow * L.c;
+        const __nv_bfloat16 *Kh = K + (size_t)h * L.nk * D;
+        float amin = INFINITY, bmax = -INFINITY;
+        int ncand = 0;
+        bool bad = false;
+        for (int e0 = 0; e0 < L.c; e0 += 32) {
+            const int e = e0 + lane;
+            const int j = e < L.c ? idr[e] : -1;
+            const bool valid = j >= 0 && j < n_valid;
+            bad |= j >= n_valid || j < -1;
+            if (valid) {
+                const uint4 *kp = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int c8 = 0; c8 < D / 8; ++c8) {
+                    const uint4 kv = __ldg(kp + c8);
+                    const float *qv = qs[warp] + c8 * 8;
+                    acc[0] = fmaf(qv[0], __uint_as_float(kv.x << 16), acc[0]);
+                    acc[1] = fmaf(qv[1], __uint_as_float(kv.x & 0xffff0000u), acc[1]);
+                    acc[2] = fmaf(qv[2], __uint_as_float(kv.y << 16), acc[2]);
+                    acc[3] = fmaf(qv[3], __uint_as_float(kv.y & 0xffff0000u), acc[3]);
+                    acc[0] = fmaf(qv[4], __uint_as_float(kv.z << 16), acc[0]);
+                    acc[1] = fmaf(qv[5], __uint_as_float(kv.z & 0xffff0000u), acc[1]);
+                    acc[2] = fmaf(qv[6], __uint_as_float(kv.w << 16), acc[2]);
+                    acc[3] = fmaf(qv[7], __uint_as_float(kv.w & 0xffff0000u), acc[3]);
+                }
+                const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                if (e < L.k) amin = fminf(amin, sc);   // Eq. 6
+                else bmax = fmaxf(bmax, sc);           // Eq. 7
+                ++ncand;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
+            bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
+            ncand += __shfl_xor_sync(kFull, ncand, o);
+        }
+        const bool any_bad = __any_sync(kFull, bad);
+        if (lane == 0) {
+            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);   // Eq. 8
+            L.flags[grow] = refresh ? 1 : 0;
+            if (!refresh) L.alpha[grow] = amin;
+            if (any_bad) atomicOr(&L.counters[2], 1ULL);
+            cpair += (unsigned long long)ncand;
+            if (refresh) {
+                const int pos = atomicAdd(&L.retry_count[h], 1);
+                L.retry_list[(size_t)h * L.nq + pos] = i;
+                atomicAdd(&L.counters[10], 1ULL);
+                crow += 1;
+                cpair += (unsigned long long)n_valid;
+                cfull += (unsigned long long)n_valid;
+            }
+        }
+        __syncwarp();
+    }
+    if (lane == 0) {
+        red_cnt[warp][0] = crow;
+        red_cnt[warp][1] = cpair;
+        red_cnt[warp][2] = cfull;
+    }
+    __syncthreads();
+    if (threadIdx.x < 3) {
+        unsigned long long s = 0;
+        for (int w = 0; w < kExactWarps; ++w) s += red_cnt[w][threadIdx.x];
+        const int slot_of[3] = {0, 1, 8};
+        if (s) atomicAdd(&L.counters[slot_of[threadIdx.x]], s);
+    }
+}
+
+}  // namespace tc
+
+CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype) {
+    CandSizes z{0, 0, 0, 0};
+    if (!route_rows_tc_supported(L, dtype)) return z;
+    const size_t blocks = (size_t)L.bh * ((L.nq + tc::kRows - 1) / tc::kRows);
+    const size_t mt = (size_t)((L.nk + tc::kKeys - 1) / tc::kKeys);
+    z.vals = blocks * tc::kRows * 4 * tc::kQCap * sizeof(float);
+    z.masks = blocks * mt * 4 * tc::kRows * sizeof(uint32_t);
+    z.meta = blocks * tc::kRows * sizeof(uint2);
+    z.und = (size_t)L.bh * L.nq * sizeof(int32_t);
+    return z;
+}
+
+size_t route_select_smem_bytes(const LedgerDev &L) { return tc::sel_layout(L.d).total; }
+
+cudaError_t route_select_prepare() {
+    cudaError_t e = cudaFuncSetAttribute(tc::route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tc::sel_layout(128).total);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::route_finish_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc::fin_smem_bytes());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(tc::route_finish_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)tc::fin_smem_bytes());
+    return e;
+}
+
+cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
+                                bool use_list, SelectMode mode, cudaStream_t s) {
+    dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
+    tc::route_select_kernel<<<grid, tc::kSelThreads, tc::sel_layout(L.d).total, s>>>(
+        L, static_cast<const __nv_bfloat16 *>(q), map, use_list ? 1 : 0);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    if (mode == SelectMode::kRelay)
+        tc::route_finish_kernel<true><<<grid, tc::kFinThreads, tc::fin_smem_bytes(), s>>>(L, layer, 0);
+    else
+        tc::route_finish_kernel<false><<<grid, tc::kFinThreads, tc::fin_smem_bytes(), s>>>(L, layer,
+                                                                                            use_list ? 1 : 0);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *k, int layer,
+                                 cudaStream_t s) {
+    CUtensorMap map;
+    cudaError_t e = tc::key_tensor_map(L, k, &map);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.und_count, 0, sizeof(int32_t), s);
+    if (e == cudaSuccess) e = launch_route_select(L, q, map, layer, false, SelectMode::kRelay, s);
+    if (e != cudaSuccess) return e;
+    const auto *Q = static_cast<const __nv_bfloat16 *>(q);
+    const auto *K = static_cast<const __nv_bfloat16 *>(k);
+    const unsigned grid = 148 * 2;   // grid-stride over the open rows (usually none)
+    if (L.d == 128) tc::relay_exact_kernel<128><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
+    else tc::relay_exact_kernel<64><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_route_retry(L, q, map, layer, s);
+}
+
+}  // namespace rr
