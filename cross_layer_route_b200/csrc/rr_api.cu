@@ -37,7 +37,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
     size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count;
     // tensor-core selection path only (size 0 otherwise)
-    size_t cand_vals, cand_masks, cand_meta, und_list, und_count;
+    size_t cand_keys, cand_masks, cand_meta, und_list, und_count;
     bool cand;
     size_t total;
 };
@@ -77,8 +77,8 @@ Layout layout_of(const rr_config *c) {
     t.g_sink = c->g_sink; t.g_recent = c->g_recent; t.c = (int)cc;
     t.mt = (c->nk + 127) / 128;
     const rr::CandSizes cs = rr::route_select_candidate_sizes(t, c->dtype);
-    L.cand = cs.vals > 0;
-    L.cand_vals = o;    o = align_up(o + cs.vals);
+    L.cand = cs.keys > 0;
+    L.cand_keys = o;    o = align_up(o + cs.keys);
     L.cand_masks = o;   o = align_up(o + cs.masks);
     L.cand_meta = o;    o = align_up(o + cs.meta);
     L.und_list = o;     o = align_up(o + cs.und);
@@ -237,7 +237,7 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
     D.retry_list = reinterpret_cast<int32_t *>(L->ws + lay.retry_list);
     D.retry_count = reinterpret_cast<int32_t *>(L->ws + lay.retry_count);
     if (lay.cand) {
-        D.cand_vals = reinterpret_cast<float *>(L->ws + lay.cand_vals);
+        D.cand_keys = reinterpret_cast<uint64_t *>(L->ws + lay.cand_keys);
         D.cand_masks = reinterpret_cast<uint32_t *>(L->ws + lay.cand_masks);
         D.cand_meta = reinterpret_cast<uint2 *>(L->ws + lay.cand_meta);
         D.und_list = reinterpret_cast<int32_t *>(L->ws + lay.und_list);
@@ -278,7 +278,7 @@ rr_status rr_relay_layer(rr_ledger *ledger, const void *d_qc, const void *d_kc, 
     if (!ledger->anchored || layer <= ledger->last_layer) return RR_ESTATE;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (is_forced_anchor(ledger, layer)) return do_full_route(ledger, d_qc, d_kc, layer, s);
-    if (ledger->dev.cand_vals) return do_relay_oneshot(ledger, d_qc, d_kc, layer, s);
+    if (ledger->dev.cand_keys) return do_relay_oneshot(ledger, d_qc, d_kc, layer, s);
     st = stage_rescore(ledger, d_qc, d_kc, layer, s);
     if (st == RR_OK) st = stage_compact(ledger, layer, s);
     if (st == RR_OK) st = stage_refresh(ledger, d_qc, d_kc, layer, s);

@@ -24,9 +24,10 @@ struct LedgerDev {
     // buffers of the tensor-core selection path (null: the allocation-free
     // entry point, whose route kernel finishes its rows itself).  Row slot
     // s = (head * blocks_per_head + block) * 128 + position in the block.
-    float *cand_vals = nullptr;      // [slots, 4, kQCap] kept scores per row quarter
-    uint32_t *cand_masks = nullptr;  // [blocks, mt, 4, 128] kept columns per (tile, quarter, row)
-    uint2 *cand_meta = nullptr;      // [slots] {kept per quarter (bytes, 0xFF = redo), threshold}
+    uint64_t *cand_keys = nullptr;   // [slots, kRowCap] kept (score, chunk) sort keys
+    uint32_t *cand_masks = nullptr;  // [blocks, mt, 4, 128] kept columns per (tile, quarter, row),
+                                     // only for heads of more than 32 key tiles
+    uint2 *cand_meta = nullptr;      // [slots] {kept keys (all ones: redo the row), threshold}
     int32_t *und_list = nullptr;     // [bh*nq] relay rows whose test needs exact rescoring
     int32_t *und_count = nullptr;    // [1]
     int mt = 0;                      // key tiles per head: ceil(nk / 128)
@@ -63,6 +64,8 @@ inline int select_capacity(int ksel) {
 // CUDA cores (rr_route_simt.cu).  prepare() sets the chosen kernel's shared
 // memory attribute on the current device.
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype);
+// The same for every kernel at its largest layout (any config), once per device.
+cudaError_t route_rows_prepare_all();
 bool route_rows_tc_supported(const LedgerDev &L, int dtype);
 cudaError_t route_rows_tc_prepare();
 cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *k, int layer,
@@ -71,7 +74,7 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
 // Tensor-core selection path (rr_select_tc.cu): the selection kernel writes
 // every row's kept scores to the candidate buffers, the finishing kernel
 // orders them and writes the ledger row.
-struct CandSizes { size_t vals, masks, meta, und; };
+struct CandSizes { size_t keys, masks, meta, und; };
 // Bytes of the buffers (all 0 when the problem does not run on the tensor cores).
 CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype);
 size_t route_select_smem_bytes(const LedgerDev &L);

@@ -37,8 +37,10 @@ static __device__ __align__(256) int32_t g_rr_static_scratch[2 * (kStaticMaxRows
 std::mutex g_setup_mutex;
 int32_t *g_scratch_addr[kMaxDevices] = {nullptr};
 
-// Per-device set-up: the device address of the static scratch, looked up
-// with the device current.  Returns nullptr on failure.
+// Per-device set-up, done once per device with that device current: the
+// device address of the static scratch, and the kernels' shared-memory
+// attributes at their largest layouts (so later calls make no host API call
+// for them).  Returns nullptr on failure.
 int32_t *static_scratch_on_current_device() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -46,6 +48,7 @@ int32_t *static_scratch_on_current_device() {
     if (!g_scratch_addr[dev]) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_rr_static_scratch) != cudaSuccess || !ptr) return nullptr;
+        if (rr::route_rows_prepare_all() != cudaSuccess) return nullptr;
         g_scratch_addr[dev] = static_cast<int32_t *>(ptr);
     }
     return g_scratch_addr[dev];
@@ -103,7 +106,6 @@ extern "C" rr_status rr_route_layer_static(const rr_config *cfg, const void *d_q
     D.seed_hi = (uint32_t)(cfg->seed >> 32);
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (rr::route_rows_prepare(D, cfg->dtype) != cudaSuccess) return RR_ECUDA;
     const int H = cfg->anchor_interval;
     const bool anchor = layer == 0 || (H > 0 && layer % H == 0);
     cudaError_t e = cudaMemsetAsync(d_counters + RR_CNT_ROWS, 0, 2 * sizeof(int64_t), s);

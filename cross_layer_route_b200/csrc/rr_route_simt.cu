@@ -289,6 +289,17 @@ cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
                                 smem);
 }
 
+cudaError_t route_rows_prepare_all() {
+    // the largest layout any config may launch: d = 256, k + m = 128
+    const int smem = (int)smem_layout(256, select_capacity(128)).total;
+    cudaError_t e = cudaFuncSetAttribute(route_rows_kernel<__nv_bfloat16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(route_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) e = route_rows_tc_prepare();
+    return e;
+}
+
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s) {
     if (route_rows_tc_supported(L, dtype)) return launch_route_rows_tc(L, q, k, layer, use_list, s);

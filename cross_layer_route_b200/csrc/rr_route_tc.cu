@@ -189,8 +189,7 @@ __global__ void __launch_bounds__(kHeapThreads, 1)
 route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                           const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    unsigned char *smem = align_smem_1024(smem_dyn);
     const int d = L.d, ksel = L.ksel;
     const Layout lay = layout_of(d, ksel, false);
     Cta c;
@@ -199,9 +198,9 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int h = blockIdx.y;
 
     if (warp == 0) {
-        if (lane == 0) producer(c, &tmap_k, d, h, 1);
+        producer(c, &tmap_k, d, h, 1);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(c, d, 1);
+        mma_issuer(c, d, 1);
     } else {
         const int sub = warp & 3;
         const int r = sub * 32 + lane;
@@ -504,8 +503,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
 route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                      const __grid_constant__ CUtensorMap tmap_k, int layer, int use_list) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    unsigned char *smem = align_smem_1024(smem_dyn);
     const int d = L.d, ksel = L.ksel;
     const Layout lay = layout_of(d, ksel, true);
     Cta c;
@@ -514,9 +512,9 @@ route_rows_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int h = blockIdx.y;
 
     if (warp == 0) {
-        if (lane == 0) producer(c, &tmap_k, d, h, 2);
+        producer(c, &tmap_k, d, h, 2);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(c, d, 2);
+        mma_issuer(c, d, 2);
     } else {
         // Four warps per TMEM sub-partition: quarter qt reads columns
         // 32*qt..32*qt+31 of every tile.  The epilogue threads meet at named
@@ -736,8 +734,7 @@ __global__ void __launch_bounds__(kPassThreads, 1)
 relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                         const __grid_constant__ CUtensorMap tmap_k, int layer) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    unsigned char *smem = align_smem_1024(smem_dyn);
     const int d = L.d;
     const Layout lay = rescore_layout(d);
     Cta c;
@@ -746,9 +743,9 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int h = blockIdx.y;
 
     if (warp == 0) {
-        if (lane == 0) producer(c, &tmap_k, d, h, 1);
+        producer(c, &tmap_k, d, h, 1);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(c, d, 1);
+        mma_issuer(c, d, 1);
     } else {
         const int ew = warp - 2;
         const int sub = warp & 3;
@@ -938,7 +935,7 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
     e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
-    if (L.cand_vals) {
+    if (L.cand_keys) {
         // selection kernel + row finishing (rr_select_tc.cu)
         e = launch_route_select(L, q, map, layer, use_list, SelectMode::kAnchor, s);
     } else {

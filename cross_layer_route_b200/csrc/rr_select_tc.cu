@@ -3,28 +3,29 @@
 // Method: "RouteRelay: Event-Triggered Cross-Layer Route Reuse for Efficient
 // Dynamic Sparse Attention" (arXiv 2609.07306), cited as RouteRelay §x.
 //
-// Full routing of a row (§2.1 Eq. 1-2, §3.1 items 1-2) takes three steps:
+// Full routing of a row (§2.1 Eq. 1-2, §3.1 items 1-2) takes two kernels:
 //
 //   route_select_kernel  (one CTA = one head x 128 query rows, the machinery
 //       of rr_tc.cuh with the query tile in TMEM as the MMA's A operand and
-//       three accumulators) scores the row block against the head's key
-//       tiles twice:
+//       two accumulators) scores the row block against the head's key tiles
+//       twice:
 //         pass 0  per row, the largest score of each of 128 column groups
 //                 (group = column mod 128); T = the (k+m)-th largest of these
 //                 maxima, found by a bit search on their 16-bit order keys
 //                 (floor), is at most the row's (k+m)-th best score since
 //                 that many distinct valid scores reach it;
 //         pass 1  every valid score >= T is kept: the thread owning (row,
-//                 quarter of the columns) appends it to its own slots in
-//                 shared memory and records the kept columns of each tile in
-//                 a 32-bit mask (device memory, one coalesced store per tile).
-//       The kept scores are then copied to the row's record in device memory.
-//   route_finish_kernel  (one CTA per row block, one warp per row) rebuilds
-//       the (score, chunk) pairs from the masks, orders them (score desc,
+//                 quarter of the columns) stores it in its slots in shared
+//                 memory (two quarters share a region, one filling it from
+//                 the bottom, the other from the top) and records the kept
+//                 columns of each tile in a 32-bit mask held in TMEM.
+//       Each thread then turns its kept scores into (score, chunk) sort keys
+//       and the row's keys go to its record in device memory.
+//   route_finish_kernel  (one warp per row) orders the keys (score desc,
 //       chunk asc) by a counting sort over 64 bins with exact ranking inside
 //       a bin, writes route | near-miss and alpha (the k-th score), draws the
 //       random sentinels and adds the global ones.  Rows whose kept scores
-//       overflow the slots go to the exact one-pass heap kernel
+//       overflow their slots go to the exact one-pass heap kernel
 //       (rr_route_tc.cu).
 //
 // The relay layer (§3.2 Eq. 5-8, §4.1-4.2) runs the same two kernels over
@@ -50,12 +51,17 @@ namespace tc {
 
 constexpr int kSelEpiWarps = 16;
 constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
-constexpr int kSelAcc = 3;                       // accumulators (TMEM columns 0..383)
-constexpr uint32_t kQCol = kSelAcc * 128;        // TMEM column of the query tile (A operand)
-constexpr int kQCap = 46;                        // kept-score slots per (row, quarter)
+constexpr int kSelAcc = 2;                       // accumulators (TMEM columns 0..255)
+constexpr uint32_t kQCol = kSelAcc * 128;        // query tile (A operand): 64 columns at most
+constexpr uint32_t kMaskCol = kQCol + 64;        // kept-column masks: [quarter][tile], 128 columns
+constexpr int kMaskTiles = 32;                   // blocks with more key tiles keep masks in device memory
+constexpr int kPairCap = 92;                     // kept-score slots shared by two quarters of a row
 constexpr int kValStride = kRows + 1;            // padded (slot, row) grid of the kept scores
-constexpr int kRowCap = 128;                     // kept scores per row the finishing handles
+constexpr int kRowCap = 160;                     // kept scores per row (the record; 5 per lane)
+constexpr int kKeysPerLane = kRowCap / 32;
 constexpr int kTopWords = 65;                    // u32 words per row of 16-bit group maxima
+constexpr int kMaskBytes = kMaskTiles * kSelEpiWarps * 32 * 4;   // masks in the key ring after pass 1
+constexpr int kChunkStride = kRows + 2;          // u16 (slot, row) grid of the kept scores' chunks
 constexpr int kHalf = 16;                        // columns per capacity check in pass 1
 
 struct SelLayout {
@@ -64,14 +70,15 @@ struct SelLayout {
     __host__ __device__ CtaLayout cta() const { return CtaLayout{0u, k, rows, bars, misc, stages}; }
 };
 
-// k (key ring, 128 KB) | vals [4][kQCap][kValStride] f32 (the group maxima
-// [kRows][kTopWords] u32 after pass 0) | rows | thr | cnt | barriers | misc
+// k (key ring, 128 KB; after pass 1 the masks [tile][epilogue thread] u32
+// and the chunk grid [2][kPairCap][kChunkStride] u16) | vals [2][kPairCap][kValStride] f32 (before pass 1 the group maxima
+// [kRows][kTopWords] u32) | rows | thr | cnt | barriers | misc
 __host__ __device__ inline SelLayout sel_layout(int d) {
     SelLayout s;
     s.stages = d == 64 ? 8 : 4;
     uint32_t o = 0;
     s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
-    s.vals = o; o = up(o + 4 * kQCap * kValStride * 4, 16);
+    s.vals = o; o = up(o + 2 * kPairCap * kValStride * 4, 16);
     s.rows = o; o = up(o + kRows * 4, 16);
     s.thr = o;  o = up(o + kRows * 4, 16);
     s.cnt = o;  o = up(o + kRows * 4, 16);
@@ -80,6 +87,8 @@ __host__ __device__ inline SelLayout sel_layout(int d) {
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
 }
+static_assert(kKeys * 128 * 2 * 4 >= kMaskBytes + 2 * kPairCap * kChunkStride * 2,
+              "the key ring holds the masks and the chunk grid");
 
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t *r) {
     asm volatile(
@@ -95,30 +104,72 @@ __device__ __forceinline__ void tc_st8(uint32_t taddr, const uint32_t *r) {
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
         : "memory");
 }
+__device__ __forceinline__ void tc_st1(uint32_t taddr, uint32_t v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// MMA issuer of the selection kernel: A (the query tile) from TMEM.
+// Pass 1's step for column J of a thread's 32: if v >= T, store v at the
+// shared address `addr`, advance `addr` by `step` bytes and set bit J of
+// `mask` (one comparison and three predicated instructions).
+template <int J>
+__device__ __forceinline__ void keep_if(float v, float T, uint32_t &addr, int32_t step, uint32_t &mask) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ge.f32 p, %2, %3;\n\t"
+        "@p st.shared.f32 [%0], %2;\n\t"
+        "@p add.s32 %0, %0, %4;\n\t"
+        "@p or.b32 %1, %1, %5;\n\t}"
+        : "+r"(addr), "+r"(mask)
+        : "f"(v), "f"(T), "r"(step), "n"(1u << J)
+        : "memory");
+}
+template <int J0, int N>
+__device__ __forceinline__ void keep_run(const float *v, float T, uint32_t &addr, int32_t step, uint32_t &mask) {
+    if constexpr (N > 0) {
+        keep_if<J0>(v[J0], T, addr, step, mask);
+        keep_run<J0 + 1, N - 1>(v, T, addr, step, mask);
+    }
+}
+
+// Larger key = better: score desc, then chunk asc (-0 counts as +0).
+__device__ __forceinline__ uint64_t sel_key(float v, int j) {
+    const float z = v == 0.0f ? 0.0f : v;
+    return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
+}
+__device__ __forceinline__ int sel_key_chunk(uint64_t key) { return (int)(0xffffu - (uint32_t)(key & 0xffffu)); }
+__device__ __forceinline__ float sel_key_score(uint64_t key) { return unord32((uint32_t)(key >> 32)); }
+
+// MMA issuer of the selection kernel (the whole warp; one elected lane
+// issues): A (the query tile) from TMEM.
+template <int kSteps>
+__device__ __forceinline__ void sel_mma_tile(uint32_t d_tmem, uint32_t a_tmem, uint64_t kdesc) {
+#pragma unroll
+    for (int kk = 0; kk < kSteps; ++kk) {
+        const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
+        tc_mma_bf16_ts_elect(d_tmem, a_tmem + (uint32_t)(kk * 8), kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
+    }
+}
+
 __device__ __forceinline__ void sel_mma_issuer(Cta &c, int d) {
     const int total = 2 * c.ntiles;
     const uint32_t k_addr = saddr(c.k_s);
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
-    const uint32_t a_tmem = c.tmem_base + kQCol;
-    const int steps = d >> 4;
+    const uint32_t tmem = __shfl_sync(kFull, c.tmem_base, 0);
+    const uint32_t a_tmem = tmem + kQCol;
     for (int g = 0; g < total; ++g) {
         const int s = g % c.stages, a = g % kSelAcc;
-        if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
-        if (!mbar_wait(&c.acc_empty[a], ((g / kSelAcc) & 1) ^ 1, c.abort_flag)) break;
+        if (!mbar_wait_warp(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
+        if (!mbar_wait_warp(&c.acc_empty[a], ((g / kSelAcc) & 1) ^ 1, c.abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
+        const uint32_t d_tmem = tmem + (uint32_t)(a * kKeys);
         const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
-        for (int kk = 0; kk < steps; ++kk) {
-            const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
-            tc_mma_bf16_ts(d_tmem, a_tmem + (uint32_t)(kk * 8), kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&c.empty[s]);
-        tc_commit(&c.acc_full[a]);
+        if (d == 128) sel_mma_tile<8>(d_tmem, a_tmem, kdesc);
+        else sel_mma_tile<4>(d_tmem, a_tmem, kdesc);
+        tc_commit_elect(&c.empty[s]);
+        tc_commit_elect(&c.acc_full[a]);
     }
-    tc_commit(c.mma_done);
+    tc_commit_elect(c.mma_done);
     const long long t0 = clock64();
     while (!mbar_test(c.mma_done, 0) && clock64() - t0 < kSpinLimit) {
     }
@@ -129,8 +180,7 @@ __global__ void __launch_bounds__(kSelThreads, 1)
 route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                     const __grid_constant__ CUtensorMap tmap_k, int use_list) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
-    unsigned char *smem = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+    unsigned char *smem = align_smem_1024(smem_dyn);
     const int d = L.d, ksel = L.ksel;
     const SelLayout lay = sel_layout(d);
     Cta c;
@@ -139,43 +189,48 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int h = blockIdx.y;
 
-    // the query tile into TMEM columns kQCol.. (row r in lane r, two bf16 per
-    // column): epilogue warp (sub-partition sub, quarter qt) writes a quarter
-    // of the row's elements for its 32 rows
-    if (warp >= 2) {
-        const int ew = warp - 2, sub = warp & 3, qt = ew >> 2;
-        const int r = sub * 32 + lane;
-        const int row = c.rows_s[r];
-        const uint32_t taddr = c.tmem_base + ((uint32_t)(sub * 32) << 16) + kQCol + (uint32_t)(qt * (d >> 3));
-        uint32_t w[16];
-        const uint4 *src = reinterpret_cast<const uint4 *>(Q + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d +
-                                                           qt * (d >> 2));
-        if (d == 128) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-            }
-            tc_st16(taddr, w);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
-            }
-            tc_st8(taddr, w);
-        }
-        tc_wait_st();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-
+    // The producer starts at once; the MMA warp waits until the epilogue
+    // warps have put the query tile into TMEM (barrier q_ready).
     if (warp == 0) {
-        if (lane == 0) producer(c, &tmap_k, d, h, 2);
+        producer(c, &tmap_k, d, h, 2);
     } else if (warp == 1) {
-        if (lane == 0) sel_mma_issuer(c, d);
+        if (mbar_wait_warp(c.q_ready, 0, c.abort_flag)) {
+            tc_fence_after();
+            sel_mma_issuer(c, d);
+        }
     } else {
+        // the query tile into TMEM columns kQCol.. (row r in lane r, two
+        // bf16 per column): epilogue warp (sub-partition sub, quarter qt)
+        // writes a quarter of the row's elements for its 32 rows
+        {
+            const int ew = warp - 2, sub = warp & 3, qt = ew >> 2;
+            const int r = sub * 32 + lane;
+            const int row = c.rows_s[r];
+            const uint32_t taddr =
+                c.tmem_base + ((uint32_t)(sub * 32) << 16) + kQCol + (uint32_t)(qt * (d >> 3));
+            uint32_t w[16];
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                Q + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d + qt * (d >> 2));
+            if (d == 128) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                }
+                tc_st16(taddr, w);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                }
+                tc_st8(taddr, w);
+            }
+            tc_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(c.q_ready);
+        }
         // Four warps per TMEM sub-partition: quarter qt reads columns
         // 32*qt..32*qt+31 of every tile.  The epilogue threads meet at named
         // barrier 1 between phases (every one of them reaches every barrier,
@@ -220,28 +275,34 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 
         // threshold of each row (kRows / kSelEpiWarps rows per warp): the
         // largest 16-bit key K that at least k + m of the row's 128 maxima
-        // reach; T = the float of key K << 16.  The search starts below the
-        // bits the largest and smallest maxima share.  Rows with at most
+        // reach; T = the float of key K << 16.  Each lane holds 4 maxima; with
+        // j = ceil((k + m) / 32), the answer lies between the smallest and the
+        // largest of the lanes' j-th largest maxima (the lanes' top j values
+        // are 32 j >= k + m values above the first; above the second each
+        // lane has fewer than j, so fewer than k + m in all), and the bit
+        // search starts below the bits those two share.  Rows with at most
         // k + m valid keys keep all of them (T = -inf).
         float *thr_s = reinterpret_cast<float *>(smem + lay.thr);
         {
             constexpr int kRowsPerWarp = kRows / kSelEpiWarps;
             const uint16_t *tops16 = reinterpret_cast<const uint16_t *>(tops);
+            const int jsel = (ksel + 31) >> 5;   // 1..2 (k + m <= 64)
             uint32_t key[kRowsPerWarp][4], K[kRowsPerWarp];
             int hb[kRowsPerWarp];
             int hbmax = -1;
 #pragma unroll
             for (int k2 = 0; k2 < kRowsPerWarp; ++k2) {
                 const int rr = ew * kRowsPerWarp + k2;
-                uint32_t kmx = 0u, kmn = 0xFFFFu;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    key[k2][i] = tops16[rr * (2 * kTopWords) + i * 32 + lane];
-                    kmx = max(kmx, key[k2][i]);
-                    kmn = min(kmn, key[k2][i]);
-                }
-                kmx = __reduce_max_sync(kFull, kmx);
-                kmn = __reduce_min_sync(kFull, kmn);
+                for (int i = 0; i < 4; ++i) key[k2][i] = tops16[rr * (2 * kTopWords) + i * 32 + lane];
+                // the lane's largest and second largest of its four keys
+                const uint32_t a0 = max(key[k2][0], key[k2][1]), b0 = min(key[k2][0], key[k2][1]);
+                const uint32_t a1 = max(key[k2][2], key[k2][3]), b1 = min(key[k2][2], key[k2][3]);
+                const uint32_t top1 = max(a0, a1);
+                const uint32_t top2 = max(min(a0, a1), max(b0, b1));
+                const uint32_t u = jsel == 1 ? top1 : top2;
+                const uint32_t kmx = __reduce_max_sync(kFull, u);
+                const uint32_t kmn = __reduce_min_sync(kFull, u);
                 const uint32_t x = kmx ^ kmn;
                 hb[k2] = x ? 31 - __clz(x) : -1;
                 K[k2] = hb[k2] >= 0 ? (kmx & ~((2u << hb[k2]) - 1u)) : kmx;
@@ -271,13 +332,23 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const float T = thr_s[r];
 
         // pass 1: keep every valid score >= T (tiles backwards: the first
-        // ones were loaded last).  This thread's slots are column r of rows
-        // qt*kQCap.. of the vals grid; a 16-column half takes the unchecked
-        // path while 16 more slots are free.
+        // ones were loaded last).  Quarters 2p and 2p+1 of row r share the
+        // slots p*kPairCap.. of column r of the vals grid: the even quarter
+        // fills them upwards, the odd one downwards, so they collide only
+        // when together they keep more than kPairCap scores (the row is then
+        // redone).  A 16-column half takes the unchecked path while 16 more
+        // slots of this thread's own count are free.  The tile's kept columns
+        // go to TMEM column kMaskCol + 32*qt + t (device memory for blocks of
+        // more than kMaskTiles tiles).
+        const int pair = qt >> 1;
+        const bool down = (qt & 1) != 0;
         float *vals = reinterpret_cast<float *>(smem + lay.vals);
-        float *pv = vals + qt * kQCap * kValStride + r;
+        float *pv = vals + (pair * kPairCap + (down ? kPairCap - 1 : 0)) * kValStride + r;
+        const int step = down ? -kValStride : kValStride;
         int cur = 0;
         const size_t blk = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+        const bool masks_in_tmem = nt <= kMaskTiles;
+        const uint32_t mask_tmem = c.tmem_base + ((uint32_t)(sub * 32) << 16) + kMaskCol + (uint32_t)(qt * 32);
         uint32_t *gmask = L.cand_masks + (blk * (size_t)L.mt * 4 + qt) * kRows + r;
         for (int i = 0; i < nt && ok; ++i) {
             const int g = nt + i;
@@ -290,25 +361,22 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             uint32_t mask = 0u;
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-                if (lim >= 32 && cur <= kQCap - kHalf) {
+                if (lim >= 32 && cur <= kPairCap - kHalf) {
                     uint32_t mh = 0u;
-#pragma unroll
-                    for (int jj = hf * kHalf; jj < (hf + 1) * kHalf; ++jj) {
-                        if (v[jj] >= T) {
-                            *pv = v[jj];
-                            pv += kValStride;
-                            mh |= 1u << jj;
-                        }
-                    }
-                    cur += __popc(mh);
+                    uint32_t addr = saddr(pv);
+                    if (hf == 0) keep_run<0, kHalf>(v, T, addr, step * 4, mh);
+                    else keep_run<kHalf, kHalf>(v, T, addr, step * 4, mh);
+                    const int n = __popc(mh);
+                    pv += n * step;
+                    cur += n;
                     mask |= mh;
                 } else {
 #pragma unroll
                     for (int jj = hf * kHalf; jj < (hf + 1) * kHalf; ++jj) {
                         if (jj < lim && v[jj] >= T) {
-                            if (cur < kQCap) {
+                            if (cur < kPairCap) {
                                 *pv = v[jj];
-                                pv += kValStride;
+                                pv += step;
                                 mask |= 1u << jj;
                             }
                             ++cur;
@@ -316,44 +384,104 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                     }
                 }
             }
-            gmask[(size_t)t * 4 * kRows] = mask;
+            if (masks_in_tmem) tc_st1(mask_tmem + (uint32_t)t, mask);
+            else gmask[(size_t)t * 4 * kRows] = mask;
         }
+        tc_wait_st();
         // kept count per quarter, one byte each (0xFF: the row is redone)
-        reinterpret_cast<uint8_t *>(smem + lay.cnt)[r * 4 + qt] = (uint8_t)(cur <= kQCap ? cur : 0xFF);
-        epi_sync();
+        reinterpret_cast<uint8_t *>(smem + lay.cnt)[r * 4 + qt] = (uint8_t)(cur <= kPairCap ? cur : 0xFF);
+        epi_sync();   // every count is written and every MMA (the key ring's last reader) is done
 
-        // hand-off: each row's kept scores to its record, quarter after
-        // quarter (one warp per row), with the counts and the threshold
+        // sort keys.  First each thread pairs its kept scores, in the order
+        // they were stored (tiles descending, columns ascending), with their
+        // chunks by walking its masks, and writes the chunks beside the
+        // scores (chunk grid [2][kPairCap][kChunkStride] u16 in the idle key
+        // ring, after the masks [tile][epilogue thread]).  Then one warp per
+        // row turns (score, chunk) into sort keys, quarters in order, and
+        // stores them to the row's record.
         const bool cta_ok = *c.abort_flag == 0;
         const uint32_t *cnt_s = reinterpret_cast<const uint32_t *>(smem + lay.cnt);
+        uint32_t *masks_s = reinterpret_cast<uint32_t *>(smem + lay.k);
+        uint16_t *chunks_s = reinterpret_cast<uint16_t *>(smem + lay.k + kMaskBytes);
+        const int et = ew * 32 + lane;   // epilogue thread 0..511
+        auto row_total = [&](int rr, int *cq) {
+            const uint32_t cw = cnt_s[rr];
+            int tot = 0;
+            bool bad = !cta_ok;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                cq[q] = (int)((cw >> (8 * q)) & 0xFFu);
+                bad |= cq[q] > kPairCap;
+                tot += cq[q];
+            }
+            bad |= cq[0] + cq[1] > kPairCap || cq[2] + cq[3] > kPairCap || tot > kRowCap;
+            return bad ? -1 : tot;
+        };
+        if (masks_in_tmem) {
+            uint32_t mk[32];
+            tc_ld32(mask_tmem, reinterpret_cast<float *>(mk));   // every lane of the warp
+#pragma unroll
+            for (int t = 0; t < kMaskTiles; ++t)
+                if (t < nt) masks_s[t * (kSelEpiWarps * 32) + et] = mk[t];
+        }
+        {
+            int cq[4];
+            const int total = row_total(r, cq);
+            const int own = (qt == 0 ? cq[0] : qt == 1 ? cq[1] : qt == 2 ? cq[2] : cq[3]);
+            if (row >= 0 && total >= 0 && own > 0) {
+                auto mask_of = [&](int t) -> uint32_t {
+                    return masks_in_tmem ? masks_s[t * (kSelEpiWarps * 32) + et] : gmask[(size_t)t * 4 * kRows];
+                };
+                uint16_t *cdst = chunks_s + (pair * kPairCap) * kChunkStride + r;
+                int t = nt - 1;
+                uint32_t m = mask_of(t);
+                for (int kk = 0; kk < own; ++kk) {
+                    while (m == 0u && t > 0) m = mask_of(--t);
+                    const int b = __ffs(m) - 1;
+                    m &= m - 1u;
+                    cdst[(down ? kPairCap - 1 - kk : kk) * kChunkStride] = (uint16_t)(t * kKeys + qt * 32 + b);
+                }
+            }
+        }
+        epi_sync();
+
+        // hand-off: each row's keys to its record (one warp per row), with
+        // the count and the threshold
         for (int k2 = 0; k2 < kRows / kSelEpiWarps; ++k2) {
             const int rr = ew * (kRows / kSelEpiWarps) + k2;
             if (c.rows_s[rr] < 0) continue;   // warp-uniform
-            const uint32_t cw = cta_ok ? cnt_s[rr] : 0xFFFFFFFFu;
+            int cq[4];
+            const int total = row_total(rr, cq);
             const size_t slot = blk * kRows + rr;
-            float *rec = L.cand_vals + slot * 4 * kQCap;
+            uint64_t *rec = L.cand_keys + slot * kRowCap;
+            const int c01 = cq[0] + cq[1], c012 = c01 + cq[2];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int n = (int)((cw >> (8 * q)) & 0xFFu);
-                if (n > kQCap) continue;
-                for (int e = lane; e < n; e += 32) rec[q * kQCap + e] = vals[(q * kQCap + e) * kValStride + rr];
+            for (int i = 0; i < kKeysPerLane; ++i) {
+                // key e: quarter q, its kk-th score (quarter pair region, upwards
+                // for even quarters, downwards for odd ones)
+                const int e = lane + 32 * i;
+                if (e < total) {
+                    const int q = e < cq[0] ? 0 : e < c01 ? 1 : e < c012 ? 2 : 3;
+                    const int kk = e - (q == 0 ? 0 : q == 1 ? cq[0] : q == 2 ? c01 : c012);
+                    const int s = (q >> 1) * kPairCap + ((q & 1) ? kPairCap - 1 - kk : kk);
+                    rec[e] = sel_key(vals[s * kValStride + rr], (int)chunks_s[s * kChunkStride + rr]);
+                }
             }
-            if (lane == 0) L.cand_meta[slot] = make_uint2(cw, __float_as_uint(thr_s[rr]));
+            if (lane == 0) L.cand_meta[slot] = make_uint2(total >= 0 ? (uint32_t)total : 0xFFFFFFFFu,
+                                                          __float_as_uint(thr_s[rr]));
         }
     }
     cta_teardown(c, L);
 }
 
 // ---- row finishing ---------------------------------------------------------------
-constexpr int kFinWarps = 16;
+constexpr int kFinWarps = 8;
 constexpr int kFinThreads = 32 * kFinWarps;
-constexpr int kMaskTilesSmem = 32;     // blocks with at most this many key tiles stage their masks
-constexpr int kMaskStride = kRows + 1;
 constexpr int kBins = 64;
 constexpr int kBitsWords = 128;        // membership bitmaps: rows with <= 4096 valid keys
 
 struct FinScratch {
-    uint64_t keys[kRowCap];            // kept (score, chunk) keys, then in bin order
+    uint64_t keys[kRowCap];            // kept keys in bin order
     uint32_t hist[kBins];              // bin counts, then bin starts
     uint32_t bits[kBitsWords];         // selected and accepted chunks
     uint32_t rbits[kBitsWords];        // relay: chunks of the old route
@@ -361,83 +489,54 @@ struct FinScratch {
     int32_t acc[32];                   // accepted random sentinels, in order
 };
 
-__host__ __device__ inline size_t fin_smem_bytes() {
-    return (size_t)kMaskTilesSmem * 4 * kMaskStride * 4 + (size_t)kFinWarps * sizeof(FinScratch);
-}
-
-// Larger key = better: score desc, then chunk asc (-0 counts as +0).
-__device__ __forceinline__ uint64_t sel_key(float v, int j) {
-    const float z = v == 0.0f ? 0.0f : v;
-    return ((uint64_t)ord32(z) << 32) | (uint32_t)(0xffffu - (uint32_t)j);
-}
-__device__ __forceinline__ int sel_key_chunk(uint64_t key) { return (int)(0xffffu - (uint32_t)(key & 0xffffu)); }
-__device__ __forceinline__ float sel_key_score(uint64_t key) { return unord32((uint32_t)(key >> 32)); }
-
 struct FinCounts {
     unsigned long long rows = 0, pairs = 0, full = 0;
 };
 
-// One warp finishes one row.  Returns with nothing written when the row is
-// handed on: kept scores overflowed (anchor: retry list; relay: exact
-// rescoring), or (relay) the test keeps the old route or needs exact scores.
-template <bool kRelay, typename MaskAt>
-__device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h, int row, size_t slot,
-                                           MaskAt mask_at, FinScratch &w, int lane, FinCounts &cnt) {
+// What a warp reads from device memory for one row, loaded one row ahead
+// so that the loads of row i+1 are in flight while row i is finished.
+struct RowIn {
+    int row;
+    size_t slot;
+    uint2 meta;
+    uint64_t key[kKeysPerLane];   // the record's first kRowCap slots (those past the count unused)
+    int32_t id[3];                // relay: the old ledger row, ids lane, lane + 32, lane + 64 (c <= 96)
+};
+
+template <bool kRelay>
+__device__ __forceinline__ void load_row(const LedgerDev &L, int h, int row, size_t slot, int lane, RowIn &in) {
+    in.row = row;
+    in.slot = slot;
+    in.meta = L.cand_meta[slot];
+    const uint64_t *rec = L.cand_keys + slot * kRowCap;
+    const int total = (int)in.meta.x;   // -1 (all ones): the row is redone, nothing to read
+#pragma unroll
+    for (int i = 0; i < kKeysPerLane; ++i) in.key[i] = lane + 32 * i < total ? rec[lane + 32 * i] : 0ull;
+    if (kRelay) {
+        const int32_t *idr = L.ids + ((size_t)h * L.nq + row) * L.c;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const int e = lane + 32 * i;
+            in.id[i] = e < L.c ? idr[e] : -1;
+        }
+    }
+}
+
+// One warp finishes one row from its sort keys.  Returns with nothing
+// written when the row is handed on: its kept scores overflowed (anchor:
+// retry list; relay: exact rescoring), or (relay) the test keeps the old
+// route or needs exact scores.
+template <bool kRelay>
+__device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h, const RowIn &in,
+                                           FinScratch &w, int lane, FinCounts &cnt) {
+    const int row = in.row;
     const int n_valid = valid_keys(row, L.nk, L.causal);
     const size_t grow = (size_t)h * L.nq + row;
     const uint32_t lt_mask = (1u << lane) - 1u;
-    const uint2 meta = L.cand_meta[slot];
+    const uint2 meta = in.meta;
     const float T = __uint_as_float(meta.y);
-    int c4[4];
-    bool redo = false;
-    int total = 0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        c4[q] = (int)((meta.x >> (8 * q)) & 0xFFu);
-        redo |= c4[q] > kQCap;
-        total += c4[q];
-    }
-    redo |= total > kRowCap || total < min(L.ksel, n_valid);
-
-    // the kept (score, chunk) pairs: mask (quarter q, tile t) holds the kept
-    // columns of that tile; a quarter's scores are stored tile by tile from
-    // the last tile down, columns ascending inside a tile
-    const int ntr = (n_valid + kKeys - 1) / kKeys;
-    const int nidx = 4 * ntr;
-    const float *rec = L.cand_vals + slot * 4 * kQCap;
-    int carry = 0;
-    if (!redo) {
-        for (int base = 0; base < nidx; base += 32) {
-            const int idx = base + lane;
-            uint32_t mk = 0u;
-            int q = 0, t = 0;
-            if (idx < nidx) {
-                q = idx / ntr;
-                t = ntr - 1 - (idx - q * ntr);
-                mk = mask_at(t, q);
-            }
-            const int pc = __popc(mk);
-            int incl = pc;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int x = __shfl_up_sync(kFull, incl, o);
-                if (lane >= o) incl += x;
-            }
-            int e = carry + incl - pc;
-            const int qs = (q > 0 ? c4[0] : 0) + (q > 1 ? c4[1] : 0) + (q > 2 ? c4[2] : 0);
-            int off = e - qs;
-            while (mk != 0u) {
-                const int b = __ffs(mk) - 1;
-                mk &= mk - 1u;
-                if (e < kRowCap && off < kQCap) w.keys[e] = sel_key(rec[q * kQCap + off], t * kKeys + q * 32 + b);
-                ++e;
-                ++off;
-            }
-            carry += __shfl_sync(kFull, incl, 31);
-        }
-        redo = carry != total;   // masks and counts disagree: redo the row
-    }
-    if (redo) {
+    const int total = (int)meta.x;   // kept keys, or -1: redo the row
+    if (total < 0 || total > kRowCap || total < min(L.ksel, n_valid)) {
         if (lane == 0) {
             if (kRelay) {
                 L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
@@ -450,14 +549,29 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         }
         return;
     }
-    __syncwarp();
-    uint64_t key[4];
-    bool live[4];
+    uint64_t key[kKeysPerLane];
+    bool live[kKeysPerLane];
+    bool bad_key = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kKeysPerLane; ++i) {
         const int e = lane + 32 * i;
         live[i] = e < total;
-        key[i] = live[i] ? w.keys[e] : 0ull;
+        key[i] = live[i] ? in.key[i] : 0ull;
+        bad_key |= live[i] && sel_key_chunk(key[i]) >= n_valid;
+    }
+    if (__any_sync(kFull, bad_key)) {   // never expected: a record that does not match the row
+        if (lane == 0) {
+            atomicOr(&L.counters[2], 4ULL);
+            if (kRelay) {
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
+                L.flags[grow] = 0;
+            } else {
+                const int pos = atomicAdd(&L.retry_count[h], 1);
+                L.retry_list[(size_t)h * L.nq + pos] = row;
+                atomicAdd(&L.counters[10], 1ULL);
+            }
+        }
+        return;
     }
 
     if constexpr (kRelay) {
@@ -475,12 +589,12 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             w.sbits[q] = 0u;
         }
         __syncwarp();
-        const int32_t *idr = L.ids + grow * L.c;
         int rt = 0, st = 0;
         bool bad = false;
-        for (int e0 = 0; e0 < L.c; e0 += 32) {
-            const int e = e0 + lane;
-            const int j = e < L.c ? idr[e] : -1;
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const int e = lane + 32 * i;
+            const int j = in.id[i];
             const bool valid = j >= 0 && j < n_valid;
             bad |= j >= n_valid || j < -1;
             if (valid) atomicOr(&(e < L.k ? w.rbits : w.sbits)[j >> 5], 1u << (j & 31));
@@ -492,7 +606,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         float amin = INFINITY, bmax = -INFINITY;
         int rf = 0, sf = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < kKeysPerLane; ++i) {
             if (!live[i]) continue;
             const int j = sel_key_chunk(key[i]);
             const float v = sel_key_score(key[i]);
@@ -547,7 +661,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     // (larger key = lower bin), then each key's rank among the keys of its bin
     uint32_t hmx = 0u, hmn = 0xFFFFFFFFu;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kKeysPerLane; ++i) {
         if (!live[i]) continue;
         const uint32_t hi = (uint32_t)(key[i] >> 32);
         hmx = max(hmx, hi);
@@ -559,10 +673,10 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     w.hist[lane] = 0u;
     w.hist[lane + 32] = 0u;
     __syncwarp();
-    int bin[4];
-    uint32_t in_bin[4];
+    int bin[kKeysPerLane];
+    uint32_t in_bin[kKeysPerLane];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kKeysPerLane; ++i) {
         bin[i] = min(kBins - 1, (int)((float)(hmx - (uint32_t)(key[i] >> 32)) * scale));
         in_bin[i] = live[i] ? atomicAdd(&w.hist[bin[i]], 1u) : 0u;
     }
@@ -581,9 +695,9 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         w.hist[2 * lane + 1] = excl + h0;
     }
     __syncwarp();
-    int start[4];
+    int start[kKeysPerLane];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kKeysPerLane; ++i) {
         start[i] = (int)w.hist[bin[i]];
         if (live[i]) w.keys[start[i] + (int)in_bin[i]] = key[i];
     }
@@ -592,10 +706,10 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     const int nm = min(L.m, n_valid - nr);
     const int nsel = nr + nm;
     int32_t *out = L.ids + grow * L.c;
-    bool sel[4];
-    int jc[4];
+    bool sel[kKeysPerLane];
+    int jc[kKeysPerLane];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < kKeysPerLane; ++i) {
         sel[i] = false;
         jc[i] = live[i] ? sel_key_chunk(key[i]) : -1;
         if (!live[i]) continue;
@@ -624,7 +738,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         for (int q = lane; q < words; q += 32) w.bits[q] = 0u;
         __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < kKeysPerLane; ++i)
             if (sel[i]) atomicOr(&w.bits[jc[i] >> 5], 1u << (jc[i] & 31));
         __syncwarp();
     }
@@ -634,7 +748,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         bool hit = false;
         for (int src = 0; src < 32; ++src) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < kKeysPerLane; ++i) {
                 const int cj = __shfl_sync(kFull, sel[i] ? jc[i] : -1, src);
                 hit |= cj == j;
             }
@@ -702,56 +816,31 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
 }
 
 template <bool kRelay>
-__global__ void __launch_bounds__(kFinThreads)
+__global__ void __launch_bounds__(kFinThreads, 3)
 route_finish_kernel(LedgerDev L, int layer, int use_list) {
-    extern __shared__ __align__(16) unsigned char fsm[];
-    __shared__ int red_row[kFinWarps];
+    __shared__ FinScratch scr[kFinWarps];
     __shared__ unsigned long long red_cnt[kFinWarps][3];
-    uint32_t *masks_s = reinterpret_cast<uint32_t *>(fsm);
-    FinScratch *scr = reinterpret_cast<FinScratch *>(fsm + (size_t)kMaskTilesSmem * 4 * kMaskStride * 4);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
     const int count = use_list ? L.head_count[h] : L.nq;
     const int row0 = blockIdx.x * kRows;
     if (row0 >= count) return;
     const int n_rows = min(kRows, count - row0);
-    // the block's key tiles, as the selection kernel counted them
-    int myrow = -1;
-    if (tid < n_rows) myrow = use_list ? L.list[(size_t)h * L.nq + row0 + tid] : row0 + tid;
-    const int wmax = __reduce_max_sync(kFull, myrow);
-    if (lane == 0) red_row[warp] = wmax;
-    __syncthreads();
-    int max_row = -1;
-    for (int i = 0; i < kFinWarps; ++i) max_row = max(max_row, red_row[i]);
-    const int kend = L.causal ? min(L.nk, max_row + 1) : L.nk;
-    const int nt = (kend + kKeys - 1) / kKeys;
     const size_t blk = (size_t)h * gridDim.x + blockIdx.x;
-    const uint32_t *gmask = L.cand_masks + blk * (size_t)L.mt * 4 * kRows;
-    const bool staged = nt <= kMaskTilesSmem;
-    if (staged) {
-        for (int e = tid; e < nt * 4 * kRows; e += blockDim.x) {
-            const int tq = e / kRows, r = e - tq * kRows;
-            masks_s[tq * kMaskStride + r] = gmask[e];
-        }
-    }
-    __syncthreads();
-
     FinCounts cnt;
-    for (int k2 = 0; k2 < kRows / kFinWarps; ++k2) {
-        const int rr = warp * (kRows / kFinWarps) + k2;
+    constexpr int kPerWarp = kRows / kFinWarps;
+    const int rr0 = warp * kPerWarp;
+    auto row_at = [&](int rr) { return use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr; };
+    RowIn cur, nxt;
+    if (rr0 < n_rows) load_row<kRelay>(L, h, row_at(rr0), blk * kRows + rr0, lane, cur);
+    for (int k2 = 0; k2 < kPerWarp; ++k2) {
+        const int rr = rr0 + k2;
         if (rr >= n_rows) break;   // warp-uniform
-        const int row = use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr;
-        const size_t slot = blk * kRows + rr;
-        if (staged) {
-            finish_one<kRelay>(
-                L, layer, h, row, slot, [&](int t, int q) { return masks_s[(t * 4 + q) * kMaskStride + rr]; },
-                scr[warp], lane, cnt);
-        } else {
-            finish_one<kRelay>(
-                L, layer, h, row, slot, [&](int t, int q) { return gmask[((size_t)t * 4 + q) * kRows + rr]; },
-                scr[warp], lane, cnt);
-        }
+        const bool more = k2 + 1 < kPerWarp && rr + 1 < n_rows;
+        if (more) load_row<kRelay>(L, h, row_at(rr + 1), blk * kRows + rr + 1, lane, nxt);
+        finish_one<kRelay>(L, layer, h, cur, scr[warp], lane, cnt);
         __syncwarp();
+        if (more) cur = nxt;
     }
     if (kRelay) {
         if (lane == 0) {
@@ -763,8 +852,8 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
         if (tid < 3) {
             unsigned long long s = 0;
             for (int i = 0; i < kFinWarps; ++i) s += red_cnt[i][tid];
-            const int slot_of[3] = {0, 1, 8};   // rows, pairs, full-routing pairs of the layer
-            if (s) atomicAdd(&L.counters[slot_of[tid]], s);
+            const int slot_of = tid == 0 ? 0 : tid == 1 ? 1 : 8;   // rows, pairs, full-routing pairs
+            if (s) atomicAdd(&L.counters[slot_of], s);
         }
     }
 }
@@ -868,8 +957,8 @@ CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype) {
     if (!route_rows_tc_supported(L, dtype)) return z;
     const size_t blocks = (size_t)L.bh * ((L.nq + tc::kRows - 1) / tc::kRows);
     const size_t mt = (size_t)((L.nk + tc::kKeys - 1) / tc::kKeys);
-    z.vals = blocks * tc::kRows * 4 * tc::kQCap * sizeof(float);
-    z.masks = blocks * mt * 4 * tc::kRows * sizeof(uint32_t);
+    z.keys = blocks * tc::kRows * tc::kRowCap * sizeof(uint64_t);
+    z.masks = mt > (size_t)tc::kMaskTiles ? blocks * mt * 4 * tc::kRows * sizeof(uint32_t) : 0;
     z.meta = blocks * tc::kRows * sizeof(uint2);
     z.und = (size_t)L.bh * L.nq * sizeof(int32_t);
     return z;
@@ -880,12 +969,6 @@ size_t route_select_smem_bytes(const LedgerDev &L) { return tc::sel_layout(L.d).
 cudaError_t route_select_prepare() {
     cudaError_t e = cudaFuncSetAttribute(tc::route_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)tc::sel_layout(128).total);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::route_finish_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc::fin_smem_bytes());
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(tc::route_finish_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)tc::fin_smem_bytes());
     return e;
 }
 
@@ -897,10 +980,9 @@ cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtenso
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (mode == SelectMode::kRelay)
-        tc::route_finish_kernel<true><<<grid, tc::kFinThreads, tc::fin_smem_bytes(), s>>>(L, layer, 0);
+        tc::route_finish_kernel<true><<<grid, tc::kFinThreads, 0, s>>>(L, layer, 0);
     else
-        tc::route_finish_kernel<false><<<grid, tc::kFinThreads, tc::fin_smem_bytes(), s>>>(L, layer,
-                                                                                            use_list ? 1 : 0);
+        tc::route_finish_kernel<false><<<grid, tc::kFinThreads, 0, s>>>(L, layer, use_list ? 1 : 0);
     return cudaGetLastError();
 }
 

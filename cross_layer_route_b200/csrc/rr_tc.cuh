@@ -9,8 +9,8 @@
 //   warp 0     TMA producer: 128-key x d tiles of Kc (bf16, 128-byte
 //              swizzle) into a ring of shared-memory stages;
 //   warp 1     allocates 512 TMEM columns (four 128x128 fp32 accumulators);
-//              one lane issues tcgen05.mma (M=128, N=128, K=16 per op) for
-//              every key tile and commits twice: to the stage's "empty"
+//              one elected lane issues tcgen05.mma (M=128, N=128, K=16 per
+//              op) for every key tile and commits twice: to the stage's "empty"
 //              barrier (the producer may refill it) and to the
 //              accumulator's "full" barrier (the epilogue may read it);
 //   warps 2-   epilogue, reading score tiles with tcgen05.ld; a warp may
@@ -42,13 +42,19 @@ constexpr int kAcc = 4;                    // TMEM accumulators (128 columns eac
 constexpr int kTmemCols = kAcc * 128;
 constexpr int kSubTileBytes = 128 * 128;   // 128 rows x 64 bf16 (one 128-byte swizzle span)
 constexpr long long kSpinLimit = 1ll << 31;
-constexpr int kNumBars = 2 * kMaxStages + 2 * kAcc + 1;
+constexpr int kNumBars = 2 * kMaxStages + 2 * kAcc + 2;
 
 __host__ __device__ inline uint32_t up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 // ---- PTX wrappers (forms from the PTX ISA for sm_100a) -----------------------
 __device__ __forceinline__ uint32_t saddr(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+// The dynamic shared-memory base rounded up to 1024 bytes (128-byte swizzled
+// operands need it).  The offset is added to the shared array itself, so the
+// compiler keeps the shared address space of every pointer derived from it.
+__device__ __forceinline__ unsigned char *align_smem_1024(unsigned char *base) {
+    return base + ((1024u - (saddr(base) & 1023u)) & 1023u);
 }
 __device__ __forceinline__ void mbar_init(uint64_t *b, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(b)), "r"(count) : "memory");
@@ -107,6 +113,60 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, u
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(saddr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(saddr(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// ---- warp-uniform issue: the whole warp runs the loop, one elected lane
+// issues the instruction (operands stay in uniform registers; a loop run
+// by a single lane pays a register move per operand and issues tcgen05.mma
+// at about half the rate) -----------------------------------------------------
+__device__ __forceinline__ void mbar_expect_tx_elect(uint64_t *b, uint32_t bytes) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(saddr(b)), "r"(bytes)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_elect(void *dst, const CUtensorMap *map, uint64_t *bar, int c0,
+                                                  int c1, int c2) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(saddr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(saddr(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            saddr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                  uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void tc_mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                                     uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// A bounded wait whose outcome the whole warp shares.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *b, uint32_t parity, volatile int *abort_flag) {
+    return __all_sync(kFull, mbar_wait(b, parity, abort_flag));
 }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -189,7 +249,7 @@ struct CtaLayout {
 struct Cta {
     unsigned char *q_s, *k_s;
     int *rows_s;
-    uint64_t *full, *empty, *acc_full, *acc_empty, *mma_done;
+    uint64_t *full, *empty, *acc_full, *acc_empty, *mma_done, *q_ready;
     uint32_t *tmem_slot;
     volatile int *abort_flag;
     int stages, n_rows, ntiles;
@@ -218,6 +278,7 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Cta
     c.acc_full = bars + 2 * kMaxStages;
     c.acc_empty = bars + 2 * kMaxStages + kAcc;
     c.mma_done = bars + 2 * kMaxStages + 2 * kAcc;
+    c.q_ready = bars + 2 * kMaxStages + 2 * kAcc + 1;
     c.tmem_slot = reinterpret_cast<uint32_t *>(smem + lay.misc);
     c.abort_flag = reinterpret_cast<volatile int *>(smem + lay.misc + 4);
     c.n_rows = min(kRows, count - row0);
@@ -237,6 +298,7 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Cta
             mbar_init(&c.acc_empty[a], (blockDim.x >> 5) - 2);
         }
         mbar_init(c.mma_done, 1);
+        mbar_init(c.q_ready, (blockDim.x >> 5) - 2);   // kernels that load the query tile into TMEM
         *c.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -277,22 +339,23 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Cta
 // (its first tiles are the ones most recently loaded).
 __device__ __forceinline__ int tile_of(int g, int ntiles) { return g < ntiles ? g : 2 * ntiles - 1 - g; }
 
-// TMA producer (one lane): `passes` sweeps over the key tiles into the ring.
-// Stage s is refilled once the MMAs that read it have completed (its empty
-// barrier, committed by the MMA lane).
+// TMA producer (the whole warp; one elected lane issues): `passes` sweeps
+// over the key tiles into the ring.  Stage s is refilled once the MMAs that
+// read it have completed (its empty barrier, committed by the MMA warp).
 __device__ __forceinline__ void producer(Cta &c, const CUtensorMap *tmap_k, int d, int h, int passes) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap_k)) : "memory");
+    if ((threadIdx.x & 31) == 0)
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap_k)) : "memory");
     const int total = passes * c.ntiles;
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
     int issued = 0;
     for (int g = 0; g < total; ++g) {
         const int s = g % c.stages;
-        if (g >= c.stages && !mbar_wait(&c.empty[s], ((g / c.stages) & 1) ^ 1, c.abort_flag)) break;
-        mbar_expect_tx(&c.full[s], stage_bytes);
+        if (g >= c.stages && !mbar_wait_warp(&c.empty[s], ((g / c.stages) & 1) ^ 1, c.abort_flag)) break;
+        mbar_expect_tx_elect(&c.full[s], stage_bytes);
         const int t = tile_of(g, c.ntiles);
         for (int kb = 0; kb < (d >> 6); ++kb)
-            tma_load_3d(c.k_s + s * stage_bytes + kb * kSubTileBytes, tmap_k, &c.full[s], kb * 64,
-                        t * kKeys, h);
+            tma_load_3d_elect(c.k_s + s * stage_bytes + kb * kSubTileBytes, tmap_k, &c.full[s], kb * 64,
+                              t * kKeys, h);
         ++issued;
     }
     // drain: every issued stage must have landed before the CTA exits
@@ -313,28 +376,30 @@ __device__ __forceinline__ void mma_tile(uint32_t d_tmem, uint64_t qdesc, uint64
 #pragma unroll
     for (int kk = 0; kk < kSteps; ++kk) {
         const uint64_t off16 = (uint64_t)((kk >> 2) * (kSubTileBytes >> 4) + (kk & 3) * 2);
-        tc_mma_bf16(d_tmem, qdesc + off16, kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
+        tc_mma_bf16_elect(d_tmem, qdesc + off16, kdesc + off16, kIdesc, kk > 0 ? 1u : 0u);
     }
 }
 
+// MMA issuer (the whole warp; one elected lane issues).
 __device__ __forceinline__ void mma_issuer(Cta &c, int d, int passes) {
     const int total = passes * c.ntiles;
     const uint64_t qdesc = sw128_desc(saddr(c.q_s));
     const uint32_t k_addr = saddr(c.k_s);
     const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
+    const uint32_t tmem = __shfl_sync(kFull, c.tmem_base, 0);
     for (int g = 0; g < total; ++g) {
         const int s = g % c.stages, a = g % kAcc;
-        if (!mbar_wait(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
-        if (!mbar_wait(&c.acc_empty[a], ((g / kAcc) & 1) ^ 1, c.abort_flag)) break;
+        if (!mbar_wait_warp(&c.full[s], (g / c.stages) & 1, c.abort_flag)) break;
+        if (!mbar_wait_warp(&c.acc_empty[a], ((g / kAcc) & 1) ^ 1, c.abort_flag)) break;
         tc_fence_after();
-        const uint32_t d_tmem = c.tmem_base + (uint32_t)(a * kKeys);
+        const uint32_t d_tmem = tmem + (uint32_t)(a * kKeys);
         const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
         if (d == 128) mma_tile<8>(d_tmem, qdesc, kdesc);
         else mma_tile<4>(d_tmem, qdesc, kdesc);
-        tc_commit(&c.empty[s]);      // the producer may refill stage s
-        tc_commit(&c.acc_full[a]);   // the epilogue may read accumulator a
+        tc_commit_elect(&c.empty[s]);      // the producer may refill stage s
+        tc_commit_elect(&c.acc_full[a]);   // the epilogue may read accumulator a
     }
-    tc_commit(c.mma_done);
+    tc_commit_elect(c.mma_done);
     const long long t0 = clock64();
     while (!mbar_test(c.mma_done, 0) && clock64() - t0 < kSpinLimit) {
     }

@@ -26,8 +26,9 @@
  *  - Every call enqueues work on `stream` (a cudaStream_t; NULL is the
  *    legacy default stream) and returns without synchronising.  Argument
  *    and state errors are returned synchronously and enqueue nothing.
- *    Errors found on the device (an out-of-range ledger id) are recorded
- *    in the ledger's error word (counters[2]), read back by rr_ledger_read.
+ *    Errors found on the device (an out-of-range ledger id, a bounded wait
+ *    that timed out) are recorded in the ledger's error word (counters[2],
+ *    see RR_CNT_ERROR), read back by rr_ledger_read.
  *  - The device that was current at rr_ledger_create must be current at
  *    every later call on that ledger.
  *  - Inputs must be finite.  Ties between equal scores are broken by the
@@ -87,7 +88,10 @@ typedef struct rr_ledger rr_ledger;
 enum {
     RR_CNT_ROWS = 0,          /* rows fully routed at the last layer */
     RR_CNT_PAIRS = 1,         /* score pairs evaluated at the last layer */
-    RR_CNT_ERROR = 2,         /* error word: bit 0 = a ledger id was out of range at relay */
+    RR_CNT_ERROR = 2,         /* error word: bit 0 = a ledger id was out of range at relay;
+                                 bit 1 = a bounded wait inside a tensor-core kernel timed out
+                                 (that launch's rows were not scored: the layer's results are
+                                 not valid, rerun it) */
     RR_CNT_ROWS_TOTAL = 3,    /* rows fully routed since rr_ledger_create */
     RR_CNT_PAIRS_TOTAL = 4,   /* score pairs since rr_ledger_create */
     RR_CNT_LAYERS = 5,        /* layers processed since rr_ledger_create */
@@ -247,18 +251,21 @@ rr_status rr_ledger_set_hysteresis(rr_ledger *ledger, int32_t min_reuse);
  * the library: about 8 MiB of device memory that every GPU loading
  * librr.so holds until the process exits.  Limits: bh * nq <= 1048576 and
  * bh <= 4096; larger problems return RR_ECAPACITY and enqueue nothing.
- * The first call on a device looks up that array's device address (set-up
- * done once per device, with the device current); make that first call
- * before any stream capture.  Every call on a device shares the one array
+ * The first call on a device looks up that array's device address and sets
+ * the kernels' shared-memory attributes (set-up done once per device, with
+ * the device current); make that first call before any stream capture.  Every call on a device shares the one array
  * and it keeps the last call's contents; nothing in it has to start at zero
  * (each call writes every list length it reads).  Calls that can overlap
  * on the GPU (different streams, or different ledgers run concurrently)
  * race on it: run them on one stream or serialise them.  The call keeps no
  * host state, so it cannot check the layer order: the caller must start a
  * sequence at layer 0 or an anchor layer and pass increasing layers.
- * Errors: RR_EINVAL (bad config, null or misaligned pointer, layer < 0),
- * RR_ECAPACITY, RR_ECUDA.  Calls no cudaMalloc, cudaFree or allocating
- * library routine. */
+ * Device-side errors land in d_counters[RR_CNT_ERROR] like the ledger's
+ * (bit 0: an out-of-range ledger id; bit 1: a bounded wait timed out and the
+ * layer's results are not valid); the caller reads that slot after the
+ * stream reaches the call.  Errors: RR_EINVAL (bad config, null or
+ * misaligned pointer, layer < 0), RR_ECAPACITY, RR_ECUDA.  Calls no
+ * cudaMalloc, cudaFree or allocating library routine. */
 rr_status rr_route_layer_static(const rr_config *cfg, const void *d_qc, const void *d_kc,
                                 int32_t layer, int32_t *d_ids, float *d_alpha,
                                 int32_t *d_anchor_layer, uint8_t *d_flags, int64_t *d_counters,

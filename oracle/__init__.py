@@ -51,7 +51,7 @@ class _Params(ctypes.Structure):
                 ("causal", ctypes.c_int32), ("max_draws", ctypes.c_int32),
                 ("gamma", ctypes.c_double), ("seed", ctypes.c_uint64),
                 ("max_age", ctypes.c_int32), ("min_reuse", ctypes.c_int32),
-                ("g_sink", ctypes.c_int32), ("g_recent", ctypes.c_int32)]
+                ("g_sink", ctypes.c_int32), ("g_recent", ctypes.c_int32), ("gamma_h", ctypes.c_double)]
 
 
 def lib():
@@ -69,7 +69,7 @@ def lib():
             _lib.rro_philox4x32_10.argtypes = [P, P, P]
             _lib.rro_random_sentinels.argtypes = [ctypes.c_uint64, i32, i32, i32, i32, P, i32, i32, i32, P]
             _lib.rro_random_sentinels.restype = i32
-            _lib.rro_head_layer.argtypes = [ctypes.POINTER(_Params), i32, i32, i32, P, P, P, P, P, P, P, P, P]
+            _lib.rro_head_layer.argtypes = [ctypes.POINTER(_Params), i32, i32, i32, P, P, P, P, P, P, P, P, P, P]
             _lib.rro_head_layer.restype = i32
             _lib.rro_exact_topk.argtypes = [ctypes.POINTER(_Params), P, P, P]
     return _lib
@@ -97,6 +97,7 @@ class Params:
     min_reuse: int = 0            # hysteresis: layers a rebuilt row is reused without the test
     g_sink: int = 0               # mandatory global sentinels: sink chunks 0..g_sink-1
     g_recent: int = 0             # ... and the row's recent chunks i-g_recent+1..i
+    gamma_h: float = 0.0          # hysteresis: larger guard margin of a refreshed row (0: off)
 
     @property
     def c(self) -> int:
@@ -106,7 +107,7 @@ class Params:
         md = self.max_draws if self.max_draws is not None else 64 * self.c
         return _Params(self.nq, self.nk, self.d, self.k, self.m, self.r, int(bool(self.causal)), md,
                        float(self.gamma), int(self.seed) & 0xFFFFFFFFFFFFFFFF, int(self.max_age),
-                       int(self.min_reuse), int(self.g_sink), int(self.g_recent))
+                       int(self.min_reuse), int(self.g_sink), int(self.g_recent), float(self.gamma_h))
 
 
 def _f32(a) -> np.ndarray:
@@ -167,10 +168,16 @@ def exact_topk(p: Params, q, k) -> np.ndarray:
 @dataclass
 class HeadLedger:
     """Ledger of one head: ids [nq, c] (route | near-miss | random), alpha,
-    anchor layer (RouteRelay Eq. 4, §4.1)."""
+    anchor layer (RouteRelay Eq. 4, §4.1), and the per-row mark of the
+    elevated guard margin (1 = the row's next test uses gamma_h)."""
     ids: np.ndarray
     alpha: np.ndarray
     anchor_layer: np.ndarray
+    elevated: np.ndarray = None
+
+    def __post_init__(self):
+        if self.elevated is None:
+            self.elevated = np.zeros(self.ids.shape[0], dtype=np.uint8)
 
     @staticmethod
     def empty(p: Params) -> "HeadLedger":
@@ -179,7 +186,7 @@ class HeadLedger:
                           np.full(p.nq, -1, dtype=np.int32))
 
     def copy(self) -> "HeadLedger":
-        return HeadLedger(self.ids.copy(), self.alpha.copy(), self.anchor_layer.copy())
+        return HeadLedger(self.ids.copy(), self.alpha.copy(), self.anchor_layer.copy(), self.elevated.copy())
 
 
 def head_layer(p: Params, bh: int, layer: int, anchor: bool, q, k, led: HeadLedger, gamma_rows=None):
@@ -198,7 +205,8 @@ def head_layer(p: Params, bh: int, layer: int, anchor: bool, q, k, led: HeadLedg
     cp = p._c()
     st = lib().rro_head_layer(ctypes.byref(cp), bh, layer, int(bool(anchor)), _ptr(q), _ptr(k),
                               _ptr(led.ids), _ptr(led.alpha), _ptr(led.anchor_layer),
-                              _ptr(flags), _ptr(beta), _ptr(counts), _ptr(g) if g is not None else None)
+                              _ptr(flags), _ptr(beta), _ptr(counts), _ptr(g) if g is not None else None,
+                              _ptr(led.elevated))
     return flags, beta, int(counts[0]), int(counts[1]), int(st)
 
 

@@ -184,6 +184,7 @@ typedef struct {
     int32_t min_reuse; /* 0: off; else a row is reused for min_reuse layers after it was built */
     int32_t g_sink;    /* mandatory global sentinels: sink chunks 0..g_sink-1 */
     int32_t g_recent;  /* ... and the row's recent chunks i-g_recent+1..i */
+    double gamma_h;    /* 0: off; else the larger guard margin of a refreshed row */
 } rro_params;
 
 static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
@@ -241,11 +242,18 @@ static void rro_rebuild_row(const rro_params *p, int32_t bh, int32_t layer,
  *     horizon of one layer", the horizon made configurable): with
  *     p->min_reuse = h > 0, a row built at layer a is reused without the
  *     test at layers a+1 .. a+h (ids kept, alpha stored).  The lifetime bound
- *     takes precedence where the two meet.  The page's optional larger guard
- *     margin after a refresh is not applied (its recovery rule is not
- *     given).
+ *     takes precedence where the two meet.
+ *     Elevated margin (reading of the same passage, "may use a larger guard
+ *     margin until its anchor margin recovers"): with p->gamma_h > 0, a row
+ *     rebuilt at a relay layer is marked elevated (elevated[i] = 1; a row
+ *     built at an anchor layer is not).  An elevated row's test uses
+ *     max(gamma_i, gamma_h) in place of gamma_i; the first time it passes
+ *     (alpha - beta > that margin: its margin has recovered) the mark is
+ *     cleared and later tests use gamma_i again.  A row kept by the horizon
+ *     without a test keeps its mark.
  * Outputs: ids [nq*c] (in/out), alpha [nq] (in/out), anchor_layer [nq]
- * (in/out), flags [nq] (out: 1 = row was fully routed at this layer),
+ * (in/out), elevated [nq] (in/out; may be NULL when gamma_h is 0), flags
+ * [nq] (out: 1 = row was fully routed at this layer),
  * beta_out [nq] (out, may be NULL; relay only), counts[2] (out: rows fully
  * routed, score pairs evaluated under the counting rule below).
  * Counting rule (reading of RouteRelay §5.2 "evaluated query-key score
@@ -257,8 +265,9 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
                        int32_t anchor, const float *q, const float *kc,
                        int32_t *ids, double *alpha, int32_t *anchor_layer,
                        uint8_t *flags, double *beta_out, int64_t *counts,
-                       const double *gamma_rows)
+                       const double *gamma_rows, uint8_t *elevated)
 {
+    const int32_t use_h = p->gamma_h > 0.0 && elevated != NULL;
     const int32_t c = p->k + p->m + p->r + p->g_sink + p->g_recent;
     double *S = (double *)malloc(sizeof(double) * (size_t)p->nq * (size_t)p->nk);
     rro_scores(q, kc, p->nq, p->nk, p->d, S);
@@ -272,6 +281,7 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
             rro_rebuild_row(p, bh, layer, i, s_row, row, &alpha[i]);
             anchor_layer[i] = layer;
             flags[i] = 1;
+            if (use_h) elevated[i] = 0;
             refreshed += 1;
             pairs += n_valid;
             if (beta_out) beta_out[i] = NAN;
@@ -290,20 +300,28 @@ int32_t rro_head_layer(const rro_params *p, int32_t bh, int32_t layer,
         }
         pairs += n_cand;
         if (beta_out) beta_out[i] = b;
-        const double g = gamma_rows ? gamma_rows[i] : p->gamma;
-        int refresh = !(a > b + g);                             /* Eq. 8 */
-        if (p->max_age > 0 && layer - anchor_layer[i] >= p->max_age)
+        double g = gamma_rows ? gamma_rows[i] : p->gamma;
+        if (use_h && elevated[i] && p->gamma_h > g) g = p->gamma_h;   /* elevated margin */
+        int refresh;
+        int tested = 0;
+        if (p->max_age > 0 && layer - anchor_layer[i] >= p->max_age) {
             refresh = 1;                                        /* lifetime bound */
-        else if (p->min_reuse > 0 && layer - anchor_layer[i] <= p->min_reuse)
+        } else if (p->min_reuse > 0 && layer - anchor_layer[i] <= p->min_reuse) {
             refresh = 0;                                        /* hysteresis horizon */
+        } else {
+            refresh = !(a > b + g);                             /* Eq. 8 */
+            tested = 1;
+        }
         flags[i] = (uint8_t)refresh;
         if (refresh) {
             rro_rebuild_row(p, bh, layer, i, s_row, row, &alpha[i]);
             anchor_layer[i] = layer;
+            if (use_h) elevated[i] = 1;                         /* refreshed at a relay layer */
             refreshed += 1;
             pairs += n_valid;
         } else {
             alpha[i] = a;
+            if (use_h && tested) elevated[i] = 0;               /* passed: the margin recovered */
         }
     }
     free(S);

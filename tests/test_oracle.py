@@ -565,6 +565,89 @@ def test_min_reuse_beyond_the_run_never_refreshes_and_the_bound_takes_precedence
         assert np.all(l - rt2.ledgers[0].anchor_layer < 2)
 
 
+# ---- hysteresis: elevated guard margin after a refresh (RouteRelay §3.2
+# "Hysteresis": a refreshed row "may use a larger guard margin until its
+# anchor margin recovers").  Reading: a row rebuilt at a relay layer is marked;
+# a marked row's test uses max(gamma_i, gamma_h); its first pass clears the
+# mark; a row built at an anchor layer is unmarked. ------------------------
+
+def _alpha_beta(S, ids_row, k):
+    r = [S[j] for j in ids_row[:k] if j >= 0]
+    s = [S[j] for j in ids_row[k:] if j >= 0]
+    return min(r), (max(s) if s else -np.inf)
+
+
+def test_elevated_margin_applies_to_refreshed_rows_until_they_pass():
+    G = 0.1
+    p = Params(nq=40, nk=40, d=8, k=4, m=3, r=2, causal=False, seed=12, gamma_h=G)
+    lq = _drifting_layers(1, 40, 8, 12, 0.12, 71)
+    rt = oracle.Router(p, bh=1, anchor_interval=6)
+    flipped = recovered = stayed = 0
+    for l, (q, k) in enumerate(lq):
+        before = rt.ledgers[0].copy()
+        res, _ = rt.step(l, q, k, recall=False)
+        flags = res[0][0]
+        after = rt.ledgers[0]
+        if oracle.is_anchor(l, 6):
+            assert np.all(after.elevated == 0) and np.all(flags == 1)
+            continue
+        S = oracle.scores(q[0], k[0])
+        for i in range(40):
+            a, b = _alpha_beta(S[i], before.ids[i], p.k)
+            margin = G if before.elevated[i] else 0.0
+            expect = int(not (a > b + margin))
+            assert flags[i] == expect, (l, i)
+            assert after.elevated[i] == expect, (l, i)   # refreshed: marked; passed: cleared
+            if before.elevated[i]:
+                flipped += int(expect == 1 and a > b)   # the larger margin decided this one
+                recovered += int(expect == 0)
+            stayed += int(expect == 0 and not before.elevated[i])
+    assert flipped > 0 and recovered > 0 and stayed > 0
+
+
+def test_elevated_margin_off_is_the_plain_test_and_gamma_rows_below_it_are_raised():
+    lq = _drifting_layers(2, 32, 8, 8, 0.12, 72)
+    base = Params(nq=32, nk=32, d=8, k=4, m=2, r=2, causal=True, seed=3)
+    a = _run(base, 2, lq, 5)
+    b = _run(Params(**{**base.__dict__, "gamma_h": 0.0}), 2, lq, 5)
+    for (la, fa, _), (lb, fb, _) in zip(a, b):
+        for h in range(2):
+            assert np.array_equal(la[h].ids, lb[h].ids) and np.array_equal(fa[h], fb[h])
+            assert not lb[h].elevated.any()
+    # a per-row margin above gamma_h is not lowered by the mark: with gamma_h
+    # below every gamma_i the run equals the run without the mark
+    g = np.full((2, 32), 0.05)
+    c = _run(Params(**{**base.__dict__, "gamma_h": 0.01}), 2, lq, 5, gamma_rows=g)
+    d = _run(base, 2, lq, 5, gamma_rows=g)
+    for (lc, fc, _), (ld, fd, _) in zip(c, d):
+        for h in range(2):
+            assert np.array_equal(lc[h].ids, ld[h].ids) and np.array_equal(fc[h], fd[h])
+
+
+def test_elevated_margin_with_the_reuse_horizon_keeps_the_mark_until_tested():
+    G, hz = 0.1, 1
+    p = Params(nq=32, nk=32, d=8, k=4, m=2, r=2, causal=False, seed=5, gamma_h=G, min_reuse=hz)
+    lq = _drifting_layers(1, 32, 8, 10, 0.2, 73)
+    rt = oracle.Router(p, bh=1, anchor_interval=100)
+    kept_marked = 0
+    for l, (q, k) in enumerate(lq):
+        before = rt.ledgers[0].copy()
+        res, _ = rt.step(l, q, k, recall=False)
+        if l == 0:
+            continue
+        flags, after = res[0][0], rt.ledgers[0]
+        S = oracle.scores(q[0], k[0])
+        for i in range(32):
+            if l - before.anchor_layer[i] <= hz:   # inside the horizon: no test, mark unchanged
+                assert flags[i] == 0 and after.elevated[i] == before.elevated[i]
+                kept_marked += int(before.elevated[i])
+            else:
+                a, b = _alpha_beta(S[i], before.ids[i], p.k)
+                expect = int(not (a > b + (G if before.elevated[i] else 0.0)))
+                assert flags[i] == expect and after.elevated[i] == expect
+    assert kept_marked > 0
+
+
 # ---- mandatory global sentinels (RouteRelay §3.1 item 3: sink and recent) ----
 
 @pytest.mark.parametrize("causal", [True, False])

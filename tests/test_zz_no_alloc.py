@@ -84,3 +84,33 @@ def test_static_entry_point_rejects_problems_beyond_its_capacity(rr):
     with pytest.raises(rr.RRError) as e:
         rr.rr_route_layer_static(cfg.to_c(), p, p, 1, p, p, p, p, p, 0)
     assert e.value.status == rr.RR_ECAPACITY
+
+
+@pytest.mark.parametrize("w", [W.C3.with_(bh=4, layers=6, anchor_interval=3),
+                               W.C5.with_(bh=2, n=640, layers=6, anchor_interval=3)],
+                         ids=["f32_causal", "bf16_causal"])
+def test_static_entry_point_allocates_nothing(rr, w):
+    """The entry point's defining property: once a device is set up (the
+    first anchor and relay calls also load the kernels), further anchor and
+    relay layers change neither torch's reserved pool nor the device's free
+    memory as the driver reports it."""
+    cfg = config_of(w, rr)
+    arrs = _static_arrays(rr, cfg)
+    st = W.LayerStream(w, "cpu")
+    xs = []
+    for _ in range(w.layers):
+        _, _, qs, ks = st.next()
+        xs.append((qs.to(DEV), ks.to(DEV)))
+    for layer in (0, 1):   # set-up calls: an anchor and a relay layer
+        _call_static(rr, cfg, xs[layer][0], xs[layer][1], layer, arrs)
+    torch.cuda.synchronize()
+    reserved0 = torch.cuda.memory_reserved(DEV)
+    free0, _ = torch.cuda.mem_get_info(DEV)
+    for layer in range(2, w.layers):   # layer 3 is a forced anchor, the others relay layers
+        _call_static(rr, cfg, xs[layer][0], xs[layer][1], layer, arrs)
+    torch.cuda.synchronize()
+    assert torch.cuda.memory_reserved(DEV) == reserved0
+    free1, _ = torch.cuda.mem_get_info(DEV)
+    assert free1 == free0, (free0, free1)
+    assert int(arrs["counters"][rr.CNT_LAST_LAYER].item()) == w.layers - 1
+    assert int(arrs["counters"][rr.CNT_ERROR].item()) == 0
