@@ -76,6 +76,10 @@ def _load():
     lib.rr_ledger_set_guard.restype = ctypes.c_int
     lib.rr_ledger_set_hysteresis.argtypes = [P, ctypes.c_int32]
     lib.rr_ledger_set_hysteresis.restype = ctypes.c_int
+    lib.rr_ledger_set_wait_budget.argtypes = [P, ctypes.c_int64]
+    lib.rr_ledger_set_wait_budget.restype = ctypes.c_int
+    lib.rr_ledger_set_hysteresis_margin.argtypes = [P, ctypes.c_float]
+    lib.rr_ledger_set_hysteresis_margin.restype = ctypes.c_int
     lib.rr_route_layer_static.argtypes = [ctypes.POINTER(rr_config), P, P, ctypes.c_int32, P, P, P, P, P, P]
     lib.rr_route_layer_static.restype = ctypes.c_int
     lib.rr_sparse_attention.argtypes = [ctypes.POINTER(rr_attn_config), P, P, P, P, P, P]
@@ -159,6 +163,16 @@ def rr_ledger_set_guard(handle, d_gamma_rows: int, max_age: int) -> None:
 
 def rr_ledger_set_hysteresis(handle, min_reuse: int) -> None:
     _check(_lib.rr_ledger_set_hysteresis(handle, min_reuse), "rr_ledger_set_hysteresis")
+
+
+def rr_ledger_set_hysteresis_margin(handle, gamma_h: float) -> None:
+    _check(_lib.rr_ledger_set_hysteresis_margin(handle, float(gamma_h)), "rr_ledger_set_hysteresis_margin")
+
+
+def rr_ledger_set_wait_budget(handle, cycles: int) -> None:
+    """Test hook (include/rr.h): the budget of the selection kernel's
+    epilogue waits, in SM cycles (0: the default, about a second)."""
+    _check(_lib.rr_ledger_set_wait_budget(handle, int(cycles)), "rr_ledger_set_wait_budget")
 
 
 def rr_route_layer_static(cfg: rr_config, d_qc: int, d_kc: int, layer: int, d_ids: int, d_alpha: int,
@@ -347,6 +361,11 @@ class RouteLedger:
     def set_hysteresis(self, min_reuse: int) -> None:
         """Minimum reuse horizon after a row is rebuilt (0: off)."""
         rr_ledger_set_hysteresis(self.handle, int(min_reuse))
+
+    def set_hysteresis_margin(self, gamma_h: float) -> None:
+        """Larger guard margin of a row rebuilt at a relay layer, until its
+        test first passes (0: off; the mark is bit 1 of the flags)."""
+        rr_ledger_set_hysteresis_margin(self.handle, float(gamma_h))
 
     def device_view(self) -> dict:
         """Zero-copy torch views of the ledger inside the workspace."""

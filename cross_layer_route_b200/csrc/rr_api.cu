@@ -156,8 +156,13 @@ rr_status stage_compact(rr_ledger *L, int32_t layer, cudaStream_t s) {
     return RR_OK;
 }
 
+// Flags byte of a row rebuilt at a relay layer: refreshed, and marked for
+// the hysteresis margin when one is set.
+uint8_t relay_rebuild_flag(const rr_ledger *L) { return (uint8_t)(1u | (L->dev.gamma_h > 0.0f ? 2u : 0u)); }
+
 rr_status stage_refresh(rr_ledger *L, const void *q, const void *k, int32_t layer, cudaStream_t s) {
     if (L->stage != 2 || layer != L->pending_layer) return RR_ESTATE;
+    L->dev.rebuild_flag = relay_rebuild_flag(L);
     cudaError_t e = rr::launch_route_rows(L->dev, L->cfg.dtype, q, k, layer, /*use_list=*/true, s);
     if (e == cudaSuccess) e = rr::launch_finalize(L->dev, layer, 0, 0, 0, s);
     if (e != cudaSuccess) return RR_ECUDA;
@@ -172,6 +177,7 @@ rr_status do_full_route(rr_ledger *L, const void *q, const void *k, int32_t laye
     if (st != RR_OK) return st;
     cudaError_t e = reset_layer_counters(L, s);
     if (e != cudaSuccess) return RR_ECUDA;
+    L->dev.rebuild_flag = 1;
     e = rr::launch_route_rows(L->dev, L->cfg.dtype, q, k, layer, /*use_list=*/false, s);
     if (e != cudaSuccess) return RR_ECUDA;
     const long long fp = full_pairs(&L->cfg);
@@ -190,6 +196,7 @@ rr_status do_relay_oneshot(rr_ledger *L, const void *q, const void *k, int32_t l
     const rr_status st = prepare(L, s);
     if (st != RR_OK) return st;
     cudaError_t e = reset_layer_counters(L, s);
+    L->dev.rebuild_flag = relay_rebuild_flag(L);
     if (e == cudaSuccess) e = rr::launch_relay_oneshot(L->dev, q, k, layer, s);
     if (e == cudaSuccess) e = rr::launch_finalize(L->dev, layer, 0, 0, 0, s);
     if (e != cudaSuccess) return RR_ECUDA;
@@ -345,6 +352,18 @@ rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int3
 rr_status rr_ledger_set_hysteresis(rr_ledger *ledger, int32_t min_reuse) {
     if (!ledger || min_reuse < 0) return RR_EINVAL;
     ledger->dev.min_reuse = min_reuse;
+    return RR_OK;
+}
+
+rr_status rr_ledger_set_wait_budget(rr_ledger *ledger, int64_t cycles) {
+    if (!ledger || cycles < 0) return RR_EINVAL;
+    ledger->dev.wait_budget = (long long)cycles;
+    return RR_OK;
+}
+
+rr_status rr_ledger_set_hysteresis_margin(rr_ledger *ledger, float gamma_h) {
+    if (!ledger || !(gamma_h >= 0.0f) || !isfinite(gamma_h)) return RR_EINVAL;
+    ledger->dev.gamma_h = gamma_h;
     return RR_OK;
 }
 

@@ -45,21 +45,29 @@ __device__ __forceinline__ bool is_global_cand(const LedgerDev &L, int row, int 
     return j >= 0 && j < n_valid && (j < L.g_sink || (j <= row && j > row - L.g_recent));
 }
 
-// The relay decision of one row (RouteRelay §3.2): refresh unless
-// alpha > beta + gamma_i (Eq. 8; gamma_i from the per-row margins when the
-// ledger has them).  A row whose ledger is max_age layers old refreshes in
-// any case (the per-row lifetime bound; max_age 0 = off); otherwise a row
-// built min_reuse or fewer layers ago is reused without the test (the
-// hysteresis horizon; min_reuse 0 = off).
-__device__ __forceinline__ bool relay_refresh(const LedgerDev &L, size_t grow, int layer,
-                                              float alpha, float beta) {
+// The relay decision of one row (RouteRelay §3.2), as the row's new flags
+// byte: bit 0 = refresh, bit 1 = the row keeps (or, refreshed at this relay
+// layer, receives) the hysteresis mark.  Refresh unless alpha > beta +
+// gamma_i (Eq. 8; gamma_i from the per-row margins when the ledger has
+// them).  A row whose ledger is max_age layers old refreshes in any case
+// (the per-row lifetime bound; max_age 0 = off); otherwise a row built
+// min_reuse or fewer layers ago is reused without the test (the hysteresis
+// horizon; min_reuse 0 = off; the mark is left as it is).  A marked row
+// tests with max(gamma_i, gamma_h) and loses the mark when it passes (the
+// "larger guard margin until its anchor margin recovers"; gamma_h 0 = off).
+// A NaN margin makes the row refresh.
+__device__ __forceinline__ uint8_t relay_decide(const LedgerDev &L, size_t grow, int layer, float alpha,
+                                                float beta) {
+    const uint8_t refreshed = (uint8_t)(1u | (L.gamma_h > 0.0f ? 2u : 0u));
+    const bool marked = L.gamma_h > 0.0f && (L.flags[grow] & 2u) != 0u;
     if (L.max_age > 0 || L.min_reuse > 0) {   // the row's age is read only when needed
         const int age = layer - L.anchor_layer[grow];
-        if (L.max_age > 0 && age >= L.max_age) return true;
-        if (L.min_reuse > 0 && age <= L.min_reuse) return false;
+        if (L.max_age > 0 && age >= L.max_age) return refreshed;
+        if (L.min_reuse > 0 && age <= L.min_reuse) return marked ? 2u : 0u;
     }
-    const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
-    return !(alpha > beta + g);
+    float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
+    if (marked && L.gamma_h > g) g = L.gamma_h;
+    return (alpha > beta + g) ? (uint8_t)0u : refreshed;
 }
 
 // ---- Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11) --------------------

@@ -44,8 +44,18 @@ struct LedgerDev {
     const float *gamma_rows = nullptr;
     int max_age = 0;
     // hysteresis: a row built at layer a is reused without the test at
-    // layers a+1 .. a+min_reuse (0: off)
+    // layers a+1 .. a+min_reuse (0: off); a row rebuilt at a relay layer is
+    // marked (flags bit 1) and tests with max(gamma_i, gamma_h) until it
+    // first passes (gamma_h 0: off)
     int min_reuse = 0;
+    float gamma_h = 0.0f;
+    // flags byte a rebuilt row receives (set by the host per launch): 1 at
+    // an anchor layer, 1 | 2 at a relay layer when gamma_h > 0
+    uint8_t rebuild_flag = 1;
+    // budget, in SM clock cycles, of the selection kernel's accumulator waits
+    // in its epilogue (0: the default, about a second); a test shortens it to
+    // make a wait run out
+    long long wait_budget = 0;
     uint32_t seed_lo, seed_hi;
 };
 

@@ -128,8 +128,9 @@ relay_rescore_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__
         }
         const bool any_bad = __any_sync(kFull, bad);
         if (lane == 0) {
-            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
-            L.flags[grow] = refresh ? 1 : 0;
+            const uint8_t fl = relay_decide(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
+            const bool refresh = (fl & 1u) != 0u;
+            L.flags[grow] = fl;
             if (!refresh) L.alpha[grow] = amin;
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
         }
@@ -157,7 +158,7 @@ __global__ void __launch_bounds__(kCompactThreads) compact_flags_kernel(LedgerDe
     unsigned long long pairs = 0;
     for (int i0 = 0; i0 < L.nq; i0 += kCompactThreads) {
         const int i = i0 + tid;
-        const bool f = i < L.nq && fl[i] != 0;
+        const bool f = i < L.nq && (fl[i] & 1u) != 0;   // bit 0: refresh (bit 1: hysteresis mark)
         const unsigned wm = __ballot_sync(kFull, f);
         if (lane == 0) warp_tot[warp] = __popc(wm);
         __syncthreads();
@@ -301,8 +302,9 @@ relay_rescore_oct_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restri
         }
         const bool any_bad = __any_sync(kFull, bad);
         if (lane == 0) {
-            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
-            L.flags[grow] = refresh ? 1 : 0;
+            const uint8_t fl = relay_decide(L, (size_t)grow, layer, amin, bmax);  // Eq. 8
+            const bool refresh = (fl & 1u) != 0u;
+            L.flags[grow] = fl;
             if (!refresh) L.alpha[grow] = amin;
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
         }

@@ -272,7 +272,7 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
         if (lane == 0) {
             L.alpha[grow] = bs[nr - 1];
             L.anchor_layer[grow] = layer;
-            L.flags[grow] = 1;
+            L.flags[grow] = L.rebuild_flag;
         }
     }
 }

@@ -273,7 +273,7 @@ route_rows_tc_heap_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
                 [&](int e) -> int & { return bi[e * kRows]; }, out + L.k + L.m, nullptr);
             L.alpha[grow] = key_score(H[(nr - 1) * kRows]);
             L.anchor_layer[grow] = layer;
-            L.flags[grow] = 1;
+            L.flags[grow] = L.rebuild_flag;
         }
     }
     cta_teardown(c, L);
@@ -491,7 +491,7 @@ __device__ __forceinline__ void finish_row(const LedgerDev &L, int layer, int h,
     if (lane < L.r) out[L.k + L.m + lane] = lane < acc ? w.acc[lane] : -1;
     if (lane == 0) {
         L.anchor_layer[grow] = layer;
-        L.flags[grow] = 1;
+        L.flags[grow] = L.rebuild_flag;
     }
 }
 
@@ -833,8 +833,9 @@ relay_rescore_tc_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             }
             if (cta_ok && row >= 0) {
                 const size_t grow = (size_t)h * L.nq + row;
-                const bool refresh = relay_refresh(L, grow, layer, a, b);   // Eq. 8
-                L.flags[grow] = refresh ? 1 : 0;
+                const uint8_t fl = relay_decide(L, grow, layer, a, b);   // Eq. 8
+                const bool refresh = (fl & 1u) != 0u;
+                L.flags[grow] = fl;
                 if (!refresh) L.alpha[grow] = a;
                 if (n & (1 << 30)) atomicOr(&L.counters[2], 1ULL);
                 pairs = (unsigned)(n & ((1 << 30) - 1));

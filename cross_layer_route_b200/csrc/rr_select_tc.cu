@@ -243,6 +243,7 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         const int n_valid = row >= 0 ? valid_keys(row, L.nk, L.causal) : 0;
         const uint32_t lane_base = c.tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(qt * 32);
         const int nt = c.ntiles;
+        const long long wait_limit = L.wait_budget > 0 ? L.wait_budget : kSpinLimit;
         bool ok = true;
         auto epi_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kSelEpiWarps * 32) : "memory"); };
 
@@ -252,7 +253,7 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
 #pragma unroll
         for (int q = 0; q < 32; ++q) m[q] = -INFINITY;
         for (int i = 0; i < nt && ok; ++i) {
-            if (!(ok = acc_wait<kSelAcc>(c, i))) break;
+            if (!(ok = acc_wait<kSelAcc>(c, i, wait_limit))) break;
             float v[32];
             tc_ld32(lane_base + (uint32_t)((i % kSelAcc) * kKeys), v);
             acc_release<kSelAcc>(c, i);   // the scores are in registers: the MMA may reuse the accumulator
@@ -353,7 +354,7 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
         for (int i = 0; i < nt && ok; ++i) {
             const int g = nt + i;
             const int t = nt - 1 - i;
-            if (!(ok = acc_wait<kSelAcc>(c, g))) break;
+            if (!(ok = acc_wait<kSelAcc>(c, g, wait_limit))) break;
             float v[32];
             tc_ld32(lane_base + (uint32_t)((g % kSelAcc) * kKeys), v);
             acc_release<kSelAcc>(c, g);
@@ -539,8 +540,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     if (total < 0 || total > kRowCap || total < min(L.ksel, n_valid)) {
         if (lane == 0) {
             if (kRelay) {
-                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
-                L.flags[grow] = 0;
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;   // flags: set by the exact rescoring
             } else {
                 const int pos = atomicAdd(&L.retry_count[h], 1);
                 L.retry_list[(size_t)h * L.nq + pos] = row;
@@ -563,8 +563,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         if (lane == 0) {
             atomicOr(&L.counters[2], 4ULL);
             if (kRelay) {
-                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
-                L.flags[grow] = 0;
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;   // flags: set by the exact rescoring
             } else {
                 const int pos = atomicAdd(&L.retry_count[h], 1);
                 L.retry_list[(size_t)h * L.nq + pos] = row;
@@ -579,8 +578,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         const int words = (n_valid + 31) >> 5;
         if (n_valid > 32 * kBitsWords) {   // no bitmap for such rows: rescore exactly
             if (lane == 0) {
-                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
-                L.flags[grow] = 0;
+                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;   // flags: set by the exact rescoring
             }
             return;
         }
@@ -624,14 +622,23 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         // sentinel was kept (the others score below T) or there is none
         const bool aexact = rf == rt;
         const bool bexact = sf > 0 || st == 0;
-        int dec = -1;   // 0 keep, 1 refresh, 2 rescore exactly
-        if (L.max_age > 0 || L.min_reuse > 0) {   // the ledger's age rules, as relay_refresh
+        // the decision of relay_decide, with one side bounded by T where the
+        // kept scores do not give it exactly
+        const bool marked = L.gamma_h > 0.0f && (L.flags[grow] & 2u) != 0u;
+        int dec = -1;            // 0 keep, 1 refresh, 2 rescore exactly
+        uint8_t keep_flag = 0;   // flags byte of a kept row
+        if (L.max_age > 0 || L.min_reuse > 0) {   // the ledger's age rules
             const int age = layer - L.anchor_layer[grow];
-            if (L.max_age > 0 && age >= L.max_age) dec = 1;
-            else if (L.min_reuse > 0 && age <= L.min_reuse) dec = aexact ? 0 : 2;
+            if (L.max_age > 0 && age >= L.max_age) {
+                dec = 1;
+            } else if (L.min_reuse > 0 && age <= L.min_reuse) {
+                dec = aexact ? 0 : 2;
+                keep_flag = marked ? 2u : 0u;   // no test: the mark stays
+            }
         }
         if (dec < 0) {
-            const float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
+            float g = L.gamma_rows ? L.gamma_rows[grow] : L.gamma;
+            if (marked && L.gamma_h > g) g = L.gamma_h;            // hysteresis margin
             if (aexact && bexact) dec = (amin > bmax + g) ? 0 : 1;   // Eq. 8
             else if (aexact) dec = (amin > T + g) ? 0 : 2;        // beta < T
             else if (sf > 0) dec = 1;                             // alpha < T <= beta
@@ -640,16 +647,13 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         if (dec == 0) {
             if (lane == 0) {
                 L.alpha[grow] = amin;
-                L.flags[grow] = 0;
+                L.flags[grow] = keep_flag;
             }
             cnt.pairs += (unsigned long long)(rt + st);
             return;
         }
-        if (dec == 2) {
-            if (lane == 0) {
-                L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
-                L.flags[grow] = 0;
-            }
+        if (dec == 2) {   // the exact rescoring writes the row's flags byte
+            if (lane == 0) L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;
             return;
         }
         cnt.pairs += (unsigned long long)(rt + st + n_valid);
@@ -811,7 +815,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     if (lane < L.r) out[L.k + L.m + lane] = lane < acc ? w.acc[lane] : -1;
     if (lane == 0) {
         L.anchor_layer[grow] = layer;
-        L.flags[grow] = 1;
+        L.flags[grow] = L.rebuild_flag;
     }
 }
 
@@ -920,8 +924,9 @@ relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_
         }
         const bool any_bad = __any_sync(kFull, bad);
         if (lane == 0) {
-            const bool refresh = relay_refresh(L, (size_t)grow, layer, amin, bmax);   // Eq. 8
-            L.flags[grow] = refresh ? 1 : 0;
+            const uint8_t fl = relay_decide(L, (size_t)grow, layer, amin, bmax);   // Eq. 8
+            const bool refresh = (fl & 1u) != 0u;
+            L.flags[grow] = fl;
             if (!refresh) L.alpha[grow] = amin;
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
             cpair += (unsigned long long)ncand;

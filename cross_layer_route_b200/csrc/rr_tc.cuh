@@ -91,10 +91,36 @@ __device__ __forceinline__ bool mbar_test_sleep(uint64_t *b, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
+// Non-blocking test of the phase (try_wait above may hold the thread for a
+// while before it answers; test_wait answers at once).
+__device__ __forceinline__ bool mbar_poll(uint64_t *b, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(saddr(b)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 // Bounded wait for the phase of the given parity.  Returns false on timeout
 // (and raises the CTA's abort flag) or when another role already aborted.
+// A limit below the default polls with test_wait, so that the limit and not
+// the hardware's own wait inside try_wait decides when the wait ends.
 __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile int *abort_flag,
                                           long long limit = kSpinLimit) {
+    if (limit < kSpinLimit) {
+        const long long t0 = clock64();
+        while (!mbar_poll(b, parity)) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > limit) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+        return true;
+    }
     if (mbar_test(b, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_test_sleep(b, parity)) {

@@ -190,8 +190,10 @@ rr_status rr_relay_refresh(rr_ledger *ledger, const void *d_qc, const void *d_kc
 /* Destination of rr_ledger_read.  Any pointer may be NULL (that part is not
  * copied).  Sizes: ids bh*nq*c int32 laid out [bh, nq, c] (route, then
  * near-miss, then random), alpha bh*nq f32, anchor_layer bh*nq int32, flags
- * bh*nq u8 (1 = the row was fully routed at the last layer), counters 16
- * int64 (the RR_CNT_* slots).  Host (pinned or pageable) or device memory. */
+ * bh*nq u8 (bit 0: the row was fully routed at the last layer; bit 1: the
+ * row carries the hysteresis mark of rr_ledger_set_hysteresis_margin, never
+ * set while that margin is 0), counters 16 int64 (the RR_CNT_* slots).  Host
+ * (pinned or pageable) or device memory. */
 typedef struct {
     int32_t *ids;
     float *alpha;
@@ -229,11 +231,24 @@ rr_status rr_ledger_set_guard(rr_ledger *ledger, const float *d_gamma_rows, int3
  * or h > 0 -- a row built at layer a (anchor or refresh) is reused without
  * the challenge test at layers a+1 .. a+h: its ids stay, its alpha is
  * stored, it counts as a stable row.  The lifetime bound of
- * rr_ledger_set_guard takes precedence where the two meet.  The page's
- * optional larger guard margin after a refresh is not applied (the page
- * gives no rule for its recovery).  Takes effect from the next relay call;
- * no CUDA call.  Returns RR_EINVAL for a NULL ledger or min_reuse < 0. */
+ * rr_ledger_set_guard takes precedence where the two meet; a row kept inside
+ * the horizon keeps its hysteresis mark (below).  Takes effect from the next
+ * relay call; no CUDA call.  Returns RR_EINVAL for a NULL ledger or
+ * min_reuse < 0. */
 rr_status rr_ledger_set_hysteresis(rr_ledger *ledger, int32_t min_reuse);
+
+/* Hysteresis, its second part (RouteRelay §3.2: a refreshed row "may use a
+ * larger guard margin until its anchor margin recovers").  gamma_h: 0 (off)
+ * or the larger margin, finite and >= 0.  Reading: a row rebuilt at a relay
+ * layer is marked (flags bit 1; a row built at an anchor layer is not); a
+ * marked row's test of Eq. 8 uses max(gamma_i, gamma_h), and the first time
+ * it passes (alpha - beta above that margin: its margin has recovered) the
+ * mark is cleared and later tests use gamma_i again.  The lifetime bound and
+ * the reuse horizon of rr_ledger_set_guard / rr_ledger_set_hysteresis come
+ * first, as in the test without the mark.  Takes effect from the next relay
+ * call; no CUDA call.  Returns RR_EINVAL for a NULL ledger or a negative or
+ * non-finite gamma_h. */
+rr_status rr_ledger_set_hysteresis_margin(rr_ledger *ledger, float gamma_h);
 
 /* One layer on caller-held ledger arrays, allocating nothing.  The paper
  * has no counterpart: this is a deployment variant for callers that cannot
@@ -270,6 +285,17 @@ rr_status rr_route_layer_static(const rr_config *cfg, const void *d_qc, const vo
                                 int32_t layer, int32_t *d_ids, float *d_alpha,
                                 int32_t *d_anchor_layer, uint8_t *d_flags, int64_t *d_counters,
                                 void *stream);
+
+/* Test hook: the budget, in SM clock cycles, of the accumulator waits in the
+ * epilogue of the tensor-core selection kernel (0, the default: about a
+ * second, which only a stalled GPU exhausts).  Every wait in the tensor-core
+ * kernels is bounded; when one runs out the CTA stops issuing, drains its
+ * copies, waits for its last MMA, frees its TMEM and sets bit 1 of the error
+ * word, and its rows are redone by the exact one-pass path.  A short budget
+ * makes that happen on purpose, so a test can check the path; production
+ * callers leave it at 0.  No CUDA call; RR_EINVAL for a NULL ledger or a
+ * negative budget. */
+rr_status rr_ledger_set_wait_budget(rr_ledger *ledger, int64_t cycles);
 
 /* Human-readable name of a status code (static string). */
 const char *rr_status_string(rr_status status);

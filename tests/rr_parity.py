@@ -23,10 +23,10 @@ TIE_REL = 1e-5
 
 
 def params_of(w, bh_offset: int = 0, max_age: int = 0, min_reuse: int = 0, g_sink: int = 0,
-              g_recent: int = 0) -> oracle.Params:
+              g_recent: int = 0, gamma_h: float = 0.0) -> oracle.Params:
     return oracle.Params(nq=w.n, nk=w.n, d=w.d, k=w.k, m=w.m, r=w.r, causal=w.causal,
                          gamma=w.gamma, seed=w.seed, max_age=max_age, min_reuse=min_reuse,
-                         g_sink=g_sink, g_recent=g_recent)
+                         g_sink=g_sink, g_recent=g_recent, gamma_h=gamma_h)
 
 
 def config_of(w, rr, bh: int | None = None, bh_offset: int = 0, g_sink: int = 0, g_recent: int = 0):
@@ -66,10 +66,15 @@ def _sorted_valid(s_row: np.ndarray, nv: int):
 
 def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndarray, k: np.ndarray,
                  prev_ids, prev_alpha, prev_anchor, gpu_ids, gpu_alpha, gpu_anchor, gpu_flags,
-                 max_report: int = 10, gamma_rows=None) -> Report:
+                 max_report: int = 10, gamma_rows=None, prev_flags=None) -> Report:
     """Runs the oracle on one head from the GPU's previous ledger and checks
     the GPU's ledger after the same layer.  gamma_rows: this head's per-row
-    guard margins (None: p.gamma)."""
+    guard margins (None: p.gamma).  Flags: bit 0 (refresh) is compared with
+    the oracle's flag, bit 1 (the hysteresis mark, p.gamma_h > 0) with the
+    oracle's mark after the layer; the oracle starts from the GPU's previous
+    marks (prev_flags bit 1)."""
+    gpu_mark = (np.asarray(gpu_flags) >> 1) & 1
+    gpu_flags = np.asarray(gpu_flags) & 1
     rep = Report(rows=p.nq)
     S = oracle.scores(q, k)
     scale = np.linalg.norm(q.astype(np.float64), axis=1) * np.linalg.norm(k.astype(np.float64), axis=1).max()
@@ -79,6 +84,9 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
     else:
         led = oracle.HeadLedger(prev_ids.astype(np.int32).copy(), prev_alpha.astype(np.float64).copy(),
                                 prev_anchor.astype(np.int32).copy())
+        if prev_flags is not None:
+            led.elevated = ((np.asarray(prev_flags) >> 1) & 1).astype(np.uint8)
+    prev_mark = None if anchor else led.elevated.copy()
     flags_o, beta_o, ref_o, pairs_o, st = oracle.head_layer(p, gh, layer, anchor, q, k, led,
                                                              gamma_rows=gamma_rows)
     assert st == 0
@@ -131,6 +139,8 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
             r_ids = [j for j in prev_ids[i, : p.k] if j >= 0]
             a = min(S[i, j] for j in r_ids) if r_ids else np.inf
             g_i = p.gamma if gamma_rows is None else float(gamma_rows[i])
+            if p.gamma_h > 0 and prev_mark[i] and p.gamma_h > g_i:
+                g_i = p.gamma_h
             age = layer - int(prev_anchor[i])
             forced = (p.max_age > 0 and age >= p.max_age) or (p.min_reuse > 0 and age <= p.min_reuse)
             if not forced and np.isfinite(beta_o[i]) and abs(a - beta_o[i] - g_i) < tol[i]:
@@ -147,6 +157,8 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
                 continue
             if not flags_o[i]:
                 rep.compared += 1
+                if int(gpu_mark[i]) != int(led.elevated[i]):
+                    bad(i, f"hysteresis mark of a kept row gpu={int(gpu_mark[i])} oracle={int(led.elevated[i])}")
                 if not np.array_equal(gpu_ids[i], prev_ids[i]):
                     bad(i, "stable row changed its ids")
                 if abs(float(gpu_alpha[i]) - a) > tol[i]:
@@ -191,12 +203,14 @@ def compare_head(p: oracle.Params, gh: int, layer: int, anchor: bool, q: np.ndar
             bad(i, f"anchor layer gpu={gpu_anchor[i]} expected {layer}")
         if int(gpu_flags[i]) != 1:
             bad(i, "fully routed row without flag")
+        if int(gpu_mark[i]) != int(led.elevated[i]):
+            bad(i, f"hysteresis mark of a rebuilt row gpu={int(gpu_mark[i])} oracle={int(led.elevated[i])}")
     return rep
 
 
 def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report_every=None,
                   gamma_rows=None, max_age: int = 0, min_reuse: int = 0, g_sink: int = 0,
-                  g_recent: int = 0):
+                  g_recent: int = 0, gamma_h: float = 0.0, check: bool = True):
     """Runs `layers` layers of workload w through the CUDA ledger `led` and
     compares every layer of the listed heads with the oracle started from
     the GPU's own previous ledger.  gamma_rows ([bh, nq] array) and max_age
@@ -205,7 +219,8 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
     import rr_workloads
     import torch
     st = rr_workloads.LayerStream(w, stream_device)
-    p = params_of(w, max_age=max_age, min_reuse=min_reuse, g_sink=g_sink, g_recent=g_recent)
+    p = params_of(w, max_age=max_age, min_reuse=min_reuse, g_sink=g_sink, g_recent=g_recent,
+                  gamma_h=gamma_h)
     total = Report()
     per_layer = []
     prev = None
@@ -215,7 +230,7 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
         kd = ks.to(device).contiguous()
         anchor = oracle.is_anchor(l, w.anchor_interval)
         led.layer(qd, kd, l)
-        after = led.read()
+        after = led.read(check=check)
         layer_rep = Report()
         qn = qf.cpu().numpy()
         kn = kf.cpu().numpy()
@@ -223,10 +238,12 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
             pi = prev["ids"][h].numpy() if prev is not None else None
             pa = prev["alpha"][h].numpy() if prev is not None else None
             pl = prev["anchor_layer"][h].numpy() if prev is not None else None
+            pf = prev["flags"][h].numpy() if prev is not None else None
             r = compare_head(p, h, l, anchor, qn[h], kn[h], pi, pa, pl, after["ids"][h].numpy(),
                              after["alpha"][h].numpy(), after["anchor_layer"][h].numpy(),
                              after["flags"][h].numpy(),
-                             gamma_rows=None if gamma_rows is None else np.asarray(gamma_rows[h]))
+                             gamma_rows=None if gamma_rows is None else np.asarray(gamma_rows[h]),
+                             prev_flags=pf)
             layer_rep.add(r)
         per_layer.append((l, anchor, layer_rep, after["counters"].clone()))
         total.add(layer_rep)

@@ -133,6 +133,14 @@ def test_trigger_setters_validate_their_arguments_without_a_cuda_call():
         assert lib.rr_ledger_set_hysteresis(h, -1) == rr.RR_EINVAL
         assert lib.rr_ledger_set_hysteresis(h, 1) == rr.RR_OK
         assert lib.rr_ledger_set_hysteresis(None, 1) == rr.RR_EINVAL
+        for bad in (-0.1, float("nan"), float("inf")):
+            assert lib.rr_ledger_set_hysteresis_margin(h, bad) == rr.RR_EINVAL
+        assert lib.rr_ledger_set_hysteresis_margin(h, 0.0) == rr.RR_OK
+        assert lib.rr_ledger_set_hysteresis_margin(h, 0.05) == rr.RR_OK
+        assert lib.rr_ledger_set_hysteresis_margin(None, 0.05) == rr.RR_EINVAL
+        assert lib.rr_ledger_set_wait_budget(h, -1) == rr.RR_EINVAL
+        assert lib.rr_ledger_set_wait_budget(h, 0) == rr.RR_OK
+        assert lib.rr_ledger_set_wait_budget(None, 0) == rr.RR_EINVAL
     finally:
         lib.rr_ledger_destroy(h)
 

@@ -353,3 +353,49 @@ def test_global_sentinels_on_equal_scores_match_the_oracle(rr, dtype, d):
     ol = oracle.HeadLedger.empty(p)
     oracle.head_layer(p, 0, 0, True, q.to(td).float()[0].numpy(), kk.to(td).float()[0].numpy(), ol)
     assert np.array_equal(out["ids"][0].numpy(), ol.ids)
+
+
+HYST_MARGIN = [
+    (W.low_drift(W.C5).with_(bh=2, n=384, layers=10), "bf16_tensor_cores"),
+    (W.low_drift(W.C3).with_(bh=2, n=256, layers=10), "f32_cuda_cores"),
+]
+
+
+@pytest.mark.parametrize("case", HYST_MARGIN, ids=[c[1] for c in HYST_MARGIN])
+def test_hysteresis_margin_marks_and_recovery(rr, case):
+    """The larger guard margin after a refresh (RouteRelay §3.2,
+    Hysteresis): rows rebuilt at a relay layer carry the mark (flags bit 1)
+    and test with max(gamma_i, gamma_h) until they first pass.  Layer by
+    layer against the oracle given the same margin: flags, marks, ids and
+    alpha."""
+    w, _ = case
+    G = 0.01
+    led = rr.RouteLedger(config_of(w, rr), DEV)
+    led.set_hysteresis_margin(G)
+    rep, per_layer = layer_stepped(w, rr, led, w.layers, range(w.bh), DEV, gamma_h=G)
+    _check(rep)
+    flags = led.read()["flags"]
+    assert int(((flags >> 1) & 1).sum()) > 0                  # some rows carry the mark
+    relay = [lr for l, a, lr, _ in per_layer if not a]
+    assert sum(lr.refreshed_gpu for lr in relay) < sum(lr.rows for lr in relay)   # some rows were kept
+
+
+def test_a_wait_that_runs_out_sets_the_error_bit_and_the_rows_are_redone(rr):
+    """Every wait in the tensor-core kernels is bounded.  With the epilogue's
+    accumulator waits cut to a few hundred cycles, a wait runs out while the
+    selection kernel's copies and MMAs are in flight: the CTA drains its
+    copies, waits for its last MMA, frees its TMEM and sets bit 1 of the
+    error word; its rows go to the exact one-pass path, so the ledger still
+    matches the oracle.  A ledger with the default budget is unaffected."""
+    w = W.C5.with_(bh=2, n=384, layers=3)
+    led = rr.RouteLedger(config_of(w, rr), DEV)
+    rr.rr_ledger_set_wait_budget(led.handle, 300)
+    rep, per_layer = layer_stepped(w, rr, led, w.layers, range(w.bh), DEV, check=False)
+    _check(rep)
+    err = [int(cnt[rr.CNT_ERROR]) for _, _, _, cnt in per_layer]
+    assert all(e & 2 for e in err), err
+    assert int(per_layer[-1][3][rr.CNT_RETRY_TOTAL]) > 0
+    fresh = rr.RouteLedger(config_of(w, rr), DEV)
+    rep2, per_layer2 = layer_stepped(w, rr, fresh, w.layers, range(w.bh), DEV)
+    _check(rep2)
+    assert all(int(cnt[rr.CNT_ERROR]) == 0 for _, _, _, cnt in per_layer2)
