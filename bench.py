@@ -210,6 +210,16 @@ def launches_per_step(w, n_anchor: int, n_relay: int, oneshot: bool) -> int:
     return 2 * n_anchor + 4 * n_relay
 
 
+def graph_mode(args, w) -> bool:
+    """Whether the timed step is replayed from a CUDA graph: always with
+    --graph on, never with --graph off, and by default for the CUDA-core
+    workloads, whose layers take microseconds and would otherwise time the
+    launch path."""
+    if args.graph == "auto":
+        return not uses_tensor_cores(w)
+    return args.graph == "on"
+
+
 def full_pairs_per_layer(w) -> int:
     if not w.causal:
         return w.bh * w.n * w.n
@@ -266,26 +276,45 @@ def run_ours(args, w, rank, world, device):
             torch.distributed.barrier()
         torch.cuda.synchronize(device)
 
+    # CUDA-graph mode: one whole step (every layer's launches) captured once
+    # and replayed K times; the per-layer split then comes from one eager
+    # step with events after the timed region
+    use_graph = graph_mode(args, w)
     for _ in range(args.warmup):
         step()
     barrier()
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        graph.replay()
+        barrier()
     c0 = led.read()["counters"].clone()
     K = args.steps
-    evs = [{n: make_events(L) for n in ("start", "compact", "refresh", "end")} for _ in range(K)]
+    K_ev = 1 if use_graph else K
+    evs = [{n: make_events(L) for n in ("start", "compact", "refresh", "end")} for _ in range(K_ev)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(smi_id(device) if args.smi_index is None else args.smi_index) as clk:
         barrier()
         t_start.record(stream)
         for s in range(K):
-            step(evs[s])
+            if graph is not None:
+                graph.replay()
+            else:
+                step(evs[s])
         t_end.record(stream)
         barrier()
     ms_total = t_start.elapsed_time(t_end)
     c1 = led.read()["counters"].clone()
+    if graph is not None:
+        step(evs[0])
+        barrier()
+        del graph
 
     anchor_layer_ms = relay_layer_ms = rescore_ms = compact_ms = refresh_ms = 0.0
-    for s in range(K):
+    for s in range(K_ev):
         for l in range(L):
             span = evs[s]["start"][l].elapsed_time(evs[s]["end"][l])
             if l in anchors:
@@ -296,11 +325,11 @@ def run_ours(args, w, rank, world, device):
                     rescore_ms += evs[s]["start"][l].elapsed_time(evs[s]["compact"][l])
                     compact_ms += evs[s]["compact"][l].elapsed_time(evs[s]["refresh"][l])
                     refresh_ms += evs[s]["refresh"][l].elapsed_time(evs[s]["end"][l])
-    n_rescore = 0 if oneshot else K * len(relays)
+    n_rescore = 0 if oneshot else K_ev * len(relays)
     # the full-routing stage: anchor layers, and the relay layers' routing
     # (one-shot: the whole relay call; staged: the refresh launches)
     route_ms = anchor_layer_ms + (relay_layer_ms if oneshot else refresh_ms)
-    n_route = K * L
+    n_route = K_ev * L
 
     ms_step = max_over_ranks(ms_total / K, world, device)
 
@@ -319,7 +348,7 @@ def run_ours(args, w, rank, world, device):
     esz = 2 if w.dtype == "bf16" else 4
     # dominant kernel: full routing (anchor + refresh).  Algorithmic work =
     # one multiply-add per (row, valid key, dim) -> 2*d flops per score pair.
-    route_flops = 2.0 * w.d * full_pairs_per_step * K
+    route_flops = 2.0 * w.d * full_pairs_per_step * K_ev
     route_tflops = route_flops / (route_ms * 1e-3) / 1e12
     if uses_tensor_cores(w):
         peak = float(peaks["bf16_tflops_sustained"])
@@ -338,7 +367,7 @@ def run_ours(args, w, rank, world, device):
         per_row = profiled_traffic_per_row("rr_select_tc.cu", "route_select_kernel__*.md")
         if per_row is not None and n_route:
             rows_routed = (w.bh * w.n * L) if oneshot else refreshed_per_step
-            traffic = round(per_row * rows_routed * K / n_route)   # bytes per launch
+            traffic = round(per_row * rows_routed * K_ev / n_route)   # bytes per launch
     roofline.update({"achieved": round(route_tflops, 3), "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(route_tflops / peak, 4), "traffic": traffic,
                      "avg_launch_ms": round(route_ms / max(n_route, 1), 4),
@@ -374,8 +403,11 @@ def run_ours(args, w, rank, world, device):
         "score_pairs_per_s": pairs_all / (ms_step * 1e-3),
         "pair_fraction": pairs_all / (full_pairs_per_layer(w) * L * world),
         "rho_relay": rho,
-        "layer_kinds": layer_kinds(w.bh * w.n, anchor_layer_ms, K * len(anchors), relay_layer_ms,
-                                   K * len(relays)),
+        "layer_kinds": layer_kinds(w.bh * w.n, anchor_layer_ms, K_ev * len(anchors), relay_layer_ms,
+                                   K_ev * len(relays)),
+        "timing": ("CUDA graph of the whole step, replayed K times; layer_kinds and roofline from one "
+                   "eager step with per-layer events after the timed region" if use_graph else
+                   "eager launches; per-layer events on the launching stream"),
         "retry_rows_per_step": retry_all,
         "relay": "one-shot (rr_relay_layer)" if oneshot else "staged (rescore, compact, refresh)",
         "roofline": roofline,
@@ -524,6 +556,36 @@ def measure_attention(args, w, state, device):
             "visible_pairs": pairs, "launches": n}
 
 
+RECALL_KIND = ("GPU vs GPU: the relayed ledger's routes against a second GPU ledger that fully routes "
+               "every layer (anchor interval 1), all rows, mean over layers; full routing itself is "
+               "checked against the oracle (parity tests; oracle_sample on sampled heads)")
+
+SMALL_WORKLOADS = (W.PR1, W.C2, W.C3, W.C4)
+
+
+def per_workload(args, device, oracle_leg: bool) -> dict:
+    """The four smaller workloads, one GPU each in turn, each timed the same
+    way as the headline one (a CUDA graph of the whole step for the
+    CUDA-core path), with recall and, when the CPU leg runs, the oracle
+    sample."""
+    keys = ("value", "unit", "ms_per_step", "steps", "score_pairs_per_s", "pair_fraction", "rho_relay",
+            "layer_kinds", "retry_rows_per_step", "roofline", "gpu_launches", "timing", "dtype", "config",
+            "clocks")
+    out = {}
+    for w in SMALL_WORKLOADS:
+        sub = argparse.Namespace(**{**vars(args), "steps": max(args.steps, 20), "relay": "oneshot"})
+        res, state = run_ours(sub, w, 0, 1, device)
+        entry = {k: res[k] for k in keys}
+        r_mean, r_min = measure_recall(w, state, device)
+        entry.update({"recall": r_mean, "recall_min_layer": r_min, "recall_kind": RECALL_KIND})
+        if oracle_leg:
+            entry["oracle_sample"] = oracle_sample(w, state)
+        out[w.name] = entry
+        del state
+        torch.cuda.empty_cache()
+    return out
+
+
 # ------------------------------------------------------- CPU baseline ------
 def cpu_baseline(w, qs, ks, threads=None, layers=2):
     """The oracle as it stands, on a bounded sample: `threads` heads (one per
@@ -546,6 +608,60 @@ def cpu_baseline(w, qs, ks, threads=None, layers=2):
             "sample": f"{T} heads x {layers} layers (anchor, relay) of {w.name}, one head per thread, "
                       f"{dt:.1f} s wall on {ncpu} host cores",
             "cpu_model": cpu_model()}
+
+
+def oracle_sample(w, state, heads=None, layers=(0, 1)):
+    """Tie-margin and mismatch counts at the bench's own size: after the
+    timed region, layers 0 (anchor) and 1 (relay) go through the GPU ledger
+    once more, and on the sampled heads each is compared with the oracle
+    started from the GPU's previous ledger (the parity tests' comparison:
+    ids, order, alpha, flags and anchor layers row by row; rows whose
+    deciding score gap is below 1e-5 x scale are counted as ties and only
+    checked for validity).  Also the oracle's recall of the relayed routes
+    at the relay layer against its own exact top-k on those heads."""
+    import numpy as np
+
+    import oracle
+    tests_dir = os.path.join(ROOT, "tests")
+    if tests_dir not in sys.path:
+        sys.path.insert(0, tests_dir)
+    import rr_parity
+
+    led, qs, ks, cfg = state
+    heads = sorted({0, w.bh - 1}) if heads is None else list(heads)
+    p = rr_parity.params_of(w)
+    rep = rr_parity.Report()
+    hits = tot = 0
+    prev = None
+    t0 = time.perf_counter()
+    for l in layers:
+        led.layer(qs[l], ks[l], l)
+        dv = led.device_view()
+        after = {n: dv[n][heads].cpu().numpy() for n in ("ids", "alpha", "anchor_layer", "flags")}
+        anchor = oracle.is_anchor(l, w.anchor_interval)
+        for j, h in enumerate(heads):
+            q = qs[l][h].float().cpu().numpy()
+            k = ks[l][h].float().cpu().numpy()
+            pv = (lambda n: None) if prev is None else (lambda n: prev[n][j])
+            rep.add(rr_parity.compare_head(p, cfg.bh_offset + h, l, anchor, q, k, pv("ids"), pv("alpha"),
+                                           pv("anchor_layer"), after["ids"][j], after["alpha"][j],
+                                           after["anchor_layer"][j], after["flags"][j],
+                                           prev_flags=pv("flags")))
+            if not anchor:
+                exact = oracle.exact_topk(p, q, k)
+                used = after["ids"][j][:, :w.k]
+                valid = exact >= 0
+                hits += int(((used[:, :, None] == exact[:, None, :]).any(1) & valid).sum())
+                tot += int(valid.sum())
+        prev = after
+    dt = time.perf_counter() - t0
+    mism = [m for m in rep.mismatches if m is not None]
+    return {"heads": heads, "layers": list(layers), "rows": rep.rows, "compared": rep.compared,
+            "ties": rep.ties, "tie_route": rep.tie_route, "tie_flag": rep.tie_flag,
+            "tie_identical": rep.tie_identical, "mismatches": len(rep.mismatches),
+            "first_mismatches": [list(map(str, m)) for m in mism[:3]],
+            "oracle_recall_relay_layer": (hits / tot) if tot else None,
+            "seconds": round(dt, 1)}
 
 
 def cpu_model() -> str:
@@ -599,6 +715,41 @@ def run_reference(args, w):
             "e2e": {"value": v, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launcher_command(argv, n: int, port: int) -> list:
+    """The command that runs this script as n ranks on one node (one rank
+    per GPU), with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__)] + list(argv)
+
+
+def resolve_world(args, env=None, device_count=None):
+    """How this process runs --gpus N: ("run", world) to go on in this process
+    as one of `world` ranks, ("launch", n) to start n ranks through the
+    launcher, or ("fail", message).  A launcher's WORLD_SIZE must equal
+    --gpus; without a launcher, --gpus N > 1 starts N ranks (never a silent
+    single rank), and needs N visible GPUs.  The reference arm's work is rank
+    0's alone, so it runs in place."""
+    env = os.environ if env is None else env
+    if "WORLD_SIZE" in env:
+        world = int(env["WORLD_SIZE"])
+        if world != args.gpus:
+            return ("fail", f"--gpus {args.gpus} but the launcher started {world} ranks")
+        return ("run", world)
+    if args.gpus <= 1 or args.impl == "reference":
+        return ("run", 1)
+    n_dev = torch.cuda.device_count() if device_count is None else device_count
+    if n_dev < args.gpus:
+        return ("fail", f"--gpus {args.gpus} needs {args.gpus} visible GPUs, found {n_dev}")
+    return ("launch", args.gpus)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -613,6 +764,12 @@ def main():
                     help="also time the sparse attention over the ledger's routes (not part of the step)")
     ap.add_argument("--relay", default="oneshot", choices=["oneshot", "staged"],
                     help="tensor-core path: time relay layers as one rr_relay_layer call or as its three stages")
+    ap.add_argument("--graph", default="auto", choices=["auto", "on", "off"],
+                    help="replay the timed step from a CUDA graph (auto: for the CUDA-core workloads)")
+    ap.add_argument("--per-workload", default="auto", choices=["auto", "on", "off"],
+                    help="also measure the four smaller workloads (auto: on for the default run on one GPU)")
+    ap.add_argument("--no-oracle-sample", action="store_true",
+                    help="skip the tie/mismatch count against the oracle on sampled heads")
     ap.add_argument("--smi-index", type=int, default=None)
     ap.add_argument("--bh", type=int, default=None, help="override BH (profiling a smaller case)")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
@@ -624,7 +781,15 @@ def main():
     if args.layers is not None:
         w = w.with_(layers=args.layers, name=f"{w.name}@L{args.layers}")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.gpus < 1:
+        ap.error("--gpus must be at least 1")
+    how, val = resolve_world(args)
+    if how == "fail":
+        print(f"bench.py: {val}", file=sys.stderr, flush=True)
+        return 2
+    if how == "launch":
+        return subprocess.call(launcher_command(sys.argv[1:], val, free_port()))
+    world = val
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 
@@ -644,6 +809,7 @@ def main():
         r_mean, r_min = measure_recall(w, state, device)
         result["recall"] = r_mean
         result["recall_min_layer"] = r_min
+        result["recall_kind"] = RECALL_KIND
     if args.attention and rank == 0:
         result["kernels"]["attention"] = measure_attention(args, w, state, device)
     if not args.no_e2e:
@@ -653,11 +819,19 @@ def main():
             e2e["value"] = w.bh * w.n * w.layers * world / (e2e["ms_per_step"] * 1e-3)
         result["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        led, qs, ks, cfg = state
-        result["cpu_baseline"] = cpu_baseline(w, qs, ks)
-        one = cpu_baseline(w, qs, ks, threads=1)
+        result["cpu_baseline"] = cpu_baseline(w, state[1], state[2])
+        one = cpu_baseline(w, state[1], state[2], threads=1)
         result["cpu_baseline"]["single_thread"] = {"value": one["value"], "unit": one["unit"],
                                                    "sample": one["sample"]}
+        if not args.no_oracle_sample:
+            result["oracle_sample"] = oracle_sample(w, state)
+    del state
+    if world == 1 and (args.per_workload == "on" or (
+            args.per_workload == "auto" and args.workload == W.C5.name and args.bh is None
+            and args.layers is None)):
+        torch.cuda.empty_cache()
+        result["per_workload"] = per_workload(args, device, oracle_leg=not args.no_cpu_baseline
+                                              and not args.no_oracle_sample)
     if rank == 0:
         print(json.dumps(result), flush=True)
     if world > 1:

@@ -81,3 +81,49 @@ def test_cpu_baseline_runs_the_oracle_on_a_bounded_sample():
     cb = bench.cpu_baseline(W.PR1, qs, ks, threads=1, layers=2)
     assert cb["kind"] == "oracle" and cb["unit"] == "rows/s" and cb["cores"] == 1 and cb["value"] > 0
     assert "1 heads x 2 layers" in cb["sample"] and isinstance(cb["cpu_model"], str)
+
+
+def _args(gpus, impl="ours"):
+    import argparse
+    return argparse.Namespace(gpus=gpus, impl=impl)
+
+
+def test_gpus_n_without_a_launcher_starts_n_ranks_or_fails():
+    # N > 1 and no launcher: start N ranks when N GPUs are visible, else fail
+    assert bench.resolve_world(_args(2), env={}, device_count=8) == ("launch", 2)
+    how, why = bench.resolve_world(_args(2), env={}, device_count=1)
+    assert how == "fail" and "--gpus 2" in why
+    assert bench.resolve_world(_args(1), env={}, device_count=0) == ("run", 1)
+    # under a launcher the rank count must be --gpus
+    assert bench.resolve_world(_args(4), env={"WORLD_SIZE": "4"}) == ("run", 4)
+    assert bench.resolve_world(_args(4), env={"WORLD_SIZE": "2"})[0] == "fail"
+    assert bench.resolve_world(_args(1), env={"WORLD_SIZE": "2"})[0] == "fail"
+    # the reference arm is rank 0's work: it runs in place and reports --gpus
+    assert bench.resolve_world(_args(8, "reference"), env={}, device_count=0) == ("run", 1)
+    cmd = bench.launcher_command(["--gpus", "2", "--steps", "3"], 2, 29555)
+    assert cmd[1:3] == ["-m", "torch.distributed.run"] and "--nproc-per-node=2" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1" and cmd[cmd.index("--master-port") + 1] == "29555"
+    assert cmd[-4:] == ["--gpus", "2", "--steps", "3"] and cmd[-5].endswith("bench.py")
+
+
+def test_bench_gpus_2_never_runs_a_single_rank_silently():
+    """The script itself, as the driver would start it without torchrun: on a
+    host with fewer than two GPUs it must exit non-zero and print no result
+    line (a one-rank line labelled n_gpus 1 is what this guards against)."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in __import__("os").environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    env["CUDA_VISIBLE_DEVICES"] = ""
+    p = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--steps", "1"], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert p.returncode != 0
+    assert '"metric"' not in p.stdout and "--gpus 2" in p.stderr
+
+
+def test_graph_mode_default_follows_the_kernel_path():
+    import argparse
+    a = argparse.Namespace(graph="auto")
+    assert bench.graph_mode(a, W.C2) and bench.graph_mode(a, W.PR1) and not bench.graph_mode(a, W.C5)
+    assert bench.graph_mode(argparse.Namespace(graph="on"), W.C5)
+    assert not bench.graph_mode(argparse.Namespace(graph="off"), W.C2)
