@@ -158,9 +158,17 @@ def profiled_traffic_per_row(kernel_file: str, summary_glob: str):
 
 
 def uses_tensor_cores(w) -> bool:
-    """Which full-routing kernel the library runs for this workload (the
-    rule of route_rows_prepare: bf16, d in {64, 128}, k + m <= 64, r <= 32)."""
-    return w.dtype == "bf16" and w.d in (64, 128) and w.k + w.m <= 64 and w.r <= 32
+    """Which full-routing kernel the library runs for this workload: the
+    selection kernel on the tensor cores for bf16 with d in {64, 128} and for
+    fp32 with d = 64 (three-way bf16 split), when k + m <= 64 and r <= 32;
+    the CUDA-core kernel otherwise."""
+    return ((w.dtype == "bf16" and w.d in (64, 128)) or (w.dtype == "f32" and w.d == 64)) \
+        and w.k + w.m <= 64 and w.r <= 32
+
+
+def uses_split(w) -> bool:
+    """fp32 on the tensor cores: Qc, Kc split into three bf16 parts each."""
+    return uses_tensor_cores(w) and w.dtype == "f32"
 
 
 def shard_offset(rank: int, w) -> int:
@@ -203,20 +211,23 @@ def launches_per_step(w, n_anchor: int, n_relay: int, oneshot: bool) -> int:
     """Our kernels launched by one step.  Tensor-core path: anchor = select,
     finish, heap retry, counters (4); one-shot relay = select, finish, exact
     rescoring, heap retry, counters (5); staged relay = rescore, compact,
-    select, finish, heap retry, counters (6).  CUDA-core path: anchor = route,
-    counters (2); relay = rescore, compact, route, counters (4)."""
+    select, finish, heap retry, counters (6); fp32 split: one more per
+    routing call (the key split; the retry runs on the CUDA cores).
+    CUDA-core path: anchor = route, counters (2); relay = rescore, compact,
+    route, counters (4)."""
     if uses_tensor_cores(w):
-        return 4 * n_anchor + (5 if oneshot else 6) * n_relay
+        x = 1 if uses_split(w) else 0
+        return (4 + x) * n_anchor + ((5 if oneshot else 6) + x) * n_relay
     return 2 * n_anchor + 4 * n_relay
 
 
 def graph_mode(args, w) -> bool:
     """Whether the timed step is replayed from a CUDA graph: always with
-    --graph on, never with --graph off, and by default for the CUDA-core
-    workloads, whose layers take microseconds and would otherwise time the
-    launch path."""
+    --graph on, never with --graph off, and by default for the workloads of
+    fewer than 2^19 rows per layer, whose layers take microseconds to tens of
+    microseconds and would otherwise time the launch path."""
     if args.graph == "auto":
-        return not uses_tensor_cores(w)
+        return w.bh * w.n < (1 << 19)
     return args.graph == "on"
 
 
@@ -350,7 +361,15 @@ def run_ours(args, w, rank, world, device):
     # one multiply-add per (row, valid key, dim) -> 2*d flops per score pair.
     route_flops = 2.0 * w.d * full_pairs_per_step * K_ev
     route_tflops = route_flops / (route_ms * 1e-3) / 1e12
-    if uses_tensor_cores(w):
+    if uses_split(w):
+        # six bf16 products per fp32 product: the arithmetic's own peak is the
+        # bf16 dense peak / 6
+        peak = float(peaks["bf16_tflops_sustained"]) / 6.0
+        roofline = {"kernel": "full routing, fp32 split in three bf16 parts: split_keys_kernel + "
+                              "route_select_kernel + route_finish_kernel (+ exact rescoring at relay layers)",
+                    "bound": "tensor",
+                    "peak_source": f"{peaks['source']} bf16 dense, sustained, / 6 (six bf16 MMAs per fp32 product)"}
+    elif uses_tensor_cores(w):
         peak = float(peaks["bf16_tflops_sustained"])
         what = ("route_select_kernel (tcgen05, query tile in TMEM, two-pass selection) + route_finish_kernel"
                 " + exact/heap fallbacks; anchor and relay layers (relay test taken from the kept scores)"
@@ -363,7 +382,7 @@ def run_ours(args, w, rank, world, device):
         roofline = {"kernel": "route_rows (CUDA cores; anchor + refresh)", "bound": "alu",
                     "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock"}
     traffic = None
-    if uses_tensor_cores(w):
+    if uses_tensor_cores(w) and not uses_split(w):
         per_row = profiled_traffic_per_row("rr_select_tc.cu", "route_select_kernel__*.md")
         if per_row is not None and n_route:
             rows_routed = (w.bh * w.n * L) if oneshot else refreshed_per_step
@@ -381,7 +400,7 @@ def run_ours(args, w, rank, world, device):
         rescore = {"bound": "hbm", "achieved_gbs": round(rescore_gbs, 1), "peak_gbs": peaks["hbm_gbs"],
                    "frac": round(rescore_gbs / peaks["hbm_gbs"], 4),
                    "avg_launch_ms": round(rescore_ms / max(n_rescore, 1), 4)}
-        if uses_tensor_cores(w):
+        if uses_tensor_cores(w) and not uses_split(w):
             # dense tiles: every valid pair of the row block is scored (2*d flops per pair)
             dense_tflops = 2.0 * w.d * full_pairs_per_layer(w) * n_rescore / (rescore_ms * 1e-3) / 1e12
             rescore = {"kernel": "relay_rescore_tc_kernel (tcgen05 dense tiles)", "bound": "tensor",

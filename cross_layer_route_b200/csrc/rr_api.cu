@@ -37,8 +37,8 @@ size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
 struct Layout {
     size_t ids, alpha, anchor_layer, flags, counters, list, head_count, retry_list, retry_count;
     // tensor-core selection path only (size 0 otherwise)
-    size_t cand_keys, cand_masks, cand_meta, und_list, und_count;
-    bool cand;
+    size_t cand_keys, cand_masks, cand_meta, und_list, und_count, ksplit;
+    bool cand, split;
     size_t total;
 };
 
@@ -83,6 +83,8 @@ Layout layout_of(const rr_config *c) {
     L.cand_meta = o;    o = align_up(o + cs.meta);
     L.und_list = o;     o = align_up(o + cs.und);
     L.und_count = o;    o = align_up(o + (L.cand ? sizeof(int32_t) : 0));
+    L.ksplit = o;       o = align_up(o + cs.ksplit);
+    L.split = cs.ksplit > 0;
     L.total = o;
     return L;
 }
@@ -249,6 +251,10 @@ rr_status rr_ledger_create(const rr_config *cfg, void *d_workspace, size_t bytes
         D.cand_meta = reinterpret_cast<uint2 *>(L->ws + lay.cand_meta);
         D.und_list = reinterpret_cast<int32_t *>(L->ws + lay.und_list);
         D.und_count = reinterpret_cast<int32_t *>(L->ws + lay.und_count);
+    }
+    if (lay.split) {
+        D.ksplit = reinterpret_cast<uint16_t *>(L->ws + lay.ksplit);
+        D.split = 1;
     }
     D.mt = (cfg->nk + 127) / 128;
     D.bh = cfg->bh; D.nq = cfg->nq; D.nk = cfg->nk; D.d = cfg->d;

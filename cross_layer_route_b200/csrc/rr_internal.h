@@ -30,6 +30,10 @@ struct LedgerDev {
     uint2 *cand_meta = nullptr;      // [slots] {kept keys (all ones: redo the row), threshold}
     int32_t *und_list = nullptr;     // [bh*nq] relay rows whose test needs exact rescoring
     int32_t *und_count = nullptr;    // [1]
+    // fp32 problems on the tensor cores: Kc split into three bf16 parts per
+    // element (hi, mid, lo: x = hi + mid + lo exactly), rows [hi | mid | lo]
+    uint16_t *ksplit = nullptr;      // [bh, nk, 3 d] bf16 bits
+    int split = 0;                   // 1: the selection kernel takes fp32 Qc/Kc split in three
     int mt = 0;                      // key tiles per head: ceil(nk / 128)
     int bh, nq, nk, d;
     int k, m, r, c, ksel;   // ksel = k + m; c = k + m + r + g_sink + g_recent
@@ -84,9 +88,19 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
 // Tensor-core selection path (rr_select_tc.cu): the selection kernel writes
 // every row's kept scores to the candidate buffers, the finishing kernel
 // orders them and writes the ledger row.
-struct CandSizes { size_t keys, masks, meta, und; };
+struct CandSizes { size_t keys, masks, meta, und, ksplit; };
 // Bytes of the buffers (all 0 when the problem does not run on the tensor cores).
 CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype);
+// fp32 problems the selection kernel takes with three-way bf16 splitting
+// (d = 64, the same selection limits as the bf16 path).
+bool route_select_split_supported(const LedgerDev &L, int dtype);
+// Full routing of fp32 rows on the tensor cores (L.split): split Kc, select,
+// finish; rows whose kept scores overflow are rebuilt on the CUDA cores.
+cudaError_t launch_route_rows_split(const LedgerDev &L, const void *q, const void *k, int layer,
+                                    bool use_list, cudaStream_t s);
+// The CUDA-core route kernel alone (rr_route_simt.cu), whatever the problem.
+cudaError_t launch_route_rows_simt(const LedgerDev &L, int dtype, const void *q, const void *k,
+                                   int layer, bool use_list, cudaStream_t s);
 size_t route_select_smem_bytes(const LedgerDev &L);
 cudaError_t route_select_prepare();
 // kAnchor: every row (or every listed row) is rebuilt.  kRelay: every row
@@ -107,6 +121,8 @@ cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *
 namespace tc {
 // Tensor map of Kc [bh, nk, d] bf16: boxes of 128 keys x 64 dims, 128-byte swizzle.
 cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map);
+// The same over bf16 key rows of row_elems elements (row_elems a multiple of 64).
+cudaError_t key_rows_tensor_map(const void *k, int row_elems, int nk, int bh, CUtensorMap *map);
 }
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s);

@@ -282,11 +282,16 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
     if (route_rows_tc_supported(L, dtype)) return route_rows_tc_prepare();
     const int smem = (int)smem_layout(L.d, select_capacity(L.ksel)).total;
+    cudaError_t e;
     if (dtype == kBF16)
-        return cudaFuncSetAttribute(route_rows_kernel<__nv_bfloat16>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    return cudaFuncSetAttribute(route_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                smem);
+        e = cudaFuncSetAttribute(route_rows_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem);
+    else
+        e = cudaFuncSetAttribute(route_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // split fp32 problems: the selection kernel, with this kernel for the
+    // rows whose kept scores overflow
+    if (e == cudaSuccess && L.split) e = route_select_prepare();
+    return e;
 }
 
 cudaError_t route_rows_prepare_all() {
@@ -303,6 +308,13 @@ cudaError_t route_rows_prepare_all() {
 cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, const void *k,
                               int layer, bool use_list, cudaStream_t s) {
     if (route_rows_tc_supported(L, dtype)) return launch_route_rows_tc(L, q, k, layer, use_list, s);
+    if (dtype == kF32 && L.split && L.cand_keys && L.ksplit)
+        return launch_route_rows_split(L, q, k, layer, use_list, s);
+    return launch_route_rows_simt(L, dtype, q, k, layer, use_list, s);
+}
+
+cudaError_t launch_route_rows_simt(const LedgerDev &L, int dtype, const void *q, const void *k,
+                                   int layer, bool use_list, cudaStream_t s) {
     const int cap = select_capacity(L.ksel);
     const size_t smem = smem_layout(L.d, cap).total;
     dim3 grid((L.nq + kTileRows - 1) / kTileRows, L.bh);

@@ -873,10 +873,14 @@ static EncodeTiledFn encode_fn() {
 }
 
 cudaError_t key_tensor_map(const LedgerDev &L, const void *k, CUtensorMap *map) {
+    return key_rows_tensor_map(k, L.d, L.nk, L.bh, map);
+}
+
+cudaError_t key_rows_tensor_map(const void *k, int row_elems, int nk, int bh, CUtensorMap *map) {
     EncodeTiledFn enc = encode_fn();
-    if (!enc) return cudaErrorNotSupported;
-    const cuuint64_t dims[3] = {(cuuint64_t)L.d, (cuuint64_t)L.nk, (cuuint64_t)L.bh};
-    const cuuint64_t strides[2] = {(cuuint64_t)L.d * 2, (cuuint64_t)L.nk * L.d * 2};
+    if (!enc || row_elems % 64 != 0) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)row_elems, (cuuint64_t)nk, (cuuint64_t)bh};
+    const cuuint64_t strides[2] = {(cuuint64_t)row_elems * 2, (cuuint64_t)nk * row_elems * 2};
     const cuuint32_t box[3] = {64u, (cuuint32_t)kKeys, 1u};
     const cuuint32_t estr[3] = {1u, 1u, 1u};
     const CUresult cr = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(k), dims,

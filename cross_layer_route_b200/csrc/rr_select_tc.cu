@@ -44,6 +44,8 @@
 // the ledger that comes out is the one the pages' two-stage procedure
 // defines, and the counters follow the pages' counting rule (c candidates per
 // relay row plus the valid keys of every refreshed row).
+#include <algorithm>
+
 #include "rr_tc.cuh"
 
 namespace rr {
@@ -52,8 +54,8 @@ namespace tc {
 constexpr int kSelEpiWarps = 16;
 constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
 constexpr int kSelAcc = 2;                       // accumulators (TMEM columns 0..255)
-constexpr uint32_t kQCol = kSelAcc * 128;        // query tile (A operand): 64 columns at most
-constexpr uint32_t kMaskCol = kQCol + 64;        // kept-column masks: [quarter][tile], 128 columns
+constexpr uint32_t kQCol = kSelAcc * 128;        // query tile (A operand): 96 columns at most
+constexpr uint32_t kMaskCol = kQCol + 96;        // kept-column masks: [quarter][tile], 128 columns
 constexpr int kMaskTiles = 32;                   // blocks with more key tiles keep masks in device memory
 constexpr int kPairCap = 92;                     // kept-score slots shared by two quarters of a row
 constexpr int kValStride = kRows + 1;            // padded (slot, row) grid of the kept scores
@@ -70,14 +72,19 @@ struct SelLayout {
     __host__ __device__ CtaLayout cta() const { return CtaLayout{0u, k, rows, bars, misc, stages}; }
 };
 
-// k (key ring, 128 KB; after pass 1 the masks [tile][epilogue thread] u32
-// and the chunk grid [2][kPairCap][kChunkStride] u16) | vals [2][kPairCap][kValStride] f32 (before pass 1 the group maxima
-// [kRows][kTopWords] u32) | rows | thr | cnt | barriers | misc
-__host__ __device__ inline SelLayout sel_layout(int d) {
+constexpr uint32_t kRingBytes = 128 * 1024;
+
+// k (key ring, 128 KB: as many stages of 128 key rows x dk bf16 as fit, at
+// most 8; after pass 1 the masks [tile][epilogue thread] u32 and the chunk
+// grid [2][kPairCap][kChunkStride] u16) | vals [2][kPairCap][kValStride] f32
+// (before pass 1 the group maxima [kRows][kTopWords] u32) | rows | thr | cnt
+// | barriers | misc.  dk: bf16 elements per key row (d, or 3 d for split fp32).
+__host__ __device__ inline SelLayout sel_layout(int dk) {
     SelLayout s;
-    s.stages = d == 64 ? 8 : 4;
+    s.stages = (int)(kRingBytes / (uint32_t)(kKeys * dk * 2));
+    if (s.stages > kMaxStages) s.stages = kMaxStages;
     uint32_t o = 0;
-    s.k = o;    o = up(o + s.stages * kKeys * d * 2, 1024);
+    s.k = o;    o = up(o + kRingBytes, 1024);
     s.vals = o; o = up(o + 2 * kPairCap * kValStride * 4, 16);
     s.rows = o; o = up(o + kRows * 4, 16);
     s.thr = o;  o = up(o + kRows * 4, 16);
@@ -87,7 +94,7 @@ __host__ __device__ inline SelLayout sel_layout(int d) {
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
 }
-static_assert(kKeys * 128 * 2 * 4 >= kMaskBytes + 2 * kPairCap * kChunkStride * 2,
+static_assert(kRingBytes >= kMaskBytes + 2 * kPairCap * kChunkStride * 2,
               "the key ring holds the masks and the chunk grid");
 
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t *r) {
@@ -140,6 +147,20 @@ __device__ __forceinline__ uint64_t sel_key(float v, int j) {
 __device__ __forceinline__ int sel_key_chunk(uint64_t key) { return (int)(0xffffu - (uint32_t)(key & 0xffffu)); }
 __device__ __forceinline__ float sel_key_score(uint64_t key) { return unord32((uint32_t)(key >> 32)); }
 
+// x = hi + mid + lo with each part a bf16 (round to nearest even at every
+// step; each remainder is exact in fp32, and the third part takes the last
+// 8 significant bits).  Bits of hi, mid, lo in b[0..2].
+__device__ __forceinline__ void split3_bf16(float x, uint32_t *b) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(x);
+    const float r1 = x - __bfloat162float(h);
+    const __nv_bfloat16 m = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(m);
+    const __nv_bfloat16 l = __float2bfloat16_rn(r2);
+    b[0] = (uint32_t)__bfloat16_as_ushort(h);
+    b[1] = (uint32_t)__bfloat16_as_ushort(m);
+    b[2] = (uint32_t)__bfloat16_as_ushort(l);
+}
+
 // MMA issuer of the selection kernel (the whole warp; one elected lane
 // issues): A (the query tile) from TMEM.
 template <int kSteps>
@@ -151,10 +172,32 @@ __device__ __forceinline__ void sel_mma_tile(uint32_t d_tmem, uint32_t a_tmem, u
     }
 }
 
-__device__ __forceinline__ void sel_mma_issuer(Cta &c, int d) {
+// Split fp32 (d = 64): the query row is [q_hi | q_mid | q_lo] in TMEM (32
+// columns per part) and the key row [k_hi | k_mid | k_lo] in three 64-wide
+// sub-tiles; the score is the sum of the six part products whose orders add
+// up to at most two (hi = order 0), smallest first: mid.mid, hi.lo, lo.hi,
+// hi.mid, mid.hi, hi.hi.  With |mid| <= 2^-8 |x| and |lo| <= 2^-16 |x|,
+// the dropped products mid.lo and lo.mid are each at most 2^-24 |q_t| |k_t|
+// and lo.lo at most 2^-32 |q_t| |k_t|: together at most 2^-23 |q| |k| per
+// score, below the fp32 rounding of the sum itself.
+__device__ __forceinline__ void sel_mma_tile_split(uint32_t d_tmem, uint32_t a_tmem, uint64_t kdesc) {
+    constexpr int kPa[6] = {1, 0, 2, 0, 1, 0};
+    constexpr int kPb[6] = {1, 2, 0, 1, 0, 0};
+#pragma unroll
+    for (int p = 0; p < 6; ++p) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t off16 = (uint64_t)(kPb[p] * (kSubTileBytes >> 4) + kk * 2);
+            tc_mma_bf16_ts_elect(d_tmem, a_tmem + (uint32_t)(kPa[p] * 32 + kk * 8), kdesc + off16, kIdesc,
+                                 (p > 0 || kk > 0) ? 1u : 0u);
+        }
+    }
+}
+
+__device__ __forceinline__ void sel_mma_issuer(Cta &c, int dk, int split) {
     const int total = 2 * c.ntiles;
     const uint32_t k_addr = saddr(c.k_s);
-    const uint32_t stage_bytes = (uint32_t)(kKeys * d * 2);
+    const uint32_t stage_bytes = (uint32_t)(kKeys * dk * 2);
     const uint32_t tmem = __shfl_sync(kFull, c.tmem_base, 0);
     const uint32_t a_tmem = tmem + kQCol;
     for (int g = 0; g < total; ++g) {
@@ -164,7 +207,8 @@ __device__ __forceinline__ void sel_mma_issuer(Cta &c, int d) {
         tc_fence_after();
         const uint32_t d_tmem = tmem + (uint32_t)(a * kKeys);
         const uint64_t kdesc = sw128_desc(k_addr + (uint32_t)s * stage_bytes);
-        if (d == 128) sel_mma_tile<8>(d_tmem, a_tmem, kdesc);
+        if (split) sel_mma_tile_split(d_tmem, a_tmem, kdesc);
+        else if (dk == 128) sel_mma_tile<8>(d_tmem, a_tmem, kdesc);
         else sel_mma_tile<4>(d_tmem, a_tmem, kdesc);
         tc_commit_elect(&c.empty[s]);
         tc_commit_elect(&c.acc_full[a]);
@@ -177,12 +221,15 @@ __device__ __forceinline__ void sel_mma_issuer(Cta &c, int d) {
 
 // ---- selection kernel ------------------------------------------------------------
 __global__ void __launch_bounds__(kSelThreads, 1)
-route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
+route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
                     const __grid_constant__ CUtensorMap tmap_k, int use_list) {
     extern __shared__ __align__(1024) unsigned char smem_dyn[];
     unsigned char *smem = align_smem_1024(smem_dyn);
     const int d = L.d, ksel = L.ksel;
-    const SelLayout lay = sel_layout(d);
+    const int split = L.split;
+    const int dk = split ? 3 * d : d;   // bf16 elements per key row in the ring
+    const SelLayout lay = sel_layout(dk);
+    const __nv_bfloat16 *Q = static_cast<const __nv_bfloat16 *>(Qv);
     Cta c;
     if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, use_list, /*q_to_smem=*/false))
         return;
@@ -192,11 +239,11 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
     // The producer starts at once; the MMA warp waits until the epilogue
     // warps have put the query tile into TMEM (barrier q_ready).
     if (warp == 0) {
-        producer(c, &tmap_k, d, h, 2);
+        producer(c, &tmap_k, dk, h, 2);
     } else if (warp == 1) {
         if (mbar_wait_warp(c.q_ready, 0, c.abort_flag)) {
             tc_fence_after();
-            sel_mma_issuer(c, d);
+            sel_mma_issuer(c, dk, split);
         }
     } else {
         // the query tile into TMEM columns kQCol.. (row r in lane r, two
@@ -211,7 +258,31 @@ route_select_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q,
             uint32_t w[16];
             const uint4 *src = reinterpret_cast<const uint4 *>(
                 Q + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d + qt * (d >> 2));
-            if (d == 128) {
+            if (split) {
+                // fp32 elements 16 qt .. 16 qt + 15, each split into bf16
+                // hi + mid + lo (x = hi + mid + lo exactly); part p goes to
+                // columns 32 p + 8 qt .. 32 p + 8 qt + 7
+                const float4 *srcf = reinterpret_cast<const float4 *>(
+                    static_cast<const float *>(Qv) + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d + qt * 16);
+                uint32_t part[3][8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 v = row >= 0 ? srcf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    const float x[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int e = 0; e < 4; e += 2) {
+                        uint32_t b0[3], b1[3];
+                        split3_bf16(x[e], b0);
+                        split3_bf16(x[e + 1], b1);
+#pragma unroll
+                        for (int p = 0; p < 3; ++p) part[p][2 * i + (e >> 1)] = b0[p] | (b1[p] << 16);
+                    }
+                }
+#pragma unroll
+                for (int p = 0; p < 3; ++p)
+                    tc_st8(c.tmem_base + ((uint32_t)(sub * 32) << 16) + kQCol + (uint32_t)(p * 32 + qt * 8),
+                           part[p]);
+            } else if (d == 128) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
@@ -869,10 +940,48 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
 // rebuilt by the heap kernel.
 constexpr int kExactWarps = 8;
 
+// The candidate's score, fp32 products of the inputs (bf16 rows: 8 elements
+// per 16-byte load; fp32 rows: 4).
 template <int D>
+__device__ __forceinline__ float exact_dot(const float *qv, const __nv_bfloat16 *krow) {
+    const uint4 *kp = reinterpret_cast<const uint4 *>(krow);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+        const uint4 kv = __ldg(kp + c8);
+        const float *q8 = qv + c8 * 8;
+        acc[0] = fmaf(q8[0], __uint_as_float(kv.x << 16), acc[0]);
+        acc[1] = fmaf(q8[1], __uint_as_float(kv.x & 0xffff0000u), acc[1]);
+        acc[2] = fmaf(q8[2], __uint_as_float(kv.y << 16), acc[2]);
+        acc[3] = fmaf(q8[3], __uint_as_float(kv.y & 0xffff0000u), acc[3]);
+        acc[0] = fmaf(q8[4], __uint_as_float(kv.z << 16), acc[0]);
+        acc[1] = fmaf(q8[5], __uint_as_float(kv.z & 0xffff0000u), acc[1]);
+        acc[2] = fmaf(q8[6], __uint_as_float(kv.w << 16), acc[2]);
+        acc[3] = fmaf(q8[7], __uint_as_float(kv.w & 0xffff0000u), acc[3]);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+template <int D>
+__device__ __forceinline__ float exact_dot(const float *qv, const float *krow) {
+    const float4 *kp = reinterpret_cast<const float4 *>(krow);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+    for (int c4 = 0; c4 < D / 4; ++c4) {
+        const float4 kv = __ldg(kp + c4);
+        const float *q4 = qv + c4 * 4;
+        acc[0] = fmaf(q4[0], kv.x, acc[0]);
+        acc[1] = fmaf(q4[1], kv.y, acc[1]);
+        acc[2] = fmaf(q4[2], kv.z, acc[2]);
+        acc[3] = fmaf(q4[3], kv.w, acc[3]);
+    }
+    return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
+
+template <int D, typename T>
 __global__ void __launch_bounds__(32 * kExactWarps)
-relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_bfloat16 *__restrict__ K,
-                   int layer) {
+relay_exact_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K, int layer) {
     __shared__ __align__(16) float qs[kExactWarps][D];
     __shared__ unsigned long long red_cnt[kExactWarps][3];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -882,10 +991,10 @@ relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_
         const int grow = L.und_list[u];
         const int h = grow / L.nq, i = grow - h * L.nq;
         const int n_valid = valid_keys(i, L.nk, L.causal);
-        for (int t = lane; t < D; t += 32) qs[warp][t] = __bfloat162float(Q[(size_t)grow * D + t]);
+        for (int t = lane; t < D; t += 32) qs[warp][t] = to_f32(Q[(size_t)grow * D + t]);
         __syncwarp();
         const int32_t *idr = L.ids + (size_t)grow * L.c;
-        const __nv_bfloat16 *Kh = K + (size_t)h * L.nk * D;
+        const T *Kh = K + (size_t)h * L.nk * D;
         float amin = INFINITY, bmax = -INFINITY;
         int ncand = 0;
         bool bad = false;
@@ -895,22 +1004,7 @@ relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_
             const bool valid = j >= 0 && j < n_valid;
             bad |= j >= n_valid || j < -1;
             if (valid) {
-                const uint4 *kp = reinterpret_cast<const uint4 *>(Kh + (size_t)j * D);
-                float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-                for (int c8 = 0; c8 < D / 8; ++c8) {
-                    const uint4 kv = __ldg(kp + c8);
-                    const float *qv = qs[warp] + c8 * 8;
-                    acc[0] = fmaf(qv[0], __uint_as_float(kv.x << 16), acc[0]);
-                    acc[1] = fmaf(qv[1], __uint_as_float(kv.x & 0xffff0000u), acc[1]);
-                    acc[2] = fmaf(qv[2], __uint_as_float(kv.y << 16), acc[2]);
-                    acc[3] = fmaf(qv[3], __uint_as_float(kv.y & 0xffff0000u), acc[3]);
-                    acc[0] = fmaf(qv[4], __uint_as_float(kv.z << 16), acc[0]);
-                    acc[1] = fmaf(qv[5], __uint_as_float(kv.z & 0xffff0000u), acc[1]);
-                    acc[2] = fmaf(qv[6], __uint_as_float(kv.w << 16), acc[2]);
-                    acc[3] = fmaf(qv[7], __uint_as_float(kv.w & 0xffff0000u), acc[3]);
-                }
-                const float sc = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+                const float sc = exact_dot<D>(qs[warp], Kh + (size_t)j * D);
                 if (e < L.k) amin = fminf(amin, sc);   // Eq. 6
                 else bmax = fmaxf(bmax, sc);           // Eq. 7
                 ++ncand;
@@ -955,17 +1049,44 @@ relay_exact_kernel(LedgerDev L, const __nv_bfloat16 *__restrict__ Q, const __nv_
     }
 }
 
+// Kc fp32 [rows, d] -> bf16 parts [rows, 3 d] = [hi | mid | lo] per row
+// (the split of split3_bf16), four elements per thread.
+__global__ void __launch_bounds__(256) split_keys_kernel(const float4 *__restrict__ K, uint16_t *__restrict__ out,
+                                                         size_t n4, int d4) {
+    for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+        const float4 v = __ldg(K + i);
+        const size_t row = i / (size_t)d4;
+        const int t = (int)(i - row * (size_t)d4) * 4;
+        const float x[4] = {v.x, v.y, v.z, v.w};
+        uint32_t b[4][3];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) split3_bf16(x[e], b[e]);
+        uint16_t *dst = out + row * (size_t)(12 * d4) + t;
+#pragma unroll
+        for (int p = 0; p < 3; ++p)
+            *reinterpret_cast<uint2 *>(dst + p * 4 * d4) =
+                make_uint2(b[0][p] | (b[1][p] << 16), b[2][p] | (b[3][p] << 16));
+    }
+}
+
 }  // namespace tc
 
+bool route_select_split_supported(const LedgerDev &L, int dtype) {
+    return dtype == kF32 && L.d == 64 && L.ksel <= 64 && L.r <= 32 && L.nk <= 65535 && L.c <= 96 &&
+           L.g_sink + L.g_recent <= 32 && route_select_smem_bytes(L) <= 232448;
+}
+
 CandSizes route_select_candidate_sizes(const LedgerDev &L, int dtype) {
-    CandSizes z{0, 0, 0, 0};
-    if (!route_rows_tc_supported(L, dtype)) return z;
+    CandSizes z{0, 0, 0, 0, 0};
+    const bool split = route_select_split_supported(L, dtype);
+    if (!route_rows_tc_supported(L, dtype) && !split) return z;
     const size_t blocks = (size_t)L.bh * ((L.nq + tc::kRows - 1) / tc::kRows);
     const size_t mt = (size_t)((L.nk + tc::kKeys - 1) / tc::kKeys);
     z.keys = blocks * tc::kRows * tc::kRowCap * sizeof(uint64_t);
     z.masks = mt > (size_t)tc::kMaskTiles ? blocks * mt * 4 * tc::kRows * sizeof(uint32_t) : 0;
     z.meta = blocks * tc::kRows * sizeof(uint2);
     z.und = (size_t)L.bh * L.nq * sizeof(int32_t);
+    if (split) z.ksplit = (size_t)L.bh * L.nk * 3 * L.d * sizeof(uint16_t);
     return z;
 }
 
@@ -980,8 +1101,8 @@ cudaError_t route_select_prepare() {
 cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
                                 bool use_list, SelectMode mode, cudaStream_t s) {
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
-    tc::route_select_kernel<<<grid, tc::kSelThreads, tc::sel_layout(L.d).total, s>>>(
-        L, static_cast<const __nv_bfloat16 *>(q), map, use_list ? 1 : 0);
+    tc::route_select_kernel<<<grid, tc::kSelThreads, tc::sel_layout(L.split ? 3 * L.d : L.d).total, s>>>(
+        L, q, map, use_list ? 1 : 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     if (mode == SelectMode::kRelay)
@@ -991,22 +1112,65 @@ cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtenso
     return cudaGetLastError();
 }
 
+namespace {
+
+// Kc of an fp32 problem into its three bf16 parts, and the tensor map of
+// the part rows.
+cudaError_t split_keys(const LedgerDev &L, const void *k, CUtensorMap *map, cudaStream_t s) {
+    const size_t n4 = (size_t)L.bh * L.nk * (L.d / 4);
+    const unsigned blocks = (unsigned)std::min<size_t>((n4 + 255) / 256, (size_t)148 * 16);
+    tc::split_keys_kernel<<<blocks, 256, 0, s>>>(static_cast<const float4 *>(k), L.ksplit, n4, L.d / 4);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = tc::key_rows_tensor_map(L.ksplit, 3 * L.d, L.nk, L.bh, map);
+    return e;
+}
+
+// Rows whose kept scores overflowed (retry lists): fp32 problems are
+// rebuilt on the CUDA cores, bf16 ones by the tensor-core heap kernel.
+cudaError_t route_retry_any(const LedgerDev &L, const void *q, const void *k, const CUtensorMap &map,
+                            int layer, cudaStream_t s) {
+    if (!L.split) return launch_route_retry(L, q, map, layer, s);
+    LedgerDev R = L;
+    R.list = L.retry_list;
+    R.head_count = L.retry_count;
+    return launch_route_rows_simt(R, kF32, q, k, layer, true, s);
+}
+
+}  // namespace
+
+cudaError_t launch_route_rows_split(const LedgerDev &L, const void *q, const void *k, int layer,
+                                    bool use_list, cudaStream_t s) {
+    CUtensorMap map;
+    cudaError_t e = split_keys(L, k, &map, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
+    if (e == cudaSuccess) e = launch_route_select(L, q, map, layer, use_list, SelectMode::kAnchor, s);
+    if (e != cudaSuccess) return e;
+    return route_retry_any(L, q, k, map, layer, s);
+}
+
 cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *k, int layer,
                                  cudaStream_t s) {
     CUtensorMap map;
-    cudaError_t e = tc::key_tensor_map(L, k, &map);
+    cudaError_t e = L.split ? split_keys(L, k, &map, s) : tc::key_tensor_map(L, k, &map);
     if (e == cudaSuccess) e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e == cudaSuccess) e = cudaMemsetAsync(L.und_count, 0, sizeof(int32_t), s);
     if (e == cudaSuccess) e = launch_route_select(L, q, map, layer, false, SelectMode::kRelay, s);
     if (e != cudaSuccess) return e;
-    const auto *Q = static_cast<const __nv_bfloat16 *>(q);
-    const auto *K = static_cast<const __nv_bfloat16 *>(k);
     const unsigned grid = 148 * 2;   // grid-stride over the open rows (usually none)
-    if (L.d == 128) tc::relay_exact_kernel<128><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
-    else tc::relay_exact_kernel<64><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
+    if (L.split) {
+        tc::relay_exact_kernel<64, float><<<grid, 32 * tc::kExactWarps, 0, s>>>(
+            L, static_cast<const float *>(q), static_cast<const float *>(k), layer);
+    } else {
+        const auto *Q = static_cast<const __nv_bfloat16 *>(q);
+        const auto *K = static_cast<const __nv_bfloat16 *>(k);
+        if (L.d == 128)
+            tc::relay_exact_kernel<128, __nv_bfloat16><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
+        else
+            tc::relay_exact_kernel<64, __nv_bfloat16><<<grid, 32 * tc::kExactWarps, 0, s>>>(L, Q, K, layer);
+    }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return launch_route_retry(L, q, map, layer, s);
+    return route_retry_any(L, q, k, map, layer, s);
 }
 
 }  // namespace rr

@@ -121,9 +121,21 @@ def test_bench_gpus_2_never_runs_a_single_rank_silently():
     assert '"metric"' not in p.stdout and "--gpus 2" in p.stderr
 
 
-def test_graph_mode_default_follows_the_kernel_path():
+def test_graph_mode_default_follows_the_step_length():
     import argparse
     a = argparse.Namespace(graph="auto")
     assert bench.graph_mode(a, W.C2) and bench.graph_mode(a, W.PR1) and not bench.graph_mode(a, W.C5)
     assert bench.graph_mode(argparse.Namespace(graph="on"), W.C5)
     assert not bench.graph_mode(argparse.Namespace(graph="off"), W.C2)
+
+
+def test_kernel_path_and_launch_count_per_workload():
+    assert bench.uses_tensor_cores(W.C5) and not bench.uses_split(W.C5)
+    for w in (W.PR1, W.C2, W.C3, W.C4):
+        assert bench.uses_tensor_cores(w) and bench.uses_split(w)
+    assert not bench.uses_tensor_cores(W.C2.with_(d=32))
+    assert not bench.uses_tensor_cores(W.C2.with_(k=48, m=24))
+    # C5: 2 anchors x 4 + 30 one-shot relays x 5; C2 (split): 4 x 5 + 28 x 6
+    assert bench.launches_per_step(W.C5, 2, 30, True) == 2 * 4 + 30 * 5
+    assert bench.launches_per_step(W.C2, 4, 28, True) == 4 * 5 + 28 * 6
+    assert bench.launches_per_step(W.C2.with_(d=32), 4, 28, True) == 4 * 2 + 28 * 4

@@ -50,7 +50,14 @@ ANCHOR_SHAPES = [
     ("only_random", 2, 100, 32, "bf16", 10, 0, 30, False),
     ("d256", 1, 96, 256, "f32", 8, 8, 8, True),
     ("seed_big", 2, 150, 64, "f32", 12, 12, 12, True),
-    # shapes of the tensor-core path (bf16, d in {64, 128}, k + m <= 64, r <= 32)
+    # fp32 on the CUDA cores at d = 64 (k + m above the selection kernel's 64)
+    ("f32_d64_cuda_cores", 2, 300, 64, "f32", 48, 24, 8, True),
+    # shapes of the tensor-core path (bf16, d in {64, 128}, k + m <= 64, r <= 32;
+    # fp32 at d = 64 with the three-way bf16 split)
+    ("split_d64_causal", 3, 1000, 64, "f32", 12, 12, 8, True),
+    ("split_exact_tile", 2, 256, 64, "f32", 40, 24, 32, False),
+    ("split_k1_r0", 2, 129, 64, "f32", 1, 0, 0, True),
+    ("split_wide_rows", 1, 4700, 64, "f32", 12, 12, 8, False),
     ("tc_d64", 3, 1000, 64, "bf16", 12, 12, 8, True),
     ("tc_d128_noncausal", 2, 300, 128, "bf16", 32, 32, 16, False),
     ("tc_small_n", 3, 70, 128, "bf16", 32, 32, 16, True),
@@ -230,7 +237,7 @@ def test_layer_order_is_enforced(rr):
     assert int(led.read()["counters"][rr.CNT_LAST_LAYER]) == 1
 
 
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 64)])
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("bf16", 64), ("f32", 64), ("f32", 32)])
 def test_equal_scores_pick_lowest_chunks(rr, dtype, d):
     """All keys equal -> every score of a row ties: the route is the k lowest
     valid chunks and the near-miss the next m (ties go to the smaller index).
@@ -254,7 +261,7 @@ def test_equal_scores_pick_lowest_chunks(rr, dtype, d):
         assert ids[0, i, k:k + nm].tolist() == list(range(nr, nr + nm))
         rand = [x for x in ids[0, i, k + m:].tolist() if x >= 0]
         assert len(rand) == min(r, nv - nr - nm) and all(nr + nm <= x < nv for x in rand)
-    if dtype == "bf16":
+    if d in (64, 128):   # tensor-core paths: every row overflows its slots and is redone
         assert int(out["counters"][rr.CNT_RETRY_TOTAL]) > 0
 
 
@@ -270,7 +277,8 @@ def test_retry_path_is_rare_on_the_full_size_workload(rr):
 
 GUARD = [
     (W.low_drift(W.C5).with_(bh=2, n=384, layers=10), "bf16_tensor_cores"),
-    (W.low_drift(W.C3).with_(bh=2, layers=8), "f32_cuda_cores"),
+    (W.low_drift(W.C3).with_(bh=2, layers=8), "f32_split_tensor_cores"),
+    (W.low_drift(W.C3).with_(bh=2, d=32, layers=8), "f32_cuda_cores"),
 ]
 
 
@@ -296,7 +304,8 @@ def test_per_row_margins_and_lifetime_bound(rr, case):
 
 HYST = [
     (W.C5.with_(bh=2, n=256, layers=8), "bf16_tensor_cores"),
-    (W.C3.with_(bh=2, n=256, layers=8), "f32_cuda_cores"),
+    (W.C3.with_(bh=2, n=256, layers=8), "f32_split_tensor_cores"),
+    (W.C3.with_(bh=2, n=256, d=32, layers=8), "f32_cuda_cores"),
 ]
 
 
@@ -319,7 +328,8 @@ def test_hysteresis_horizon(rr, case):
 
 GLOBALS = [
     (W.C5.with_(bh=2, n=384, layers=5), "bf16_tensor_cores"),
-    (W.C3.with_(bh=2, n=256, layers=5), "f32_cuda_cores"),
+    (W.C3.with_(bh=2, n=256, layers=5), "f32_split_tensor_cores"),
+    (W.C3.with_(bh=2, n=256, d=32, layers=5), "f32_cuda_cores"),
 ]
 
 
@@ -333,7 +343,7 @@ def test_global_sentinels_layer_by_layer(rr, case):
     _check(rep)
 
 
-@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64), ("f32", 32)])
 def test_global_sentinels_on_equal_scores_match_the_oracle(rr, dtype, d):
     """All scores of a row tie, so route, near-miss and globals are fixed by
     the index order and the random draws by the exclusion set: every id must
@@ -357,7 +367,8 @@ def test_global_sentinels_on_equal_scores_match_the_oracle(rr, dtype, d):
 
 HYST_MARGIN = [
     (W.low_drift(W.C5).with_(bh=2, n=384, layers=10), "bf16_tensor_cores"),
-    (W.low_drift(W.C3).with_(bh=2, n=256, layers=10), "f32_cuda_cores"),
+    (W.low_drift(W.C3).with_(bh=2, n=256, layers=10), "f32_split_tensor_cores"),
+    (W.low_drift(W.C3).with_(bh=2, n=256, d=32, layers=10), "f32_cuda_cores"),
 ]
 
 
