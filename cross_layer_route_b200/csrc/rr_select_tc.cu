@@ -62,7 +62,6 @@ constexpr int kValStride = kRows + 1;            // padded (slot, row) grid of t
 constexpr int kRowCap = 160;                     // kept scores per row (the record; 5 per lane)
 constexpr int kKeysPerLane = kRowCap / 32;
 constexpr int kTopWords = 65;                    // u32 words per row of 16-bit group maxima
-constexpr int kMaskBytes = kMaskTiles * kSelEpiWarps * 32 * 4;   // masks in the key ring after pass 1
 constexpr int kChunkStride = kRows + 2;          // u16 (slot, row) grid of the kept scores' chunks
 constexpr int kHalf = 16;                        // columns per capacity check in pass 1
 
@@ -75,8 +74,8 @@ struct SelLayout {
 constexpr uint32_t kRingBytes = 128 * 1024;
 
 // k (key ring, 128 KB: as many stages of 128 key rows x dk bf16 as fit, at
-// most 8; after pass 1 the masks [tile][epilogue thread] u32 and the chunk
-// grid [2][kPairCap][kChunkStride] u16) | vals [2][kPairCap][kValStride] f32
+// most 8; after pass 1 the chunk grid [2][kPairCap][kChunkStride] u16) |
+// vals [2][kPairCap][kValStride] f32
 // (before pass 1 the group maxima [kRows][kTopWords] u32) | rows | thr | cnt
 // | barriers | misc.  dk: bf16 elements per key row (d, or 3 d for split fp32).
 __host__ __device__ inline SelLayout sel_layout(int dk) {
@@ -94,8 +93,7 @@ __host__ __device__ inline SelLayout sel_layout(int dk) {
     s.total = o + 1024;   // slack for aligning the dynamic base to 1024
     return s;
 }
-static_assert(kRingBytes >= kMaskBytes + 2 * kPairCap * kChunkStride * 2,
-              "the key ring holds the masks and the chunk grid");
+static_assert(kRingBytes >= 2 * kPairCap * kChunkStride * 2, "the key ring holds the chunk grid");
 
 __device__ __forceinline__ void tc_st16(uint32_t taddr, const uint32_t *r) {
     asm volatile(
@@ -466,16 +464,13 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
 
         // sort keys.  First each thread pairs its kept scores, in the order
         // they were stored (tiles descending, columns ascending), with their
-        // chunks by walking its masks, and writes the chunks beside the
+        // chunks by walking its tile masks, and writes the chunks beside the
         // scores (chunk grid [2][kPairCap][kChunkStride] u16 in the idle key
-        // ring, after the masks [tile][epilogue thread]).  Then one warp per
-        // row turns (score, chunk) into sort keys, quarters in order, and
-        // stores them to the row's record.
+        // ring).  Then one warp per row turns (score, chunk) into sort keys,
+        // quarters in order, and stores them to the row's record.
         const bool cta_ok = *c.abort_flag == 0;
         const uint32_t *cnt_s = reinterpret_cast<const uint32_t *>(smem + lay.cnt);
-        uint32_t *masks_s = reinterpret_cast<uint32_t *>(smem + lay.k);
-        uint16_t *chunks_s = reinterpret_cast<uint16_t *>(smem + lay.k + kMaskBytes);
-        const int et = ew * 32 + lane;   // epilogue thread 0..511
+        uint16_t *chunks_s = reinterpret_cast<uint16_t *>(smem + lay.k);
         auto row_total = [&](int rr, int *cq) {
             const uint32_t cw = cnt_s[rr];
             int tot = 0;
@@ -489,29 +484,41 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
             bad |= cq[0] + cq[1] > kPairCap || cq[2] + cq[3] > kPairCap || tot > kRowCap;
             return bad ? -1 : tot;
         };
-        if (masks_in_tmem) {
-            uint32_t mk[32];
-            tc_ld32(mask_tmem, reinterpret_cast<float *>(mk));   // every lane of the warp
-#pragma unroll
-            for (int t = 0; t < kMaskTiles; ++t)
-                if (t < nt) masks_s[t * (kSelEpiWarps * 32) + et] = mk[t];
-        }
         {
             int cq[4];
             const int total = row_total(r, cq);
             const int own = (qt == 0 ? cq[0] : qt == 1 ? cq[1] : qt == 2 ? cq[2] : cq[3]);
-            if (row >= 0 && total >= 0 && own > 0) {
-                auto mask_of = [&](int t) -> uint32_t {
-                    return masks_in_tmem ? masks_s[t * (kSelEpiWarps * 32) + et] : gmask[(size_t)t * 4 * kRows];
-                };
-                uint16_t *cdst = chunks_s + (pair * kPairCap) * kChunkStride + r;
-                int t = nt - 1;
-                uint32_t m = mask_of(t);
-                for (int kk = 0; kk < own; ++kk) {
-                    while (m == 0u && t > 0) m = mask_of(--t);
-                    const int b = __ffs(m) - 1;
-                    m &= m - 1u;
-                    cdst[(down ? kPairCap - 1 - kk : kk) * kChunkStride] = (uint16_t)(t * kKeys + qt * 32 + b);
+            const bool walk = row >= 0 && total >= 0 && own > 0;
+            uint16_t *cp = chunks_s + (pair * kPairCap + (down ? kPairCap - 1 : 0)) * kChunkStride + r;
+            const int cstep = down ? -kChunkStride : kChunkStride;
+            if (masks_in_tmem) {
+                // the thread's tile masks in registers (a warp-wide load),
+                // walked tiles descending, columns ascending
+                uint32_t mk[kMaskTiles];
+                tc_ld32(mask_tmem, reinterpret_cast<float *>(mk));
+                if (walk) {
+#pragma unroll
+                    for (int t = kMaskTiles - 1; t >= 0; --t) {
+                        if (t < nt) {
+                            uint32_t m = mk[t];
+                            const int base = t * kKeys + qt * 32;
+                            while (m != 0u) {
+                                *cp = (uint16_t)(base + __ffs(m) - 1);
+                                cp += cstep;
+                                m &= m - 1u;
+                            }
+                        }
+                    }
+                }
+            } else if (walk) {
+                for (int t = nt - 1; t >= 0; --t) {
+                    uint32_t m = gmask[(size_t)t * 4 * kRows];
+                    const int base = t * kKeys + qt * 32;
+                    while (m != 0u) {
+                        *cp = (uint16_t)(base + __ffs(m) - 1);
+                        cp += cstep;
+                        m &= m - 1u;
+                    }
                 }
             }
         }
