@@ -38,7 +38,7 @@
 // keeps its ids and stores alpha; a challenged row is rebuilt from the same
 // kept scores at this layer.  Rows the bound cannot settle are rescored
 // exactly (relay_exact_kernel, candidate key rows gathered) and, if
-// challenged, rebuilt by the heap kernel.  On B200 the dense score tiles cost
+// challenged, rebuilt there from their kept scores.  On B200 the dense score tiles cost
 // less than the per-score work of the test, so one pass that both tests and
 // re-routes is cheaper than a rescoring pass followed by a re-route pass;
 // the ledger that comes out is the one the pages' two-stage procedure
@@ -942,9 +942,10 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
 
 // ---- exact rescoring of the relay rows the kept scores leave open ------------------
 // One warp per listed row: alpha and beta from the row's candidate key rows
-// (Eq. 5-7, fp32 products of the bf16 inputs), the decision of Eq. 8 with
-// the ledger's age rules; a challenged row goes to the retry list and is
-// rebuilt by the heap kernel.
+// (Eq. 5-7, fp32 products of the inputs), the decision of Eq. 8 with the
+// ledger's age rules; a challenged row is rebuilt by the same warp from its
+// kept scores (the finishing step of an anchor row), or, when its record
+// overflowed, goes to the retry list.
 constexpr int kExactWarps = 8;
 
 // The candidate's score, fp32 products of the inputs (bf16 rows: 8 elements
@@ -990,7 +991,9 @@ template <int D, typename T>
 __global__ void __launch_bounds__(32 * kExactWarps)
 relay_exact_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K, int layer) {
     __shared__ __align__(16) float qs[kExactWarps][D];
+    __shared__ FinScratch fin[kExactWarps];
     __shared__ unsigned long long red_cnt[kExactWarps][3];
+    const size_t slots_per_head = (size_t)((L.nq + kRows - 1) / kRows) * kRows;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n = *L.und_count;
     unsigned long long crow = 0, cpair = 0, cfull = 0;
@@ -1024,21 +1027,31 @@ relay_exact_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K
             ncand += __shfl_xor_sync(kFull, ncand, o);
         }
         const bool any_bad = __any_sync(kFull, bad);
+        uint32_t fl = 0u;
+        if (lane == 0) fl = relay_decide(L, (size_t)grow, layer, amin, bmax);   // Eq. 8
+        fl = __shfl_sync(kFull, fl, 0);
+        const bool refresh = (fl & 1u) != 0u;
         if (lane == 0) {
-            const uint8_t fl = relay_decide(L, (size_t)grow, layer, amin, bmax);   // Eq. 8
-            const bool refresh = (fl & 1u) != 0u;
-            L.flags[grow] = fl;
-            if (!refresh) L.alpha[grow] = amin;
+            if (!refresh) {
+                L.flags[grow] = (uint8_t)fl;
+                L.alpha[grow] = amin;
+            }
             if (any_bad) atomicOr(&L.counters[2], 1ULL);
             cpair += (unsigned long long)ncand;
             if (refresh) {
-                const int pos = atomicAdd(&L.retry_count[h], 1);
-                L.retry_list[(size_t)h * L.nq + pos] = i;
-                atomicAdd(&L.counters[10], 1ULL);
                 crow += 1;
                 cpair += (unsigned long long)n_valid;
                 cfull += (unsigned long long)n_valid;
             }
+        }
+        if (refresh) {
+            // the row is rebuilt at this layer from the same kept scores (its
+            // record from the selection kernel); a record that overflowed
+            // goes to the retry list
+            RowIn in;
+            load_row<false>(L, h, i, (size_t)h * slots_per_head + i, lane, in);
+            FinCounts unused;
+            finish_one<false>(L, layer, h, in, fin[warp], lane, unused);
         }
         __syncwarp();
     }
