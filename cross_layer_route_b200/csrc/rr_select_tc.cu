@@ -556,6 +556,8 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
 // ---- row finishing ---------------------------------------------------------------
 constexpr int kFinWarps = 8;
 constexpr int kFinThreads = 32 * kFinWarps;
+constexpr int kFinSub = 4;                     // finishing CTAs per selection row block
+constexpr int kFinRows = kRows / kFinSub;      // rows per finishing CTA (4 per warp)
 constexpr int kBins = 64;
 constexpr int kBitsWords = 128;        // membership bitmaps: rows with <= 4096 valid keys
 
@@ -905,21 +907,25 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h = blockIdx.y;
     const int count = use_list ? L.head_count[h] : L.nq;
-    const int row0 = blockIdx.x * kRows;
+    // CTA (x, h) finishes rows 32 (x % 4) .. 32 (x % 4) + 31 of the
+    // selection kernel's row block x / 4 of head h
+    const int bsel = blockIdx.x / kFinSub, part = blockIdx.x % kFinSub;
+    const int row0 = bsel * kRows + part * kFinRows;
     if (row0 >= count) return;
-    const int n_rows = min(kRows, count - row0);
-    const size_t blk = (size_t)h * gridDim.x + blockIdx.x;
+    const int n_rows = min(kFinRows, count - row0);
+    const size_t blk = (size_t)h * ((L.nq + kRows - 1) / kRows) + bsel;
+    const size_t slot0 = blk * kRows + (size_t)part * kFinRows;
     FinCounts cnt;
-    constexpr int kPerWarp = kRows / kFinWarps;
+    constexpr int kPerWarp = kFinRows / kFinWarps;
     const int rr0 = warp * kPerWarp;
     auto row_at = [&](int rr) { return use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr; };
     RowIn cur, nxt;
-    if (rr0 < n_rows) load_row<kRelay>(L, h, row_at(rr0), blk * kRows + rr0, lane, cur);
+    if (rr0 < n_rows) load_row<kRelay>(L, h, row_at(rr0), slot0 + rr0, lane, cur);
     for (int k2 = 0; k2 < kPerWarp; ++k2) {
         const int rr = rr0 + k2;
         if (rr >= n_rows) break;   // warp-uniform
         const bool more = k2 + 1 < kPerWarp && rr + 1 < n_rows;
-        if (more) load_row<kRelay>(L, h, row_at(rr + 1), blk * kRows + rr + 1, lane, nxt);
+        if (more) load_row<kRelay>(L, h, row_at(rr + 1), slot0 + rr + 1, lane, nxt);
         finish_one<kRelay>(L, layer, h, cur, scr[warp], lane, cnt);
         __syncwarp();
         if (more) cur = nxt;
@@ -1125,10 +1131,11 @@ cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtenso
         L, q, map, use_list ? 1 : 0);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+    dim3 fgrid(grid.x * tc::kFinSub, L.bh);
     if (mode == SelectMode::kRelay)
-        tc::route_finish_kernel<true><<<grid, tc::kFinThreads, 0, s>>>(L, layer, 0);
+        tc::route_finish_kernel<true><<<fgrid, tc::kFinThreads, 0, s>>>(L, layer, 0);
     else
-        tc::route_finish_kernel<false><<<grid, tc::kFinThreads, 0, s>>>(L, layer, use_list ? 1 : 0);
+        tc::route_finish_kernel<false><<<fgrid, tc::kFinThreads, 0, s>>>(L, layer, use_list ? 1 : 0);
     return cudaGetLastError();
 }
 
