@@ -558,12 +558,13 @@ constexpr int kFinWarps = 8;
 constexpr int kFinThreads = 32 * kFinWarps;
 constexpr int kFinSub = 4;                     // finishing CTAs per selection row block
 constexpr int kFinRows = kRows / kFinSub;      // rows per finishing CTA (4 per warp)
-constexpr int kBins = 64;
+constexpr int kBins = 128;
+static_assert(kBins == 4 * 32, "four bins per lane in the finishing sort");
 constexpr int kBitsWords = 128;        // membership bitmaps: rows with <= 4096 valid keys
 
 struct FinScratch {
     uint64_t keys[kRowCap];            // kept keys in bin order
-    uint32_t hist[kBins];              // bin counts, then bin starts
+    alignas(16) uint32_t hist[kBins];  // bin counts, then bin starts (4 per lane)
     uint32_t bits[kBitsWords];         // selected and accepted chunks
     uint32_t rbits[kBitsWords];        // relay: chunks of the old route
     uint32_t sbits[kBitsWords];        // relay: chunks of the old sentinels
@@ -655,18 +656,14 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
 
     if constexpr (kRelay) {
         // relay test of the old ledger row (§3.2 Eq. 5-8) from the kept scores
-        const int words = (n_valid + 31) >> 5;
         if (n_valid > 32 * kBitsWords) {   // no bitmap for such rows: rescore exactly
             if (lane == 0) {
                 L.und_list[atomicAdd(L.und_count, 1)] = (int)grow;   // flags: set by the exact rescoring
             }
             return;
         }
-        for (int q = lane; q < words; q += 32) {
-            w.rbits[q] = 0u;
-            w.sbits[q] = 0u;
-        }
-        __syncwarp();
+        // rbits / sbits are all zero here: cleared when the warp starts and,
+        // after every row, at the words that row set
         int rt = 0, st = 0;
         bool bad = false;
 #pragma unroll
@@ -691,6 +688,16 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             if ((w.rbits[j >> 5] >> (j & 31)) & 1u) { amin = fminf(amin, v); ++rf; }   // Eq. 6
             if ((w.sbits[j >> 5] >> (j & 31)) & 1u) { bmax = fmaxf(bmax, v); ++sf; }   // Eq. 7
         }
+        __syncwarp();   // every lane has looked its keys up: clear the words this row set
+#pragma unroll
+        for (int i = 0; i < 3; ++i) {
+            const int j = in.id[i];
+            if (j >= 0 && j < n_valid) {
+                w.rbits[j >> 5] = 0u;
+                w.sbits[j >> 5] = 0u;
+            }
+        }
+        __syncwarp();
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
@@ -741,8 +748,10 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         cnt.full += (unsigned long long)n_valid;
     }
 
-    // order: counting sort of the kept keys over 64 bins of their score key
-    // (larger key = lower bin), then each key's rank among the keys of its bin
+    // order: counting sort of the kept keys over 128 bins of their score key
+    // (larger key = lower bin; bin = (largest key - key) >> shift, the shift
+    // putting the key range in 64..128 bins), then each key's rank among the
+    // keys of its bin
     uint32_t hmx = 0u, hmn = 0xFFFFFFFFu;
 #pragma unroll
     for (int i = 0; i < kKeysPerLane; ++i) {
@@ -753,30 +762,29 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     }
     hmx = __reduce_max_sync(kFull, hmx);
     hmn = __reduce_min_sync(kFull, hmn);
-    const float scale = (float)kBins / ((float)(hmx - hmn) + 1.0f);
-    w.hist[lane] = 0u;
-    w.hist[lane + 32] = 0u;
+    const int shift = max(0, 25 - __clz(hmx - hmn));   // (hmx - hmn) >> shift < 128
+    reinterpret_cast<uint4 *>(w.hist)[lane] = make_uint4(0u, 0u, 0u, 0u);
     __syncwarp();
     int bin[kKeysPerLane];
     uint32_t in_bin[kKeysPerLane];
 #pragma unroll
     for (int i = 0; i < kKeysPerLane; ++i) {
-        bin[i] = min(kBins - 1, (int)((float)(hmx - (uint32_t)(key[i] >> 32)) * scale));
+        bin[i] = (int)min((uint32_t)(kBins - 1), (hmx - (uint32_t)(key[i] >> 32)) >> shift);
         in_bin[i] = live[i] ? atomicAdd(&w.hist[bin[i]], 1u) : 0u;
     }
     __syncwarp();
     {
-        const uint32_t h0 = w.hist[2 * lane], h1 = w.hist[2 * lane + 1];
-        uint32_t incl = h0 + h1;
+        const uint4 hv = reinterpret_cast<const uint4 *>(w.hist)[lane];
+        uint32_t incl = hv.x + hv.y + hv.z + hv.w;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t x = __shfl_up_sync(kFull, incl, o);
             if (lane >= o) incl += x;
         }
-        const uint32_t excl = incl - h0 - h1;
+        const uint32_t excl = incl - (hv.x + hv.y + hv.z + hv.w);
         __syncwarp();
-        w.hist[2 * lane] = excl;
-        w.hist[2 * lane + 1] = excl + h0;
+        reinterpret_cast<uint4 *>(w.hist)[lane] =
+            make_uint4(excl, excl + hv.x, excl + hv.x + hv.y, excl + hv.x + hv.y + hv.z);
     }
     __syncwarp();
     int start[kKeysPerLane];
@@ -919,6 +927,13 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
     constexpr int kPerWarp = kFinRows / kFinWarps;
     const int rr0 = warp * kPerWarp;
     auto row_at = [&](int rr) { return use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr; };
+    if (kRelay) {   // the relay test's bitmaps start clear (each row clears what it sets)
+        for (int q = lane; q < kBitsWords; q += 32) {
+            scr[warp].rbits[q] = 0u;
+            scr[warp].sbits[q] = 0u;
+        }
+        __syncwarp();
+    }
     RowIn cur, nxt;
     if (rr0 < n_rows) load_row<kRelay>(L, h, row_at(rr0), slot0 + rr0, lane, cur);
     for (int k2 = 0; k2 < kPerWarp; ++k2) {
