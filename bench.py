@@ -598,6 +598,7 @@ def per_workload(args, device, oracle_leg: bool) -> dict:
         r_mean, r_min = measure_recall(w, state, device)
         entry.update({"recall": r_mean, "recall_min_layer": r_min, "recall_kind": RECALL_KIND})
         if oracle_leg:
+            entry["cpu_baseline"] = cpu_baseline(w, state[1], state[2])
             entry["oracle_sample"] = oracle_sample(w, state)
         out[w.name] = entry
         del state
@@ -790,11 +791,15 @@ def main():
     ap.add_argument("--no-oracle-sample", action="store_true",
                     help="skip the tie/mismatch count against the oracle on sampled heads")
     ap.add_argument("--smi-index", type=int, default=None)
+    ap.add_argument("--low-drift", action="store_true",
+                    help="the supplementary low-drift variant of the workload (sigma / sqrt(d) per element)")
     ap.add_argument("--bh", type=int, default=None, help="override BH (profiling a smaller case)")
     ap.add_argument("--layers", type=int, default=None, help="override the layer count")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     w = W.BY_NAME[args.workload]
+    if args.low_drift:
+        w = W.low_drift(w)
     if args.bh is not None:
         w = w.with_(bh=args.bh, name=f"{w.name}@bh{args.bh}")
     if args.layers is not None:
@@ -847,7 +852,7 @@ def main():
     del state
     if world == 1 and (args.per_workload == "on" or (
             args.per_workload == "auto" and args.workload == W.C5.name and args.bh is None
-            and args.layers is None)):
+            and args.layers is None and not args.low_drift)):
         torch.cuda.empty_cache()
         result["per_workload"] = per_workload(args, device, oracle_leg=not args.no_cpu_baseline
                                               and not args.no_oracle_sample)
