@@ -383,7 +383,12 @@ def run_ours(args, w, rank, world, device):
                     "peak_source": "148 SMs x 128 fp32 lanes x 2 flop x max SM clock"}
     traffic = None
     if uses_tensor_cores(w) and not uses_split(w):
-        per_row = profiled_traffic_per_row("rr_select_tc.cu", "route_select_kernel__*.md")
+        # DRAM bytes per routed row of the two kernels of a routing call, from
+        # the committed ncu summaries of the 64-head case (traffic grows with
+        # the rows routed), while their source is unchanged
+        parts = [profiled_traffic_per_row("rr_select_tc.cu", g)
+                 for g in ("route_select_kernel__*.md", "route_finish_kernel__*.md")]
+        per_row = sum(parts) if all(x is not None for x in parts) else None
         if per_row is not None and n_route:
             rows_routed = (w.bh * w.n * L) if oneshot else refreshed_per_step
             traffic = round(per_row * rows_routed * K_ev / n_route)   # bytes per launch
