@@ -908,7 +908,7 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
 }
 
 template <bool kRelay>
-__global__ void __launch_bounds__(kFinThreads, 3)
+__global__ void __launch_bounds__(kFinThreads, 4)
 route_finish_kernel(LedgerDev L, int layer, int use_list) {
     __shared__ FinScratch scr[kFinWarps];
     __shared__ unsigned long long red_cnt[kFinWarps][3];
@@ -934,16 +934,13 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
         }
         __syncwarp();
     }
-    RowIn cur, nxt;
-    if (rr0 < n_rows) load_row<kRelay>(L, h, row_at(rr0), slot0 + rr0, lane, cur);
     for (int k2 = 0; k2 < kPerWarp; ++k2) {
         const int rr = rr0 + k2;
         if (rr >= n_rows) break;   // warp-uniform
-        const bool more = k2 + 1 < kPerWarp && rr + 1 < n_rows;
-        if (more) load_row<kRelay>(L, h, row_at(rr + 1), slot0 + rr + 1, lane, nxt);
+        RowIn cur;
+        load_row<kRelay>(L, h, row_at(rr), slot0 + rr, lane, cur);
         finish_one<kRelay>(L, layer, h, cur, scr[warp], lane, cnt);
         __syncwarp();
-        if (more) cur = nxt;
     }
     if (kRelay) {
         if (lane == 0) {
