@@ -566,8 +566,7 @@ struct FinScratch {
     uint64_t keys[kRowCap];            // kept keys in bin order
     alignas(16) uint32_t hist[kBins];  // bin counts, then bin starts (4 per lane)
     uint32_t bits[kBitsWords];         // selected and accepted chunks
-    uint32_t rbits[kBitsWords];        // relay: chunks of the old route
-    uint32_t sbits[kBitsWords];        // relay: chunks of the old sentinels
+    uint32_t cbits[2 * kBitsWords];    // relay: chunks of the old route (bit 0) and sentinels (bit 1)
     int32_t acc[32];                   // accepted random sentinels, in order
 };
 
@@ -662,8 +661,9 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             }
             return;
         }
-        // rbits / sbits are all zero here: cleared when the warp starts and,
-        // after every row, at the words that row set
+        // the old row's chunks, two bits each in cbits (bit 0: route, bit 1:
+        // sentinel; 16 chunks per word).  cbits is all zero here: cleared when
+        // the warp starts and, after every row, at the words that row set.
         int rt = 0, st = 0;
         bool bad = false;
 #pragma unroll
@@ -672,10 +672,13 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             const int j = in.id[i];
             const bool valid = j >= 0 && j < n_valid;
             bad |= j >= n_valid || j < -1;
-            if (valid) atomicOr(&(e < L.k ? w.rbits : w.sbits)[j >> 5], 1u << (j & 31));
-            rt += __popc(__ballot_sync(kFull, valid && e < L.k));
-            st += __popc(__ballot_sync(kFull, valid && e >= L.k));
+            const bool route = e < L.k;
+            if (valid) atomicOr(&w.cbits[j >> 4], (route ? 1u : 2u) << ((j & 15) << 1));
+            rt += valid && route ? 1 : 0;
+            st += valid && !route ? 1 : 0;
         }
+        rt = (int)__reduce_add_sync(kFull, (unsigned)rt);
+        st = (int)__reduce_add_sync(kFull, (unsigned)st);
         if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.counters[2], 1ULL);
         __syncwarp();
         float amin = INFINITY, bmax = -INFINITY;
@@ -684,18 +687,18 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         for (int i = 0; i < kKeysPerLane; ++i) {
             if (!live[i]) continue;
             const int j = sel_key_chunk(key[i]);
-            const float v = sel_key_score(key[i]);
-            if ((w.rbits[j >> 5] >> (j & 31)) & 1u) { amin = fminf(amin, v); ++rf; }   // Eq. 6
-            if ((w.sbits[j >> 5] >> (j & 31)) & 1u) { bmax = fmaxf(bmax, v); ++sf; }   // Eq. 7
+            const uint32_t cb = (w.cbits[j >> 4] >> ((j & 15) << 1)) & 3u;
+            if (cb != 0u) {
+                const float v = sel_key_score(key[i]);
+                if (cb & 1u) { amin = fminf(amin, v); ++rf; }   // Eq. 6
+                if (cb & 2u) { bmax = fmaxf(bmax, v); ++sf; }   // Eq. 7
+            }
         }
         __syncwarp();   // every lane has looked its keys up: clear the words this row set
 #pragma unroll
         for (int i = 0; i < 3; ++i) {
             const int j = in.id[i];
-            if (j >= 0 && j < n_valid) {
-                w.rbits[j >> 5] = 0u;
-                w.sbits[j >> 5] = 0u;
-            }
+            if (j >= 0 && j < n_valid) w.cbits[j >> 4] = 0u;
         }
         __syncwarp();
 #pragma unroll
@@ -927,11 +930,8 @@ route_finish_kernel(LedgerDev L, int layer, int use_list) {
     constexpr int kPerWarp = kFinRows / kFinWarps;
     const int rr0 = warp * kPerWarp;
     auto row_at = [&](int rr) { return use_list ? L.list[(size_t)h * L.nq + row0 + rr] : row0 + rr; };
-    if (kRelay) {   // the relay test's bitmaps start clear (each row clears what it sets)
-        for (int q = lane; q < kBitsWords; q += 32) {
-            scr[warp].rbits[q] = 0u;
-            scr[warp].sbits[q] = 0u;
-        }
+    if (kRelay) {   // the relay test's chunk map starts clear (each row clears what it sets)
+        for (int q = lane; q < 2 * kBitsWords; q += 32) scr[warp].cbits[q] = 0u;
         __syncwarp();
     }
     for (int k2 = 0; k2 < kPerWarp; ++k2) {

@@ -410,3 +410,35 @@ def test_a_wait_that_runs_out_sets_the_error_bit_and_the_rows_are_redone(rr):
     rep2, per_layer2 = layer_stepped(w, rr, fresh, w.layers, range(w.bh), DEV)
     _check(rep2)
     assert all(int(cnt[rr.CNT_ERROR]) == 0 for _, _, _, cnt in per_layer2)
+
+
+def test_split_fp32_scores_stay_within_the_split_error_bound(rr):
+    """fp32 rows run on the tensor cores as six bf16 products of a three-way
+    split (hi + mid + lo = x exactly); the dropped products add at most
+    2^-23 |q||k| per score and the fp32 accumulation of 24 MMA steps a few
+    2^-24 |q||k| more.  alpha (the k-th best score of every row, §3.2 Eq. 6)
+    is checked against the fp64 k-th score on every row of a causal anchor:
+    the worst error must stay below 2^-19 of the row's scale, 50 times inside
+    the 1e-5 tie margin and about 2000 times below a bf16 rounding of the
+    inputs."""
+    w = W.C4.with_(bh=2, layers=1)
+    cfg = config_of(w, rr)
+    led = rr.RouteLedger(cfg, DEV)
+    st = W.LayerStream(w, "cpu")
+    qf, kf, qs, ks = st.next()
+    led.full_route(qs.to(DEV), ks.to(DEV), 0)
+    alpha = led.read()["alpha"].numpy().astype(np.float64)
+    worst = 0.0
+    for h in range(w.bh):
+        q = qf[h].double().numpy()
+        k = kf[h].double().numpy()
+        S = q @ k.T
+        scale = np.linalg.norm(q, axis=1) * np.linalg.norm(k, axis=1).max()
+        for i in range(w.n):
+            nv = i + 1
+            if nv < w.k:
+                continue
+            kth = np.sort(S[i, :nv])[::-1][w.k - 1]
+            worst = max(worst, abs(alpha[h, i] - kth) / scale[i])
+    assert worst <= 2.0 ** -19, worst
+    print(f"worst alpha error / row scale: {worst:.3e}")
