@@ -39,6 +39,10 @@ template <int DH, int CH>
 struct Shape {
     static constexpr int kWarps = CH / 16;              // 16 query rows per warp
     static constexpr int kThreads = 32 * kWarps;
+    // CTAs per SM the register budget is fitted to: three for chunks of up
+    // to 64 tokens (at most 170 registers a thread, no spills); one for
+    // chunks of 128 (eight warps, whose fragments would spill at three)
+    static constexpr int kMinBlocks = kThreads >= 256 ? 1 : 3;
     static constexpr int kRow = DH + 8;                  // padded smem row (elements)
     static constexpr int kTile = CH * kRow;              // one staged K or V chunk (elements)
     static constexpr int kListBytes = kMaxWidth * 4 + 16;
@@ -109,7 +113,7 @@ __device__ __forceinline__ void stage_chunk(const __nv_bfloat16 *__restrict__ kh
 }
 
 template <int DH, int CH>
-__global__ void __launch_bounds__(Shape<DH, CH>::kThreads)
+__global__ void __launch_bounds__(Shape<DH, CH>::kThreads, Shape<DH, CH>::kMinBlocks)
 sparse_attention_kernel(rr_attn_config cfg, const __nv_bfloat16 *__restrict__ q,
                         const __nv_bfloat16 *__restrict__ k, const __nv_bfloat16 *__restrict__ v,
                         const int32_t *__restrict__ route, float *__restrict__ out, float scale_log2) {
