@@ -228,11 +228,29 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
     const int dk = split ? 3 * d : d;   // bf16 elements per key row in the ring
     const SelLayout lay = sel_layout(dk);
     const __nv_bfloat16 *Q = static_cast<const __nv_bfloat16 *>(Qv);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int h = blockIdx.y;
+
+    // Each epilogue thread starts loading its quarter of its query row (the
+    // row the set-up below will list for it) before the set-up, so that the
+    // loads are in flight while barriers and TMEM are prepared: 64 bytes
+    // (d = 128 bf16, or 16 fp32 elements of a split row), or 32 (d = 64 bf16).
+    uint4 qpre[4];
+    if (warp >= 2) {
+        const int qt = (warp - 2) >> 2, r = (warp & 3) * 32 + lane;
+        const int count = use_list ? L.head_count[h] : L.nq;
+        const int rp = blockIdx.x * kRows + r;
+        const int row = rp < count ? (use_list ? L.list[(size_t)h * L.nq + rp] : rp) : -1;
+        const size_t base = ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d;
+        const uint4 *src = split ? reinterpret_cast<const uint4 *>(static_cast<const float *>(Qv) + base + qt * 16)
+                                 : reinterpret_cast<const uint4 *>(Q + base + qt * (d >> 2));
+        const int n16 = (split || d == 128) ? 4 : 2;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) qpre[i] = (row >= 0 && i < n16) ? src[i] : make_uint4(0u, 0u, 0u, 0u);
+    }
     Cta c;
     if (!cta_setup(c, smem, lay.cta(), L, Q, L.list, L.head_count, use_list, /*q_to_smem=*/false))
         return;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int h = blockIdx.y;
 
     // The producer starts at once; the MMA warp waits until the epilogue
     // warps have put the query tile into TMEM (barrier q_ready).
@@ -249,24 +267,18 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
         // writes a quarter of the row's elements for its 32 rows
         {
             const int ew = warp - 2, sub = warp & 3, qt = ew >> 2;
-            const int r = sub * 32 + lane;
-            const int row = c.rows_s[r];
             const uint32_t taddr =
                 c.tmem_base + ((uint32_t)(sub * 32) << 16) + kQCol + (uint32_t)(qt * (d >> 3));
             uint32_t w[16];
-            const uint4 *src = reinterpret_cast<const uint4 *>(
-                Q + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d + qt * (d >> 2));
             if (split) {
                 // fp32 elements 16 qt .. 16 qt + 15, each split into bf16
                 // hi + mid + lo (x = hi + mid + lo exactly); part p goes to
                 // columns 32 p + 8 qt .. 32 p + 8 qt + 7
-                const float4 *srcf = reinterpret_cast<const float4 *>(
-                    static_cast<const float *>(Qv) + ((size_t)h * L.nq + (row >= 0 ? row : 0)) * d + qt * 16);
                 uint32_t part[3][8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float4 v = row >= 0 ? srcf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    const float x[4] = {v.x, v.y, v.z, v.w};
+                    const float x[4] = {__uint_as_float(qpre[i].x), __uint_as_float(qpre[i].y),
+                                        __uint_as_float(qpre[i].z), __uint_as_float(qpre[i].w)};
 #pragma unroll
                     for (int e = 0; e < 4; e += 2) {
                         uint32_t b0[3], b1[3];
@@ -283,15 +295,13 @@ route_select_kernel(LedgerDev L, const void *__restrict__ Qv,
             } else if (d == 128) {
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                    w[4 * i] = qpre[i].x; w[4 * i + 1] = qpre[i].y; w[4 * i + 2] = qpre[i].z; w[4 * i + 3] = qpre[i].w;
                 }
                 tc_st16(taddr, w);
             } else {
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
-                    const uint4 v = row >= 0 ? src[i] : make_uint4(0u, 0u, 0u, 0u);
-                    w[4 * i] = v.x; w[4 * i + 1] = v.y; w[4 * i + 2] = v.z; w[4 * i + 3] = v.w;
+                    w[4 * i] = qpre[i].x; w[4 * i + 1] = qpre[i].y; w[4 * i + 2] = qpre[i].z; w[4 * i + 3] = qpre[i].w;
                 }
                 tc_st8(taddr, w);
             }

@@ -351,8 +351,13 @@ __device__ __forceinline__ bool cta_setup(Cta &c, unsigned char *smem, const Cta
         *reinterpret_cast<uint4 *>(c.q_s + kb * kSubTileBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = v;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    int max_row = -1;
-    for (int e = 0; e < c.n_rows; ++e) max_row = max(max_row, c.rows_s[e]);
+    // the block's last row bounds its key tiles under the causal mask; rows
+    // from a list may come in any order
+    int max_row = row0 + c.n_rows - 1;
+    if (use_list) {
+        max_row = -1;
+        for (int e = 0; e < c.n_rows; ++e) max_row = max(max_row, c.rows_s[e]);
+    }
     const int kend = L.causal ? min(L.nk, max_row + 1) : L.nk;
     c.ntiles = (kend + kKeys - 1) / kKeys;
     __syncthreads();
