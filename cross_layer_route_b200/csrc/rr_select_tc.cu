@@ -691,18 +691,18 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
         st = (int)__reduce_add_sync(kFull, (unsigned)st);
         if (__any_sync(kFull, bad) && lane == 0) atomicOr(&L.counters[2], 1ULL);
         __syncwarp();
-        float amin = INFINITY, bmax = -INFINITY;
+        // alpha and beta as order keys of the scores (the sort keys' top
+        // words), reduced across the warp as unsigned integers
+        uint32_t amin_k = 0xFFFFFFFFu, bmax_k = 0u;
         int rf = 0, sf = 0;
 #pragma unroll
         for (int i = 0; i < kKeysPerLane; ++i) {
             if (!live[i]) continue;
             const int j = sel_key_chunk(key[i]);
             const uint32_t cb = (w.cbits[j >> 4] >> ((j & 15) << 1)) & 3u;
-            if (cb != 0u) {
-                const float v = sel_key_score(key[i]);
-                if (cb & 1u) { amin = fminf(amin, v); ++rf; }   // Eq. 6
-                if (cb & 2u) { bmax = fmaxf(bmax, v); ++sf; }   // Eq. 7
-            }
+            const uint32_t ok = (uint32_t)(key[i] >> 32);
+            if (cb & 1u) { amin_k = min(amin_k, ok); ++rf; }   // Eq. 6
+            if (cb & 2u) { bmax_k = max(bmax_k, ok); ++sf; }   // Eq. 7
         }
         __syncwarp();   // every lane has looked its keys up: clear the words this row set
 #pragma unroll
@@ -711,13 +711,12 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             if (j >= 0 && j < n_valid) w.cbits[j >> 4] = 0u;
         }
         __syncwarp();
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            amin = fminf(amin, __shfl_xor_sync(kFull, amin, o));
-            bmax = fmaxf(bmax, __shfl_xor_sync(kFull, bmax, o));
-        }
+        amin_k = __reduce_min_sync(kFull, amin_k);
+        bmax_k = __reduce_max_sync(kFull, bmax_k);
         rf = (int)__reduce_add_sync(kFull, (unsigned)rf);
         sf = (int)__reduce_add_sync(kFull, (unsigned)sf);
+        const float amin = rf > 0 ? unord32(amin_k) : INFINITY;
+        const float bmax = sf > 0 ? unord32(bmax_k) : -INFINITY;
         // alpha is exact when every route chunk was kept; beta when a
         // sentinel was kept (the others score below T) or there is none
         const bool aexact = rf == rt;
@@ -817,7 +816,9 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
     for (int i = 0; i < kKeysPerLane; ++i) {
         sel[i] = false;
         jc[i] = live[i] ? sel_key_chunk(key[i]) : -1;
-        if (!live[i]) continue;
+        // a key with nsel or more keys in the bins above it is not selected:
+        // no rank needed (these are the lowest, most crowded bins)
+        if (!live[i] || start[i] >= nsel) continue;
         const int end = bin[i] + 1 < kBins ? (int)w.hist[bin[i] + 1] : total;
         int rank = 0;
         for (int p = start[i]; p < end; ++p) rank += w.keys[p] > key[i] ? 1 : 0;
@@ -828,8 +829,9 @@ __device__ __forceinline__ void finish_one(const LedgerDev &L, int layer, int h,
             if (pos == nr - 1) L.alpha[grow] = sel_key_score(key[i]);
         }
     }
-    for (int sl = lane; sl < L.k + L.m; sl += 32) {   // padding of short rows
-        if (sl < L.k ? sl >= nr : sl - L.k >= nm) out[sl] = -1;
+    if (nsel < L.k + L.m) {   // padding of short rows
+        for (int sl = lane; sl < L.k + L.m; sl += 32)
+            if (sl < L.k ? sl >= nr : sl - L.k >= nm) out[sl] = -1;
     }
 
     // random sentinels (§3.1 item 2, §3.4): Philox4x32-10 words keyed
