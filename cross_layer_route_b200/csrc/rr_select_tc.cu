@@ -59,7 +59,7 @@ constexpr uint32_t kMaskCol = kQCol + 96;        // kept-column masks: [quarter]
 constexpr int kMaskTiles = 32;                   // blocks with more key tiles keep masks in device memory
 constexpr int kPairCap = 92;                     // kept-score slots shared by two quarters of a row
 constexpr int kValStride = kRows + 1;            // padded (slot, row) grid of the kept scores
-constexpr int kRowCap = 160;                     // kept scores per row (the record; 5 per lane)
+constexpr int kRowCap = 128;                     // kept scores per row (the record; 4 per lane)
 constexpr int kKeysPerLane = kRowCap / 32;
 constexpr int kTopWords = 65;                    // u32 words per row of 16-bit group maxima
 constexpr int kChunkStride = kRows + 2;          // u16 (slot, row) grid of the kept scores' chunks
