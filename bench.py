@@ -209,10 +209,10 @@ def sum_over_ranks(xs, world: int, device=None) -> list:
 
 def launches_per_step(w, n_anchor: int, n_relay: int, oneshot: bool) -> int:
     """Our kernels launched by one step.  Tensor-core path: anchor = select,
-    finish, heap retry, counters (4); one-shot relay = select, finish, exact
-    rescoring, heap retry, counters (5); staged relay = rescore, compact,
-    select, finish, heap retry, counters (6); fp32 split: one more per
-    routing call (the key split; the retry runs on the CUDA cores).
+    finish, retry (CUDA cores, usually an empty list), counters (4); one-shot
+    relay = select, finish, exact rescoring, retry, counters (5); staged
+    relay = rescore, compact, select, finish, retry, counters (6); fp32
+    split: one more per routing call (the key split).
     CUDA-core path: anchor = route, counters (2); relay = rescore, compact,
     route, counters (4)."""
     if uses_tensor_cores(w):
@@ -372,9 +372,9 @@ def run_ours(args, w, rank, world, device):
     elif uses_tensor_cores(w):
         peak = float(peaks["bf16_tflops_sustained"])
         what = ("route_select_kernel (tcgen05, query tile in TMEM, two-pass selection) + route_finish_kernel"
-                " + exact/heap fallbacks; anchor and relay layers (relay test taken from the kept scores)"
+                " + exact fallbacks; anchor and relay layers (relay test taken from the kept scores)"
                 if oneshot else
-                "route_select_kernel + route_finish_kernel + heap fallback; anchor layers and refresh launches")
+                "route_select_kernel + route_finish_kernel + exact fallback; anchor layers and refresh launches")
         roofline = {"kernel": "full routing: " + what, "bound": "tensor",
                     "peak_source": f"{peaks['source']} bf16 dense, sustained (timed inside a long step)"}
     else:

@@ -99,8 +99,10 @@ bool route_select_split_supported(const LedgerDev &L, int dtype);
 cudaError_t launch_route_rows_split(const LedgerDev &L, const void *q, const void *k, int layer,
                                     bool use_list, cudaStream_t s);
 // The CUDA-core route kernel alone (rr_route_simt.cu), whatever the problem.
+// max_tiles > 0 caps the grid's tiles of 32 rows per head; each CTA then
+// strides over the head's remaining tiles (the retry lists, usually empty).
 cudaError_t launch_route_rows_simt(const LedgerDev &L, int dtype, const void *q, const void *k,
-                                   int layer, bool use_list, cudaStream_t s);
+                                   int layer, bool use_list, cudaStream_t s, int max_tiles = 0);
 size_t route_select_smem_bytes(const LedgerDev &L);
 cudaError_t route_select_prepare();
 // kAnchor: every row (or every listed row) is rebuilt.  kRelay: every row
@@ -109,7 +111,12 @@ cudaError_t route_select_prepare();
 enum class SelectMode { kAnchor = 0, kRelay = 1 };
 cudaError_t launch_route_select(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
                                 bool use_list, SelectMode mode, cudaStream_t s);
-// Exact heap selection of the rows in the per-head retry lists (rr_route_tc.cu).
+// Exact routing on the CUDA cores of the rows in the per-head retry lists
+// (rows whose kept scores overflowed on the selection path; rr_select_tc.cu).
+cudaError_t launch_retry_rows_simt(const LedgerDev &L, const void *q, const void *k, int layer,
+                                   cudaStream_t s);
+// Exact heap selection of the rows in the per-head retry lists of the fused
+// kernel route_rows_tc_kernel (rr_route_tc.cu).
 cudaError_t launch_route_retry(const LedgerDev &L, const void *q, const CUtensorMap &map, int layer,
                                cudaStream_t s);
 // One relay layer on the tensor-core selection path: route every row, take

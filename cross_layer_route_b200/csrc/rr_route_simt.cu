@@ -142,145 +142,149 @@ route_rows_kernel(LedgerDev L, const T *__restrict__ Q, const T *__restrict__ K,
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int d = L.d, nq = L.nq, nk = L.nk;
     const int count = use_list ? L.head_count[h] : nq;
-    const int row0 = blockIdx.x * kTileRows;
-    if (row0 >= count) return;
-    const int n_rows = min(kTileRows, count - row0);
+    // tiles of 32 rows, grid-stride (a grid narrower than the rows, as the
+    // retry lists use, takes several tiles per CTA)
+    for (int row0 = blockIdx.x * kTileRows; row0 < count; row0 += gridDim.x * kTileRows) {
+        __syncthreads();   // the previous tile's rows, queries and buffers are done with
+        const int n_rows = min(kTileRows, count - row0);
 
-    if (tid < kTileRows) {
-        int row = -1;
-        if (tid < n_rows) row = use_list ? L.list[(size_t)h * nq + row0 + tid] : row0 + tid;
-        rows_s[tid] = row;
-    }
-    __syncthreads();
-    // query tile -> shared (fp32), zero rows for empty slots
-    const int d4 = d >> 2;
-    for (int e = tid; e < kTileRows * d4; e += kThreads) {
-        const int rr_ = e / d4, t = (e - rr_ * d4) * 4;
-        const int row = rows_s[rr_];
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (row >= 0) Elem<T>::load4(Q + ((size_t)h * nq + row) * d + t, v);
-        *reinterpret_cast<float4 *>(Qs + rr_ * d + t) = make_float4(v[0], v[1], v[2], v[3]);
-    }
-    int max_row = -1;
-    for (int e = 0; e < n_rows; ++e) max_row = max(max_row, rows_s[e]);
-    const int kend = L.causal ? min(nk, max_row + 1) : nk;
-
-    // per-row selection state (warp-uniform)
-    int my_rows[kRowsPerWarp], my_kend[kRowsPerWarp], cnt[kRowsPerWarp];
-    float thr[kRowsPerWarp];
-#pragma unroll
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        my_rows[r] = rows_s[warp * kRowsPerWarp + r];
-        my_kend[r] = my_rows[r] >= 0 ? valid_keys(my_rows[r], nk, L.causal) : 0;
-        cnt[r] = 0;
-        thr[r] = -INFINITY;
-    }
-
-    for (int kc0 = 0; kc0 < kend; kc0 += kKeyTile) {
-        __syncthreads();  // previous key tile fully consumed
-        for (int e = tid; e < kKeyTile * d4; e += kThreads) {
-            const int key = e / d4, t = (e - key * d4) * 4;
-            const int j = kc0 + key;
-            float v[4] = {0.f, 0.f, 0.f, 0.f};
-            if (j < kend) Elem<T>::load4(K + ((size_t)h * nk + j) * d + t, v);
-#pragma unroll
-            for (int u = 0; u < 4; ++u) Ks[(t + u) * kKeyStride + key] = v[u];
+        if (tid < kTileRows) {
+            int row = -1;
+            if (tid < n_rows) row = use_list ? L.list[(size_t)h * nq + row0 + tid] : row0 + tid;
+            rows_s[tid] = row;
         }
         __syncthreads();
+        // query tile -> shared (fp32), zero rows for empty slots
+        const int d4 = d >> 2;
+        for (int e = tid; e < kTileRows * d4; e += kThreads) {
+            const int rr_ = e / d4, t = (e - rr_ * d4) * 4;
+            const int row = rows_s[rr_];
+            float v[4] = {0.f, 0.f, 0.f, 0.f};
+            if (row >= 0) Elem<T>::load4(Q + ((size_t)h * nq + row) * d + t, v);
+            *reinterpret_cast<float4 *>(Qs + rr_ * d + t) = make_float4(v[0], v[1], v[2], v[3]);
+        }
+        int max_row = -1;
+        for (int e = 0; e < n_rows; ++e) max_row = max(max_row, rows_s[e]);
+        const int kend = L.causal ? min(nk, max_row + 1) : nk;
 
-        float acc[kRowsPerWarp][2];
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) acc[r][0] = acc[r][1] = 0.f;
-        const float4 *Q4 = reinterpret_cast<const float4 *>(Qs + warp * kRowsPerWarp * d);
-        for (int t = 0; t < d; t += 4) {
-            float4 qv[kRowsPerWarp];
-#pragma unroll
-            for (int r = 0; r < kRowsPerWarp; ++r) qv[r] = Q4[r * d4 + (t >> 2)];
-#pragma unroll
-            for (int tt = 0; tt < 4; ++tt) {
-                const float k0 = Ks[(t + tt) * kKeyStride + lane];
-                const float k1 = Ks[(t + tt) * kKeyStride + lane + 32];
-#pragma unroll
-                for (int r = 0; r < kRowsPerWarp; ++r) {
-                    const float qq = tt == 0 ? qv[r].x : tt == 1 ? qv[r].y : tt == 2 ? qv[r].z : qv[r].w;
-                    acc[r][0] = fmaf(qq, k0, acc[r][0]);
-                    acc[r][1] = fmaf(qq, k1, acc[r][1]);
-                }
-            }
+        // per-row selection state (warp-uniform)
+        int my_rows[kRowsPerWarp], my_kend[kRowsPerWarp], cnt[kRowsPerWarp];
+        float thr[kRowsPerWarp];
+    #pragma unroll
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            my_rows[r] = rows_s[warp * kRowsPerWarp + r];
+            my_kend[r] = my_rows[r] >= 0 ? valid_keys(my_rows[r], nk, L.causal) : 0;
+            cnt[r] = 0;
+            thr[r] = -INFINITY;
         }
 
-#pragma unroll
-        for (int r = 0; r < kRowsPerWarp; ++r) {
-            float *bs = bs_all + (warp * kRowsPerWarp + r) * cap;
-            int *bi = bi_all + (warp * kRowsPerWarp + r) * cap;
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-                const int j = kc0 + lane + 32 * u;
-                const float v = acc[r][u];
-                const bool p = j < my_kend[r] && v >= thr[r];
-                const unsigned msk = __ballot_sync(kFull, p);
-                if (msk) {
-                    const int pos = cnt[r] + __popc(msk & lanemask_lt());
-                    if (p) { bs[pos] = v; bi[pos] = j; }
-                    cnt[r] += __popc(msk);
-                    if (cnt[r] > cap - 32) {
-                        __syncwarp();
-                        warp_sort_best_first(bs, bi, cnt[r], cap);
-                        cnt[r] = min(cnt[r], L.ksel);
-                        thr[r] = cnt[r] == L.ksel ? bs[L.ksel - 1] : -INFINITY;
+        for (int kc0 = 0; kc0 < kend; kc0 += kKeyTile) {
+            __syncthreads();  // previous key tile fully consumed
+            for (int e = tid; e < kKeyTile * d4; e += kThreads) {
+                const int key = e / d4, t = (e - key * d4) * 4;
+                const int j = kc0 + key;
+                float v[4] = {0.f, 0.f, 0.f, 0.f};
+                if (j < kend) Elem<T>::load4(K + ((size_t)h * nk + j) * d + t, v);
+    #pragma unroll
+                for (int u = 0; u < 4; ++u) Ks[(t + u) * kKeyStride + key] = v[u];
+            }
+            __syncthreads();
+
+            float acc[kRowsPerWarp][2];
+    #pragma unroll
+            for (int r = 0; r < kRowsPerWarp; ++r) acc[r][0] = acc[r][1] = 0.f;
+            const float4 *Q4 = reinterpret_cast<const float4 *>(Qs + warp * kRowsPerWarp * d);
+            for (int t = 0; t < d; t += 4) {
+                float4 qv[kRowsPerWarp];
+    #pragma unroll
+                for (int r = 0; r < kRowsPerWarp; ++r) qv[r] = Q4[r * d4 + (t >> 2)];
+    #pragma unroll
+                for (int tt = 0; tt < 4; ++tt) {
+                    const float k0 = Ks[(t + tt) * kKeyStride + lane];
+                    const float k1 = Ks[(t + tt) * kKeyStride + lane + 32];
+    #pragma unroll
+                    for (int r = 0; r < kRowsPerWarp; ++r) {
+                        const float qq = tt == 0 ? qv[r].x : tt == 1 ? qv[r].y : tt == 2 ? qv[r].z : qv[r].w;
+                        acc[r][0] = fmaf(qq, k0, acc[r][0]);
+                        acc[r][1] = fmaf(qq, k1, acc[r][1]);
+                    }
+                }
+            }
+
+    #pragma unroll
+            for (int r = 0; r < kRowsPerWarp; ++r) {
+                float *bs = bs_all + (warp * kRowsPerWarp + r) * cap;
+                int *bi = bi_all + (warp * kRowsPerWarp + r) * cap;
+    #pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int j = kc0 + lane + 32 * u;
+                    const float v = acc[r][u];
+                    const bool p = j < my_kend[r] && v >= thr[r];
+                    const unsigned msk = __ballot_sync(kFull, p);
+                    if (msk) {
+                        const int pos = cnt[r] + __popc(msk & lanemask_lt());
+                        if (p) { bs[pos] = v; bi[pos] = j; }
+                        cnt[r] += __popc(msk);
+                        if (cnt[r] > cap - 32) {
+                            __syncwarp();
+                            warp_sort_best_first(bs, bi, cnt[r], cap);
+                            cnt[r] = min(cnt[r], L.ksel);
+                            thr[r] = cnt[r] == L.ksel ? bs[L.ksel - 1] : -INFINITY;
+                        }
                     }
                 }
             }
         }
-    }
 
-    // finish every row of this warp: best-first order, ledger row write
-#pragma unroll 1
-    for (int r = 0; r < kRowsPerWarp; ++r) {
-        const int row = my_rows[r];
-        if (row < 0) continue;
-        float *bs = bs_all + (warp * kRowsPerWarp + r) * cap;
-        int *bi = bi_all + (warp * kRowsPerWarp + r) * cap;
-        __syncwarp();
-        warp_sort_best_first(bs, bi, cnt[r], cap);
-        const int n_valid = my_kend[r];
-        const int nr = min(L.k, n_valid);
-        const int nm = min(L.m, n_valid - nr);
-        const size_t grow = (size_t)h * nq + row;
-        int32_t *out = L.ids + grow * L.c;
-        for (int e = lane; e < L.k + L.m; e += 32) {
-            int id = -1;
-            if (e < L.k) id = e < nr ? bi[e] : -1;
-            else id = (e - L.k) < nm ? bi[nr + e - L.k] : -1;
-            out[e] = id;
+        // finish every row of this warp: best-first order, ledger row write
+    #pragma unroll 1
+        for (int r = 0; r < kRowsPerWarp; ++r) {
+            const int row = my_rows[r];
+            if (row < 0) continue;
+            float *bs = bs_all + (warp * kRowsPerWarp + r) * cap;
+            int *bi = bi_all + (warp * kRowsPerWarp + r) * cap;
+            __syncwarp();
+            warp_sort_best_first(bs, bi, cnt[r], cap);
+            const int n_valid = my_kend[r];
+            const int nr = min(L.k, n_valid);
+            const int nm = min(L.m, n_valid - nr);
+            const size_t grow = (size_t)h * nq + row;
+            int32_t *out = L.ids + grow * L.c;
+            for (int e = lane; e < L.k + L.m; e += 32) {
+                int id = -1;
+                if (e < L.k) id = e < nr ? bi[e] : -1;
+                else id = (e - L.k) < nm ? bi[nr + e - L.k] : -1;
+                out[e] = id;
+            }
+            // mandatory global sentinels (g <= 32), after the random block
+            const int g = L.g_sink + L.g_recent;
+            int n_glob = 0;
+            if (g > 0) {
+                const int jg = lane < g ? global_cand(L, row, lane) : -1;
+                const bool keep = lane < g && global_cand_listable(L, lane, jg, n_valid) &&
+                                  !in_list(bi, nr + nm, jg);
+                const unsigned km = __ballot_sync(kFull, keep);
+                n_glob = __popc(km);
+                int32_t *gout = out + L.k + L.m + L.r;
+                if (keep) gout[__popc(km & lanemask_lt())] = jg;
+                if (lane >= n_glob && lane < g) gout[lane] = -1;
+            }
+            draw_random_sentinels(L, L.bh_offset + h, row, layer, n_valid, bi, nr + nm, n_glob,
+                                  rnd_all + warp * kRandMax, out + L.k + L.m);
+            if (lane == 0) {
+                L.alpha[grow] = bs[nr - 1];
+                L.anchor_layer[grow] = layer;
+                L.flags[grow] = L.rebuild_flag;
+            }
         }
-        // mandatory global sentinels (g <= 32), after the random block
-        const int g = L.g_sink + L.g_recent;
-        int n_glob = 0;
-        if (g > 0) {
-            const int jg = lane < g ? global_cand(L, row, lane) : -1;
-            const bool keep = lane < g && global_cand_listable(L, lane, jg, n_valid) &&
-                              !in_list(bi, nr + nm, jg);
-            const unsigned km = __ballot_sync(kFull, keep);
-            n_glob = __popc(km);
-            int32_t *gout = out + L.k + L.m + L.r;
-            if (keep) gout[__popc(km & lanemask_lt())] = jg;
-            if (lane >= n_glob && lane < g) gout[lane] = -1;
-        }
-        draw_random_sentinels(L, L.bh_offset + h, row, layer, n_valid, bi, nr + nm, n_glob,
-                              rnd_all + warp * kRandMax, out + L.k + L.m);
-        if (lane == 0) {
-            L.alpha[grow] = bs[nr - 1];
-            L.anchor_layer[grow] = layer;
-            L.flags[grow] = L.rebuild_flag;
-        }
-    }
+    }   // row tiles
 }
 
 }  // namespace
 
 cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
-    if (route_rows_tc_supported(L, dtype)) return route_rows_tc_prepare();
+    // this kernel also rebuilds the retry lists of the tensor-core selection
+    // path, so its attribute is set in every case
     const int smem = (int)smem_layout(L.d, select_capacity(L.ksel)).total;
     cudaError_t e;
     if (dtype == kBF16)
@@ -291,6 +295,7 @@ cudaError_t route_rows_prepare(const LedgerDev &L, int dtype) {
     // split fp32 problems: the selection kernel, with this kernel for the
     // rows whose kept scores overflow
     if (e == cudaSuccess && L.split) e = route_select_prepare();
+    if (e == cudaSuccess && route_rows_tc_supported(L, dtype)) e = route_rows_tc_prepare();
     return e;
 }
 
@@ -314,10 +319,12 @@ cudaError_t launch_route_rows(const LedgerDev &L, int dtype, const void *q, cons
 }
 
 cudaError_t launch_route_rows_simt(const LedgerDev &L, int dtype, const void *q, const void *k,
-                                   int layer, bool use_list, cudaStream_t s) {
+                                   int layer, bool use_list, cudaStream_t s, int max_tiles) {
     const int cap = select_capacity(L.ksel);
     const size_t smem = smem_layout(L.d, cap).total;
-    dim3 grid((L.nq + kTileRows - 1) / kTileRows, L.bh);
+    int tiles = (L.nq + kTileRows - 1) / kTileRows;
+    if (max_tiles > 0 && tiles > max_tiles) tiles = max_tiles;   // the CTAs stride over the rest
+    dim3 grid(tiles, L.bh);
     if (dtype == kBF16)
         route_rows_kernel<__nv_bfloat16><<<grid, kThreads, smem, s>>>(
             L, static_cast<const __nv_bfloat16 *>(q), static_cast<const __nv_bfloat16 *>(k), layer,

@@ -941,8 +941,11 @@ cudaError_t launch_route_rows_tc(const LedgerDev &L, const void *q, const void *
     if (e != cudaSuccess) return e;
     dim3 grid((L.nq + tc::kRows - 1) / tc::kRows, L.bh);
     if (L.cand_keys) {
-        // selection kernel + row finishing (rr_select_tc.cu)
+        // selection kernel + row finishing (rr_select_tc.cu); overflowed rows
+        // on the CUDA cores
         e = launch_route_select(L, q, map, layer, use_list, SelectMode::kAnchor, s);
+        if (e != cudaSuccess) return e;
+        return launch_retry_rows_simt(L, q, k, layer, s);
     } else {
         const size_t smem2 = tc::layout_of(L.d, L.ksel, true).total;
         tc::route_rows_tc_kernel<<<grid, tc::kPassThreads, smem2, s>>>(

@@ -25,8 +25,8 @@
 //       chunk asc) by a counting sort over 64 bins with exact ranking inside
 //       a bin, writes route | near-miss and alpha (the k-th score), draws the
 //       random sentinels and adds the global ones.  Rows whose kept scores
-//       overflow their slots go to the exact one-pass heap kernel
-//       (rr_route_tc.cu).
+//       overflow their slots go to a retry list and are routed exactly on
+//       the CUDA cores (route_rows_kernel, rr_route_simt.cu).
 //
 // The relay layer (§3.2 Eq. 5-8, §4.1-4.2) runs the same two kernels over
 // every row and takes the relay decision in route_finish_kernel from the
@@ -1176,18 +1176,19 @@ cudaError_t split_keys(const LedgerDev &L, const void *k, CUtensorMap *map, cuda
     return e;
 }
 
-// Rows whose kept scores overflowed (retry lists): fp32 problems are
-// rebuilt on the CUDA cores, bf16 ones by the tensor-core heap kernel.
-cudaError_t route_retry_any(const LedgerDev &L, const void *q, const void *k, const CUtensorMap &map,
-                            int layer, cudaStream_t s) {
-    if (!L.split) return launch_route_retry(L, q, map, layer, s);
+}  // namespace
+
+// Rows whose kept scores overflowed (retry lists) are rebuilt exactly on the
+// CUDA cores.  The lists are short (usually empty), so the grid is narrow:
+// about four CTAs per SM over all heads, each striding over its head's list.
+cudaError_t launch_retry_rows_simt(const LedgerDev &L, const void *q, const void *k, int layer,
+                                   cudaStream_t s) {
     LedgerDev R = L;
     R.list = L.retry_list;
     R.head_count = L.retry_count;
-    return launch_route_rows_simt(R, kF32, q, k, layer, true, s);
+    const int max_tiles = std::max(1, (4 * 148 + L.bh - 1) / L.bh);
+    return launch_route_rows_simt(R, L.split ? kF32 : kBF16, q, k, layer, true, s, max_tiles);
 }
-
-}  // namespace
 
 cudaError_t launch_route_rows_split(const LedgerDev &L, const void *q, const void *k, int layer,
                                     bool use_list, cudaStream_t s) {
@@ -1196,7 +1197,7 @@ cudaError_t launch_route_rows_split(const LedgerDev &L, const void *q, const voi
     if (e == cudaSuccess) e = cudaMemsetAsync(L.retry_count, 0, (size_t)L.bh * sizeof(int32_t), s);
     if (e == cudaSuccess) e = launch_route_select(L, q, map, layer, use_list, SelectMode::kAnchor, s);
     if (e != cudaSuccess) return e;
-    return route_retry_any(L, q, k, map, layer, s);
+    return launch_retry_rows_simt(L, q, k, layer, s);
 }
 
 cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *k, int layer,
@@ -1221,7 +1222,7 @@ cudaError_t launch_relay_oneshot(const LedgerDev &L, const void *q, const void *
     }
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    return route_retry_any(L, q, k, map, layer, s);
+    return launch_retry_rows_simt(L, q, k, layer, s);
 }
 
 }  // namespace rr
