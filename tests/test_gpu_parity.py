@@ -265,6 +265,38 @@ def test_equal_scores_pick_lowest_chunks(rr, dtype, d):
         assert int(out["counters"][rr.CNT_RETRY_TOTAL]) > 0
 
 
+def test_retry_lists_longer_than_the_retry_grid(rr):
+    """Equal keys again, with 640 heads: the retry launch has one CTA per head
+    (about four per SM over all heads), and each head's 172 overflowing rows
+    (the rows with more than 128 valid chunks) take six tiles of 32, so every
+    retry CTA strides over several tiles.  Checked on every row of every
+    head, after the anchor layer and after a relay layer (equal scores:
+    alpha = beta, every row challenged and rebuilt)."""
+    bh, n, d, k, m, r = 640, 300, 64, 8, 6, 4
+    cfg = rr.Config(bh=bh, nq=n, nk=n, d=d, k=k, m_near=m, r_rand=r, dtype="bf16", causal=True)
+    g = torch.Generator().manual_seed(11)
+    q = torch.randn((bh, n, d), generator=g).to(torch.bfloat16).to(DEV)
+    kk = torch.randn((bh, 1, d), generator=g).expand(bh, n, d).contiguous().to(torch.bfloat16).to(DEV)
+    led = rr.RouteLedger(cfg, DEV)
+    nv = np.arange(1, n + 1)
+    nr = np.minimum(k, nv)
+    nm = np.minimum(m, nv - nr)
+    want = np.full((n, k + m), -1, dtype=np.int64)
+    for i in range(n):
+        want[i, :nr[i]] = np.arange(nr[i])
+        want[i, k:k + nm[i]] = np.arange(nr[i], nr[i] + nm[i])
+    for layer, call in ((0, led.full_route), (1, led.relay_layer)):
+        call(q, kk, layer)
+        out = led.read()
+        ids = out["ids"].numpy().astype(np.int64)
+        assert np.array_equal(ids[:, :, :k + m], np.broadcast_to(want, (bh, n, k + m))), layer
+        rand = ids[:, :, k + m:]
+        lo = (nr + nm)[None, :, None]
+        ok = (rand == -1) | ((rand >= lo) & (rand < nv[None, :, None]))
+        assert ok.all(), layer
+        assert int(out["counters"][rr.CNT_RETRY_TOTAL]) >= (layer + 1) * bh * (n - 128)
+
+
 def test_retry_path_is_rare_on_the_full_size_workload(rr):
     """On the bf16 workload the three-pass certificate should hold for nearly
     every row (the retry path is a safety net, not the common case)."""
