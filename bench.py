@@ -137,22 +137,32 @@ def make_inputs(w, device, seed):
     return qs, ks
 
 
+def code_sha256(path: str) -> str:
+    """sha256 of a C/CUDA source's code: comments removed, each line stripped
+    of surrounding blanks, blank lines dropped (a comment-only edit keeps it)."""
+    import hashlib
+    import re
+    text = open(path, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    lines = [re.sub(r"//.*$", "", ln).strip() for ln in text.splitlines()]
+    return hashlib.sha256("\n".join(ln for ln in lines if ln).encode()).hexdigest()
+
+
 def profiled_traffic_per_row(kernel_file: str, summary_glob: str):
     """DRAM bytes per routed row from a committed ncu summary, or None when
-    the kernel source changed since the counters were taken."""
+    the kernel source's code changed since the counters were taken."""
     import glob
-    import hashlib
     src = os.path.join(ROOT, "cross_layer_route_b200", "csrc", kernel_file)
     if not os.path.exists(src):
         return None
-    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    sha = code_sha256(src)
     for path in glob.glob(os.path.join(ROOT, "profiles", summary_glob)):
         vals = {}
         for line in open(path):
-            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_row", "source_sha256"):
+            if ":" in line and line.split(":")[0] in ("traffic_bytes_per_row", "code_sha256"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-        if vals.get("source_sha256") == sha and "traffic_bytes_per_row" in vals:
+        if vals.get("code_sha256") == sha and "traffic_bytes_per_row" in vals:
             return float(vals["traffic_bytes_per_row"])
     return None
 

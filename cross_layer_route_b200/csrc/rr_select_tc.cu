@@ -22,7 +22,7 @@
 //       Each thread then turns its kept scores into (score, chunk) sort keys
 //       and the row's keys go to its record in device memory.
 //   route_finish_kernel  (one warp per row) orders the keys (score desc,
-//       chunk asc) by a counting sort over 64 bins with exact ranking inside
+//       chunk asc) by a counting sort over 128 bins with exact ranking inside
 //       a bin, writes route | near-miss and alpha (the k-th score), draws the
 //       random sentinels and adds the global ones.  Rows whose kept scores
 //       overflow their slots go to a retry list and are routed exactly on

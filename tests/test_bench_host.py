@@ -45,12 +45,16 @@ def test_profiled_traffic_needs_the_profiled_source(tmp_path, monkeypatch):
     (tmp_path / "cross_layer_route_b200" / "csrc").mkdir(parents=True)
     (tmp_path / "profiles").mkdir()
     src = tmp_path / "cross_layer_route_b200" / "csrc" / "k.cu"
-    src.write_text("kernel v1\n")
-    sha = hashlib.sha256(b"kernel v1\n").hexdigest()
-    (tmp_path / "profiles" / "k__case.md").write_text(f"x\ntraffic_bytes_per_row: 1234\nsource_sha256: {sha}\n")
+    src.write_text("int k(int x) {  // v1\n    return x + 1;\n}\n")
+    sha = hashlib.sha256(b"int k(int x) {\nreturn x + 1;\n}").hexdigest()
+    assert bench.code_sha256(str(src)) == sha
+    (tmp_path / "profiles" / "k__case.md").write_text(f"x\ntraffic_bytes_per_row: 1234\ncode_sha256: {sha}\n")
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.profiled_traffic_per_row("k.cu", "k__*.md") == 1234.0
-    src.write_text("kernel v2\n")                       # the kernel changed: the counters are stale
+    # comments and blank lines only: the same code, the counters still hold
+    src.write_text("/* the kernel */\nint k(int x) {  // v1, reworded\n\n    return x + 1;\n}\n")
+    assert bench.profiled_traffic_per_row("k.cu", "k__*.md") == 1234.0
+    src.write_text("int k(int x) {\n    return x + 2;\n}\n")   # the code changed: the counters are stale
     assert bench.profiled_traffic_per_row("k.cu", "k__*.md") is None
 
 
