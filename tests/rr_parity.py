@@ -217,7 +217,6 @@ def layer_stepped(w, rr, led, layers, heads, device, stream_device="cpu", report
     must match what the ledger was given with set_guard.  Returns (total
     report, per-layer list)."""
     import rr_workloads
-    import torch
     st = rr_workloads.LayerStream(w, stream_device)
     p = params_of(w, max_age=max_age, min_reuse=min_reuse, g_sink=g_sink, g_recent=g_recent,
                   gamma_h=gamma_h)

@@ -9,7 +9,6 @@ wrong counting rule).
 import math
 import os
 import subprocess
-import sys
 
 import numpy as np
 import pytest
