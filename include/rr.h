@@ -99,8 +99,8 @@ enum {
     RR_CNT_DRAW_CAP = 7,      /* rows whose random draws hit the draw cap and were filled in order */
     RR_CNT_FULL_PAIRS = 8,    /* score pairs of the rows fully routed at the last layer */
     RR_CNT_FULL_PAIRS_TOTAL = 9, /* the same, since rr_ledger_create */
-    RR_CNT_RETRY_TOTAL = 10,  /* rows whose tensor-core selection took the one-pass exact
-                                 path (kept scores overflowed the two-pass buffer), since create */
+    RR_CNT_RETRY_TOTAL = 10,  /* rows whose tensor-core selection was redone exactly (kept
+                                 scores overflowed the record, or a wait ran out), since create */
     RR_NUM_COUNTERS = 16      /* slots 11..15 are reserved (0) */
 };
 
@@ -111,8 +111,10 @@ enum {
  * [bh*nq] u8, counters [16] int64 -- plus the library's per-layer scratch
  * (refresh lists and counts; for problems routed on the tensor cores also
  * the kept scores each row hands from the selection kernel to the kernel
- * that orders them: 120 x 6 bytes + 4 per row, rows rounded up to 128 per
- * head).  Pure host arithmetic. */
+ * that orders them: 128 sort keys of 8 bytes and an 8-byte count and
+ * threshold per row, rows rounded up to 128 per head, the list of relay rows
+ * left for exact rescoring, and for fp32 problems the keys split into three
+ * bf16 parts, 3 d bf16 per key row).  Pure host arithmetic. */
 size_t rr_ledger_workspace_bytes(const rr_config *cfg);
 
 /* Validates cfg, carves the ledger out of d_workspace (device memory of at
@@ -291,7 +293,7 @@ rr_status rr_route_layer_static(const rr_config *cfg, const void *d_qc, const vo
  * second, which only a stalled GPU exhausts).  Every wait in the tensor-core
  * kernels is bounded; when one runs out the CTA stops issuing, drains its
  * copies, waits for its last MMA, frees its TMEM and sets bit 1 of the error
- * word, and its rows are redone by the exact one-pass path.  A short budget
+ * word, and its rows are redone exactly on the retry path.  A short budget
  * makes that happen on purpose, so a test can check the path; production
  * callers leave it at 0.  No CUDA call; RR_EINVAL for a NULL ledger or a
  * negative budget. */
